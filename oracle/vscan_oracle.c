@@ -1,0 +1,379 @@
+/*
+ * vscan_oracle.c -- plain fp64 CPU oracle for the routed visual selective scan.
+ *
+ * TEST INFRASTRUCTURE ONLY. This file is the slow, obviously-correct statement
+ * of what the routed selective scan computes. It is used by the tests, by
+ * __graft_entry__.smoke() and by the cpu_baseline / reference legs of bench.py,
+ * and by nothing else. It shares no code, header, table or helper with the
+ * CUDA library under vision_selective_state_b200/csrc, and it never calls it.
+ *
+ * Every step follows the pages it cites, in their order and notation:
+ *
+ *   [Vim]   "Vision Mamba: Bidirectional State Space Models for Images"
+ *           (abhik.ai review): sec. 3 "Choose the state update from the current
+ *           content", sec. 4 "Keep a running state, then read it", sec. 5 "Align
+ *           the backward scan before combining", and the prose section "Two
+ *           scans meet at the same token".
+ *   [EVM]   "EfficientVMamba: Atrous Selective Scan for Light Weight Visual
+ *           Mamba" (abhik.ai review): sec. 1 "Gather spatial residues into
+ *           ordered streams", sec. 2 "Update an independent state inside each
+ *           group", sec. 3 "Invert the routing, then crop the padding", and the
+ *           prose section "Merge restores coordinates instead of adding
+ *           directions".
+ *   [FVim]  "Fast Vision Mamba: Pooling Spatial Dimensions for Accelerated
+ *           Processing" (gptget.net summary): "Methodology" list.
+ *   [NoD]   "Norm or Direction? Decoding Vision Mambas for High-Resolution
+ *           Vision": sec. 3 Background, Eq. 1-2 and "2D Selective Scan (SS2D)".
+ *
+ * Readings taken where the pages are silent or ambiguous (each one is listed
+ * with its reason in the design notes at the repository root):
+ *   - merge of several directions: summed, then multiplied by merge_scale
+ *     (1 = sum as in SS2D and Vim's Algorithm 1; 0.5 = the released Vim average);
+ *   - atrous padding slots carry u = rawDelta = B = C = 0, so Delta is
+ *     softplus(bias) and the state still decays across them;
+ *   - pooled route: u, rawDelta, B and C are mean-pooled over the pooled axis
+ *     before the bias and softplus; the whole scan (including D*u) runs on the
+ *     pooled tokens; the result is repeated over the pooled axis and then gated
+ *     with the un-pooled z of every grid token;
+ *   - input write is Delta*B*u (the released convention), not exact ZOH;
+ *   - softplus is the exact log(1 + e^x), evaluated without a threshold.
+ */
+#include <math.h>
+#include <omp.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Route kinds. The numbering is part of the oracle's own interface. */
+#define OR_BIDIR 0   /* [Vim] forward + whole-sequence reverse               */
+#define OR_CROSS4 1  /* [NoD] SS2D: row fwd, row rev, column fwd, column rev  */
+#define OR_ATROUS2 2 /* [EVM] p=2 residue groups, right/bottom zero padding   */
+#define OR_POOL_W 3  /* [FVim] mean over columns -> length h, fwd + bwd      */
+#define OR_POOL_H 4  /* [FVim] mean over rows    -> length w, fwd + bwd      */
+
+#define OR_OK 0
+#define OR_EINVAL -1
+#define OR_ENOMEM -6
+#define OR_EOWNER -9 /* a real pixel was written by zero or by two atrous streams */
+
+/* ------------------------------------------------------------------------- */
+/* Geometry: number of directions K, sequence length L per direction and the  */
+/* number of tokens per image in the token array (grid + optional CLS).        */
+/* ------------------------------------------------------------------------- */
+int oracle_geometry(int kind, int h, int w, int cls_pos, int* K, int* L, int* tokens)
+{
+    if (h <= 0 || w <= 0) return OR_EINVAL;
+    int hw = h * w;
+    switch (kind) {
+    case OR_BIDIR:
+        /* [Vim] "Insert the class token": CLS sits at floor(P/2) of the P
+         * patches, giving P + 1 tokens; both scans run over all of them. */
+        if (cls_pos != -1 && cls_pos != hw / 2) return OR_EINVAL;
+        *K = 2;
+        *tokens = hw + (cls_pos >= 0 ? 1 : 0);
+        *L = *tokens;
+        return OR_OK;
+    case OR_CROSS4:
+        if (cls_pos != -1) return OR_EINVAL;
+        *K = 4; *L = hw; *tokens = hw;
+        return OR_OK;
+    case OR_ATROUS2:
+        if (cls_pos != -1) return OR_EINVAL;
+        /* [EVM] sec. 1: four lists of ceil(H/2) x ceil(W/2). */
+        *K = 4; *L = ((h + 1) / 2) * ((w + 1) / 2); *tokens = hw;
+        return OR_OK;
+    case OR_POOL_W:
+        if (cls_pos != -1) return OR_EINVAL;
+        *K = 2; *L = h; *tokens = hw;
+        return OR_OK;
+    case OR_POOL_H:
+        if (cls_pos != -1) return OR_EINVAL;
+        *K = 2; *L = w; *tokens = hw;
+        return OR_OK;
+    default:
+        return OR_EINVAL;
+    }
+}
+
+/*
+ * Route coordinates, written as explicit coordinate loops.
+ * out[k*L + t] = index (into the token array, or into the pooled sequence for
+ * the pooled routes) visited by step t of direction k, or -1 for a padding slot.
+ */
+int oracle_route(int kind, int h, int w, int cls_pos, int64_t* out)
+{
+    int K, L, tokens;
+    int rc = oracle_geometry(kind, h, w, cls_pos, &K, &L, &tokens);
+    if (rc != OR_OK) return rc;
+
+    if (kind == OR_BIDIR || kind == OR_POOL_W || kind == OR_POOL_H) {
+        /* [Vim] "Two scans meet at the same token": the forward scan takes the
+         * sequence in order, the backward scan the entire reversed sequence. */
+        for (int t = 0; t < L; ++t) {
+            out[0 * L + t] = t;
+            out[1 * L + t] = L - 1 - t;
+        }
+        return OR_OK;
+    }
+
+    if (kind == OR_CROSS4) {
+        /* [NoD] SS2D: the four traversals are the row-major order, its reverse,
+         * the column-major order and its reverse. Tokens are stored row-major
+         * (columns fastest), as the Vim patch flattening fixes. */
+        int64_t* row = out + 0 * (int64_t)L;
+        int64_t* col = out + 2 * (int64_t)L;
+        int t = 0;
+        for (int r = 0; r < h; ++r)
+            for (int c = 0; c < w; ++c) row[t++] = (int64_t)r * w + c;
+        t = 0;
+        for (int c = 0; c < w; ++c)
+            for (int r = 0; r < h; ++r) col[t++] = (int64_t)r * w + c;
+        for (int s = 0; s < L; ++s) {
+            out[1 * (int64_t)L + s] = row[L - 1 - s];
+            out[3 * (int64_t)L + s] = col[L - 1 - s];
+        }
+        return OR_OK;
+    }
+
+    /* OR_ATROUS2. [EVM] sec. 1: O_k[t] = X[2 r_t + m_k, 2 c_t + n_k] with
+     * offsets (m_k, n_k) = (0,0), (1,0), (0,1), (1,1) in (row, column); groups
+     * 0 and 2 walk their residue sub-grid row-major, groups 1 and 3 walk it
+     * column-major; coordinates beyond the H x W map are right/bottom padding. */
+    const int dy[4] = {0, 1, 0, 1};
+    const int dx[4] = {0, 0, 1, 1};
+    int rows = (h + 1) / 2, cols = (w + 1) / 2;
+    for (int k = 0; k < 4; ++k) {
+        int t = 0;
+        if (k == 0 || k == 2) {
+            for (int a = 0; a < rows; ++a)
+                for (int b = 0; b < cols; ++b) {
+                    int y = 2 * a + dy[k], x = 2 * b + dx[k];
+                    out[(int64_t)k * L + t++] = (y < h && x < w) ? (int64_t)y * w + x : -1;
+                }
+        } else {
+            for (int a = 0; a < cols; ++a)
+                for (int b = 0; b < rows; ++b) {
+                    int y = 2 * b + dy[k], x = 2 * a + dx[k];
+                    out[(int64_t)k * L + t++] = (y < h && x < w) ? (int64_t)y * w + x : -1;
+                }
+        }
+    }
+    return OR_OK;
+}
+
+/* softplus(x) = log(1 + e^x), evaluated as max(x, 0) + log1p(e^-|x|), which is
+ * the same real function written so that no term overflows. [Vim] sec. 3. */
+static double softplus(double x)
+{
+    return (x > 0.0 ? x : 0.0) + log1p(exp(-fabs(x)));
+}
+
+/* SiLU(z) = z * sigma(z), sigma(z) = 1 / (1 + e^-z). [Vim] sec. 5 and the
+ * prose under "Inside the released Vim block". */
+static double silu(double z)
+{
+    return z / (1.0 + exp(-z));
+}
+
+/*
+ * One selective scan over one sequence of one channel, [Vim] sec. 4 and
+ * [EVM] sec. 2:
+ *     h_t = exp(dt_t * A) (.) h_{t-1} + dt_t * B_t * u_t,   h_{-1} = 0
+ *     y_t = sum_n C_{t,n} h_{t,n} + D * u_t
+ * dt is the already-discretized step (after bias and softplus).
+ * B and C are [L][N]; A is [N]; u, dt, y are [L]. h is caller scratch [N].
+ */
+void oracle_scan_sequence(int L, int N, const double* u, const double* dt, const double* A,
+                          const double* B, const double* C, double D, double* h, double* y)
+{
+    for (int n = 0; n < N; ++n) h[n] = 0.0;
+    for (int t = 0; t < L; ++t) {
+        double read = 0.0;
+        for (int n = 0; n < N; ++n) {
+            double retention = exp(dt[t] * A[n]);
+            double write = dt[t] * B[(int64_t)t * N + n] * u[t];
+            h[n] = retention * h[n] + write;
+            read += C[(int64_t)t * N + n] * h[n];
+        }
+        y[t] = read + D * u[t];
+    }
+}
+
+/*
+ * Routed forward pass.
+ *
+ * Layouts (row-major, element strides):
+ *   u, delta : [Ki][batch][tokens][D]   delta is the raw step, before bias/softplus
+ *   B, C     : [Ki][batch][tokens][N]
+ *   A        : [Kp][D][N]
+ *   Dskip    : [Kp][D]      (nullable: no skip term)
+ *   bias     : [Kp][D]      (nullable: no bias)
+ *   z        : [batch][tokens][D] (nullable: no gate); the gate is shared by all
+ *              directions ([Vim] "Inside the released Vim block").
+ *   y        : [batch][tokens][D]   output
+ * Ki = K when per_dir_inputs, else 1; Kp = K when per_dir_params, else 1.
+ * Every (batch, channel) pair is independent; channels and batches are
+ * processed by OpenMP threads (nthreads <= 0: the OpenMP default).
+ */
+int oracle_forward(int kind, int h, int w, int cls_pos, int batch, int D, int N,
+                   const double* u, const double* delta, const double* A,
+                   const double* B, const double* C, const double* Dskip,
+                   const double* bias, const double* z, int delta_softplus,
+                   double merge_scale, int per_dir_inputs, int per_dir_params,
+                   double* y, int nthreads)
+{
+    int K, L, tokens;
+    int rc = oracle_geometry(kind, h, w, cls_pos, &K, &L, &tokens);
+    if (rc != OR_OK) return rc;
+    if (batch < 0 || D <= 0 || N <= 0) return OR_EINVAL;
+    if (batch == 0) return OR_OK;
+
+    int64_t* route = (int64_t*)malloc(sizeof(int64_t) * (size_t)K * L);
+    if (!route) return OR_ENOMEM;
+    rc = oracle_route(kind, h, w, cls_pos, route);
+    if (rc != OR_OK) { free(route); return rc; }
+
+    const int pooled = (kind == OR_POOL_W || kind == OR_POOL_H);
+    const int64_t in_dir = per_dir_inputs ? (int64_t)batch * tokens * D : 0;
+    const int64_t bc_dir = per_dir_inputs ? (int64_t)batch * tokens * N : 0;
+    const int64_t a_dir = per_dir_params ? (int64_t)D * N : 0;
+    const int64_t v_dir = per_dir_params ? (int64_t)D : 0;
+
+    int failed = 0; /* bit 0: scratch allocation failed; bit 1: atrous owner check failed */
+    int64_t pairs = (int64_t)batch * D;
+    int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+
+#pragma omp parallel num_threads(nt) reduction(| : failed)
+    {
+        /* per-thread scratch */
+        double* su = (double*)malloc(sizeof(double) * L);
+        double* sdt = (double*)malloc(sizeof(double) * L);
+        double* sB = (double*)malloc(sizeof(double) * (size_t)L * N);
+        double* sC = (double*)malloc(sizeof(double) * (size_t)L * N);
+        double* sy = (double*)malloc(sizeof(double) * L);
+        double* hs = (double*)malloc(sizeof(double) * N);
+        double* acc = (double*)malloc(sizeof(double) * (pooled ? L : tokens));
+        int* owners = (int*)malloc(sizeof(int) * tokens);
+        int bad = (!su || !sdt || !sB || !sC || !sy || !hs || !acc || !owners);
+        if (bad) failed |= 1;
+
+#pragma omp for schedule(static)
+        for (int64_t pr = 0; pr < pairs; ++pr) {
+            if (bad) continue;
+            int bi = (int)(pr / D);
+            int d = (int)(pr % D);
+
+            for (int i = 0; i < (pooled ? L : tokens); ++i) acc[i] = 0.0;
+            for (int i = 0; i < tokens; ++i) owners[i] = 0;
+
+            for (int k = 0; k < K; ++k) {
+                const double* uk = u + k * in_dir + (int64_t)bi * tokens * D;
+                const double* dk = delta + k * in_dir + (int64_t)bi * tokens * D;
+                const double* Bk = B + k * bc_dir + (int64_t)bi * tokens * N;
+                const double* Ck = C + k * bc_dir + (int64_t)bi * tokens * N;
+                const double* Ak = A + k * a_dir + (int64_t)d * N;
+                double Dk = Dskip ? Dskip[k * v_dir + d] : 0.0;
+                double bk = bias ? bias[k * v_dir + d] : 0.0;
+
+                /* Gather: one sequence step per route step. */
+                for (int t = 0; t < L; ++t) {
+                    int64_t q = route[(int64_t)k * L + t];
+                    double uu = 0.0, dd = 0.0;
+                    if (!pooled) {
+                        if (q >= 0) { /* a real token */
+                            uu = uk[q * D + d];
+                            dd = dk[q * D + d];
+                            for (int n = 0; n < N; ++n) {
+                                sB[(int64_t)t * N + n] = Bk[q * N + n];
+                                sC[(int64_t)t * N + n] = Ck[q * N + n];
+                            }
+                        } else { /* [EVM] sec. 1: padding supplies zeros */
+                            for (int n = 0; n < N; ++n) {
+                                sB[(int64_t)t * N + n] = 0.0;
+                                sC[(int64_t)t * N + n] = 0.0;
+                            }
+                        }
+                    } else {
+                        /* [FVim] Methodology: mean-pool one spatial axis. For
+                         * POOL_W pooled token q is grid row q averaged over its
+                         * w columns; for POOL_H it is column q averaged over
+                         * its h rows. */
+                        int cnt = (kind == OR_POOL_W) ? w : h;
+                        double su_ = 0.0, sd_ = 0.0;
+                        for (int n = 0; n < N; ++n) {
+                            sB[(int64_t)t * N + n] = 0.0;
+                            sC[(int64_t)t * N + n] = 0.0;
+                        }
+                        for (int j = 0; j < cnt; ++j) {
+                            int64_t tok = (kind == OR_POOL_W) ? q * w + j : (int64_t)j * w + q;
+                            su_ += uk[tok * D + d];
+                            sd_ += dk[tok * D + d];
+                            for (int n = 0; n < N; ++n) {
+                                sB[(int64_t)t * N + n] += Bk[tok * N + n];
+                                sC[(int64_t)t * N + n] += Ck[tok * N + n];
+                            }
+                        }
+                        uu = su_ / cnt;
+                        dd = sd_ / cnt;
+                        for (int n = 0; n < N; ++n) {
+                            sB[(int64_t)t * N + n] /= cnt;
+                            sC[(int64_t)t * N + n] /= cnt;
+                        }
+                    }
+                    /* Discretization, [Vim] sec. 3 and sec. 4: bias, then softplus. */
+                    double x = dd + bk;
+                    su[t] = uu;
+                    sdt[t] = delta_softplus ? softplus(x) : x;
+                }
+
+                oracle_scan_sequence(L, N, su, sdt, Ak, sB, sC, Dk, hs, sy);
+
+                /* Scatter back to the original coordinates. */
+                for (int t = 0; t < L; ++t) {
+                    int64_t q = route[(int64_t)k * L + t];
+                    if (q < 0) continue; /* [EVM] sec. 3: crop padding */
+                    if (kind == OR_ATROUS2) {
+                        /* [EVM] sec. 3: one owner per coordinate, assignment. */
+                        acc[q] = sy[t];
+                        owners[q] += 1;
+                    } else {
+                        /* [Vim] sec. 5 / [NoD] SS2D: aligned outputs are added. */
+                        acc[q] += sy[t];
+                    }
+                }
+            }
+
+            if (kind == OR_ATROUS2) {
+                for (int i = 0; i < tokens; ++i)
+                    if (owners[i] != 1) failed |= 2;
+            }
+
+            /* Merge scale, repeat (pooled routes), then the shared SiLU gate. */
+            double* yb = y + (int64_t)bi * tokens * D;
+            const double* zb = z ? z + (int64_t)bi * tokens * D : 0;
+            for (int i = 0; i < tokens; ++i) {
+                double v;
+                if (!pooled) {
+                    v = acc[i];
+                } else {
+                    int r = i / w, c = i % w;
+                    v = acc[kind == OR_POOL_W ? r : c];
+                }
+                v *= merge_scale;
+                if (zb) v *= silu(zb[(int64_t)i * D + d]);
+                yb[(int64_t)i * D + d] = v;
+            }
+        }
+        free(su); free(sdt); free(sB); free(sC); free(sy); free(hs); free(acc); free(owners);
+    }
+    free(route);
+    if (failed & 1) return OR_ENOMEM;
+    if (failed & 2) return OR_EOWNER;
+    return OR_OK;
+}
+
+/* Number of OpenMP threads oracle_forward uses when nthreads <= 0. */
+int oracle_default_threads(void)
+{
+    return omp_get_max_threads();
+}
