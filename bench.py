@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Throughput of the routed visual selective scan on B200, as one JSON line.
+
+A step is one pass of the whole fused path (gather, discretization,
+recurrence, read-out, merge, gate, store) over one batch of every grid of the
+selected workload. The default workload is the EfficientVMamba atrous p=2 scan:
+batch 8, d_inner 192, N 16, float32, on the 56x56 grid and on the odd 55x57
+grid (zero-padded to 56x58); one step runs both.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank scans its own
+seeded copy of the workload (weak scaling, no collective on the data path);
+the timed region is bracketed by a barrier and a synchronize, and the time
+is the maximum over ranks. --impl reference times the fp64 CPU oracle on the
+host cores instead (rank 0 only).
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "scan throughput tokens·ch/s at 1 B200; achieved HBM GB/s vs peak"
+UNIT = "tokens·ch/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=4000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="1",
+                   help="configuration index 0-4 or a workload name (default 1: atrous 56x56 + 55x57)")
+    p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline budget")
+    return p.parse_args()
+
+
+def select(spec):
+    if spec.isdigit():
+        names = workloads.CONFIG_GROUPS[int(spec)]
+    else:
+        names = [spec]
+    return [workloads.WORKLOADS[n] for n in names]
+
+
+def workload_label(wls):
+    w0 = wls[0]
+    grids = "+".join(f"{w.h}x{w.w}" for w in wls)
+    cls = "_cls" if w0.cls_pos >= 0 else ""
+    return f"{w0.route}_{grids}{cls}_b{w0.batch}_d{w0.D}_n{w0.N}_{w0.dtype}"
+
+
+def algorithmic_bytes(wl):
+    """Compulsory HBM bytes of one forward: read u, raw delta, z, B, C; write y."""
+    eb = 2 if wl.dtype == "bf16" else 4
+    per_token = (3 * wl.D + 2 * wl.N) * eb + wl.D * eb
+    params = (wl.D * wl.N + 2 * wl.D) * 4
+    return wl.batch * wl.tokens * per_token + params
+
+
+def seq_geometry(wl):
+    K = {"bidir": 2, "cross4": 4, "atrous2": 4, "pool_w": 2, "pool_h": 2}[wl.route]
+    if wl.route == "atrous2":
+        L = ((wl.h + 1) // 2) * ((wl.w + 1) // 2)
+    elif wl.route == "pool_w":
+        L = wl.h
+    elif wl.route == "pool_h":
+        L = wl.w
+    else:
+        L = wl.tokens
+    return K, L
+
+
+def updates(wl):
+    """Recurrence steps x states of one forward (padding steps included)."""
+    K, L = seq_geometry(wl)
+    return wl.batch * K * L * wl.D * wl.N
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured", float(d.get("sm_max_mhz", 1965.0))
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback", 1965.0
+
+
+def source_digest():
+    csrc = os.path.join(ROOT, "vision_selective_state_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """dram read+write bytes per launch from a committed ncu summary, if the
+    kernel sources have not changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    digest = source_digest()
+    with open(path) as f:
+        for ln in f:
+            if ln.startswith("#") or not ln.strip():
+                continue
+            k, wl, dig, val = ln.split()[:4]
+            if k == kernel and wl == workload and dig == digest:
+                return float(val)
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML during a region."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, interval=0.02):
+        self.index, self.interval = index, interval
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.nvml = None
+            self.error = str(e)
+
+    def _reason_mask(self):
+        fn = getattr(self.nvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(self.nvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return fn(self.handle)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample_once()
+            self._stop.wait(self.interval)
+
+    def sample_once(self):
+        if self.nvml is None:
+            return
+        try:
+            self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
+            mask = self._reason_mask()
+            for bit, name in self.REASONS.items():
+                if mask & bit:
+                    self.reasons.add(name)
+        except Exception:  # noqa: BLE001
+            pass
+
+    def start(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        self.sample_once()
+
+    def summary(self):
+        if self.nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "error": getattr(self, "error", "nvml unavailable")}
+        reasons = sorted(self.reasons - {"gpu_idle"})
+        return {"sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples),
+                "source": "nvml, 20 ms interval, during the timed region"}
+
+
+# ------------------------------------------------------------------ distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_time(wls, channels, threads=0):
+    """Seconds the fp64 oracle takes for the given channel subset of every grid."""
+    import oracle
+    total = 0.0
+    for wl in wls:
+        x = workloads.channel_slice(workloads.draw(wl), channels)
+        t0 = time.perf_counter()
+        oracle.forward(wl.route, wl.h, wl.w, x["u"], x["delta"], x["A"], x["B"], x["C"], x["Dskip"],
+                       x["bias"], x["z"] if wl.gate else None, cls_pos=wl.cls_pos, threads=threads)
+        total += time.perf_counter() - t0
+    return total
+
+
+def cpu_baseline(wls, budget_s):
+    """The oracle as it stands, on the host cores, on a bounded channel sample."""
+    import oracle
+    cores = oracle.default_threads()
+    D = wls[0].D
+    t1 = oracle_time(wls, list(range(min(cores, D))))
+    per_channel = t1 / min(cores, D)
+    nch = int(max(1, min(D, budget_s / max(per_channel, 1e-9))))
+    chans = list(range(nch))
+    t = oracle_time(wls, chans)
+    units = sum(w.batch * w.tokens * nch for w in wls)
+    return {"value": units / t, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"all images and tokens of every grid, {nch} of {D} channels, one pass, fp64",
+            "seconds": round(t, 3)}
+
+
+def run_reference(args, wls):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    cores = oracle.default_threads()
+    D = wls[0].D
+    probe = oracle_time(wls, [0])
+    steps_total = args.steps + args.warmup
+    budget = 150.0  # seconds for the whole run
+    nch = int(max(1, min(D, budget / steps_total / max(probe, 1e-6))))
+    chans = list(range(nch))
+    for _ in range(args.warmup):
+        oracle_time(wls, chans)
+    t = 0.0
+    for _ in range(args.steps):
+        t += oracle_time(wls, chans)
+    units = sum(w.batch * w.tokens * nch for w in wls) * args.steps
+    value = units / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic, seeded (page-workload shapes and value recipe)",
+        "config": config_block(wls, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: all images and tokens of every grid, {nch} of {D} channels"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_block(wls, n):
+    w0 = wls[0]
+    return {"workload": workload_label(wls), "route": w0.route,
+            "grids": [f"{w.h}x{w.w}" for w in wls], "batch": w0.batch, "d_inner": w0.D,
+            "d_state": w0.N, "io_dtype": w0.dtype, "gate": w0.gate, "merge_scale": w0.merge_scale,
+            "parallelism": f"replicas x{n} (one full workload per GPU, no collective)"}
+
+
+# ------------------------------------------------------------------ our path
+def run_ours(args, wls):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    import vision_selective_state_b200 as vs
+
+    stream = torch.cuda.Stream(dev)
+    td = {"f32": torch.float32, "bf16": torch.bfloat16}
+    # Rotate several device copies of every input so that no step finds its
+    # inputs in the 126 MB L2 left by the previous step.
+    step_bytes = sum(algorithmic_bytes(w) for w in wls)
+    rot = max(2, -(-3 * L2_BYTES // step_bytes) + 1)
+    rot = min(rot, 8)
+    plans, host_sets, routes = [], [], []
+    for wi, wl in enumerate(wls):
+        seeded = wl.with_(seed=wl.seed + 1000 * rank)
+        x = workloads.draw(seeded)
+        route = vs.Route(wl.route, wl.h, wl.w, wl.cls_pos)
+        routes.append(route)
+        dt = td[wl.dtype]
+        host = {k: torch.from_numpy(x[k]).to(dt) for k in ("u", "delta", "B", "C", "z")}
+        host.update({k: torch.from_numpy(np.ascontiguousarray(x[k], dtype=np.float32))
+                     for k in ("A", "Dskip", "bias")})
+        host_sets.append(host)
+        ws_bytes = vs.workspace_size(route, host["u"], host["B"])
+        per = []
+        for r in range(rot):
+            d = {k: v.to(dev) for k, v in host.items()}
+            out = torch.empty_like(d["u"])
+            ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+            per.append(vs.Plan(route, d["u"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], d["bias"],
+                               d["z"] if wl.gate else None, out=out, workspace=ws,
+                               merge_scale=wl.merge_scale))
+        plans.append(per)
+    launches_per_forward = 2 if wls[0].route in ("pool_w", "pool_h") else 1
+    torch.cuda.synchronize(dev)
+
+    # warm-up
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            for per in plans:
+                per[i % rot].run(stream)
+    stream.synchronize()
+
+    K = args.steps
+    nfw = len(wls)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(nfw)] for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if dev.index is not None else local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    wall0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for i in range(K):
+            for j, per in enumerate(plans):
+                a, b = ev[i][j]
+                a.record(stream)
+                per[i % rot].run(stream)
+                b.record(stream)
+        t_end.record(stream)
+    stream.synchronize()
+    wall = time.perf_counter() - wall0
+    sampler.stop()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+
+    elapsed_ms = t_start.elapsed_time(t_end)
+    per_launch_ms = [[ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(K)] for j in range(nfw)]
+    t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t_max.item())
+
+    units_step = sum(w.token_channels for w in wls)
+    value = units_step * K * world / (elapsed_ms * 1e-3)
+
+    # roofline of the dominant kernel (the fused scan: one launch per forward for
+    # the streaming routes; for the pooled route the bracket also holds the small
+    # B/C pooling pre-pass)
+    hbm_peak, peak_src, sm_max = peaks()
+    bytes_all = sum(algorithmic_bytes(w) * K for w in wls)
+    ms_all = sum(sum(v) for v in per_launch_ms)
+    achieved = bytes_all / (ms_all * 1e-3) / 1e9
+    kname = {"atrous2": "stream_scan_kernel<ATROUS2>", "bidir": "stream_scan_kernel<BIDIR>",
+             "cross4": "stream_scan_kernel<CROSS4>", "pool_w": "pool_scan_kernel",
+             "pool_h": "pool_scan_kernel"}[wls[0].route]
+    traffic = recorded_traffic(kname, workload_label(wls))
+    upd_all = sum(updates(w) * K for w in wls)
+    sfu_peak = 16 * 148 * sm_max * 1e6  # one exp per state update on the SFU
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "kernel": kname, "launch_ms_avg": round(ms_all / (K * nfw), 5),
+                "algorithmic_bytes_per_launch": [algorithmic_bytes(w) for w in wls],
+                "sfu": {"state_updates_per_s": upd_all / (ms_all * 1e-3), "peak": sfu_peak,
+                        "frac": round(upd_all / (ms_all * 1e-3) / sfu_peak, 4),
+                        "note": "one ex2 per state update, 16 SFU results/clk/SM x 148 SMs at max clock"}}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if wls[0].dtype == "f32" else "bf16",
+        "data": "synthetic, seeded (page-workload shapes and value recipe)",
+        "config": dict(config_block(wls, world),
+                       l2=f"rotating {rot} device copies of the inputs ({rot * step_bytes / 2**20:.0f} MiB) > 126 MiB L2"),
+        "roofline": roofline,
+        "gpu_launches": K * nfw * launches_per_forward,
+        "clocks": sampler.summary(),
+        "wall_s_timed_region": round(wall, 4),
+    }
+
+    # end to end through the host-buffer entry point
+    if not args.no_e2e:
+        hplans, h2d, d2h = [], 0, 0
+        for wl, route, host in zip(wls, routes, host_sets):
+            pin = {k: v.pin_memory() for k, v in host.items()}
+            out = torch.empty_like(pin["u"]).pin_memory()
+            nbytes = vs.host_buffer_size(route, pin["u"], pin["B"], z=wl.gate)
+            buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+            hplans.append(vs.HostPlan(route, pin["u"], pin["delta"], pin["A"], pin["B"], pin["C"],
+                                      pin["Dskip"], pin["bias"], pin["z"] if wl.gate else None,
+                                      out=out, device_buffer=buf, merge_scale=wl.merge_scale))
+            h2d += sum(pin[k].numel() * pin[k].element_size()
+                       for k in ("u", "delta", "B", "C", "z", "A", "Dskip", "bias"))
+            d2h += out.numel() * out.element_size()
+        E = max(1, min(args.e2e_steps, K))
+        with torch.cuda.stream(stream):
+            for hp in hplans:
+                hp.run(stream)
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(E):
+                for hp in hplans:
+                    hp.run(stream)
+            e1.record(stream)
+        stream.synchronize()
+        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        line["e2e"] = {"value": units_step * E * world / (float(e_ms.item()) * 1e-3), "unit": UNIT,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": E,
+                       "path": "vscan_forward_host (pinned host buffers, copies inside the timed region)"}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wls, args.cpu_seconds)
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for r in routes:
+        r.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    wls = select(args.workload)
+    if args.impl == "reference":
+        run_reference(args, wls)
+    else:
+        run_ours(args, wls)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,220 @@
+/*
+ * vscan.h -- C ABI of the routed visual selective scan library (libvscan.so).
+ *
+ * The library computes, on one NVIDIA B200 (sm_100a), the Mamba S6 selective
+ * scan run over image-token sequences under a spatial routing, fused with the
+ * gather, the discretization, the read-out, the SiLU gate and the
+ * direction-merging scatter:
+ *
+ *   for every image b, channel d and direction k of the route:
+ *     (u_t, rawDelta_t, B_t, C_t) = tokens gathered in the route's order
+ *     Delta_t = softplus(rawDelta_t + bias_d)
+ *     h_t     = exp(Delta_t * A_d) (.) h_{t-1} + Delta_t * B_t * u_t,  h_{-1} = 0
+ *     y_t     = sum_n C_{t,n} h_{t,n} + D_d * u_t
+ *   then y is scattered back to the grid, the directions are summed and scaled
+ *   by merge_scale, and the result is gated: Y = merge_scale * sum_k y_k * SiLU(z).
+ *
+ * Sources (page title and section):
+ *   - "Vision Mamba: Bidirectional State Space Models for Images": sec. 3-4
+ *     (discretization, recurrence, read-out, released Delta*B*u write), sec. 5
+ *     and "Two scans meet at the same token" (bidirectional route, flip back,
+ *     shared SiLU gate), sec. 2 (middle CLS at floor(P/2)).
+ *   - "EfficientVMamba: Atrous Selective Scan for Light Weight Visual Mamba":
+ *     sec. 1-3 (p = 2 atrous groups, right/bottom zero padding, merge by
+ *     inverse permutation and crop).
+ *   - "Norm or Direction? Decoding Vision Mambas for High-Resolution Vision":
+ *     sec. 3, Eq. 1-2 and "2D Selective Scan (SS2D)" (four traversals, summed).
+ *   - "Fast Vision Mamba: Pooling Spatial Dimensions for Accelerated
+ *     Processing": Methodology (mean-pool one axis, scan forward and backward,
+ *     repeat the outputs over the pooled axis).
+ *
+ * Conventions for every function below:
+ *   - Return value: VSCAN_OK (0) or a negative vscan_status. Nothing throws
+ *     across the ABI. After a non-OK status, vscan_last_error() returns a
+ *     message for the calling thread.
+ *   - Argument checks happen on the host before any CUDA call; a rejected call
+ *     launches nothing and changes no memory.
+ *   - "device pointer" means memory the caller allocated on the current CUDA
+ *     device; "stream" is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Work is enqueued on that stream; no function synchronizes it
+ *     unless its comment says so.
+ *   - The library owns only the vscan_route objects it creates. Every tensor,
+ *     the workspace and every host buffer are owned by the caller.
+ */
+#ifndef VSCAN_H
+#define VSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum vscan_status {
+    VSCAN_OK = 0,
+    VSCAN_ERR_INVALID_ARGUMENT = -1, /* null pointer, bad enum, non-positive size */
+    VSCAN_ERR_SHAPE = -2,            /* size combination the route cannot take     */
+    VSCAN_ERR_ALIGNMENT = -3,        /* pointer or channel count not 16-byte aligned */
+    VSCAN_ERR_UNSUPPORTED = -4,      /* valid but not implemented (e.g. N > 16)    */
+    VSCAN_ERR_CUDA = -5,             /* a CUDA runtime call failed                 */
+    VSCAN_ERR_WORKSPACE = -6         /* workspace missing or smaller than required */
+} vscan_status;
+
+/* Spatial routings. The token array of one image is row-major over the h x w
+ * grid (columns fastest), with the CLS token inserted at cls_pos for BIDIR. */
+typedef enum vscan_route_kind {
+    /* Vim: forward over the assembled sequence (grid + optional middle CLS) and
+     * backward over the whole reversed sequence; outputs aligned and added.
+     * "Vision Mamba ...", sec. 2 and 5. K = 2, L = h*w (+1 with CLS). */
+    VSCAN_ROUTE_BIDIR = 0,
+    /* VMamba SS2D: k0 row-major, k1 row-major reversed, k2 column-major,
+     * k3 column-major reversed; the four outputs are summed at the original
+     * coordinates. "Norm or Direction? ...", sec. 3. K = 4, L = h*w. */
+    VSCAN_ROUTE_CROSS4 = 1,
+    /* EfficientVMamba p = 2: group k takes grid coordinates
+     * (2 r + m_k, 2 c + n_k), (m_k, n_k) = (0,0), (1,0), (0,1), (1,1); groups 0
+     * and 2 row-major, 1 and 3 column-major, on the grid zero-padded
+     * right/bottom to even size; each real pixel has one owner (no summation)
+     * and padding outputs are cropped. "EfficientVMamba ...", sec. 1-3.
+     * K = 4, L = ceil(h/2) * ceil(w/2). */
+    VSCAN_ROUTE_ATROUS2 = 2,
+    /* FastVim: u, rawDelta, B, C mean-pooled over the columns of every grid
+     * row (length h), scanned forward and backward, summed, repeated over the
+     * columns and gated with the un-pooled z. "Fast Vision Mamba ...",
+     * Methodology. K = 2, L = h. */
+    VSCAN_ROUTE_POOL_W = 3,
+    /* FastVim alternate axis: mean over the rows of every column, L = w. */
+    VSCAN_ROUTE_POOL_H = 4
+} vscan_route_kind;
+
+typedef enum vscan_dtype {
+    VSCAN_F32 = 0, /* IEEE float32 */
+    VSCAN_BF16 = 1 /* bfloat16; state and accumulation stay float32 */
+} vscan_dtype;
+
+/* Opaque, immutable route description (host memory only). */
+typedef struct vscan_route vscan_route;
+
+/*
+ * Arguments of one forward pass. All tensors are dense, row-major, with the
+ * channel (or state) axis contiguous. "tokens" is the route's token count per
+ * image (vscan_route_info), Ki = K if per_dir_inputs else 1, Kp = K if
+ * per_dir_params else 1.
+ */
+typedef struct vscan_args {
+    int32_t batch;          /* images, >= 0 (0 = nothing to do)                      */
+    int32_t channels;       /* D (expanded width); multiple of 4 (f32) or 8 (bf16)   */
+    int32_t d_state;        /* N, 1..16                                              */
+    int32_t dtype;          /* vscan_dtype of u, delta, B, C, z and y                */
+    const void* u;          /* device, [Ki][batch][tokens][D]                        */
+    const void* delta;      /* device, [Ki][batch][tokens][D], raw step before bias  */
+    const void* B;          /* device, [Ki][batch][tokens][N]                        */
+    const void* C;          /* device, [Ki][batch][tokens][N]                        */
+    const void* z;          /* device, [batch][tokens][D], or NULL for no gate       */
+    void* y;                /* device, [batch][tokens][D], written (not accumulated) */
+    const float* A;         /* device, [Kp][D][N] float32 (negative for stability)   */
+    const float* Dskip;     /* device, [Kp][D] float32, or NULL for no skip term     */
+    const float* delta_bias;/* device, [Kp][D] float32, or NULL for no bias          */
+    int32_t per_dir_inputs; /* 0: u, delta, B, C shared by all directions; 1: per k  */
+    int32_t per_dir_params; /* 0: A, Dskip, delta_bias shared; 1: leading K axis     */
+    int32_t delta_softplus; /* 1: Delta = softplus(raw + bias); 0: Delta = raw + bias */
+    float merge_scale;      /* scales the merged output: 1 = sum, 0.5 = Vim average  */
+    void* workspace;        /* device scratch of >= vscan_workspace_size() bytes     */
+    uint64_t workspace_bytes;
+    int32_t seq_chunks;     /* 0 = library choice; 1 = one sequential pass per
+                               direction; 2..8 = split each sequence into that many
+                               chunks combined by an affine-pair prefix scan
+                               (only for routes whose tile fits on chip)            */
+    int32_t reserved;       /* must be 0                                             */
+} vscan_args;
+
+/*
+ * Describe a route. Host only: no CUDA call, no device memory.
+ *   kind    : vscan_route_kind.
+ *   h, w    : grid rows and columns, >= 1.
+ *   cls_pos : BIDIR only: index of the CLS token in the token array, which
+ *             must be floor(h*w/2) ("Vision Mamba ...", sec. 2), or -1 for no
+ *             CLS; every other route requires -1.
+ * On success *out receives a route to be released with vscan_destroy.
+ * Errors: VSCAN_ERR_INVALID_ARGUMENT (null out, bad kind, h or w < 1, a
+ * sequence longer than 2^24 tokens), VSCAN_ERR_SHAPE (cls_pos not allowed).
+ */
+vscan_status vscan_create_route(vscan_route** out, int32_t kind, int32_t h, int32_t w,
+                                int32_t cls_pos);
+
+/* Release a route. NULL is a no-op. Always returns VSCAN_OK. */
+vscan_status vscan_destroy(vscan_route* route);
+
+/*
+ * Geometry of a route (host only). Any output pointer may be NULL.
+ *   K        : directions (2 or 4).
+ *   seq_len  : steps per direction.
+ *   tokens   : tokens per image in the token array (h*w, +1 with CLS).
+ *   padded_h, padded_w : working grid (ATROUS2: rounded up to even; else h, w).
+ */
+vscan_status vscan_route_info(const vscan_route* route, int32_t* K, int32_t* seq_len,
+                              int32_t* tokens, int32_t* padded_h, int32_t* padded_w);
+
+/*
+ * Write the route's index maps into a device buffer of K * seq_len int32:
+ * out[k * seq_len + t] = token index visited at step t of direction k (for
+ * the pooled routes: the pooled-sequence index), or -1 for an ATROUS2 padding
+ * slot. The maps are produced on the GPU by the same index functions the scan
+ * kernels evaluate. Enqueued on stream.
+ */
+vscan_status vscan_route_indices(const vscan_route* route, int32_t* dev_out, void* stream);
+
+/*
+ * Device scratch bytes vscan_forward needs for these arguments (host only).
+ * BIDIR and CROSS4 hold per-direction partial outputs until the last direction
+ * of a token adds them up; POOL_W/POOL_H hold the pooled B and C; ATROUS2
+ * needs none (every pixel has one owner).
+ */
+vscan_status vscan_workspace_size(const vscan_route* route, const vscan_args* args,
+                                  uint64_t* bytes);
+
+/*
+ * Run the fused routed scan on the device. Enqueued on stream; allocates
+ * nothing; never synchronizes. The output y is fully overwritten. Concurrent
+ * calls on different streams must use different workspaces.
+ * Errors: INVALID_ARGUMENT / SHAPE / ALIGNMENT / UNSUPPORTED for bad
+ * arguments (nothing launched), WORKSPACE if the workspace is too small,
+ * CUDA if a launch failed (message from the CUDA runtime).
+ */
+vscan_status vscan_forward(const vscan_route* route, const vscan_args* args, void* stream);
+
+/*
+ * Bytes of device memory vscan_forward_host needs in its device_buffer for
+ * these arguments (host only): device copies of every input and of y, plus
+ * the workspace, each rounded up to 256 bytes.
+ */
+vscan_status vscan_host_buffer_size(const vscan_route* route, const vscan_args* host_args,
+                                    uint64_t* bytes);
+
+/*
+ * End-to-end call with HOST tensors. host_args holds host pointers (page-locked
+ * memory gives asynchronous copies) with the same layouts as vscan_forward;
+ * its workspace fields are ignored. The call enqueues on stream: host-to-device
+ * copies of the inputs into device_buffer, the forward pass, and the
+ * device-to-host copy of y into host_args->y. The caller synchronizes the
+ * stream before reading y. device_buffer is caller-owned device memory of at
+ * least vscan_host_buffer_size() bytes.
+ */
+vscan_status vscan_forward_host(const vscan_route* route, const vscan_args* host_args,
+                                void* device_buffer, uint64_t device_buffer_bytes, void* stream);
+
+/* Message for the last non-OK status on this thread ("" if none). */
+const char* vscan_last_error(void);
+
+/* Static name of a status code. */
+const char* vscan_status_string(int32_t status);
+
+/* Library ABI version; changes whenever vscan_args changes layout. */
+int32_t vscan_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSCAN_H */

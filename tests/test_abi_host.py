@@ -1,0 +1,135 @@
+"""Host-side checks of the C ABI: no GPU needed, no kernel launched.
+
+Every call here either is host-only by contract (route creation, geometry,
+workspace sizing) or fails argument validation, which the library performs
+before its first CUDA call. No call with plausible-looking fake device pointers
+is ever allowed to pass validation.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT, read_golden
+
+import oracle as O
+
+abi = pytest.importorskip("vision_selective_state_b200._abi")
+vs = pytest.importorskip("vision_selective_state_b200")
+
+HEADER = os.path.join(ROOT, "include", "vscan.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(vscan_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    names = declared_functions()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_struct_layout_matches_the_header():
+    # int32 x4, 6 pointers, 3 pointers, int32 x3, float, pointer, uint64, int32 x2
+    assert ctypes.sizeof(abi.VscanArgs) == 16 + 48 + 24 + 12 + 4 + 8 + 8 + 8
+    assert abi.lib.vscan_abi_version() == abi.ABI_VERSION
+
+
+def test_status_strings():
+    for code, name in abi.STATUS.items():
+        assert abi.lib.vscan_status_string(code).decode() == name
+
+
+@pytest.mark.parametrize("kind", ["bidir", "cross4", "atrous2", "pool_w", "pool_h"])
+@pytest.mark.parametrize("h,w", [(1, 1), (3, 5), (14, 14), (55, 57), (56, 56), (128, 128)])
+def test_route_geometry_matches_the_oracle(kind, h, w):
+    cls = (h * w) // 2 if kind == "bidir" else -1
+    r = vs.Route(kind, h, w, cls)
+    K, L, T = O.geometry(kind, h, w, cls)
+    assert (r.K, r.seq_len, r.tokens) == (K, L, T)
+    if kind == "atrous2":
+        assert (r.padded_h, r.padded_w) == (h + h % 2, w + w % 2)
+    r.close()
+
+
+def test_vim_sequence_lengths_fixture():
+    for ln in read_golden("vim_sequence_lengths.txt"):
+        h, w, cls, tokens = map(int, ln.split())
+        r = vs.Route("bidir", h, w, cls)
+        assert (r.K, r.seq_len, r.tokens) == (2, tokens, tokens)
+
+
+@pytest.mark.parametrize("kind,h,w,cls,status", [
+    ("bidir", 14, 14, 97, -2), ("bidir", 0, 4, -1, -1), ("cross4", 4, 4, 8, -2),
+    ("atrous2", 3, -1, -1, -1), ("pool_w", 4, 4, 0, -2), (7, 4, 4, -1, -1),
+])
+def test_invalid_routes_are_rejected(kind, h, w, cls, status):
+    handle = ctypes.c_void_p()
+    code = abi.ROUTES[kind] if isinstance(kind, str) else kind
+    got = abi.lib.vscan_create_route(ctypes.byref(handle), code, h, w, cls)
+    assert got == status
+    assert handle.value is None
+    assert abi.lib.vscan_last_error().decode()
+
+
+def _args(**kw):
+    a = abi.VscanArgs()
+    a.batch, a.channels, a.d_state, a.dtype = 2, 16, 16, abi.F32
+    a.delta_softplus, a.merge_scale = 1, 1.0
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_workspace_sizes():
+    n = ctypes.c_uint64()
+    for kind, expect in (("atrous2", 0), ("bidir", 2 * 2 * 197 * 16 * 4), ("cross4", 4 * 2 * 36 * 16 * 4)):
+        h, w, cls = (14, 14, 98) if kind == "bidir" else (6, 6, -1)
+        r = vs.Route(kind, h, w, cls)
+        assert abi.lib.vscan_workspace_size(r.handle, ctypes.byref(_args()), ctypes.byref(n)) == 0
+        assert n.value == (expect + 255) // 256 * 256
+    r = vs.Route("pool_w", 8, 8)
+    assert abi.lib.vscan_workspace_size(r.handle, ctypes.byref(_args()), ctypes.byref(n)) == 0
+    assert n.value == 2 * ((2 * 8 * 16 * 4 + 255) // 256 * 256)
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("channels", 6, -3), ("channels", 0, -1), ("d_state", 17, -4), ("d_state", 0, -1),
+    ("dtype", 5, -1), ("batch", -1, -1), ("reserved", 1, -1), ("seq_chunks", 9, -1),
+    ("per_dir_inputs", 2, -1), ("merge_scale", float("nan"), -1),
+])
+def test_bad_arguments_fail_before_any_cuda_call(field, value, status):
+    r = vs.Route("atrous2", 5, 5)
+    a = _args(**{field: value})
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(a), None) == status
+    n = ctypes.c_uint64()
+    assert abi.lib.vscan_workspace_size(r.handle, ctypes.byref(a), ctypes.byref(n)) == status
+
+
+def test_null_and_misaligned_pointers_are_rejected():
+    r = vs.Route("atrous2", 5, 5)
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args()), None) == -1  # u is NULL
+    fake = dict(u=0x1000, delta=0x2000, B=0x3000, C=0x4000, y=0x5000, A=0x6000)
+    a = _args(**dict(fake, delta=0x2004))
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(a), None) == -3
+    rb = vs.Route("bidir", 5, 5, 12)
+    a = _args(**fake)  # BIDIR needs a workspace; none given
+    assert abi.lib.vscan_forward(rb.handle, ctypes.byref(a), None) == -6
+    a = _args(**fake, workspace=0x7000, workspace_bytes=64)
+    assert abi.lib.vscan_forward(rb.handle, ctypes.byref(a), None) == -6
+    assert "workspace" in abi.lib.vscan_last_error().decode()
+    hb = _args(**fake)
+    n = ctypes.c_uint64()
+    assert abi.lib.vscan_host_buffer_size(rb.handle, ctypes.byref(hb), ctypes.byref(n)) == 0
+    assert abi.lib.vscan_forward_host(rb.handle, ctypes.byref(hb), None, 0, None) == -6
+
+
+def test_pooled_route_length_limit():
+    r = vs.Route("pool_w", 4000, 2)
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args()), None) == -4

@@ -1,0 +1,231 @@
+"""Routed visual selective scan on NVIDIA B200: Python binding of libvscan.so.
+
+The binding only marshals PyTorch tensors (device memory and streams) into the
+C ABI declared in include/vscan.h; every step of the scan runs in the CUDA
+kernels of the library. Tensors are channels-last:
+
+    u, delta, z, y : [batch, tokens, D]   (leading K axis for per-direction u/delta)
+    B, C           : [batch, tokens, N]   (leading K axis for per-direction B/C)
+    A              : [D, N] float32        ([K, D, N] per direction)
+    Dskip, bias    : [D] float32           ([K, D] per direction)
+
+u, delta, B, C, z and y share one dtype: torch.float32 or torch.bfloat16.
+"""
+import ctypes
+
+import torch
+
+from ._abi import BF16, F32, ROUTES, VscanArgs, VscanError, check, lib
+
+__all__ = ["Route", "forward", "forward_host", "workspace_size", "host_buffer_size", "VscanError",
+           "ROUTES"]
+
+
+class Route:
+    """An immutable route description (vscan_create_route / vscan_destroy)."""
+
+    def __init__(self, kind, h, w, cls_pos=-1):
+        self.kind_name = kind if isinstance(kind, str) else {v: k for k, v in ROUTES.items()}[kind]
+        self.kind = ROUTES[kind] if isinstance(kind, str) else int(kind)
+        self.h, self.w, self.cls_pos = int(h), int(w), int(cls_pos)
+        handle = ctypes.c_void_p()
+        check(lib.vscan_create_route(ctypes.byref(handle), self.kind, self.h, self.w, self.cls_pos))
+        self._handle = handle
+        vals = [ctypes.c_int32() for _ in range(5)]
+        check(lib.vscan_route_info(self._handle, *[ctypes.byref(v) for v in vals]))
+        self.K, self.seq_len, self.tokens, self.padded_h, self.padded_w = (v.value for v in vals)
+
+    @property
+    def handle(self):
+        if self._handle is None:
+            raise ValueError("route was closed")
+        return self._handle
+
+    def close(self):
+        if getattr(self, "_handle", None) is not None:
+            lib.vscan_destroy(self._handle)
+            self._handle = None
+
+    def __del__(self):
+        self.close()
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def indices(self, device="cuda", stream=None):
+        """[K, seq_len] int32 maps computed on the GPU by the kernels' index functions."""
+        out = torch.empty((self.K, self.seq_len), dtype=torch.int32, device=device)
+        s = _stream(stream, out.device)
+        check(lib.vscan_route_indices(self.handle, ctypes.c_void_p(out.data_ptr()), s))
+        return out
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _args(route, u, delta, A, B, C, Dskip, delta_bias, z, y, delta_softplus, merge_scale,
+          per_dir_inputs, per_dir_params, workspace, seq_chunks):
+    for name, t in (("u", u), ("delta", delta), ("B", B), ("C", C), ("z", z), ("y", y),
+                    ("A", A), ("Dskip", Dskip), ("delta_bias", delta_bias)):
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    for name, t in (("A", A), ("Dskip", Dskip), ("delta_bias", delta_bias)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    lead = 1 if per_dir_inputs else 0
+    batch, tokens, D = u.shape[lead:]
+    N = B.shape[-1]
+    if tokens != route.tokens:
+        raise ValueError(f"u has {tokens} tokens per image, the route has {route.tokens}")
+    code = _dtype_code(u)
+    for name, t in (("delta", delta), ("B", B), ("C", C), ("z", z), ("y", y)):
+        if t is not None and t.dtype != u.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} != u dtype {u.dtype}")
+    a = VscanArgs()
+    a.batch, a.channels, a.d_state, a.dtype = batch, D, N, code
+    a.u, a.delta, a.B, a.C, a.z, a.y = (_ptr(u), _ptr(delta), _ptr(B), _ptr(C), _ptr(z), _ptr(y))
+    a.A, a.Dskip, a.delta_bias = _ptr(A), _ptr(Dskip), _ptr(delta_bias)
+    a.per_dir_inputs, a.per_dir_params = int(bool(per_dir_inputs)), int(bool(per_dir_params))
+    a.delta_softplus = int(bool(delta_softplus))
+    a.merge_scale = float(merge_scale)
+    if workspace is not None:
+        a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    a.seq_chunks = int(seq_chunks)
+    a.reserved = 0
+    return a
+
+
+def workspace_size(route, u, B, *, per_dir_inputs=False, per_dir_params=False):
+    """Bytes of device scratch vscan_forward needs (host-only query)."""
+    lead = 1 if per_dir_inputs else 0
+    a = VscanArgs()
+    a.batch, _, a.channels = u.shape[lead:]
+    a.d_state = B.shape[-1]
+    a.dtype = _dtype_code(u)
+    a.per_dir_inputs, a.per_dir_params = int(bool(per_dir_inputs)), int(bool(per_dir_params))
+    a.delta_softplus, a.merge_scale = 1, 1.0
+    n = ctypes.c_uint64()
+    check(lib.vscan_workspace_size(route.handle, ctypes.byref(a), ctypes.byref(n)))
+    return n.value
+
+
+def forward(route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, delta_softplus=True,
+            merge_scale=1.0, per_dir_inputs=False, per_dir_params=False, out=None, workspace=None,
+            seq_chunks=0, stream=None):
+    """Routed selective scan on the GPU (vscan_forward). Returns y [batch, tokens, D]."""
+    lead = 1 if per_dir_inputs else 0
+    if out is None:
+        out = torch.empty(u.shape[lead:], dtype=u.dtype, device=u.device)
+    if workspace is None:
+        need = workspace_size(route, u, B, per_dir_inputs=per_dir_inputs, per_dir_params=per_dir_params)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=u.device)
+    a = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus, merge_scale,
+              per_dir_inputs, per_dir_params, workspace, seq_chunks)
+    check(lib.vscan_forward(route.handle, ctypes.byref(a), _stream(stream, u.device)))
+    return out
+
+
+def host_buffer_size(route, u, B, *, z=True, Dskip=True, delta_bias=True, per_dir_inputs=False,
+                     per_dir_params=False):
+    """Bytes of device memory forward_host needs (host-only query)."""
+    lead = 1 if per_dir_inputs else 0
+    a = VscanArgs()
+    a.batch, _, a.channels = u.shape[lead:]
+    a.d_state = B.shape[-1]
+    a.dtype = _dtype_code(u)
+    a.per_dir_inputs, a.per_dir_params = int(bool(per_dir_inputs)), int(bool(per_dir_params))
+    a.delta_softplus, a.merge_scale = 1, 1.0
+    # only nullness matters for the size query
+    a.z = ctypes.c_void_p(1) if z else None
+    a.Dskip = ctypes.c_void_p(1) if Dskip else None
+    a.delta_bias = ctypes.c_void_p(1) if delta_bias else None
+    n = ctypes.c_uint64()
+    check(lib.vscan_host_buffer_size(route.handle, ctypes.byref(a), ctypes.byref(n)))
+    return n.value
+
+
+def forward_host(route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, out,
+                 device_buffer, delta_softplus=True, merge_scale=1.0, per_dir_inputs=False,
+                 per_dir_params=False, stream=None):
+    """End-to-end call with host (CPU, ideally pinned) tensors (vscan_forward_host).
+
+    Enqueues the host-to-device copies, the scan and the copy of y into `out`
+    (a host tensor) on the stream; synchronize the stream before reading `out`.
+    """
+    for t in (u, delta, A, B, C, Dskip, delta_bias, z, out):
+        if t is not None and t.is_cuda:
+            raise ValueError("forward_host takes host tensors")
+    a = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus, merge_scale,
+              per_dir_inputs, per_dir_params, None, 0)
+    nbytes = device_buffer.numel() * device_buffer.element_size()
+    check(lib.vscan_forward_host(route.handle, ctypes.byref(a), ctypes.c_void_p(device_buffer.data_ptr()),
+                                 nbytes, _stream(stream, device_buffer.device)))
+    return out
+
+
+class Plan:
+    """A forward call with its arguments marshalled once (for repeated launches).
+
+    Holds references to every tensor it points at; run() is one vscan_forward call.
+    """
+
+    def __init__(self, route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, out,
+                 workspace, delta_softplus=True, merge_scale=1.0, per_dir_inputs=False,
+                 per_dir_params=False, seq_chunks=0):
+        self.route = route
+        self._keep = (u, delta, A, B, C, Dskip, delta_bias, z, out, workspace)
+        self.out = out
+        self.args = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus,
+                          merge_scale, per_dir_inputs, per_dir_params, workspace, seq_chunks)
+        self._ref = ctypes.byref(self.args)
+
+    def run(self, stream):
+        """Enqueue the forward pass on a torch.cuda.Stream."""
+        check(lib.vscan_forward(self.route.handle, self._ref, ctypes.c_void_p(stream.cuda_stream)))
+
+
+__all__.append("Plan")
+
+
+class HostPlan:
+    """An end-to-end forward_host call with its arguments marshalled once."""
+
+    def __init__(self, route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, out,
+                 device_buffer, delta_softplus=True, merge_scale=1.0, per_dir_inputs=False,
+                 per_dir_params=False):
+        for t in (u, delta, A, B, C, Dskip, delta_bias, z, out):
+            if t is not None and t.is_cuda:
+                raise ValueError("HostPlan takes host tensors")
+        self.route = route
+        self._keep = (u, delta, A, B, C, Dskip, delta_bias, z, out, device_buffer)
+        self.out = out
+        self.args = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus,
+                          merge_scale, per_dir_inputs, per_dir_params, None, 0)
+        self._ref = ctypes.byref(self.args)
+        self._buf = ctypes.c_void_p(device_buffer.data_ptr())
+        self._nbytes = device_buffer.numel() * device_buffer.element_size()
+
+    def run(self, stream):
+        check(lib.vscan_forward_host(self.route.handle, self._ref, self._buf, self._nbytes,
+                                     ctypes.c_void_p(stream.cuda_stream)))
+
+
+__all__.append("HostPlan")

@@ -1,0 +1,402 @@
+// C ABI of the routed selective scan (declared in include/vscan.h).
+//
+// Host side only: argument checks, workspace sizing, kernel selection and
+// launch, and the host-buffer (end-to-end) entry point. Every check runs before
+// the first CUDA call, so a rejected call launches nothing.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "vscan.h"
+#include "vscan_pool.cuh"
+#include "vscan_route.cuh"
+#include "vscan_stream.cuh"
+
+struct vscan_route {
+    vscan::RouteGeom g;
+};
+
+namespace {
+
+constexpr int32_t kAbiVersion = 1;
+thread_local std::string g_last_error;
+
+vscan_status fail(vscan_status s, const char* fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+vscan_status cuda_fail(cudaError_t e, const char* what)
+{
+    return fail(VSCAN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
+
+size_t elem_bytes(int32_t dtype) { return dtype == VSCAN_BF16 ? 2 : 4; }
+
+bool is_pool(int kind) { return kind == vscan::RK_POOL_W || kind == vscan::RK_POOL_H; }
+
+// Checks that do not depend on where the tensors live.
+vscan_status check_shape(const vscan_route* r, const vscan_args* a)
+{
+    if (!r) return fail(VSCAN_ERR_INVALID_ARGUMENT, "route is NULL");
+    if (!a) return fail(VSCAN_ERR_INVALID_ARGUMENT, "args is NULL");
+    if (a->reserved != 0) return fail(VSCAN_ERR_INVALID_ARGUMENT, "args.reserved must be 0");
+    if (a->dtype != VSCAN_F32 && a->dtype != VSCAN_BF16)
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "unknown dtype %d", a->dtype);
+    if (a->batch < 0) return fail(VSCAN_ERR_INVALID_ARGUMENT, "batch %d < 0", a->batch);
+    if (a->channels < 1) return fail(VSCAN_ERR_INVALID_ARGUMENT, "channels %d < 1", a->channels);
+    if (a->d_state < 1) return fail(VSCAN_ERR_INVALID_ARGUMENT, "d_state %d < 1", a->d_state);
+    if (a->d_state > 16) return fail(VSCAN_ERR_UNSUPPORTED, "d_state %d > 16", a->d_state);
+    const int vec = a->dtype == VSCAN_F32 ? 4 : 8;
+    if (a->channels % vec != 0)
+        return fail(VSCAN_ERR_ALIGNMENT, "channels %d is not a multiple of %d (16-byte rows)", a->channels, vec);
+    if (a->per_dir_inputs != 0 && a->per_dir_inputs != 1)
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "per_dir_inputs must be 0 or 1");
+    if (a->per_dir_params != 0 && a->per_dir_params != 1)
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "per_dir_params must be 0 or 1");
+    if (a->delta_softplus != 0 && a->delta_softplus != 1)
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "delta_softplus must be 0 or 1");
+    if (!std::isfinite(a->merge_scale)) return fail(VSCAN_ERR_INVALID_ARGUMENT, "merge_scale is not finite");
+    if (a->seq_chunks < 0 || a->seq_chunks > 8)
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "seq_chunks %d outside 0..8", a->seq_chunks);
+    if (a->batch > 65535) return fail(VSCAN_ERR_UNSUPPORTED, "batch %d > 65535", a->batch);
+    if (is_pool(r->g.kind)) {
+        const int Ki = a->per_dir_inputs ? 2 : 1;
+        if (vscan::pool_scan_smem_bytes(Ki, r->g.L) > 200 * 1024)
+            return fail(VSCAN_ERR_UNSUPPORTED, "pooled length %d too long for the on-chip tile", r->g.L);
+    }
+    return VSCAN_OK;
+}
+
+vscan_status check_pointers(const vscan_args* a, bool device)
+{
+    if (a->batch == 0) return VSCAN_OK;
+    const char* names[] = {"u", "delta", "B", "C", "y", "A"};
+    const void* ptrs[] = {a->u, a->delta, a->B, a->C, a->y, a->A};
+    for (int i = 0; i < 6; ++i)
+        if (!ptrs[i]) return fail(VSCAN_ERR_INVALID_ARGUMENT, "%s is NULL", names[i]);
+    if (device) {
+        const char* vn[] = {"u", "delta", "B", "C", "z", "y"};
+        const void* vp[] = {a->u, a->delta, a->B, a->C, a->z, a->y};
+        for (int i = 0; i < 6; ++i)
+            if (vp[i] && !aligned16(vp[i]))
+                return fail(VSCAN_ERR_ALIGNMENT, "%s is not 16-byte aligned", vn[i]);
+    }
+    return VSCAN_OK;
+}
+
+uint64_t workspace_need(const vscan_route* r, const vscan_args* a)
+{
+    const vscan::RouteGeom& g = r->g;
+    if (a->batch == 0) return 0;
+    if (g.kind == vscan::RK_BIDIR || g.kind == vscan::RK_CROSS4)
+        return round256((uint64_t)g.K * a->batch * g.tokens * a->channels * sizeof(float));
+    if (is_pool(g.kind)) {
+        const int Ki = a->per_dir_inputs ? 2 : 1;
+        return 2 * round256((uint64_t)Ki * a->batch * g.L * a->d_state * sizeof(float));
+    }
+    return 0;
+}
+
+template <int RK, typename T>
+void launch_stream(const vscan::ScanParams& p, cudaStream_t s)
+{
+    constexpr int K = (RK == vscan::RK_BIDIR) ? 2 : 4;
+    const dim3 grid((p.D + vscan::ST_CH - 1) / vscan::ST_CH, p.batch);
+    const size_t smem = K * sizeof(vscan::StreamStage);
+    if (p.N == 16)
+        vscan::stream_scan_kernel<RK, T, true><<<grid, 32 * K, smem, s>>>(p);
+    else
+        vscan::stream_scan_kernel<RK, T, false><<<grid, 32 * K, smem, s>>>(p);
+}
+
+template <typename T>
+cudaError_t launch_pool(const vscan::PoolParams& p, cudaStream_t s)
+{
+    const dim3 g1(p.g.L, p.batch, p.Ki);
+    vscan::pool_bc_kernel<T><<<g1, 128, 0, s>>>(p);
+    const size_t smem = vscan::pool_scan_smem_bytes(p.Ki, p.g.L);
+    cudaError_t e = cudaFuncSetAttribute(vscan::pool_scan_kernel<T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (e != cudaSuccess) return e;
+    const dim3 g2((p.D + vscan::PL_CH - 1) / vscan::PL_CH, p.batch);
+    vscan::pool_scan_kernel<T><<<g2, vscan::PL_THREADS, smem, s>>>(p);
+    return cudaSuccess;
+}
+
+template <typename T>
+vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s)
+{
+    const vscan::RouteGeom& g = r->g;
+    const long long plane = (long long)a->batch * g.tokens;
+    if (is_pool(g.kind)) {
+        vscan::PoolParams p{};
+        p.g = g;
+        p.batch = a->batch; p.D = a->channels; p.N = a->d_state;
+        p.Ki = a->per_dir_inputs ? 2 : 1;
+        p.u = a->u; p.delta = a->delta; p.B = a->B; p.C = a->C; p.z = a->z; p.y = a->y;
+        p.A = a->A; p.Dskip = a->Dskip; p.bias = a->delta_bias;
+        p.in_dir = a->per_dir_inputs ? plane * a->channels : 0;
+        p.bc_dir = a->per_dir_inputs ? plane * a->d_state : 0;
+        p.a_dir = a->per_dir_params ? a->channels * a->d_state : 0;
+        p.v_dir = a->per_dir_params ? a->channels : 0;
+        p.softplus = a->delta_softplus;
+        p.merge_scale = a->merge_scale;
+        const uint64_t half = workspace_need(r, a) / 2;
+        p.pB = static_cast<float*>(a->workspace);
+        p.pC = reinterpret_cast<float*>(static_cast<char*>(a->workspace) + half);
+        cudaError_t e = launch_pool<T>(p, s);
+        if (e != cudaSuccess) return cuda_fail(e, "configuring the pooled-scan kernel");
+    } else {
+        vscan::ScanParams p{};
+        p.g = g;
+        p.batch = a->batch; p.D = a->channels; p.N = a->d_state;
+        p.u = a->u; p.delta = a->delta; p.B = a->B; p.C = a->C; p.z = a->z; p.y = a->y;
+        p.A = a->A; p.Dskip = a->Dskip; p.bias = a->delta_bias;
+        p.in_dir = a->per_dir_inputs ? plane * a->channels : 0;
+        p.bc_dir = a->per_dir_inputs ? plane * a->d_state : 0;
+        p.a_dir = a->per_dir_params ? a->channels * a->d_state : 0;
+        p.v_dir = a->per_dir_params ? a->channels : 0;
+        p.softplus = a->delta_softplus;
+        p.merge_scale = a->merge_scale;
+        p.scratch = static_cast<float*>(a->workspace);
+        switch (g.kind) {
+        case vscan::RK_BIDIR: launch_stream<vscan::RK_BIDIR, T>(p, s); break;
+        case vscan::RK_CROSS4: launch_stream<vscan::RK_CROSS4, T>(p, s); break;
+        default: launch_stream<vscan::RK_ATROUS2, T>(p, s); break;
+        }
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return VSCAN_OK;
+}
+
+vscan_status forward_device(const vscan_route* r, const vscan_args* a, cudaStream_t s)
+{
+    const uint64_t need = workspace_need(r, a);
+    if (need > 0) {
+        if (!a->workspace || a->workspace_bytes < need)
+            return fail(VSCAN_ERR_WORKSPACE, "workspace of %llu bytes needed, %llu given",
+                        (unsigned long long)need, (unsigned long long)(a->workspace ? a->workspace_bytes : 0));
+        if (!aligned16(a->workspace)) return fail(VSCAN_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
+    }
+    if (a->batch == 0) return VSCAN_OK;
+    return a->dtype == VSCAN_F32 ? dispatch<float>(r, a, s) : dispatch<__nv_bfloat16>(r, a, s);
+}
+
+__global__ void route_map_kernel(vscan::RouteGeom g, int32_t* out)
+{
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx < (long long)g.K * g.L) {
+        const int k = (int)(idx / g.L);
+        const int t = (int)(idx - (long long)k * g.L);
+        out[idx] = vscan::route_token_any(g, k, t);
+    }
+}
+
+struct HostLayout {
+    size_t u, delta, B, C, z, y, A, Dskip, bias, ws, total;
+};
+
+HostLayout host_layout(const vscan_route* r, const vscan_args* a)
+{
+    const vscan::RouteGeom& g = r->g;
+    const size_t eb = elem_bytes(a->dtype);
+    const size_t Ki = a->per_dir_inputs ? g.K : 1;
+    const size_t Kp = a->per_dir_params ? g.K : 1;
+    const size_t plane = (size_t)a->batch * g.tokens;
+    HostLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off += round256(bytes); return o; };
+    L.u = take(Ki * plane * a->channels * eb);
+    L.delta = take(Ki * plane * a->channels * eb);
+    L.B = take(Ki * plane * a->d_state * eb);
+    L.C = take(Ki * plane * a->d_state * eb);
+    L.z = take(a->z ? plane * a->channels * eb : 0);
+    L.y = take(plane * a->channels * eb);
+    L.A = take(Kp * a->channels * a->d_state * sizeof(float));
+    L.Dskip = take(a->Dskip ? Kp * a->channels * sizeof(float) : 0);
+    L.bias = take(a->delta_bias ? Kp * a->channels * sizeof(float) : 0);
+    L.ws = take(workspace_need(r, a));
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+vscan_status vscan_create_route(vscan_route** out, int32_t kind, int32_t h, int32_t w, int32_t cls_pos)
+{
+    if (!out) return fail(VSCAN_ERR_INVALID_ARGUMENT, "out is NULL");
+    *out = nullptr;
+    if (kind < vscan::RK_BIDIR || kind > vscan::RK_POOL_H)
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "unknown route kind %d", kind);
+    if (h < 1 || w < 1) return fail(VSCAN_ERR_INVALID_ARGUMENT, "grid %dx%d is empty", h, w);
+    if ((long long)h * w > (1LL << 24))
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "grid %dx%d has more than 2^24 tokens", h, w);
+    vscan::RouteGeom g{};
+    if (!vscan::make_geom(kind, h, w, cls_pos, &g)) {
+        if (kind == vscan::RK_BIDIR)
+            return fail(VSCAN_ERR_SHAPE, "cls_pos %d must be -1 or floor(h*w/2) = %lld", cls_pos,
+                        (long long)h * w / 2);
+        return fail(VSCAN_ERR_SHAPE, "cls_pos %d must be -1 for route kind %d", cls_pos, kind);
+    }
+    vscan_route* r = new (std::nothrow) vscan_route;
+    if (!r) return fail(VSCAN_ERR_INVALID_ARGUMENT, "out of host memory");
+    r->g = g;
+    *out = r;
+    return VSCAN_OK;
+}
+
+vscan_status vscan_destroy(vscan_route* route)
+{
+    delete route;
+    return VSCAN_OK;
+}
+
+vscan_status vscan_route_info(const vscan_route* r, int32_t* K, int32_t* seq_len, int32_t* tokens,
+                              int32_t* padded_h, int32_t* padded_w)
+{
+    if (!r) return fail(VSCAN_ERR_INVALID_ARGUMENT, "route is NULL");
+    if (K) *K = r->g.K;
+    if (seq_len) *seq_len = r->g.L;
+    if (tokens) *tokens = r->g.tokens;
+    const bool atrous = r->g.kind == vscan::RK_ATROUS2;
+    if (padded_h) *padded_h = atrous ? 2 * r->g.rows : r->g.h;
+    if (padded_w) *padded_w = atrous ? 2 * r->g.cols : r->g.w;
+    return VSCAN_OK;
+}
+
+vscan_status vscan_route_indices(const vscan_route* r, int32_t* dev_out, void* stream)
+{
+    if (!r) return fail(VSCAN_ERR_INVALID_ARGUMENT, "route is NULL");
+    if (!dev_out) return fail(VSCAN_ERR_INVALID_ARGUMENT, "dev_out is NULL");
+    const long long n = (long long)r->g.K * r->g.L;
+    const int threads = 256;
+    const unsigned blocks = (unsigned)((n + threads - 1) / threads);
+    route_map_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(r->g, dev_out);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "route map kernel launch");
+    return VSCAN_OK;
+}
+
+vscan_status vscan_workspace_size(const vscan_route* r, const vscan_args* a, uint64_t* bytes)
+{
+    if (!bytes) return fail(VSCAN_ERR_INVALID_ARGUMENT, "bytes is NULL");
+    vscan_status st = check_shape(r, a);
+    if (st != VSCAN_OK) return st;
+    *bytes = workspace_need(r, a);
+    return VSCAN_OK;
+}
+
+vscan_status vscan_forward(const vscan_route* r, const vscan_args* a, void* stream)
+{
+    vscan_status st = check_shape(r, a);
+    if (st != VSCAN_OK) return st;
+    st = check_pointers(a, true);
+    if (st != VSCAN_OK) return st;
+    return forward_device(r, a, static_cast<cudaStream_t>(stream));
+}
+
+vscan_status vscan_host_buffer_size(const vscan_route* r, const vscan_args* a, uint64_t* bytes)
+{
+    if (!bytes) return fail(VSCAN_ERR_INVALID_ARGUMENT, "bytes is NULL");
+    vscan_status st = check_shape(r, a);
+    if (st != VSCAN_OK) return st;
+    *bytes = host_layout(r, a).total;
+    return VSCAN_OK;
+}
+
+vscan_status vscan_forward_host(const vscan_route* r, const vscan_args* ha, void* device_buffer,
+                                uint64_t device_buffer_bytes, void* stream)
+{
+    vscan_status st = check_shape(r, ha);
+    if (st != VSCAN_OK) return st;
+    st = check_pointers(ha, false);
+    if (st != VSCAN_OK) return st;
+    if (ha->batch == 0) return VSCAN_OK;
+    const HostLayout L = host_layout(r, ha);
+    if (!device_buffer || device_buffer_bytes < L.total)
+        return fail(VSCAN_ERR_WORKSPACE, "device buffer of %llu bytes needed, %llu given",
+                    (unsigned long long)L.total, (unsigned long long)(device_buffer ? device_buffer_bytes : 0));
+    if ((reinterpret_cast<uintptr_t>(device_buffer) & 255u) != 0)
+        return fail(VSCAN_ERR_ALIGNMENT, "device buffer is not 256-byte aligned");
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* base = static_cast<char*>(device_buffer);
+    const vscan::RouteGeom& g = r->g;
+    const size_t eb = elem_bytes(ha->dtype);
+    const size_t Ki = ha->per_dir_inputs ? g.K : 1;
+    const size_t Kp = ha->per_dir_params ? g.K : 1;
+    const size_t plane = (size_t)ha->batch * g.tokens;
+
+    vscan_args da = *ha;
+    da.u = base + L.u;
+    da.delta = base + L.delta;
+    da.B = base + L.B;
+    da.C = base + L.C;
+    da.z = ha->z ? base + L.z : nullptr;
+    da.y = base + L.y;
+    da.A = reinterpret_cast<const float*>(base + L.A);
+    da.Dskip = ha->Dskip ? reinterpret_cast<const float*>(base + L.Dskip) : nullptr;
+    da.delta_bias = ha->delta_bias ? reinterpret_cast<const float*>(base + L.bias) : nullptr;
+    da.workspace = base + L.ws;
+    da.workspace_bytes = workspace_need(r, ha);
+
+    struct Copy { void* dst; const void* src; size_t bytes; };
+    const Copy in[] = {
+        {const_cast<void*>(da.u), ha->u, Ki * plane * ha->channels * eb},
+        {const_cast<void*>(da.delta), ha->delta, Ki * plane * ha->channels * eb},
+        {const_cast<void*>(da.B), ha->B, Ki * plane * ha->d_state * eb},
+        {const_cast<void*>(da.C), ha->C, Ki * plane * ha->d_state * eb},
+        {const_cast<void*>(da.z), ha->z, ha->z ? plane * ha->channels * eb : 0},
+        {const_cast<float*>(da.A), ha->A, Kp * ha->channels * ha->d_state * sizeof(float)},
+        {const_cast<float*>(da.Dskip), ha->Dskip, ha->Dskip ? Kp * ha->channels * sizeof(float) : 0},
+        {const_cast<float*>(da.delta_bias), ha->delta_bias, ha->delta_bias ? Kp * ha->channels * sizeof(float) : 0},
+    };
+    for (const Copy& c : in) {
+        if (c.bytes == 0) continue;
+        cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    }
+    st = forward_device(r, &da, s);
+    if (st != VSCAN_OK) return st;
+    cudaError_t e = cudaMemcpyAsync(ha->y, da.y, plane * ha->channels * eb, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+    return VSCAN_OK;
+}
+
+const char* vscan_last_error(void) { return g_last_error.c_str(); }
+
+const char* vscan_status_string(int32_t status)
+{
+    switch (status) {
+    case VSCAN_OK: return "VSCAN_OK";
+    case VSCAN_ERR_INVALID_ARGUMENT: return "VSCAN_ERR_INVALID_ARGUMENT";
+    case VSCAN_ERR_SHAPE: return "VSCAN_ERR_SHAPE";
+    case VSCAN_ERR_ALIGNMENT: return "VSCAN_ERR_ALIGNMENT";
+    case VSCAN_ERR_UNSUPPORTED: return "VSCAN_ERR_UNSUPPORTED";
+    case VSCAN_ERR_CUDA: return "VSCAN_ERR_CUDA";
+    case VSCAN_ERR_WORKSPACE: return "VSCAN_ERR_WORKSPACE";
+    default: return "VSCAN_UNKNOWN_STATUS";
+    }
+}
+
+int32_t vscan_abi_version(void) { return kAbiVersion; }
+
+}  // extern "C"

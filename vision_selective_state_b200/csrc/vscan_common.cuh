@@ -1,0 +1,105 @@
+// Device helpers shared by the routed-scan kernels: element loads/stores for
+// the two I/O types, the discretization functions and the gate.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace vscan {
+
+constexpr unsigned FULL_MASK = 0xffffffffu;
+constexpr float LOG2E = 1.4426950408889634f;
+
+// ---- element I/O -----------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float load_elem(const T* p);
+
+template <>
+__device__ __forceinline__ float load_elem<float>(const float* p) { return __ldg(p); }
+
+template <>
+__device__ __forceinline__ float load_elem<__nv_bfloat16>(const __nv_bfloat16* p)
+{
+    return __bfloat162float(__ldg(p));
+}
+
+template <typename T>
+__device__ __forceinline__ void store_elem(T* p, float v);
+
+template <>
+__device__ __forceinline__ void store_elem<float>(float* p, float v) { *p = v; }
+
+template <>
+__device__ __forceinline__ void store_elem<__nv_bfloat16>(__nv_bfloat16* p, float v)
+{
+    *p = __float2bfloat16_rn(v);
+}
+
+// Four consecutive elements starting at a 4-element-aligned address.
+template <typename T>
+__device__ __forceinline__ float4 load4(const T* p);
+
+template <>
+__device__ __forceinline__ float4 load4<float>(const float* p)
+{
+    return __ldg(reinterpret_cast<const float4*>(p));
+}
+
+template <>
+__device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p)
+{
+    const uint2 raw = __ldg(reinterpret_cast<const uint2*>(p));
+    float4 r;
+    r.x = __uint_as_float(raw.x << 16);
+    r.y = __uint_as_float(raw.x & 0xffff0000u);
+    r.z = __uint_as_float(raw.y << 16);
+    r.w = __uint_as_float(raw.y & 0xffff0000u);
+    return r;
+}
+
+template <typename T>
+__device__ __forceinline__ void store4(T* p, float4 v);
+
+template <>
+__device__ __forceinline__ void store4<float>(float* p, float4 v)
+{
+    *reinterpret_cast<float4*>(p) = v;
+}
+
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 v)
+{
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 raw;
+    raw.x = *reinterpret_cast<uint32_t*>(&a);
+    raw.y = *reinterpret_cast<uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(p) = raw;
+}
+
+// ---- discretization ---------------------------------------------------------
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32). The retention
+// exp(Delta * A) is evaluated as 2^(Delta * A * log2 e), with A pre-scaled.
+__device__ __forceinline__ float fast_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// softplus(x) = log(1 + e^x) ("Vision Mamba ...", sec. 3). Above 20 the two
+// differ by less than 2^-28 relative, so x itself is returned, as PyTorch's
+// softplus does.
+__device__ __forceinline__ float softplus_f(float x)
+{
+    return x > 20.0f ? x : log1pf(expf(x));
+}
+
+// SiLU(z) = z * sigma(z), signed and unbounded ("Vision Mamba ...", sec. 5).
+__device__ __forceinline__ float silu_f(float z)
+{
+    return z / (1.0f + expf(-z));
+}
+
+}  // namespace vscan

@@ -1,0 +1,276 @@
+// Pooled route (FastVim): POOL_W and POOL_H.
+//
+// "Fast Vision Mamba: Pooling Spatial Dimensions for Accelerated Processing",
+// Methodology: reshape the tokens to (h, w), mean-pool one spatial axis, run the
+// forward and backward selective scans on the pooled tokens only, repeat the
+// outputs along the pooled axis. The gate uses the un-pooled z of each token.
+//
+// Two kernels:
+//   pool_bc_kernel    mean-pools B and C (shared by all channels) into the
+//                     workspace: [Ki][batch][Lp][N] float32 each.
+//   pool_scan_kernel  one CTA per (image, 32-channel tile): pools u and raw
+//                     Delta of the tile into shared memory (HBM stream), runs
+//                     both scan directions on the Lp pooled steps, then streams
+//                     the repeated, gated output over every grid token.
+// The pooled-route memory traffic is the compulsory one: u, Delta and z read
+// once, y written once; B and C are read once by the small pre-pass.
+#pragma once
+
+#include "vscan_common.cuh"
+#include "vscan_route.cuh"
+
+namespace vscan {
+
+struct PoolParams {
+    RouteGeom g;
+    int batch, D, N, Ki;
+    const void* u;
+    const void* delta;
+    const void* B;
+    const void* C;
+    const void* z;
+    void* y;
+    const float* A;
+    const float* Dskip;
+    const float* bias;
+    long long in_dir;
+    long long bc_dir;
+    int a_dir;
+    int v_dir;
+    int softplus;
+    float merge_scale;
+    float* pB;  // [Ki][batch][Lp][N]
+    float* pC;  // [Ki][batch][Lp][N]
+};
+
+constexpr int PL_CH = 32;       // channels per CTA
+constexpr int PL_THREADS = 256;
+
+// Token of the grid that is the j-th member of pooled index i.
+__device__ __forceinline__ int pool_member(const RouteGeom& g, int i, int j)
+{
+    return (g.kind == RK_POOL_W) ? i * g.w + j : j * g.w + i;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(128) pool_bc_kernel(const PoolParams p)
+{
+    __shared__ float part_b[8][16];
+    __shared__ float part_c[8][16];
+    const int i = blockIdx.x, b = blockIdx.y, k = blockIdx.z;
+    const int n = threadIdx.x & 15, jl = threadIdx.x >> 4;
+    const int N = p.N;
+    const int cnt = (p.g.kind == RK_POOL_W) ? p.g.w : p.g.h;
+    const long long img = (long long)b * p.g.tokens;
+    const T* Bb = static_cast<const T*>(p.B) + k * p.bc_dir + img * N;
+    const T* Cb = static_cast<const T*>(p.C) + k * p.bc_dir + img * N;
+    float sb = 0.f, sc = 0.f;
+    if (n < N) {
+        for (int j = jl; j < cnt; j += 8) {
+            const long long tok = pool_member(p.g, i, j);
+            sb += load_elem<T>(Bb + tok * N + n);
+            sc += load_elem<T>(Cb + tok * N + n);
+        }
+    }
+    part_b[jl][n] = sb;
+    part_c[jl][n] = sc;
+    __syncthreads();
+    if (jl == 0 && n < N) {
+        float tb = 0.f, tc = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            tb += part_b[q][n];
+            tc += part_c[q][n];
+        }
+        const float inv = 1.0f / (float)cnt;
+        const long long o = (((long long)k * p.batch + b) * p.g.L + i) * N + n;
+        p.pB[o] = tb * inv;
+        p.pC[o] = tc * inv;
+    }
+}
+
+// Dynamic shared memory (floats): pd[Ki][Lp][32] (pooled raw Delta),
+// pu[Ki][Lp][32] (pooled u), Y[2][Lp][32] (per-direction outputs).
+inline size_t pool_scan_smem_bytes(int Ki, int Lp)
+{
+    return sizeof(float) * (size_t)(2 * Ki + 2) * Lp * PL_CH;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams p)
+{
+    extern __shared__ __align__(16) float psm[];
+    const int Lp = p.g.L;
+    const int Ki = p.Ki;
+    float* pd = psm;                          // [Ki][Lp][32]
+    float* pu = psm + (size_t)Ki * Lp * PL_CH;  // [Ki][Lp][32]
+    float* Y = pu + (size_t)Ki * Lp * PL_CH;    // [2][Lp][32]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = blockIdx.y;
+    const int c0 = blockIdx.x * PL_CH;
+    const int D = p.D, N = p.N;
+    const int tokens = p.g.tokens;
+    const long long img = (long long)b * tokens;
+    const int cnt = (p.g.kind == RK_POOL_W) ? p.g.w : p.g.h;
+    const float inv_cnt = 1.0f / (float)cnt;
+
+    // ---- phase 1: mean-pool u and raw Delta of the channel tile ---------------
+    {
+        const int jl = lane >> 3;   // token sub-lane 0..3
+        const int q = lane & 7;     // channel quad of the tile
+        const int ch = c0 + 4 * q;
+        const bool cval = ch < D;
+        for (int k = 0; k < Ki; ++k) {
+            const T* ub = static_cast<const T*>(p.u) + k * p.in_dir + img * D + ch;
+            const T* db = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + ch;
+            for (int i = warp; i < Lp; i += PL_THREADS / 32) {
+                float4 au = make_float4(0.f, 0.f, 0.f, 0.f), ad = au;
+                if (cval) {
+                    int j = jl;
+                    for (; j + 12 < cnt; j += 16) {
+                        float4 u4[4], d4[4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const long long tok = pool_member(p.g, i, j + 4 * r);
+                            u4[r] = load4<T>(ub + tok * D);
+                            d4[r] = load4<T>(db + tok * D);
+                        }
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            au.x += u4[r].x; au.y += u4[r].y; au.z += u4[r].z; au.w += u4[r].w;
+                            ad.x += d4[r].x; ad.y += d4[r].y; ad.z += d4[r].z; ad.w += d4[r].w;
+                        }
+                    }
+                    for (; j < cnt; j += 4) {
+                        const long long tok = pool_member(p.g, i, j);
+                        const float4 u1 = load4<T>(ub + tok * D);
+                        const float4 d1 = load4<T>(db + tok * D);
+                        au.x += u1.x; au.y += u1.y; au.z += u1.z; au.w += u1.w;
+                        ad.x += d1.x; ad.y += d1.y; ad.z += d1.z; ad.w += d1.w;
+                    }
+                }
+#pragma unroll
+                for (int m = 8; m <= 16; m <<= 1) {
+                    au.x += __shfl_xor_sync(FULL_MASK, au.x, m);
+                    au.y += __shfl_xor_sync(FULL_MASK, au.y, m);
+                    au.z += __shfl_xor_sync(FULL_MASK, au.z, m);
+                    au.w += __shfl_xor_sync(FULL_MASK, au.w, m);
+                    ad.x += __shfl_xor_sync(FULL_MASK, ad.x, m);
+                    ad.y += __shfl_xor_sync(FULL_MASK, ad.y, m);
+                    ad.z += __shfl_xor_sync(FULL_MASK, ad.z, m);
+                    ad.w += __shfl_xor_sync(FULL_MASK, ad.w, m);
+                }
+                if (jl == 0) {
+                    float* du_ = pu + ((size_t)k * Lp + i) * PL_CH + 4 * q;
+                    float* dd_ = pd + ((size_t)k * Lp + i) * PL_CH + 4 * q;
+                    du_[0] = au.x * inv_cnt; du_[1] = au.y * inv_cnt; du_[2] = au.z * inv_cnt; du_[3] = au.w * inv_cnt;
+                    dd_[0] = ad.x * inv_cnt; dd_[1] = ad.y * inv_cnt; dd_[2] = ad.z * inv_cnt; dd_[3] = ad.w * inv_cnt;
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- phase 2: both directions over the Lp pooled steps ----------------------
+    {
+        const int kd = warp >> 2;          // direction 0 (forward) / 1 (backward)
+        const int cg = warp & 3;           // 8-channel group of the tile
+        const int ki = (Ki > 1) ? kd : 0;  // input plane
+        const int cc = lane >> 2, grp = lane & 3;
+        const int c = 8 * cg + cc;
+        const int d = c0 + c;
+        const bool dvalid = d < D;
+        float a2[4];
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const int n = 4 * grp + s;
+            a2[s] = (dvalid && n < N) ? __ldg(p.A + (long long)kd * p.a_dir + (long long)d * N + n) * LOG2E : 0.f;
+        }
+        const float Dd = (dvalid && p.Dskip) ? __ldg(p.Dskip + kd * p.v_dir + d) : 0.f;
+        const float bias = (dvalid && p.bias) ? __ldg(p.bias + kd * p.v_dir + d) : 0.f;
+        const float* pBk = p.pB + ((long long)ki * p.batch + b) * Lp * N;
+        const float* pCk = p.pC + ((long long)ki * p.batch + b) * Lp * N;
+        const float* pdk = pd + (size_t)ki * Lp * PL_CH;
+        const float* puk = pu + (size_t)ki * Lp * PL_CH;
+        float* Yk = Y + (size_t)kd * Lp * PL_CH;
+        float h[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int t0 = 0; t0 < Lp; t0 += 4) {
+            float yp[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int t = t0 + jj;
+                float acc = 0.f;
+                if (t < Lp) {
+                    const int i = kd == 0 ? t : Lp - 1 - t;
+                    // Delta = softplus(mean raw Delta + bias): the bias and
+                    // softplus act on the pooled token.
+                    const float x = pdk[(size_t)i * PL_CH + c] + bias;
+                    const float dsp = p.softplus ? softplus_f(x) : x;
+                    const float du = dsp * puk[(size_t)i * PL_CH + c];
+                    float bv[4], cv[4];
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        const int n = 4 * grp + s;
+                        bv[s] = n < N ? __ldg(pBk + (size_t)i * N + n) : 0.f;
+                        cv[s] = n < N ? __ldg(pCk + (size_t)i * N + n) : 0.f;
+                    }
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        const float e = fast_exp2(dsp * a2[s]);
+                        h[s] = fmaf(e, h[s], du * bv[s]);
+                        acc = fmaf(cv[s], h[s], acc);
+                    }
+                }
+                yp[jj] = acc;
+            }
+            const bool hi = grp & 2;
+            float x0 = hi ? yp[2] : yp[0];
+            float x1 = hi ? yp[3] : yp[1];
+            const float s0 = hi ? yp[0] : yp[2];
+            const float s1 = hi ? yp[1] : yp[3];
+            x0 += __shfl_xor_sync(FULL_MASK, s0, 2);
+            x1 += __shfl_xor_sync(FULL_MASK, s1, 2);
+            const bool odd = grp & 1;
+            float keep = odd ? x1 : x0;
+            const float send = odd ? x0 : x1;
+            keep += __shfl_xor_sync(FULL_MASK, send, 1);
+            const int t = t0 + grp;
+            if (t < Lp) {
+                const int i = kd == 0 ? t : Lp - 1 - t;
+                Yk[(size_t)i * PL_CH + c] = fmaf(Dd, puk[(size_t)i * PL_CH + c], keep);
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- phase 3: repeat over the pooled axis, merge, gate, store ---------------
+    {
+        const int q = tid & 7;        // channel quad
+        const int tl = tid >> 3;      // token lane 0..31
+        const int ch = c0 + 4 * q;
+        if (ch < D) {
+            const float* Y0 = Y;
+            const float* Y1 = Y + (size_t)Lp * PL_CH;
+            const T* zb = p.z ? static_cast<const T*>(p.z) + img * D + ch : nullptr;
+            T* yb = static_cast<T*>(p.y) + img * D + ch;
+            const float scale = p.merge_scale;
+            for (int tok = tl; tok < tokens; tok += 32) {
+                const int r = tok / p.g.w;
+                const int col = tok - r * p.g.w;
+                const int i = (p.g.kind == RK_POOL_W) ? r : col;
+                const float4 f = *reinterpret_cast<const float4*>(Y0 + (size_t)i * PL_CH + 4 * q);
+                const float4 g = *reinterpret_cast<const float4*>(Y1 + (size_t)i * PL_CH + 4 * q);
+                float4 o = make_float4((f.x + g.x) * scale, (f.y + g.y) * scale,
+                                       (f.z + g.z) * scale, (f.w + g.w) * scale);
+                if (zb) {
+                    const float4 zz = load4<T>(zb + (long long)tok * D);
+                    o.x *= silu_f(zz.x); o.y *= silu_f(zz.y); o.z *= silu_f(zz.z); o.w *= silu_f(zz.w);
+                }
+                store4<T>(yb + (long long)tok * D, o);
+            }
+        }
+    }
+}
+
+}  // namespace vscan
