@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline budget")
+    p.add_argument("--rotate", type=int, default=0,
+                   help="device copies of the inputs cycled through (0: enough to exceed 3x L2)")
     return p.parse_args()
 
 
@@ -210,6 +212,26 @@ def dist_env():
     return world, rank, local
 
 
+def replica(wl, rank):
+    """The workload one rank scans: same shapes, its own seeded values."""
+    return wl.with_(seed=wl.seed + 1000 * rank)
+
+
+def max_over_ranks(value, device=None):
+    """The largest value over all ranks (the job's time is its slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step, steps, world, elapsed_ms_max):
+    """Whole-job throughput: units every rank processed / the slowest rank's time."""
+    return units_per_rank_step * steps * world / (elapsed_ms_max * 1e-3)
+
+
 # ------------------------------------------------------------------ CPU oracle
 def oracle_time(wls, channels, threads=0):
     """Seconds the fp64 oracle takes for the given channel subset of every grid."""
@@ -299,11 +321,10 @@ def run_ours(args, wls):
     # inputs in the 126 MB L2 left by the previous step.
     step_bytes = sum(algorithmic_bytes(w) for w in wls)
     rot = max(2, -(-3 * L2_BYTES // step_bytes) + 1)
-    rot = min(rot, 8)
+    rot = min(rot, 8) if args.rotate <= 0 else args.rotate
     plans, host_sets, routes = [], [], []
     for wi, wl in enumerate(wls):
-        seeded = wl.with_(seed=wl.seed + 1000 * rank)
-        x = workloads.draw(seeded)
+        x = workloads.draw(replica(wl, rank))
         route = vs.Route(wl.route, wl.h, wl.w, wl.cls_pos)
         routes.append(route)
         dt = td[wl.dtype]
@@ -359,15 +380,11 @@ def run_ours(args, wls):
     if world > 1:
         dist.barrier()
 
-    elapsed_ms = t_start.elapsed_time(t_end)
     per_launch_ms = [[ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(K)] for j in range(nfw)]
-    t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(t_max.item())
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
 
     units_step = sum(w.token_channels for w in wls)
-    value = units_step * K * world / (elapsed_ms * 1e-3)
+    value = job_throughput(units_step, K, world, elapsed_ms)
 
     # roofline of the dominant kernel (the fused scan: one launch per forward for
     # the streaming routes; for the pooled route the bracket also holds the small
@@ -398,7 +415,8 @@ def run_ours(args, wls):
         "dtype": "f32" if wls[0].dtype == "f32" else "bf16",
         "data": "synthetic, seeded (page-workload shapes and value recipe)",
         "config": dict(config_block(wls, world),
-                       l2=f"rotating {rot} device copies of the inputs ({rot * step_bytes / 2**20:.0f} MiB) > 126 MiB L2"),
+                       l2=f"rotating {rot} device copies of the inputs ({rot * step_bytes / 2**20:.0f} MiB; "
+                          f"each step's inputs were last touched {rot - 1} steps earlier)"),
         "roofline": roofline,
         "gpu_launches": K * nfw * launches_per_forward,
         "clocks": sampler.summary(),
@@ -435,10 +453,8 @@ def run_ours(args, wls):
                     hp.run(stream)
             e1.record(stream)
         stream.synchronize()
-        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        line["e2e"] = {"value": units_step * E * world / (float(e_ms.item()) * 1e-3), "unit": UNIT,
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        line["e2e"] = {"value": job_throughput(units_step, E, world, e_ms), "unit": UNIT,
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": E,
                        "path": "vscan_forward_host (pinned host buffers, copies inside the timed region)"}
 

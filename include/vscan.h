@@ -123,9 +123,11 @@ typedef struct vscan_args {
     void* workspace;        /* device scratch of >= vscan_workspace_size() bytes     */
     uint64_t workspace_bytes;
     int32_t seq_chunks;     /* 0 = library choice; 1 = one sequential pass per
-                               direction; 2..8 = split each sequence into that many
-                               chunks combined by an affine-pair prefix scan
-                               (only for routes whose tile fits on chip)            */
+                               direction (streaming kernel); 2, 4 or 8 = split each
+                               sequence into that many chunks joined by a prefix
+                               scan of affine pairs (BIDIR, CROSS4 and ATROUS2 when
+                               the image's token tile fits on chip, else
+                               VSCAN_ERR_UNSUPPORTED); ignored by the pooled routes */
     int32_t reserved;       /* must be 0                                             */
 } vscan_args;
 

@@ -102,6 +102,7 @@ def test_workspace_sizes():
 @pytest.mark.parametrize("field,value,status", [
     ("channels", 6, -3), ("channels", 0, -1), ("d_state", 17, -4), ("d_state", 0, -1),
     ("dtype", 5, -1), ("batch", -1, -1), ("reserved", 1, -1), ("seq_chunks", 9, -1),
+    ("seq_chunks", 3, -1), ("seq_chunks", -1, -1),
     ("per_dir_inputs", 2, -1), ("merge_scale", float("nan"), -1),
 ])
 def test_bad_arguments_fail_before_any_cuda_call(field, value, status):
@@ -128,6 +129,14 @@ def test_null_and_misaligned_pointers_are_rejected():
     n = ctypes.c_uint64()
     assert abi.lib.vscan_host_buffer_size(rb.handle, ctypes.byref(hb), ctypes.byref(n)) == 0
     assert abi.lib.vscan_forward_host(rb.handle, ctypes.byref(hb), None, 0, None) == -6
+
+
+def test_chunked_scan_needs_the_tile_on_chip():
+    big = vs.Route("cross4", 56, 56)
+    assert abi.lib.vscan_forward(big.handle, ctypes.byref(_args(seq_chunks=4)), None) == -4
+    small = vs.Route("cross4", 14, 14)
+    # passes the shape checks, then stops at the NULL tensors
+    assert abi.lib.vscan_forward(small.handle, ctypes.byref(_args(seq_chunks=4)), None) == -1
 
 
 def test_pooled_route_length_limit():

@@ -28,8 +28,13 @@ ROUTES = ["bidir", "cross4", "atrous2", "pool_w", "pool_h"]
 def _case(route, h, w, D, N, dtype, batch=2, seed=1, a_mode="random", pdi=False, pdp=False, cls=None, **opts):
     wl = small_workload(route, h, w, D, N, dtype, batch, seed, cls)
     x = workloads.draw(wl, a_mode=a_mode, per_dir_inputs=pdi, per_dir_params=pdp)
+    if opts.get("delta_softplus") is False:
+        # without softplus the step is raw delta + bias: keep it positive (stable decay)
+        x["delta"] = np.abs(x["delta"])
+        x["bias"] = np.full_like(x["bias"], 0.01)
     r = vs.Route(route, h, w, wl.cls_pos)
     y = run_gpu(r, to_device(x, dtype), per_dir_inputs=pdi, per_dir_params=pdp, **opts)
+    opts.pop("seq_chunks", None)  # a launch choice of the CUDA path only
     ref = run_oracle(route, h, w, wl.cls_pos, x, per_dir_inputs=pdi, per_dir_params=pdp, **opts)
     err = rel_err(y.float().cpu().numpy(), ref)
     assert err <= TOL[dtype], (route, h, w, D, N, dtype, err)
@@ -63,6 +68,17 @@ def test_optional_terms(route):
     _case(route, 8, 9, 16, 16, "f32", skip=False, bias=False)
     _case(route, 8, 9, 16, 16, "f32", merge_scale=0.5)
     _case(route, 8, 9, 16, 16, "f32", delta_softplus=False, a_mode="s4d")
+
+
+@pytest.mark.parametrize("route", ["bidir", "cross4", "atrous2"])
+@pytest.mark.parametrize("nc", [1, 2, 4, 8])
+@pytest.mark.parametrize("h,w", [(1, 1), (3, 5), (14, 14), (9, 13)])
+def test_resident_chunked_scan(route, nc, h, w):
+    """The chunked parallel scan (affine-pair prefix over chunks) against the oracle,
+    with chunk boundaries falling on every kind of step (pads, CLS, ragged ends)."""
+    _case(route, h, w, 12, 16, "f32", seq_chunks=nc)
+    _case(route, h, w, 16, 7, "bf16", seq_chunks=nc, pdi=True, pdp=True)
+    _case(route, h, w, 8, 16, "f32", seq_chunks=nc, merge_scale=0.5, gate=False)
 
 
 def test_bidirectional_without_cls_and_long_sequences():

@@ -13,6 +13,7 @@
 
 #include "vscan.h"
 #include "vscan_pool.cuh"
+#include "vscan_resident.cuh"
 #include "vscan_route.cuh"
 #include "vscan_stream.cuh"
 
@@ -23,6 +24,7 @@ struct vscan_route {
 namespace {
 
 constexpr int32_t kAbiVersion = 1;
+constexpr size_t kMaxSmem = 200 * 1024;  // dynamic shared memory the kernels may ask for
 thread_local std::string g_last_error;
 
 vscan_status fail(vscan_status s, const char* fmt, ...)
@@ -49,6 +51,13 @@ size_t elem_bytes(int32_t dtype) { return dtype == VSCAN_BF16 ? 2 : 4; }
 
 bool is_pool(int kind) { return kind == vscan::RK_POOL_W || kind == vscan::RK_POOL_H; }
 
+size_t resident_bytes(const vscan_route* r, const vscan_args* a)
+{
+    const int Ki = a->per_dir_inputs ? r->g.K : 1;
+    const int Kd = (a->per_dir_inputs || a->per_dir_params) ? r->g.K : 1;
+    return vscan::resident_smem_bytes(r->g.kind, r->g.tokens, Ki, Kd);
+}
+
 // Checks that do not depend on where the tensors live.
 vscan_status check_shape(const vscan_route* r, const vscan_args* a)
 {
@@ -71,15 +80,33 @@ vscan_status check_shape(const vscan_route* r, const vscan_args* a)
     if (a->delta_softplus != 0 && a->delta_softplus != 1)
         return fail(VSCAN_ERR_INVALID_ARGUMENT, "delta_softplus must be 0 or 1");
     if (!std::isfinite(a->merge_scale)) return fail(VSCAN_ERR_INVALID_ARGUMENT, "merge_scale is not finite");
-    if (a->seq_chunks < 0 || a->seq_chunks > 8)
-        return fail(VSCAN_ERR_INVALID_ARGUMENT, "seq_chunks %d outside 0..8", a->seq_chunks);
+    if (a->seq_chunks != 0 && a->seq_chunks != 1 && a->seq_chunks != 2 && a->seq_chunks != 4 &&
+        a->seq_chunks != 8)
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "seq_chunks %d is not 0, 1, 2, 4 or 8", a->seq_chunks);
     if (a->batch > 65535) return fail(VSCAN_ERR_UNSUPPORTED, "batch %d > 65535", a->batch);
     if (is_pool(r->g.kind)) {
         const int Ki = a->per_dir_inputs ? 2 : 1;
-        if (vscan::pool_scan_smem_bytes(Ki, r->g.L) > 200 * 1024)
+        if (vscan::pool_scan_smem_bytes(Ki, r->g.L) > kMaxSmem)
             return fail(VSCAN_ERR_UNSUPPORTED, "pooled length %d too long for the on-chip tile", r->g.L);
+    } else if (a->seq_chunks > 1) {
+        if (resident_bytes(r, a) > kMaxSmem)
+            return fail(VSCAN_ERR_UNSUPPORTED, "seq_chunks > 1 needs the token tile on chip; %d tokens do not fit",
+                        r->g.tokens);
     }
     return VSCAN_OK;
+}
+
+// Chunks per sequence for the streaming routes: 1 = streaming kernel, 2/4/8 =
+// resident chunked kernel. The library picks the resident kernel when the tile
+// fits on chip and the streaming kernel would leave most SMs idle.
+int choose_chunks(const vscan_route* r, const vscan_args* a)
+{
+    if (is_pool(r->g.kind)) return 1;
+    if (a->seq_chunks >= 1) return a->seq_chunks;
+    if (resident_bytes(r, a) > kMaxSmem) return 1;
+    const long long stream_warps = (long long)a->batch * ((a->channels + vscan::ST_CH - 1) / vscan::ST_CH) * r->g.K;
+    if (stream_warps >= 4LL * 148) return 1;
+    return r->g.L >= 128 ? 8 : (r->g.L >= 32 ? 4 : 2);
 }
 
 vscan_status check_pointers(const vscan_args* a, bool device)
@@ -112,16 +139,48 @@ uint64_t workspace_need(const vscan_route* r, const vscan_args* a)
     return 0;
 }
 
-template <int RK, typename T>
-void launch_stream(const vscan::ScanParams& p, cudaStream_t s)
+template <int RK, typename T, bool N16>
+cudaError_t launch_stream_n(const vscan::ScanParams& p, cudaStream_t s)
 {
     constexpr int K = (RK == vscan::RK_BIDIR) ? 2 : 4;
+    const size_t smem = vscan::stream_smem_bytes<T>(K);
+    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     const dim3 grid((p.D + vscan::ST_CH - 1) / vscan::ST_CH, p.batch);
-    const size_t smem = K * sizeof(vscan::StreamStage);
-    if (p.N == 16)
-        vscan::stream_scan_kernel<RK, T, true><<<grid, 32 * K, smem, s>>>(p);
-    else
-        vscan::stream_scan_kernel<RK, T, false><<<grid, 32 * K, smem, s>>>(p);
+    vscan::stream_scan_kernel<RK, T, N16><<<grid, 32 * K, smem, s>>>(p);
+    return cudaSuccess;
+}
+
+template <int RK, typename T>
+cudaError_t launch_stream(const vscan::ScanParams& p, cudaStream_t s)
+{
+    return p.N == 16 ? launch_stream_n<RK, T, true>(p, s) : launch_stream_n<RK, T, false>(p, s);
+}
+
+template <int RK, typename T, int NC>
+cudaError_t launch_resident_nc(const vscan::ScanParams& p, size_t smem, cudaStream_t s)
+{
+    constexpr int CH = vscan::ResidentShape<RK>::CH;
+    cudaError_t e = cudaFuncSetAttribute(vscan::resident_scan_kernel<RK, T, NC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((p.D + CH - 1) / CH, p.batch);
+    vscan::resident_scan_kernel<RK, T, NC><<<grid, 64 * NC, smem, s>>>(p);
+    return cudaSuccess;
+}
+
+template <int RK, typename T>
+cudaError_t launch_resident(const vscan::ScanParams& p, int nc, cudaStream_t s)
+{
+    const int Ki = p.in_dir ? p.g.K : 1;
+    const int Kd = (p.in_dir || p.v_dir) ? p.g.K : 1;
+    const size_t smem = vscan::resident_smem_bytes(RK, p.g.tokens, Ki, Kd);
+    switch (nc) {
+    case 2: return launch_resident_nc<RK, T, 2>(p, smem, s);
+    case 4: return launch_resident_nc<RK, T, 4>(p, smem, s);
+    default: return launch_resident_nc<RK, T, 8>(p, smem, s);
+    }
 }
 
 template <typename T>
@@ -174,10 +233,23 @@ vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s)
         p.softplus = a->delta_softplus;
         p.merge_scale = a->merge_scale;
         p.scratch = static_cast<float*>(a->workspace);
-        switch (g.kind) {
-        case vscan::RK_BIDIR: launch_stream<vscan::RK_BIDIR, T>(p, s); break;
-        case vscan::RK_CROSS4: launch_stream<vscan::RK_CROSS4, T>(p, s); break;
-        default: launch_stream<vscan::RK_ATROUS2, T>(p, s); break;
+        const int nc = choose_chunks(r, a);
+        if (nc > 1) {
+            cudaError_t e;
+            switch (g.kind) {
+            case vscan::RK_BIDIR: e = launch_resident<vscan::RK_BIDIR, T>(p, nc, s); break;
+            case vscan::RK_CROSS4: e = launch_resident<vscan::RK_CROSS4, T>(p, nc, s); break;
+            default: e = launch_resident<vscan::RK_ATROUS2, T>(p, nc, s); break;
+            }
+            if (e != cudaSuccess) return cuda_fail(e, "configuring the resident scan kernel");
+        } else {
+            cudaError_t e;
+            switch (g.kind) {
+            case vscan::RK_BIDIR: e = launch_stream<vscan::RK_BIDIR, T>(p, s); break;
+            case vscan::RK_CROSS4: e = launch_stream<vscan::RK_CROSS4, T>(p, s); break;
+            default: e = launch_stream<vscan::RK_ATROUS2, T>(p, s); break;
+            }
+            if (e != cudaSuccess) return cuda_fail(e, "configuring the streaming scan kernel");
         }
     }
     cudaError_t e = cudaGetLastError();

@@ -36,6 +36,9 @@ __device__ __forceinline__ void store_elem<__nv_bfloat16>(__nv_bfloat16* p, floa
     *p = __float2bfloat16_rn(v);
 }
 
+__device__ __forceinline__ float to_float(float v) { return v; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
+
 // Four consecutive elements starting at a 4-element-aligned address.
 template <typename T>
 __device__ __forceinline__ float4 load4(const T* p);

@@ -1,0 +1,276 @@
+// Resident chunked routed selective scan, for grids whose channel tile fits on
+// chip (e.g. Vim-Tiny's 197 tokens): more parallelism per sequence at the cost
+// of a second pass over each chunk.
+//
+// The CTA stages the whole token array of one image and a tile of CH channels
+// in shared memory, with the step Delta = softplus(raw Delta + bias)
+// discretized once per token and channel while staging. Each direction's sequence is cut into NC chunks; lane
+// (chunk j, group g) of a channel runs its chunk sequentially for states
+// 4g..4g+3:
+//   pass 1  from a zero state: P = prod_t dA_t and H = the chunk's end state,
+//           i.e. the chunk as one affine map h -> P (.) h + H;
+//   combine an inclusive warp-shuffle scan of the affine pairs over the chunk
+//           lanes, (P1, H1) then (P2, H2) -> (P1 P2, P2 H1 + H2), gives every
+//           chunk the state entering it;
+//   pass 2  from that state: recurrence and read-out, y summed over the four
+//           group lanes, written to a per-direction output plane in shared
+//           memory at the token's grid position.
+// A CTA barrier then merges the planes (sum; ATROUS2 has one owner per token
+// and a single plane), scales, gates with SiLU(z) and stores.
+//
+// The recurrence, discretization and merge follow "Vision Mamba ...", sec. 3-5,
+// and "EfficientVMamba ...", sec. 1-3, exactly as the streaming kernel does;
+// "Fast Vision Mamba ..." cites the log-depth parallel scan this realizes.
+#pragma once
+
+#include "vscan_common.cuh"
+#include "vscan_route.cuh"
+#include "vscan_stream.cuh"
+
+namespace vscan {
+
+constexpr int RS_THREADS = 512;
+
+template <int RK>
+struct ResidentShape {
+    static constexpr int K = (RK == RK_BIDIR) ? 2 : 4;
+    static constexpr int CH = (K == 2) ? 8 : 4;               // channels per CTA
+    static constexpr int PLANES = (RK == RK_ATROUS2) ? 1 : K;  // output planes
+};
+
+// Shared-memory bytes of the resident kernel, or 0 if RK is not supported.
+// Ki: input planes (u, B, C); Kd: planes of the discretized step (K when the
+// inputs or the bias differ per direction, else 1).
+inline size_t resident_smem_bytes(int kind, int tokens, int Ki, int Kd)
+{
+    int CH, PLANES;
+    switch (kind) {
+    case RK_BIDIR: CH = 8; PLANES = 2; break;
+    case RK_CROSS4: CH = 4; PLANES = 4; break;
+    case RK_ATROUS2: CH = 4; PLANES = 1; break;
+    default: return 0;
+    }
+    const size_t per_token = (size_t)Ki * (CH + 32) + (size_t)Kd * CH + (size_t)PLANES * CH;
+    return per_token * tokens * sizeof(float);
+}
+
+template <int RK, typename T, int NC>
+__global__ void __launch_bounds__(RS_THREADS) resident_scan_kernel(const ScanParams p)
+{
+    using S = ResidentShape<RK>;
+    constexpr int K = S::K, CH = S::CH, PLANES = S::PLANES;
+    constexpr int LPC = 4 * NC;        // lanes per channel
+    constexpr int CPW = 32 / LPC;      // channels per warp
+    constexpr int WPD = CH / CPW;      // warps per direction
+    static_assert(CPW >= 1 && CH % CPW == 0, "chunk count must be 2, 4 or 8");
+
+    extern __shared__ __align__(16) float rsm[];
+    const int tokens = p.g.tokens, L = p.g.L, D = p.D, N = p.N;
+    const int Ki = p.in_dir ? K : 1;
+    const int Kd = (p.in_dir || p.v_dir) ? K : 1;
+    float* su = rsm;                                  // [Ki][tokens][CH]  u
+    float* sp = su + (size_t)Ki * tokens * CH;        // [Kd][tokens][CH]  softplus(raw delta + bias)
+    float* sB = sp + (size_t)Kd * tokens * CH;        // [Ki][tokens][16]
+    float* sC = sB + (size_t)Ki * tokens * 16;        // [Ki][tokens][16]
+    float* sY = sC + (size_t)Ki * tokens * 16;        // [PLANES][tokens][CH]
+
+    const int tid = threadIdx.x;
+    const int nthreads = K * WPD * 32;
+    const int b = blockIdx.y;
+    const int c0 = blockIdx.x * CH;
+    const long long img = (long long)b * tokens;
+    constexpr int BATCH = 4;  // independent loads in flight per thread while staging
+
+    // ---- stage the tile: u, the discretized step (once per token and channel), B, C
+    {
+        const int n_u = Ki * tokens * CH, n_d = Kd * tokens * CH;
+        for (int base = tid; base < n_u + n_d; base += BATCH * nthreads) {
+            float v[BATCH];
+#pragma unroll
+            for (int r = 0; r < BATCH; ++r) {
+                const int e = base + r * nthreads;
+                v[r] = 0.f;
+                if (e < n_u + n_d) {
+                    const bool is_u = e < n_u;
+                    const int ee = is_u ? e : e - n_u;
+                    const int kk = ee / (tokens * CH);
+                    const int rem = ee - kk * tokens * CH;
+                    const int tok = rem / CH, c = rem - tok * CH;
+                    const int d = c0 + c;
+                    if (d < D) {
+                        const int ki = is_u ? kk : (Ki > 1 ? kk : 0);
+                        const long long o = ki * p.in_dir + (img + tok) * D + d;
+                        v[r] = load_elem<T>(static_cast<const T*>(is_u ? p.u : p.delta) + o);
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < BATCH; ++r) {
+                const int e = base + r * nthreads;
+                if (e < n_u) {
+                    su[e] = v[r];
+                } else if (e < n_u + n_d) {
+                    const int ee = e - n_u;
+                    const int kd = ee / (tokens * CH);
+                    const int c = (ee - kd * tokens * CH) % CH;
+                    const int d = c0 + c;
+                    const float bias = (d < D && p.bias) ? __ldg(p.bias + kd * p.v_dir + d) : 0.f;
+                    const float x = v[r] + bias;
+                    sp[ee] = p.softplus ? softplus_f(x) : x;
+                }
+            }
+        }
+        const int n_bc = Ki * tokens * 16;
+        for (int base = tid; base < n_bc; base += BATCH * nthreads) {
+            float vb[BATCH], vc[BATCH];
+#pragma unroll
+            for (int r = 0; r < BATCH; ++r) {
+                const int e = base + r * nthreads;
+                vb[r] = 0.f;
+                vc[r] = 0.f;
+                if (e < n_bc) {
+                    const int k = e / (tokens * 16);
+                    const int rem = e - k * tokens * 16;
+                    const int tok = rem >> 4, n = rem & 15;
+                    if (n < N) {
+                        const long long o = k * p.bc_dir + (img + tok) * N + n;
+                        vb[r] = load_elem<T>(static_cast<const T*>(p.B) + o);
+                        vc[r] = load_elem<T>(static_cast<const T*>(p.C) + o);
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < BATCH; ++r) {
+                const int e = base + r * nthreads;
+                if (e < n_bc) {
+                    sB[e] = vb[r];
+                    sC[e] = vc[r];
+                }
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- roles ------------------------------------------------------------------
+    const int warp = tid >> 5, lane = tid & 31;
+    const int k = warp / WPD;
+    const int wi = warp - k * WPD;
+    const int cl = lane / LPC;
+    const int r = lane - cl * LPC;
+    const int j = r >> 2;          // chunk
+    const int grp = r & 3;         // states 4*grp .. 4*grp+3
+    const int c = wi * CPW + cl;   // channel within the tile
+    const int d = c0 + c;
+    const bool dvalid = d < D;
+    const int ki = Ki > 1 ? k : 0;
+    float a2[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        const int n = 4 * grp + s;
+        a2[s] = (dvalid && n < N) ? __ldg(p.A + (long long)k * p.a_dir + (long long)d * N + n) * LOG2E : 0.f;
+    }
+    const float Dd = (dvalid && p.Dskip) ? __ldg(p.Dskip + k * p.v_dir + d) : 0.f;
+    const float bias = (dvalid && p.bias) ? __ldg(p.bias + k * p.v_dir + d) : 0.f;
+    const float dsp_pad = p.softplus ? softplus_f(bias) : bias;  // ATROUS2 padding step
+    const float* suk = su + (size_t)ki * tokens * CH;
+    const float* spk = sp + (size_t)(Kd > 1 ? k : 0) * tokens * CH;
+    const float4* sBk = reinterpret_cast<const float4*>(sB + (size_t)ki * tokens * 16);
+    const float4* sCk = reinterpret_cast<const float4*>(sC + (size_t)ki * tokens * 16);
+    float* sYk = sY + (size_t)(PLANES == 1 ? 0 : k) * tokens * CH;
+
+    const int Lc = (L + NC - 1) / NC;
+    const int t0 = j * Lc;
+
+    // One step: discretized delta, delta*u, u, and this lane's B/C quads.
+    auto step = [&](int t, float& dsp, float& du, float& uu, float4& Bv, float4& Cv, int& pos) {
+        pos = (t < L) ? route_token<RK>(p.g, k, t) : -2;
+        dsp = 0.f; du = 0.f; uu = 0.f;
+        Bv = make_float4(0.f, 0.f, 0.f, 0.f);
+        Cv = Bv;
+        if (pos >= 0) {
+            uu = suk[(size_t)pos * CH + c];
+            dsp = spk[(size_t)pos * CH + c];
+            Bv = sBk[(size_t)pos * 4 + grp];
+            Cv = sCk[(size_t)pos * 4 + grp];
+            du = dsp * uu;
+        } else if (pos == -1) {
+            dsp = dsp_pad;
+        }
+    };
+
+    // ---- pass 1: each chunk as an affine map -------------------------------------
+    float P[4] = {1.f, 1.f, 1.f, 1.f}, H[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int i = 0; i < Lc; ++i) {
+        float dsp, du, uu;
+        float4 Bv, Cv;
+        int pos;
+        step(t0 + i, dsp, du, uu, Bv, Cv, pos);
+        const float bv[4] = {Bv.x, Bv.y, Bv.z, Bv.w};
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const float e = fast_exp2(dsp * a2[s]);
+            P[s] *= e;
+            H[s] = fmaf(e, H[s], du * bv[s]);
+        }
+    }
+
+    // ---- combine: inclusive shuffle scan of (P, H) over the chunk lanes ----------
+#pragma unroll
+    for (int off = 1; off < NC; off <<= 1) {
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const float Pp = __shfl_up_sync(FULL_MASK, P[s], 4 * off, LPC);
+            const float Hp = __shfl_up_sync(FULL_MASK, H[s], 4 * off, LPC);
+            if (j >= off) {
+                H[s] = fmaf(P[s], Hp, H[s]);
+                P[s] *= Pp;
+            }
+        }
+    }
+    float h[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        const float hin = __shfl_up_sync(FULL_MASK, H[s], 4, LPC);
+        h[s] = (j > 0) ? hin : 0.f;
+    }
+
+    // ---- pass 2: recurrence from the entering state, read-out ---------------------
+#pragma unroll 4
+    for (int i = 0; i < Lc; ++i) {
+        float dsp, du, uu;
+        float4 Bv, Cv;
+        int pos;
+        step(t0 + i, dsp, du, uu, Bv, Cv, pos);
+        const float bv[4] = {Bv.x, Bv.y, Bv.z, Bv.w};
+        const float cv[4] = {Cv.x, Cv.y, Cv.z, Cv.w};
+        float acc = 0.f;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const float e = fast_exp2(dsp * a2[s]);
+            h[s] = fmaf(e, h[s], du * bv[s]);
+            acc = fmaf(cv[s], h[s], acc);
+        }
+        acc += __shfl_xor_sync(FULL_MASK, acc, 1);
+        acc += __shfl_xor_sync(FULL_MASK, acc, 2);
+        if (grp == 0 && pos >= 0) sYk[(size_t)pos * CH + c] = fmaf(Dd, uu, acc);
+    }
+    __syncthreads();
+
+    // ---- merge the directions, gate, store ----------------------------------------
+    const T* zb = p.z ? static_cast<const T*>(p.z) + img * D : nullptr;
+    T* yb = static_cast<T*>(p.y) + img * D;
+    for (int e = tid; e < tokens * CH; e += nthreads) {
+        const int tok = e / CH, cc = e - tok * CH;
+        const int dd = c0 + cc;
+        if (dd >= D) continue;
+        float acc = 0.f;
+#pragma unroll
+        for (int pl = 0; pl < PLANES; ++pl) acc += sY[(size_t)pl * tokens * CH + e];
+        float o = acc * p.merge_scale;
+        if (zb) o *= silu_f(load_elem<T>(zb + (long long)tok * D + dd));
+        store_elem<T>(yb + (long long)tok * D + dd, o);
+    }
+}
+
+}  // namespace vscan

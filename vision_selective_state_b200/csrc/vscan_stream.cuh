@@ -4,11 +4,16 @@
 // all K directions of the route: warp k runs direction k. Inside a warp,
 // lane = 4*c + g owns channel c of the tile and the four states 4g..4g+3, so the
 // N = 16 states of a channel sit on 4 adjacent lanes and the read-out sum over
-// n is a 4-lane reduction. Each warp walks its direction's sequence in chunks
-// of 16 steps: the chunk's route tokens are gathered from HBM into registers
-// one chunk ahead (channels-last rows, so every gathered token is a contiguous
-// channel segment), then discretized once per (token, channel) into shared
-// memory, then consumed by the recurrence.
+// n is a 4-lane reduction.
+//
+// Data movement. Each warp walks its direction's sequence in chunks of 16
+// steps. For every chunk it gathers the route's tokens with cp.async straight
+// into a shared-memory stage: the 8-channel segments of u, raw Delta and z
+// (channels-last rows, so every gathered token is one contiguous 16- or
+// 32-byte piece) and the B and C rows, with zero fill for ATROUS2 padding.
+// NSTAGE chunks are in flight, so the gather latency is hidden behind the
+// recurrence of the chunks before it. Once a stage lands, the warp discretizes
+// it once per (step, channel) and runs the recurrence:
 //
 // Per step and state ("Vision Mamba ...", sec. 4; "EfficientVMamba", sec. 2):
 //     dA = 2^(Delta * A * log2 e)          (one SFU op)
@@ -52,17 +57,58 @@ struct ScanParams {
     float* scratch;    // merge routes: [K][batch][tokens][D] float32
 };
 
-constexpr int ST_TOK = 16;  // steps per staged chunk
-constexpr int ST_CH = 8;    // channels per warp
+constexpr int ST_TOK = 16;   // steps per chunk
+constexpr int ST_CH = 8;     // channels per warp
+constexpr int NSTAGE = 4;    // chunks in flight per warp
 
-struct __align__(16) StreamStage {
-    float4 B[ST_TOK][4];        // B[t][4q..4q+3]
-    float4 C[ST_TOK][4];
-    float dsp[ST_TOK][ST_CH];   // Delta after bias + softplus
-    float du[ST_TOK][ST_CH];    // Delta * u
-    float uu[ST_TOK][ST_CH];    // u (skip term)
-    int pos[ST_TOK];            // token index, -1 pad, -2 past the end
+// ---- cp.async (sm_80+ form, 16- and 4-byte) ------------------------------------
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid)
+{
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    const int n = valid ? 16 : 0;  // 0: fill the 16 bytes with zeros, read nothing
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
+}
+
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool valid)
+{
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    const int n = valid ? 4 : 0;
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+// Raw gathered chunk, in the I/O type.
+template <typename T>
+struct __align__(16) RawStage {
+    T u[ST_TOK][ST_CH];
+    T d[ST_TOK][ST_CH];
+    T z[ST_TOK][ST_CH];
+    T B[ST_TOK][16];
+    T C[ST_TOK][16];
+    int pos[ST_TOK];  // token index, -1 pad, -2 past the end
 };
+
+// Discretized chunk (float32), written once per chunk by the warp.
+struct __align__(16) PrepStage {
+    float4 B[ST_TOK][4];
+    float4 C[ST_TOK][4];
+    float dsp[ST_TOK][ST_CH];  // Delta after bias + softplus
+    float du[ST_TOK][ST_CH];   // Delta * u
+    float uu[ST_TOK][ST_CH];   // u (skip term)
+};
+
+template <typename T>
+struct WarpSmem {
+    RawStage<T> raw[NSTAGE];
+    PrepStage prep;
+};
+
+template <typename T>
+constexpr size_t stream_smem_bytes(int K) { return K * sizeof(WarpSmem<T>); }
 
 // Direction that adds up token p: the one visiting p in the latest chunk.
 template <int RK>
@@ -86,13 +132,14 @@ __global__ void __launch_bounds__(128) stream_scan_kernel(const ScanParams p)
 {
     constexpr bool MERGE = (RK == RK_BIDIR || RK == RK_CROSS4);
     constexpr int K = (RK == RK_BIDIR) ? 2 : 4;
+    constexpr bool F32 = sizeof(T) == 4;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    StreamStage* stages = reinterpret_cast<StreamStage*>(smem_raw);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int k = warp;
-    StreamStage& st = stages[warp];
+    WarpSmem<T>& sm = reinterpret_cast<WarpSmem<T>*>(smem_raw)[warp];
+    PrepStage& pr = sm.prep;
 
     const int b = blockIdx.y;
     const int c0 = blockIdx.x * ST_CH;
@@ -110,144 +157,137 @@ __global__ void __launch_bounds__(128) stream_scan_kernel(const ScanParams p)
     }
     const float Dd = (dvalid && p.Dskip) ? __ldg(p.Dskip + k * p.v_dir + d) : 0.f;
 
-    // Staging role: channel ce of the tile, steps (lane >> 3) + 4i.
+    // Prep role: channel ce of the tile, steps (lane >> 3) + 4i.
     const int ce = lane & 7;
-    const int ds = c0 + ce;
-    const bool svalid = ds < D;
-    const float bias_s = (svalid && p.bias) ? __ldg(p.bias + k * p.v_dir + ds) : 0.f;
+    const bool evalid = c0 + ce < D;
+    const float bias_e = (evalid && p.bias) ? __ldg(p.bias + k * p.v_dir + c0 + ce) : 0.f;
 
     const long long img = (long long)b * tokens;
-    const T* u_base = static_cast<const T*>(p.u) + k * p.in_dir + img * D;
-    const T* d_base = static_cast<const T*>(p.delta) + k * p.in_dir + img * D;
+    const T* u_base = static_cast<const T*>(p.u) + k * p.in_dir + img * D + c0;
+    const T* d_base = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + c0;
+    const T* z_base = p.z ? static_cast<const T*>(p.z) + img * D + c0 : nullptr;
     const T* B_base = static_cast<const T*>(p.B) + k * p.bc_dir + img * N;
     const T* C_base = static_cast<const T*>(p.C) + k * p.bc_dir + img * N;
-    const T* z_base = p.z ? static_cast<const T*>(p.z) + img * D : nullptr;
     T* y_base = static_cast<T*>(p.y) + img * D;
 
-    float h[4] = {0.f, 0.f, 0.f, 0.f};
-
-    // Registers holding the next chunk while the current one is computed.
-    float ru[4], rd[4];
-    float rb[8], rc[8];
-    int rpos = -2;
-
-    auto load_chunk = [&](int chunk) {
+    // Gather one chunk into raw stage s. Every lane issues the same number of
+    // cp.async operations and one commit, so group counting stays uniform.
+    auto issue = [&](int chunk, int s) {
+        RawStage<T>& st = sm.raw[s];
         const int t = chunk * ST_TOK + (lane & 15);
-        rpos = (t < L) ? route_token<RK>(p.g, k, t) : -2;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int j = (lane >> 3) + 4 * i;
-            const int pj = __shfl_sync(FULL_MASK, rpos, j);
-            if (pj >= 0 && svalid) {
-                ru[i] = load_elem<T>(u_base + (long long)pj * D + ds);
-                rd[i] = load_elem<T>(d_base + (long long)pj * D + ds);
+        const int mypos = (t < L) ? route_token<RK>(p.g, k, t) : -2;
+        if (lane < 16) st.pos[lane] = mypos;
+        if (F32) {
+            // u, Delta, z: 16 steps x 32 bytes; lane -> (step lane>>1, 4-channel half lane&1)
+            const int j = lane >> 1, hf = lane & 1;
+            const int pj = __shfl_sync(FULL_MASK, mypos, j);
+            const bool ok = pj >= 0 && (c0 + 4 * hf) < D;
+            const long long off = (long long)(ok ? pj : 0) * D + 4 * hf;
+            cp_async16(&st.u[j][4 * hf], u_base + off, ok);
+            cp_async16(&st.d[j][4 * hf], d_base + off, ok);
+            if (z_base) cp_async16(&st.z[j][4 * hf], z_base + off, ok);
+        } else {
+            // 16 steps x 16 bytes: lanes 0-15 take u (and z), lanes 16-31 take Delta
+            const int j = lane & 15;
+            const int pj = __shfl_sync(FULL_MASK, mypos, j);
+            const bool ok = pj >= 0;
+            const long long off = (long long)(ok ? pj : 0) * D;
+            if (lane < 16) {
+                cp_async16(&st.u[j][0], u_base + off, ok);
+                if (z_base) cp_async16(&st.z[j][0], z_base + off, ok);
             } else {
-                ru[i] = 0.f;
-                rd[i] = 0.f;
+                cp_async16(&st.d[j][0], d_base + off, ok);
             }
         }
         if (N16) {
-            if (sizeof(T) == 4) {
-                // 16 steps x 4 float4 per tensor: lane takes (step f>>2, quad f&3), f = lane + 32i
+            if (F32) {
+                // 16 steps x 4 quads x 16 bytes per tensor: f = lane + 32i -> (step f>>2, quad f&3)
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     const int f = lane + 32 * i;
-                    const int pj = __shfl_sync(FULL_MASK, rpos, f >> 2);
-                    float4 vb = make_float4(0.f, 0.f, 0.f, 0.f), vc = vb;
-                    if (pj >= 0) {
-                        vb = load4<T>(B_base + (long long)pj * 16 + 4 * (f & 3));
-                        vc = load4<T>(C_base + (long long)pj * 16 + 4 * (f & 3));
-                    }
-                    rb[4 * i + 0] = vb.x; rb[4 * i + 1] = vb.y; rb[4 * i + 2] = vb.z; rb[4 * i + 3] = vb.w;
-                    rc[4 * i + 0] = vc.x; rc[4 * i + 1] = vc.y; rc[4 * i + 2] = vc.z; rc[4 * i + 3] = vc.w;
+                    const int pj = __shfl_sync(FULL_MASK, mypos, f >> 2);
+                    const bool ok = pj >= 0;
+                    const long long off = (long long)(ok ? pj : 0) * 16 + 4 * (f & 3);
+                    cp_async16(&st.B[f >> 2][4 * (f & 3)], B_base + off, ok);
+                    cp_async16(&st.C[f >> 2][4 * (f & 3)], C_base + off, ok);
                 }
             } else {
-                // 16 steps x 2 halves of 8 bf16: lane takes (step lane>>1, half lane&1)
-                const int pj = __shfl_sync(FULL_MASK, rpos, lane >> 1);
-                float4 b0 = make_float4(0.f, 0.f, 0.f, 0.f), b1 = b0, q0 = b0, q1 = b0;
-                if (pj >= 0) {
-                    const T* pb = B_base + (long long)pj * 16 + 8 * (lane & 1);
-                    const T* pc = C_base + (long long)pj * 16 + 8 * (lane & 1);
-                    b0 = load4<T>(pb); b1 = load4<T>(pb + 4);
-                    q0 = load4<T>(pc); q1 = load4<T>(pc + 4);
-                }
-                rb[0] = b0.x; rb[1] = b0.y; rb[2] = b0.z; rb[3] = b0.w;
-                rb[4] = b1.x; rb[5] = b1.y; rb[6] = b1.z; rb[7] = b1.w;
-                rc[0] = q0.x; rc[1] = q0.y; rc[2] = q0.z; rc[3] = q0.w;
-                rc[4] = q1.x; rc[5] = q1.y; rc[6] = q1.z; rc[7] = q1.w;
+                // 16 steps x 2 halves x 16 bytes: lane -> (step lane>>1, half lane&1)
+                const int j = lane >> 1, hf = lane & 1;
+                const int pj = __shfl_sync(FULL_MASK, mypos, j);
+                const bool ok = pj >= 0;
+                const long long off = (long long)(ok ? pj : 0) * 16 + 8 * hf;
+                cp_async16(&st.B[j][8 * hf], B_base + off, ok);
+                cp_async16(&st.C[j][8 * hf], C_base + off, ok);
             }
         } else {
-            // Any N <= 16: 16 steps x 16 state slots, lane takes slot e = lane + 32i.
+            // Any N <= 16: element loads (the 16-byte path needs 16-float rows).
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int e = lane + 32 * i;
-                const int n = e & 15;
-                const int pj = __shfl_sync(FULL_MASK, rpos, e >> 4);
-                float vb = 0.f, vc = 0.f;
+                const int n = e & 15, j = e >> 4;
+                const int pj = __shfl_sync(FULL_MASK, mypos, j);
+                T vb = T(0.f), vc = T(0.f);
                 if (pj >= 0 && n < N) {
-                    vb = load_elem<T>(B_base + (long long)pj * N + n);
-                    vc = load_elem<T>(C_base + (long long)pj * N + n);
+                    vb = B_base[(long long)pj * N + n];
+                    vc = C_base[(long long)pj * N + n];
                 }
-                rb[i] = vb;
-                rc[i] = vc;
+                st.B[j][n] = vb;
+                st.C[j][n] = vc;
             }
         }
+        cp_async_commit();
     };
 
-    auto commit_chunk = [&]() {
+    // Discretize a landed raw stage into the prep buffers (once per step and channel).
+    auto prepare = [&](const RawStage<T>& st) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int j = (lane >> 3) + 4 * i;
-            const int pj = __shfl_sync(FULL_MASK, rpos, j);
-            const float x = rd[i] + bias_s;
+            const int pj = st.pos[j];
+            float uu = to_float(st.u[j][ce]);
+            const float x = to_float(st.d[j][ce]) + bias_e;
             float dsp = p.softplus ? softplus_f(x) : x;
-            float uu = ru[i];
-            if (pj == -2 || !svalid) {  // past the end: a no-op step
+            if (pj == -2 || !evalid) {  // past the end: a no-op step
                 dsp = 0.f;
                 uu = 0.f;
             }
-            st.dsp[j][ce] = dsp;
-            st.du[j][ce] = dsp * uu;
-            st.uu[j][ce] = uu;
+            pr.dsp[j][ce] = dsp;
+            pr.du[j][ce] = dsp * uu;
+            pr.uu[j][ce] = uu;
         }
-        if (N16) {
-            if (sizeof(T) == 4) {
+        // B and C to float32: 16 steps x 16 states each, lane -> 8 values per tensor
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int f = lane + 32 * i;
-                    st.B[f >> 2][f & 3] = make_float4(rb[4 * i], rb[4 * i + 1], rb[4 * i + 2], rb[4 * i + 3]);
-                    st.C[f >> 2][f & 3] = make_float4(rc[4 * i], rc[4 * i + 1], rc[4 * i + 2], rc[4 * i + 3]);
-                }
-            } else {
-                const int j = lane >> 1, q = 2 * (lane & 1);
-                st.B[j][q] = make_float4(rb[0], rb[1], rb[2], rb[3]);
-                st.B[j][q + 1] = make_float4(rb[4], rb[5], rb[6], rb[7]);
-                st.C[j][q] = make_float4(rc[0], rc[1], rc[2], rc[3]);
-                st.C[j][q + 1] = make_float4(rc[4], rc[5], rc[6], rc[7]);
-            }
-        } else {
-            float* sb = reinterpret_cast<float*>(&st.B[0][0]);
-            float* sc = reinterpret_cast<float*>(&st.C[0][0]);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int e = lane + 32 * i;
-                sb[e] = rb[i];
-                sc[e] = rc[i];
-            }
+        for (int i = 0; i < 2; ++i) {
+            const int f = lane + 32 * i;  // (step f>>2, quad f&3)
+            const int j = f >> 2, q = f & 3;
+            pr.B[j][q] = make_float4(to_float(st.B[j][4 * q]), to_float(st.B[j][4 * q + 1]),
+                                     to_float(st.B[j][4 * q + 2]), to_float(st.B[j][4 * q + 3]));
+            pr.C[j][q] = make_float4(to_float(st.C[j][4 * q]), to_float(st.C[j][4 * q + 1]),
+                                     to_float(st.C[j][4 * q + 2]), to_float(st.C[j][4 * q + 3]));
         }
-        if (lane < 16) st.pos[lane] = rpos;
     };
 
+    float h[4] = {0.f, 0.f, 0.f, 0.f};
     const int nchunks = (L + ST_TOK - 1) / ST_TOK;
-    load_chunk(0);
-    commit_chunk();
-    __syncwarp();
+
+#pragma unroll
+    for (int s = 0; s < NSTAGE - 1; ++s) {
+        if (s < nchunks) issue(s, s);
+        else cp_async_commit();
+    }
 
     for (int chunk = 0; chunk < nchunks; ++chunk) {
-        const bool more = chunk + 1 < nchunks;
-        if (more) load_chunk(chunk + 1);
+        const int ahead = chunk + NSTAGE - 1;
+        if (ahead < nchunks) issue(ahead, ahead % NSTAGE);
+        else cp_async_commit();
+        cp_async_wait<NSTAGE - 1>();
+        __syncwarp();
+        const RawStage<T>& st = sm.raw[chunk % NSTAGE];
+        prepare(st);
+        __syncwarp();
 
-        // ---- recurrence over the 16 staged steps -----------------------------
+        // ---- recurrence over the 16 steps ----------------------------------------
         float yv[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -255,10 +295,10 @@ __global__ void __launch_bounds__(128) stream_scan_kernel(const ScanParams p)
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
                 const int j = 4 * q + jj;
-                const float dsp = st.dsp[j][cc];
-                const float du = st.du[j][cc];
-                const float4 Bv = st.B[j][grp];
-                const float4 Cv = st.C[j][grp];
+                const float dsp = pr.dsp[j][cc];
+                const float du = pr.du[j][cc];
+                const float4 Bv = pr.B[j][grp];
+                const float4 Cv = pr.C[j][grp];
                 const float e0 = fast_exp2(dsp * a2[0]);
                 const float e1 = fast_exp2(dsp * a2[1]);
                 const float e2 = fast_exp2(dsp * a2[2]);
@@ -285,27 +325,26 @@ __global__ void __launch_bounds__(128) stream_scan_kernel(const ScanParams p)
             float keep = odd ? a1 : a0;
             const float send = odd ? a0 : a1;
             keep += __shfl_xor_sync(FULL_MASK, send, 1);
-            yv[q] = fmaf(Dd, st.uu[4 * q + grp][cc], keep);
+            yv[q] = fmaf(Dd, pr.uu[4 * q + grp][cc], keep);
         }
 
-        // ---- merge, gate and store --------------------------------------------
+        // ---- merge, gate and store ------------------------------------------------
         if (!MERGE) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const int pj = st.pos[4 * q + grp];
+                const int j = 4 * q + grp;
+                const int pj = st.pos[j];
                 if (pj >= 0 && dvalid) {
                     float o = yv[q] * p.merge_scale;
-                    if (z_base) o *= silu_f(load_elem<T>(z_base + (long long)pj * D + d));
+                    if (z_base) o *= silu_f(to_float(st.z[j][cc]));
                     store_elem<T>(y_base + (long long)pj * D + d, o);
                 }
             }
         } else {
             bool mine[4];
-            int pos4[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int pj = st.pos[4 * q + grp];
-                pos4[q] = pj;
                 mine[q] = false;
                 if (pj >= 0 && dvalid) {
                     if (finalizer<RK>(p.g, pj) == k) {
@@ -319,7 +358,8 @@ __global__ void __launch_bounds__(128) stream_scan_kernel(const ScanParams p)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 if (mine[q]) {
-                    const int pj = pos4[q];
+                    const int j = 4 * q + grp;
+                    const int pj = st.pos[j];
                     float acc = yv[q];
 #pragma unroll
                     for (int kk = 0; kk < K; ++kk) {
@@ -327,16 +367,14 @@ __global__ void __launch_bounds__(128) stream_scan_kernel(const ScanParams p)
                         acc += p.scratch[(((long long)kk * p.batch + b) * tokens + pj) * D + d];
                     }
                     float o = acc * p.merge_scale;
-                    if (z_base) o *= silu_f(load_elem<T>(z_base + (long long)pj * D + d));
+                    if (z_base) o *= silu_f(to_float(st.z[j][cc]));
                     store_elem<T>(y_base + (long long)pj * D + d, o);
                 }
             }
         }
-
-        __syncwarp();
-        if (more) commit_chunk();
         __syncwarp();
     }
+    cp_async_wait<0>();
 }
 
 }  // namespace vscan
