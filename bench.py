@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline budget")
+    p.add_argument("--batch", type=int, default=0,
+                   help="override the workload's batch (small profiling captures only)")
     p.add_argument("--rotate", type=int, default=0,
                    help="device copies of the inputs cycled through (0: enough to exceed 3x L2)")
     return p.parse_args()
@@ -472,6 +474,8 @@ def run_ours(args, wls):
 def main():
     args = parse()
     wls = select(args.workload)
+    if args.batch > 0:
+        wls = [w.with_(batch=args.batch) for w in wls]
     if args.impl == "reference":
         run_reference(args, wls)
     else:

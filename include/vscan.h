@@ -169,12 +169,20 @@ vscan_status vscan_route_indices(const vscan_route* route, int32_t* dev_out, voi
 
 /*
  * Device scratch bytes vscan_forward needs for these arguments (host only).
- * BIDIR and CROSS4 hold per-direction partial outputs until the last direction
- * of a token adds them up; POOL_W/POOL_H hold the pooled B and C; ATROUS2
- * needs none (every pixel has one owner).
+ * BIDIR and CROSS4 park per-direction partial outputs until the last
+ * direction of a token adds them up ([K][batch][tokens][D] float32); POOL_W
+ * and POOL_H hold the pooled B and C; ATROUS2 needs none (one owner per pixel).
  */
 vscan_status vscan_workspace_size(const vscan_route* route, const vscan_args* args,
                                   uint64_t* bytes);
+
+/*
+ * Number of kernel launches vscan_forward makes for these arguments (host
+ * only): 1 for BIDIR, CROSS4 and ATROUS2 (streaming or resident chunked
+ * scan), 2 for the pooled routes (B/C pooling, then the fused
+ * pool-scan-repeat), 0 for an empty batch.
+ */
+vscan_status vscan_plan_info(const vscan_route* route, const vscan_args* args, int32_t* kernels);
 
 /*
  * Run the fused routed scan on the device. Enqueued on stream; allocates

@@ -131,6 +131,18 @@ def test_null_and_misaligned_pointers_are_rejected():
     assert abi.lib.vscan_forward_host(rb.handle, ctypes.byref(hb), None, 0, None) == -6
 
 
+def test_plan_info_counts_launches():
+    n = ctypes.c_int32()
+    for kind, h, w, cls, chunks, expect in (("atrous2", 56, 56, -1, 0, 1), ("cross4", 56, 56, -1, 0, 1),
+                                            ("bidir", 64, 64, 2048, 1, 1), ("bidir", 14, 14, 98, 4, 1),
+                                            ("pool_w", 8, 8, -1, 0, 2)):
+        r = vs.Route(kind, h, w, cls)
+        assert abi.lib.vscan_plan_info(r.handle, ctypes.byref(_args(seq_chunks=chunks)), ctypes.byref(n)) == 0
+        assert n.value == expect, kind
+    r = vs.Route("atrous2", 4, 4)
+    assert abi.lib.vscan_plan_info(r.handle, ctypes.byref(_args(batch=0)), ctypes.byref(n)) == 0 and n.value == 0
+
+
 def test_chunked_scan_needs_the_tile_on_chip():
     big = vs.Route("cross4", 56, 56)
     assert abi.lib.vscan_forward(big.handle, ctypes.byref(_args(seq_chunks=4)), None) == -4

@@ -81,6 +81,14 @@ def test_resident_chunked_scan(route, nc, h, w):
     _case(route, h, w, 8, 16, "f32", seq_chunks=nc, merge_scale=0.5, gate=False)
 
 
+@pytest.mark.parametrize("route,h,w", [("bidir", 14, 14), ("cross4", 9, 13), ("atrous2", 9, 13),
+                                       ("bidir", 31, 33), ("cross4", 31, 33), ("atrous2", 31, 33)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_streaming_kernel_full_state_rows(route, h, w, dtype):
+    """The streaming kernel (seq_chunks=1) with N = 16, both I/O types, short and long sequences."""
+    _case(route, h, w, 16, 16, dtype, seq_chunks=1)
+
+
 def test_bidirectional_without_cls_and_long_sequences():
     _case("bidir", 10, 10, 16, 16, "f32", cls=-1)
     _case("bidir", 40, 40, 16, 16, "f32", batch=1)       # L = 1601, CLS 800

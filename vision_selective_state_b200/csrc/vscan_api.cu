@@ -84,6 +84,8 @@ vscan_status check_shape(const vscan_route* r, const vscan_args* a)
         a->seq_chunks != 8)
         return fail(VSCAN_ERR_INVALID_ARGUMENT, "seq_chunks %d is not 0, 1, 2, 4 or 8", a->seq_chunks);
     if (a->batch > 65535) return fail(VSCAN_ERR_UNSUPPORTED, "batch %d > 65535", a->batch);
+    if ((long long)r->g.tokens * a->channels >= (1LL << 31))
+        return fail(VSCAN_ERR_UNSUPPORTED, "tokens x channels of one image must be below 2^31");
     if (is_pool(r->g.kind)) {
         const int Ki = a->per_dir_inputs ? 2 : 1;
         if (vscan::pool_scan_smem_bytes(Ki, r->g.L) > kMaxSmem)
@@ -130,7 +132,7 @@ uint64_t workspace_need(const vscan_route* r, const vscan_args* a)
 {
     const vscan::RouteGeom& g = r->g;
     if (a->batch == 0) return 0;
-    if (g.kind == vscan::RK_BIDIR || g.kind == vscan::RK_CROSS4)
+    if (g.kind == vscan::RK_BIDIR || g.kind == vscan::RK_CROSS4)  // one parking plane per direction
         return round256((uint64_t)g.K * a->batch * g.tokens * a->channels * sizeof(float));
     if (is_pool(g.kind)) {
         const int Ki = a->per_dir_inputs ? 2 : 1;
@@ -139,17 +141,35 @@ uint64_t workspace_need(const vscan_route* r, const vscan_args* a)
     return 0;
 }
 
+template <int RK, typename T, bool N16, int KC, int MODE>
+cudaError_t launch_stream_mode(vscan::ScanParams p, int k_base, int grid_z, cudaStream_t s)
+{
+    const size_t smem = vscan::stream_smem_bytes<T, KC, MODE>();
+    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16, KC, MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    p.k_base = k_base;
+    const dim3 grid((p.D + vscan::ST_CH - 1) / vscan::ST_CH, p.batch, grid_z);
+    vscan::stream_scan_kernel<RK, T, N16, KC, MODE>
+        <<<grid, vscan::StreamShape<T, KC, MODE>::THREADS, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+// ATROUS2: every pixel has one owner; float32 I/O runs one direction per CTA
+//   (grid.z = 4), bf16 I/O all four directions per CTA.
+// BIDIR, CROSS4: all directions of an image tile in one CTA, merged by parking.
 template <int RK, typename T, bool N16>
 cudaError_t launch_stream_n(const vscan::ScanParams& p, cudaStream_t s)
 {
-    constexpr int K = (RK == vscan::RK_BIDIR) ? 2 : 4;
-    const size_t smem = vscan::stream_smem_bytes<T>(K);
-    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const dim3 grid((p.D + vscan::ST_CH - 1) / vscan::ST_CH, p.batch);
-    vscan::stream_scan_kernel<RK, T, N16><<<grid, 32 * K, smem, s>>>(p);
-    return cudaSuccess;
+    using namespace vscan;
+    if constexpr (RK == RK_ATROUS2) {
+        if constexpr (sizeof(T) == 4) return launch_stream_mode<RK, T, N16, 1, MODE_OWNER>(p, 0, 4, s);
+        else return launch_stream_mode<RK, T, N16, 4, MODE_OWNER>(p, 0, 1, s);
+    } else if constexpr (RK == RK_BIDIR) {
+        return launch_stream_mode<RK, T, N16, 2, MODE_PARK>(p, 0, 1, s);
+    } else {
+        return launch_stream_mode<RK, T, N16, 4, MODE_PARK>(p, 0, 1, s);
+    }
 }
 
 template <int RK, typename T>
@@ -383,6 +403,18 @@ vscan_status vscan_forward(const vscan_route* r, const vscan_args* a, void* stre
     st = check_pointers(a, true);
     if (st != VSCAN_OK) return st;
     return forward_device(r, a, static_cast<cudaStream_t>(stream));
+}
+
+vscan_status vscan_plan_info(const vscan_route* r, const vscan_args* a, int32_t* kernels)
+{
+    if (!kernels) return fail(VSCAN_ERR_INVALID_ARGUMENT, "kernels is NULL");
+    vscan_status st = check_shape(r, a);
+    if (st != VSCAN_OK) return st;
+    if (a->batch == 0) *kernels = 0;
+    else if (is_pool(r->g.kind)) *kernels = 2;
+    else if (choose_chunks(r, a) > 1) *kernels = 1;
+    else *kernels = 1;
+    return VSCAN_OK;
 }
 
 vscan_status vscan_host_buffer_size(const vscan_route* r, const vscan_args* a, uint64_t* bytes)

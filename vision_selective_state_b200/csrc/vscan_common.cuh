@@ -91,18 +91,41 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
-// softplus(x) = log(1 + e^x) ("Vision Mamba ...", sec. 3). Above 20 the two
-// differ by less than 2^-28 relative, so x itself is returned, as PyTorch's
-// softplus does.
-__device__ __forceinline__ float softplus_f(float x)
+__device__ __forceinline__ float fast_rcp(float x)
 {
-    return x > 20.0f ? x : log1pf(expf(x));
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
-// SiLU(z) = z * sigma(z), signed and unbounded ("Vision Mamba ...", sec. 5).
+constexpr float LN2 = 0.69314718055994531f;
+
+// softplus(x) = log(1 + e^x) ("Vision Mamba ...", sec. 3), evaluated as
+//     max(x, 0) + ln 2 * t * P(t),   t = 2^(-|x| log2 e) in (0, 1],
+// i.e. max(x, 0) + log(1 + e^-|x|) with log2(1 + t) = t * P(t). P is a degree-8
+// least-squares fit of log2(1 + t) / t on [0, 1] made by fit_log2p1.py
+// (relative error 1.4e-7 in float32). One SFU op.
+__device__ __forceinline__ float softplus_f(float x)
+{
+    const float t = fast_exp2(-fabsf(x) * LOG2E);
+    float p = 7.366087753e-03f;
+    p = fmaf(p, t, -4.182628542e-02f);
+    p = fmaf(p, t, 1.116363406e-01f);
+    p = fmaf(p, t, -1.960704774e-01f);
+    p = fmaf(p, t, 2.751406133e-01f);
+    p = fmaf(p, t, -3.582780361e-01f);
+    p = fmaf(p, t, 4.806761742e-01f);
+    p = fmaf(p, t, -7.213394046e-01f);
+    p = fmaf(p, t, 1.442695022e+00f);
+    return fmaxf(x, 0.f) + LN2 * (t * p);
+}
+
+// SiLU(z) = z * sigma(z) = z / (1 + e^-z), signed and unbounded ("Vision
+// Mamba ...", sec. 5). Two SFU ops (2^x and the reciprocal); for z below about
+// -88, e^-z overflows to +inf and the result is a signed zero.
 __device__ __forceinline__ float silu_f(float z)
 {
-    return z / (1.0f + expf(-z));
+    return z * fast_rcp(1.0f + fast_exp2(-z * LOG2E));
 }
 
 }  // namespace vscan

@@ -245,7 +245,10 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
     __syncthreads();
 
     // ---- phase 3: repeat over the pooled axis, merge, gate, store ---------------
+    // Eight tokens per thread per round, loads first, so that each thread keeps
+    // 128 bytes of z in flight.
     {
+        constexpr int U = 8;
         const int q = tid & 7;        // channel quad
         const int tl = tid >> 3;      // token lane 0..31
         const int ch = c0 + 4 * q;
@@ -255,19 +258,30 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
             const T* zb = p.z ? static_cast<const T*>(p.z) + img * D + ch : nullptr;
             T* yb = static_cast<T*>(p.y) + img * D + ch;
             const float scale = p.merge_scale;
-            for (int tok = tl; tok < tokens; tok += 32) {
-                const int r = tok / p.g.w;
-                const int col = tok - r * p.g.w;
-                const int i = (p.g.kind == RK_POOL_W) ? r : col;
-                const float4 f = *reinterpret_cast<const float4*>(Y0 + (size_t)i * PL_CH + 4 * q);
-                const float4 g = *reinterpret_cast<const float4*>(Y1 + (size_t)i * PL_CH + 4 * q);
-                float4 o = make_float4((f.x + g.x) * scale, (f.y + g.y) * scale,
-                                       (f.z + g.z) * scale, (f.w + g.w) * scale);
-                if (zb) {
-                    const float4 zz = load4<T>(zb + (long long)tok * D);
-                    o.x *= silu_f(zz.x); o.y *= silu_f(zz.y); o.z *= silu_f(zz.z); o.w *= silu_f(zz.w);
+            for (int tok0 = tl; tok0 < tokens; tok0 += 32 * U) {
+                float4 zz[U];
+#pragma unroll
+                for (int v = 0; v < U; ++v) {
+                    const int tok = tok0 + 32 * v;
+                    zz[v] = (zb && tok < tokens) ? load4<T>(zb + (long long)tok * D) : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-                store4<T>(yb + (long long)tok * D, o);
+#pragma unroll
+                for (int v = 0; v < U; ++v) {
+                    const int tok = tok0 + 32 * v;
+                    if (tok >= tokens) break;
+                    const int r = tok / p.g.w;
+                    const int col = tok - r * p.g.w;
+                    const int i = (p.g.kind == RK_POOL_W) ? r : col;
+                    const float4 f = *reinterpret_cast<const float4*>(Y0 + (size_t)i * PL_CH + 4 * q);
+                    const float4 g = *reinterpret_cast<const float4*>(Y1 + (size_t)i * PL_CH + 4 * q);
+                    float4 o = make_float4((f.x + g.x) * scale, (f.y + g.y) * scale,
+                                           (f.z + g.z) * scale, (f.w + g.w) * scale);
+                    if (zb) {
+                        o.x *= silu_f(zz[v].x); o.y *= silu_f(zz[v].y);
+                        o.z *= silu_f(zz[v].z); o.w *= silu_f(zz[v].w);
+                    }
+                    store4<T>(yb + (long long)tok * D, o);
+                }
             }
         }
     }

@@ -1,40 +1,46 @@
 // Streaming routed selective scan: BIDIR, CROSS4 and ATROUS2 routes.
 //
-// Work decomposition. One CTA covers one image b and a tile of 8 channels for
-// all K directions of the route: warp k runs direction k. Inside a warp,
-// lane = 4*c + g owns channel c of the tile and the four states 4g..4g+3, so the
-// N = 16 states of a channel sit on 4 adjacent lanes and the read-out sum over
-// n is a 4-lane reduction.
+// One CTA covers one image b, a tile of 8 channels and KC directions of the
+// route, and runs them as a software pipeline over 16-step chunks with two
+// kinds of warps:
 //
-// Data movement. Each warp walks its direction's sequence in chunks of 16
-// steps. For every chunk it gathers the route's tokens with cp.async straight
-// into a shared-memory stage: the 8-channel segments of u, raw Delta and z
-// (channels-last rows, so every gathered token is one contiguous 16- or
-// 32-byte piece) and the B and C rows, with zero fill for ATROUS2 padding.
-// NSTAGE chunks are in flight, so the gather latency is hidden behind the
-// recurrence of the chunks before it. Once a stage lands, the warp discretizes
-// it once per (step, channel) and runs the recurrence:
+//   consumer warp (one per direction) runs only the recurrence. Lane 4*c + g
+//     owns channel c of the tile and states 4g..4g+3, so the 16 states of a
+//     channel sit on 4 adjacent lanes and the read-out sum over n is a 4-lane
+//     reduction. Per step and state ("Vision Mamba ...", sec. 4;
+//     "EfficientVMamba", sec. 2), two states per packed f32x2 instruction:
+//         dA = 2^(Delta * A * log2 e)        (one SFU op)
+//         h  = dA * h + (Delta * u) * B      (FMUL + FFMA)
+//         y += C * h                         (FFMA)
 //
-// Per step and state ("Vision Mamba ...", sec. 4; "EfficientVMamba", sec. 2):
-//     dA = 2^(Delta * A * log2 e)          (one SFU op)
-//     h  = dA * h + (Delta * u) * B        (FMUL + FFMA)
-//     y += C * h                           (FFMA)
+//   producer warp (one per direction) does everything that happens once per
+//     (step, channel): it gathers the route's tokens for chunk tau+1+LOOK with
+//     cp.async into a shared-memory ring (zero fill for ATROUS2 padding;
+//     channels-last rows make every gathered token one contiguous segment),
+//     discretizes chunk tau+1 (Delta = softplus(raw + bias), Delta*u, B and C
+//     as float32), and finishes chunk tau-1.
 //
-// Merge. ATROUS2 gives every pixel one owner ("EfficientVMamba", sec. 3), so
-// each direction gates and stores its own outputs. BIDIR and CROSS4 add the
-// K aligned outputs of every token ("Vision Mamba ...", sec. 5; SS2D): the
-// direction that visits a token in the latest 16-step chunk (ties: larger k)
-// is its finalizer. Every other direction parks its contribution in the fp32
-// workspace; after the CTA barrier that closes the chunk, the finalizer adds
-// the parked values to its own, scales, gates with SiLU(z) and stores. All
-// directions of a token live in the same CTA, so no atomics and no second pass
-// over y are needed.
+// All warps meet at one CTA barrier per chunk, so the gather of chunk tau+4,
+// the discretization of tau+1, the recurrence of tau and the epilogue of tau-1
+// overlap.
+//
+// How a direction's output y_k (including its skip term D*u) becomes y
+// (merge: "Vision Mamba ...", sec. 5; "EfficientVMamba", sec. 3; SS2D):
+//   MODE_OWNER    ATROUS2: every pixel has one owner; y = s * y_k * SiLU(z).
+//   MODE_PARK     all KC = K directions in one CTA (BIDIR, CROSS4): the
+//                 direction that visits a token in the latest chunk (ties:
+//                 larger k) adds it up. The others park y_k in the fp32
+//                 workspace; one barrier later the finalizer adds the parked
+//                 values to its own, scales, gates and stores.
+// Neither mode uses atomics or a separate pass over y.
 #pragma once
 
 #include "vscan_common.cuh"
 #include "vscan_route.cuh"
 
 namespace vscan {
+
+enum StreamMode : int { MODE_OWNER = 0, MODE_PARK = 1 };
 
 struct ScanParams {
     RouteGeom g;
@@ -54,14 +60,15 @@ struct ScanParams {
     int v_dir;         // elements between directions of Dskip / bias (0 or D)
     int softplus;
     float merge_scale;
-    float* scratch;    // merge routes: [K][batch][tokens][D] float32
+    int k_base;        // first direction of this launch (direction = k_base + blockIdx.z*KC + local)
+    float* scratch;    // PARK: [K][batch][tokens][D] float32
 };
 
-constexpr int ST_TOK = 16;   // steps per chunk
-constexpr int ST_CH = 8;     // channels per warp
-constexpr int NSTAGE = 4;    // chunks in flight per warp
+constexpr int ST_TOK = 16;  // steps per chunk
+constexpr int ST_CH = 8;    // channels per CTA
+constexpr int ST_LOOK = 3;  // chunks between a gather and its discretization
 
-// ---- cp.async (sm_80+ form, 16- and 4-byte) ------------------------------------
+// ---- cp.async (16-byte, L2 only) ------------------------------------------------
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid)
 {
     const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
@@ -69,46 +76,68 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool va
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
 }
 
-__device__ __forceinline__ void cp_async4(void* smem, const void* gmem, bool valid)
-{
-    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-    const int n = valid ? 4 : 0;
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
-}
-
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
-// Raw gathered chunk, in the I/O type.
+// Gathered per-token rows of one direction's chunk, in the I/O type.
 template <typename T>
-struct __align__(16) RawStage {
+struct __align__(16) TokStage {
     T u[ST_TOK][ST_CH];
     T d[ST_TOK][ST_CH];
     T z[ST_TOK][ST_CH];
+    int pos[ST_TOK];  // token index, -1 pad, -2 past the end
+    int fin[ST_TOK];  // MODE_PARK: 1 if this direction adds up the token
+};
+
+// Gathered B and C rows of one direction's chunk, in the I/O type.
+template <typename T>
+struct __align__(16) BCStage {
     T B[ST_TOK][16];
     T C[ST_TOK][16];
-    int pos[ST_TOK];  // token index, -1 pad, -2 past the end
 };
 
-// Discretized chunk (float32), written once per chunk by the warp.
-struct __align__(16) PrepStage {
+// Discretized chunk of one direction; with CONV, float32 copies of B and C.
+template <bool CONV>
+struct PrepStage;
+
+template <>
+struct __align__(16) PrepStage<true> {
     float4 B[ST_TOK][4];
     float4 C[ST_TOK][4];
-    float dsp[ST_TOK][ST_CH];  // Delta after bias + softplus
-    float du[ST_TOK][ST_CH];   // Delta * u
-    float uu[ST_TOK][ST_CH];   // u (skip term)
+    float2 dd[ST_TOK][ST_CH];  // {Delta after bias + softplus (0 past the end), Delta * u}
 };
 
-template <typename T>
-struct WarpSmem {
-    RawStage<T> raw[NSTAGE];
-    PrepStage prep;
+template <>
+struct __align__(16) PrepStage<false> {
+    float2 dd[ST_TOK][ST_CH];
 };
 
-template <typename T>
-constexpr size_t stream_smem_bytes(int K) { return K * sizeof(WarpSmem<T>); }
+template <typename T, int KC, int MODE>
+struct StreamShape {
+    static constexpr bool F32 = sizeof(T) == 4;
+    static constexpr bool PARK = MODE == MODE_PARK;
+    // token slot of chunk c lives from its gather (tau = c-1-LOOK) to its last
+    // epilogue use (tau = c+1, or c+2 when parking)
+    static constexpr int NR = ST_LOOK + (PARK ? 4 : 3);
+    // B/C slot: until discretized at tau = c-1 (bf16) or consumed at tau = c (f32)
+    static constexpr int NBC = ST_LOOK + (F32 ? 2 : 1);
+    static constexpr int NY = PARK ? 3 : 2;  // output ring
+    static constexpr int THREADS = 64 * KC;  // a consumer and a producer per direction
+};
+
+template <typename T, int KC, int MODE>
+struct StreamSmem {
+    using S = StreamShape<T, KC, MODE>;
+    TokStage<T> tok[KC][S::NR];
+    BCStage<T> bc[KC][S::NBC];
+    PrepStage<!S::F32> prep[KC][2];
+    float yout[KC][S::NY][ST_TOK][ST_CH];
+};
+
+template <typename T, int KC, int MODE>
+constexpr size_t stream_smem_bytes() { return sizeof(StreamSmem<T, KC, MODE>); }
 
 // Direction that adds up token p: the one visiting p in the latest chunk.
 template <int RK>
@@ -127,252 +156,320 @@ __device__ __forceinline__ int finalizer(const RouteGeom& g, int p)
     return best_k;
 }
 
-template <int RK, typename T, bool N16>
-__global__ void __launch_bounds__(128) stream_scan_kernel(const ScanParams p)
+template <int RK, typename T, bool N16, int KC, int MODE>
+__global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan_kernel(const ScanParams p)
 {
-    constexpr bool MERGE = (RK == RK_BIDIR || RK == RK_CROSS4);
-    constexpr int K = (RK == RK_BIDIR) ? 2 : 4;
-    constexpr bool F32 = sizeof(T) == 4;
+    using S = StreamShape<T, KC, MODE>;
+    constexpr int NR = S::NR, NBC = S::NBC, NY = S::NY;
+    constexpr bool PARK = S::PARK;
+    constexpr bool F32 = S::F32;
+    constexpr int KR = (RK == RK_BIDIR) ? 2 : 4;  // directions of the route
     extern __shared__ __align__(16) unsigned char smem_raw[];
+    StreamSmem<T, KC, MODE>& sm = *reinterpret_cast<StreamSmem<T, KC, MODE>*>(smem_raw);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int k = warp;
-    WarpSmem<T>& sm = reinterpret_cast<WarpSmem<T>*>(smem_raw)[warp];
-    PrepStage& pr = sm.prep;
-
     const int b = blockIdx.y;
     const int c0 = blockIdx.x * ST_CH;
     const int D = p.D, N = p.N, L = p.g.L, tokens = p.g.tokens;
-
-    // Compute role: channel cc, states 4*grp .. 4*grp+3.
-    const int cc = lane >> 2, grp = lane & 3;
-    const int d = c0 + cc;
-    const bool dvalid = d < D;
-    float a2[4];
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        const int n = 4 * grp + s;
-        a2[s] = (dvalid && n < N) ? __ldg(p.A + (long long)k * p.a_dir + (long long)d * N + n) * LOG2E : 0.f;
-    }
-    const float Dd = (dvalid && p.Dskip) ? __ldg(p.Dskip + k * p.v_dir + d) : 0.f;
-
-    // Prep role: channel ce of the tile, steps (lane >> 3) + 4i.
-    const int ce = lane & 7;
-    const bool evalid = c0 + ce < D;
-    const float bias_e = (evalid && p.bias) ? __ldg(p.bias + k * p.v_dir + c0 + ce) : 0.f;
-
-    const long long img = (long long)b * tokens;
-    const T* u_base = static_cast<const T*>(p.u) + k * p.in_dir + img * D + c0;
-    const T* d_base = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + c0;
-    const T* z_base = p.z ? static_cast<const T*>(p.z) + img * D + c0 : nullptr;
-    const T* B_base = static_cast<const T*>(p.B) + k * p.bc_dir + img * N;
-    const T* C_base = static_cast<const T*>(p.C) + k * p.bc_dir + img * N;
-    T* y_base = static_cast<T*>(p.y) + img * D;
-
-    // Gather one chunk into raw stage s. Every lane issues the same number of
-    // cp.async operations and one commit, so group counting stays uniform.
-    auto issue = [&](int chunk, int s) {
-        RawStage<T>& st = sm.raw[s];
-        const int t = chunk * ST_TOK + (lane & 15);
-        const int mypos = (t < L) ? route_token<RK>(p.g, k, t) : -2;
-        if (lane < 16) st.pos[lane] = mypos;
-        if (F32) {
-            // u, Delta, z: 16 steps x 32 bytes; lane -> (step lane>>1, 4-channel half lane&1)
-            const int j = lane >> 1, hf = lane & 1;
-            const int pj = __shfl_sync(FULL_MASK, mypos, j);
-            const bool ok = pj >= 0 && (c0 + 4 * hf) < D;
-            const long long off = (long long)(ok ? pj : 0) * D + 4 * hf;
-            cp_async16(&st.u[j][4 * hf], u_base + off, ok);
-            cp_async16(&st.d[j][4 * hf], d_base + off, ok);
-            if (z_base) cp_async16(&st.z[j][4 * hf], z_base + off, ok);
-        } else {
-            // 16 steps x 16 bytes: lanes 0-15 take u (and z), lanes 16-31 take Delta
-            const int j = lane & 15;
-            const int pj = __shfl_sync(FULL_MASK, mypos, j);
-            const bool ok = pj >= 0;
-            const long long off = (long long)(ok ? pj : 0) * D;
-            if (lane < 16) {
-                cp_async16(&st.u[j][0], u_base + off, ok);
-                if (z_base) cp_async16(&st.z[j][0], z_base + off, ok);
-            } else {
-                cp_async16(&st.d[j][0], d_base + off, ok);
-            }
-        }
-        if (N16) {
-            if (F32) {
-                // 16 steps x 4 quads x 16 bytes per tensor: f = lane + 32i -> (step f>>2, quad f&3)
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int f = lane + 32 * i;
-                    const int pj = __shfl_sync(FULL_MASK, mypos, f >> 2);
-                    const bool ok = pj >= 0;
-                    const long long off = (long long)(ok ? pj : 0) * 16 + 4 * (f & 3);
-                    cp_async16(&st.B[f >> 2][4 * (f & 3)], B_base + off, ok);
-                    cp_async16(&st.C[f >> 2][4 * (f & 3)], C_base + off, ok);
-                }
-            } else {
-                // 16 steps x 2 halves x 16 bytes: lane -> (step lane>>1, half lane&1)
-                const int j = lane >> 1, hf = lane & 1;
-                const int pj = __shfl_sync(FULL_MASK, mypos, j);
-                const bool ok = pj >= 0;
-                const long long off = (long long)(ok ? pj : 0) * 16 + 8 * hf;
-                cp_async16(&st.B[j][8 * hf], B_base + off, ok);
-                cp_async16(&st.C[j][8 * hf], C_base + off, ok);
-            }
-        } else {
-            // Any N <= 16: element loads (the 16-byte path needs 16-float rows).
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int e = lane + 32 * i;
-                const int n = e & 15, j = e >> 4;
-                const int pj = __shfl_sync(FULL_MASK, mypos, j);
-                T vb = T(0.f), vc = T(0.f);
-                if (pj >= 0 && n < N) {
-                    vb = B_base[(long long)pj * N + n];
-                    vc = C_base[(long long)pj * N + n];
-                }
-                st.B[j][n] = vb;
-                st.C[j][n] = vc;
-            }
-        }
-        cp_async_commit();
-    };
-
-    // Discretize a landed raw stage into the prep buffers (once per step and channel).
-    auto prepare = [&](const RawStage<T>& st) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int j = (lane >> 3) + 4 * i;
-            const int pj = st.pos[j];
-            float uu = to_float(st.u[j][ce]);
-            const float x = to_float(st.d[j][ce]) + bias_e;
-            float dsp = p.softplus ? softplus_f(x) : x;
-            if (pj == -2 || !evalid) {  // past the end: a no-op step
-                dsp = 0.f;
-                uu = 0.f;
-            }
-            pr.dsp[j][ce] = dsp;
-            pr.du[j][ce] = dsp * uu;
-            pr.uu[j][ce] = uu;
-        }
-        // B and C to float32: 16 steps x 16 states each, lane -> 8 values per tensor
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int f = lane + 32 * i;  // (step f>>2, quad f&3)
-            const int j = f >> 2, q = f & 3;
-            pr.B[j][q] = make_float4(to_float(st.B[j][4 * q]), to_float(st.B[j][4 * q + 1]),
-                                     to_float(st.B[j][4 * q + 2]), to_float(st.B[j][4 * q + 3]));
-            pr.C[j][q] = make_float4(to_float(st.C[j][4 * q]), to_float(st.C[j][4 * q + 1]),
-                                     to_float(st.C[j][4 * q + 2]), to_float(st.C[j][4 * q + 3]));
-        }
-    };
-
-    float h[4] = {0.f, 0.f, 0.f, 0.f};
     const int nchunks = (L + ST_TOK - 1) / ST_TOK;
+    const int last_tau = nchunks + (PARK ? 1 : 0);
+    const long long img = (long long)b * tokens;
 
+    if (warp < KC) {
+        // =============================== consumer =================================
+        const int kl = warp;
+        const int k = p.k_base + blockIdx.z * KC + kl;
+        const int cc = lane >> 2, grp = lane & 3;
+        const int d = c0 + cc;
+        const bool dvalid = d < D;
+        float a2[4];
 #pragma unroll
-    for (int s = 0; s < NSTAGE - 1; ++s) {
-        if (s < nchunks) issue(s, s);
-        else cp_async_commit();
-    }
-
-    for (int chunk = 0; chunk < nchunks; ++chunk) {
-        const int ahead = chunk + NSTAGE - 1;
-        if (ahead < nchunks) issue(ahead, ahead % NSTAGE);
-        else cp_async_commit();
-        cp_async_wait<NSTAGE - 1>();
-        __syncwarp();
-        const RawStage<T>& st = sm.raw[chunk % NSTAGE];
-        prepare(st);
-        __syncwarp();
-
-        // ---- recurrence over the 16 steps ----------------------------------------
-        float yv[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float yp[4];
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int j = 4 * q + jj;
-                const float dsp = pr.dsp[j][cc];
-                const float du = pr.du[j][cc];
-                const float4 Bv = pr.B[j][grp];
-                const float4 Cv = pr.C[j][grp];
-                const float e0 = fast_exp2(dsp * a2[0]);
-                const float e1 = fast_exp2(dsp * a2[1]);
-                const float e2 = fast_exp2(dsp * a2[2]);
-                const float e3 = fast_exp2(dsp * a2[3]);
-                h[0] = fmaf(e0, h[0], du * Bv.x);
-                h[1] = fmaf(e1, h[1], du * Bv.y);
-                h[2] = fmaf(e2, h[2], du * Bv.z);
-                h[3] = fmaf(e3, h[3], du * Bv.w);
-                float acc = Cv.x * h[0];
-                acc = fmaf(Cv.y, h[1], acc);
-                acc = fmaf(Cv.z, h[2], acc);
-                acc = fmaf(Cv.w, h[3], acc);
-                yp[jj] = acc;
-            }
-            // Reduce-scatter over the 4 state-group lanes: lane grp keeps step 4q+grp.
-            const bool hi = grp & 2;
-            float a0 = hi ? yp[2] : yp[0];
-            float a1 = hi ? yp[3] : yp[1];
-            const float s0 = hi ? yp[0] : yp[2];
-            const float s1 = hi ? yp[1] : yp[3];
-            a0 += __shfl_xor_sync(FULL_MASK, s0, 2);
-            a1 += __shfl_xor_sync(FULL_MASK, s1, 2);
-            const bool odd = grp & 1;
-            float keep = odd ? a1 : a0;
-            const float send = odd ? a0 : a1;
-            keep += __shfl_xor_sync(FULL_MASK, send, 1);
-            yv[q] = fmaf(Dd, pr.uu[4 * q + grp][cc], keep);
+        for (int s = 0; s < 4; ++s) {
+            const int n = 4 * grp + s;
+            a2[s] = (dvalid && n < N) ? __ldg(p.A + (long long)k * p.a_dir + (long long)d * N + n) * LOG2E : 0.f;
         }
+        const float2 a01 = make_float2(a2[0], a2[1]), a23 = make_float2(a2[2], a2[3]);
+        float2 h01 = make_float2(0.f, 0.f), h23 = h01;
+        __syncthreads();  // prologue: chunk 0 discretized
 
-        // ---- merge, gate and store ------------------------------------------------
-        if (!MERGE) {
+        for (int tau = 0; tau <= last_tau; ++tau) {
+            if (tau < nchunks) {
+                const auto& pr = sm.prep[kl][tau & 1];
+                const BCStage<T>& bcs = sm.bc[kl][tau % NBC];
+                float* yo = &sm.yout[kl][tau % NY][0][0];
+                float yv[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int j = 4 * q + grp;
-                const int pj = st.pos[j];
-                if (pj >= 0 && dvalid) {
-                    float o = yv[q] * p.merge_scale;
-                    if (z_base) o *= silu_f(to_float(st.z[j][cc]));
-                    store_elem<T>(y_base + (long long)pj * D + d, o);
-                }
-            }
-        } else {
-            bool mine[4];
+                for (int q = 0; q < 4; ++q) {
+                    float yp[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int pj = st.pos[4 * q + grp];
-                mine[q] = false;
-                if (pj >= 0 && dvalid) {
-                    if (finalizer<RK>(p.g, pj) == k) {
-                        mine[q] = true;
-                    } else {
-                        p.scratch[(((long long)k * p.batch + b) * tokens + pj) * D + d] = yv[q];
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = 4 * q + jj;
+                        const float2 dd = pr.dd[j][cc];
+                        float4 Bv, Cv;
+                        if constexpr (F32) {
+                            Bv = *reinterpret_cast<const float4*>(&bcs.B[j][4 * grp]);
+                            Cv = *reinterpret_cast<const float4*>(&bcs.C[j][4 * grp]);
+                        } else {
+                            Bv = pr.B[j][grp];
+                            Cv = pr.C[j][grp];
+                        }
+                        const float2 dsp2 = make_float2(dd.x, dd.x);
+                        const float2 du2 = make_float2(dd.y, dd.y);
+                        const float2 x01 = __fmul2_rn(dsp2, a01);
+                        const float2 x23 = __fmul2_rn(dsp2, a23);
+                        const float2 e01 = make_float2(fast_exp2(x01.x), fast_exp2(x01.y));
+                        const float2 e23 = make_float2(fast_exp2(x23.x), fast_exp2(x23.y));
+                        h01 = __ffma2_rn(e01, h01, __fmul2_rn(du2, make_float2(Bv.x, Bv.y)));
+                        h23 = __ffma2_rn(e23, h23, __fmul2_rn(du2, make_float2(Bv.z, Bv.w)));
+                        float2 acc = __fmul2_rn(make_float2(Cv.x, Cv.y), h01);
+                        acc = __ffma2_rn(make_float2(Cv.z, Cv.w), h23, acc);
+                        yp[jj] = acc.x + acc.y;
                     }
+                    // Reduce-scatter over the 4 state-group lanes: lane grp keeps step 4q+grp.
+                    const bool hi = grp & 2;
+                    float x0 = hi ? yp[2] : yp[0];
+                    float x1 = hi ? yp[3] : yp[1];
+                    const float s0 = hi ? yp[0] : yp[2];
+                    const float s1 = hi ? yp[1] : yp[3];
+                    x0 += __shfl_xor_sync(FULL_MASK, s0, 2);
+                    x1 += __shfl_xor_sync(FULL_MASK, s1, 2);
+                    const bool odd = grp & 1;
+                    float keep = odd ? x1 : x0;
+                    const float send = odd ? x0 : x1;
+                    keep += __shfl_xor_sync(FULL_MASK, send, 1);
+                    yv[q] = keep;
                 }
+                // stores after every load of the chunk, so none of them waits on a store
+#pragma unroll
+                for (int q = 0; q < 4; ++q) yo[(4 * q + grp) * ST_CH + cc] = yv[q];
             }
             __syncthreads();
+        }
+        return;
+    }
+
+    // ================================= producer ===================================
+    const int kl = warp - KC;
+    const int k = p.k_base + blockIdx.z * KC + kl;  // direction this producer serves
+    const int ce = lane & 7;  // channel of the tile this lane discretizes / stores
+    const int dch = c0 + ce;
+    const bool evalid = dch < D;
+    const float bias_k = (evalid && p.bias) ? __ldg(p.bias + k * p.v_dir + dch) : 0.f;
+    const float Dk = (evalid && p.Dskip) ? __ldg(p.Dskip + k * p.v_dir + dch) : 0.f;
+    const T* z_base = p.z ? static_cast<const T*>(p.z) + img * D + c0 : nullptr;
+    T* y_base = static_cast<T*>(p.y) + img * D + dch;  // + token * D (fits in int32)
+    // parked contributions of direction kk for this image and channel: + token * D
+    auto park = [&](int kk) { return p.scratch + ((long long)kk * p.batch + b) * tokens * D + dch; };
+
+    // Gather chunk `chunk` into token slot chunk % NR and B/C slot chunk % NBC.
+    auto issue = [&](int chunk) {
+        if (chunk < nchunks) {
+            auto& st = sm.tok[kl][chunk % NR];
+            BCStage<T>& sb = sm.bc[kl][chunk % NBC];
+            const T* u_base = static_cast<const T*>(p.u) + k * p.in_dir + img * D + c0;
+            const T* d_base = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + c0;
+            const T* B_base = static_cast<const T*>(p.B) + k * p.bc_dir + img * N;
+            const T* C_base = static_cast<const T*>(p.C) + k * p.bc_dir + img * N;
+            const int t = chunk * ST_TOK + (lane & 15);
+            const int mypos = (t < L) ? route_token<RK>(p.g, k, t) : -2;
+            if (lane < 16) {
+                st.pos[lane] = mypos;
+                if constexpr (PARK) st.fin[lane] = (mypos >= 0 && finalizer<RK>(p.g, mypos) == k) ? 1 : 0;
+            }
+            if (F32) {
+                // u, Delta, z: 16 steps x 32 bytes; lane -> (step lane>>1, 4-channel half lane&1)
+                const int j = lane >> 1, hf = lane & 1;
+                const int pj = __shfl_sync(FULL_MASK, mypos, j);
+                const bool ok = pj >= 0 && (c0 + 4 * hf) < D;
+                const long long off = (long long)(ok ? pj : 0) * D + 4 * hf;
+                cp_async16(&st.u[j][4 * hf], u_base + off, ok);
+                cp_async16(&st.d[j][4 * hf], d_base + off, ok);
+                if (z_base) cp_async16(&st.z[j][4 * hf], z_base + off, ok);
+            } else {
+                // 16 steps x 16 bytes: lanes 0-15 take u and z, lanes 16-31 take Delta
+                const int j = lane & 15;
+                const int pj = __shfl_sync(FULL_MASK, mypos, j);
+                const bool ok = pj >= 0;
+                const long long off = (long long)(ok ? pj : 0) * D;
+                if (lane < 16) {
+                    cp_async16(&st.u[j][0], u_base + off, ok);
+                    if (z_base) cp_async16(&st.z[j][0], z_base + off, ok);
+                } else {
+                    cp_async16(&st.d[j][0], d_base + off, ok);
+                }
+            }
+            if (N16) {
+                if (F32) {
+                    // 16 steps x 4 quads x 16 bytes per tensor: f = lane + 32i -> (step f>>2, quad f&3)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if (mine[q]) {
-                    const int j = 4 * q + grp;
-                    const int pj = st.pos[j];
-                    float acc = yv[q];
-#pragma unroll
-                    for (int kk = 0; kk < K; ++kk) {
-                        if (kk == k) continue;
-                        acc += p.scratch[(((long long)kk * p.batch + b) * tokens + pj) * D + d];
+                    for (int i = 0; i < 2; ++i) {
+                        const int f = lane + 32 * i;
+                        const int pj = __shfl_sync(FULL_MASK, mypos, f >> 2);
+                        const bool ok = pj >= 0;
+                        const long long off = (long long)(ok ? pj : 0) * 16 + 4 * (f & 3);
+                        cp_async16(&sb.B[f >> 2][4 * (f & 3)], B_base + off, ok);
+                        cp_async16(&sb.C[f >> 2][4 * (f & 3)], C_base + off, ok);
                     }
-                    float o = acc * p.merge_scale;
-                    if (z_base) o *= silu_f(to_float(st.z[j][cc]));
-                    store_elem<T>(y_base + (long long)pj * D + d, o);
+                } else {
+                    // 16 steps x 2 halves x 16 bytes: lane -> (step lane>>1, half lane&1)
+                    const int j = lane >> 1, hf = lane & 1;
+                    const int pj = __shfl_sync(FULL_MASK, mypos, j);
+                    const bool ok = pj >= 0;
+                    const long long off = (long long)(ok ? pj : 0) * 16 + 8 * hf;
+                    cp_async16(&sb.B[j][8 * hf], B_base + off, ok);
+                    cp_async16(&sb.C[j][8 * hf], C_base + off, ok);
+                }
+            } else {
+                // Any N <= 16: element loads (the 16-byte path needs rows of 16 states).
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int e = lane + 32 * i;
+                    const int n = e & 15, j = e >> 4;
+                    const int pj = __shfl_sync(FULL_MASK, mypos, j);
+                    T vb = T(0.f), vc = T(0.f);
+                    if (pj >= 0 && n < N) {
+                        vb = B_base[(long long)pj * N + n];
+                        vc = C_base[(long long)pj * N + n];
+                    }
+                    sb.B[j][n] = vb;
+                    sb.C[j][n] = vc;
                 }
             }
         }
-        __syncwarp();
+        cp_async_commit();  // one group per chunk, possibly empty
+    };
+
+    // Discretize chunk c: once per (step, channel); loads first, then math, then stores.
+    auto prepare = [&](int c) {
+        const auto& st = sm.tok[kl][c % NR];
+        auto& pr = sm.prep[kl][c & 1];
+        float xd[4], xu[4];
+        bool live[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int j = (lane >> 3) + 4 * r;
+            xd[r] = to_float(st.d[j][ce]);
+            xu[r] = to_float(st.u[j][ce]);
+            live[r] = st.pos[j] != -2 && evalid;  // past the end: a no-op step
+        }
+        float4 cb[2], cv[2];
+        if constexpr (!F32) {
+            const BCStage<T>& sb = sm.bc[kl][c % NBC];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int f = lane + 32 * r;  // (step f>>2, quad f&3)
+                const int j = f >> 2, q = f & 3;
+                cb[r] = make_float4(to_float(sb.B[j][4 * q]), to_float(sb.B[j][4 * q + 1]),
+                                    to_float(sb.B[j][4 * q + 2]), to_float(sb.B[j][4 * q + 3]));
+                cv[r] = make_float4(to_float(sb.C[j][4 * q]), to_float(sb.C[j][4 * q + 1]),
+                                    to_float(sb.C[j][4 * q + 2]), to_float(sb.C[j][4 * q + 3]));
+            }
+        }
+        float2 out[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const float x = xd[r] + bias_k;
+            const float dsp = live[r] ? (p.softplus ? softplus_f(x) : x) : 0.f;
+            out[r] = make_float2(dsp, live[r] ? dsp * xu[r] : 0.f);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) pr.dd[(lane >> 3) + 4 * r][ce] = out[r];
+        if constexpr (!F32) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int f = lane + 32 * r;
+                pr.B[f >> 2][f & 3] = cb[r];
+                pr.C[f >> 2][f & 3] = cv[r];
+            }
+        }
+    };
+
+    // Epilogue of chunk c: add the skip term, then store (one owner) or park / keep.
+    auto finish_a = [&](int c) {
+        const auto& st = sm.tok[kl][c % NR];
+        float* yo = &sm.yout[kl][c % NY][0][0];
+        int pj[4], fin[4];
+        float yk[4], zz[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int j = (lane >> 3) + 4 * r;
+            pj[r] = evalid ? st.pos[j] : -1;
+            fin[r] = PARK ? st.fin[j] : 1;
+            yk[r] = fmaf(Dk, to_float(st.u[j][ce]), yo[j * ST_CH + ce]);
+            zz[r] = z_base ? to_float(st.z[j][ce]) : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int j = (lane >> 3) + 4 * r;
+            if (pj[r] < 0) continue;
+            if constexpr (MODE == MODE_OWNER) {
+                float o = yk[r] * p.merge_scale;
+                if (z_base) o *= silu_f(zz[r]);
+                store_elem<T>(y_base + pj[r] * D, o);
+            } else if (fin[r]) {
+                yo[j * ST_CH + ce] = yk[r];
+            } else {
+                park(k)[pj[r] * D] = yk[r];
+            }
+        }
+    };
+
+    // MODE_PARK, second half (chunk c, one barrier after finish_a): the finalizer
+    // adds the parked contributions, scales, gates and stores. The parked values
+    // are loaded at the top of the iteration (fetch_b) and used at its end.
+    float parked[4];
+    auto fetch_b = [&](int c) {
+        const auto& st = sm.tok[kl][c % NR];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int j = (lane >> 3) + 4 * r;
+            const int pj = st.pos[j];
+            float acc = 0.f;
+            if (evalid && pj >= 0 && st.fin[j]) {
+#pragma unroll
+                for (int kk = 0; kk < KR; ++kk) {
+                    if (kk == k) continue;
+                    acc += park(kk)[pj * D];
+                }
+            }
+            parked[r] = acc;
+        }
+    };
+    auto finish_b = [&](int c) {
+        const auto& st = sm.tok[kl][c % NR];
+        const float* yo = &sm.yout[kl][c % NY][0][0];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int j = (lane >> 3) + 4 * r;
+            const int pj = st.pos[j];
+            if (!evalid || pj < 0 || !st.fin[j]) continue;
+            float o = (yo[j * ST_CH + ce] + parked[r]) * p.merge_scale;
+            if (z_base) o *= silu_f(to_float(st.z[j][ce]));
+            store_elem<T>(y_base + pj * D, o);
+        }
+    };
+
+    // Prologue: gathers for chunks 0..LOOK in flight, chunk 0 discretized.
+#pragma unroll
+    for (int c = 0; c <= ST_LOOK; ++c) issue(c);
+    cp_async_wait<ST_LOOK>();
+    __syncwarp();
+    if (nchunks > 0) prepare(0);
+    __syncthreads();
+
+    for (int tau = 0; tau <= last_tau; ++tau) {
+        const bool do_b = PARK && tau >= 2 && tau - 2 < nchunks;
+        if (do_b) fetch_b(tau - 2);
+        issue(tau + 1 + ST_LOOK);
+        if (tau + 1 < nchunks) {
+            cp_async_wait<ST_LOOK>();  // chunk tau+1 has landed (this lane's copies)
+            __syncwarp();              // ... and every lane's
+            prepare(tau + 1);
+        }
+        if (tau >= 1 && tau - 1 < nchunks) finish_a(tau - 1);
+        if (do_b) finish_b(tau - 2);
+        __syncthreads();
     }
     cp_async_wait<0>();
 }
