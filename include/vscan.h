@@ -195,6 +195,34 @@ vscan_status vscan_plan_info(const vscan_route* route, const vscan_args* args, i
 vscan_status vscan_forward(const vscan_route* route, const vscan_args* args, void* stream);
 
 /*
+ * Pooled-route forward pass that allocates nothing and needs no workspace.
+ * (An addition of this library; the pages have no counterpart.)
+ *
+ * For callers that cannot allocate device memory: a plugin whose host runtime
+ * owns all device memory, or a latency-bound loop that must not call
+ * cudaMalloc (which can synchronize the device and fail under memory pressure).
+ * The only scratch of the pooled routes, the pooled B and C, is placed in a
+ * fixed 4 MiB array inside the library instead of the caller's workspace; the
+ * caller still passes every input and the output, as for vscan_forward, and
+ * args->workspace is ignored.
+ *   - Routes: VSCAN_ROUTE_POOL_W and VSCAN_ROUTE_POOL_H only (else
+ *     VSCAN_ERR_UNSUPPORTED).
+ *   - Limit: 2 * Ki * batch * pooled_length * d_state * 4 bytes must not
+ *     exceed 4 MiB (e.g. batch 32, length 128, N 16 uses 512 KiB); larger
+ *     calls return VSCAN_ERR_UNSUPPORTED with the sizes in vscan_last_error().
+ *   - Every GPU that loads the library holds the 4 MiB until the process exits.
+ *   - The first call on a device, with that device current, resolves the
+ *     array's device address (cudaGetSymbolAddress) and keeps it; make that
+ *     first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero (every element read is written
+ *     first by the same call), but calls that overlap on the GPU (different
+ *     streams, no ordering between them) race on it: order them.
+ * Errors and the other conventions are those of vscan_forward.
+ */
+vscan_status vscan_forward_pooled_noalloc(const vscan_route* route, const vscan_args* args, void* stream);
+
+/*
  * Bytes of device memory vscan_forward_host needs in its device_buffer for
  * these arguments (host only): device copies of every input and of y, plus
  * the workspace, each rounded up to 256 bytes.

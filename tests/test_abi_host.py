@@ -151,6 +151,17 @@ def test_chunked_scan_needs_the_tile_on_chip():
     assert abi.lib.vscan_forward(small.handle, ctypes.byref(_args(seq_chunks=4)), None) == -1
 
 
+def test_noalloc_pooled_forward_rejects_before_any_cuda_call():
+    fake = dict(u=0x1000, delta=0x2000, B=0x3000, C=0x4000, y=0x5000, A=0x6000)
+    r = vs.Route("cross4", 8, 8)  # not a pooled route
+    assert abi.lib.vscan_forward_pooled_noalloc(r.handle, ctypes.byref(_args(**fake)), None) == -4
+    # 2 planes x 256 images x 256 pooled steps x 16 states x 4 bytes = 8 MiB > 4 MiB
+    big = vs.Route("pool_w", 256, 2)
+    a = _args(**fake, batch=256)
+    assert abi.lib.vscan_forward_pooled_noalloc(big.handle, ctypes.byref(a), None) == -4
+    assert "fixed scratch" in abi.lib.vscan_last_error().decode()
+
+
 def test_pooled_route_length_limit():
     r = vs.Route("pool_w", 4000, 2)
     assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args()), None) == -4

@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "vscan.h"
@@ -328,6 +329,36 @@ HostLayout host_layout(const vscan_route* r, const vscan_args* a)
     return L;
 }
 
+// ---- fixed scratch for vscan_forward_pooled_noalloc ---------------------------------
+// The pooled routes need scratch only for the pooled B and C
+// (2 x Ki x batch x L x N floats). This array holds it for callers that cannot
+// allocate device memory; every GPU that loads the library keeps it until exit.
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch, resolved once per device: in host code the
+// symbol is only a host-side stand-in and must never be passed to a kernel.
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mutex;
+void* g_static_addr[kMaxDevices] = {};
+
+vscan_status static_scratch_address(void** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(VSCAN_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(g_static_mutex);
+    if (!g_static_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the fixed scratch");
+        g_static_addr[dev] = p;
+    }
+    *out = g_static_addr[dev];
+    return VSCAN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -483,6 +514,30 @@ vscan_status vscan_forward_host(const vscan_route* r, const vscan_args* ha, void
     cudaError_t e = cudaMemcpyAsync(ha->y, da.y, plane * ha->channels * eb, cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
     return VSCAN_OK;
+}
+
+vscan_status vscan_forward_pooled_noalloc(const vscan_route* r, const vscan_args* a, void* stream)
+{
+    vscan_status st = check_shape(r, a);
+    if (st != VSCAN_OK) return st;
+    st = check_pointers(a, true);
+    if (st != VSCAN_OK) return st;
+    if (!is_pool(r->g.kind))
+        return fail(VSCAN_ERR_UNSUPPORTED, "vscan_forward_pooled_noalloc takes POOL_W or POOL_H routes only");
+    const uint64_t need = workspace_need(r, a);
+    if (need > kStaticScratchBytes)
+        return fail(VSCAN_ERR_UNSUPPORTED,
+                    "pooled B/C need %llu bytes of scratch; the fixed scratch holds %llu "
+                    "(2 x planes x batch x pooled length x d_state floats)",
+                    (unsigned long long)need, (unsigned long long)kStaticScratchBytes);
+    if (a->batch == 0) return VSCAN_OK;
+    void* scratch = nullptr;
+    st = static_scratch_address(&scratch);
+    if (st != VSCAN_OK) return st;
+    vscan_args b = *a;
+    b.workspace = scratch;
+    b.workspace_bytes = kStaticScratchBytes;
+    return forward_device(r, &b, static_cast<cudaStream_t>(stream));
 }
 
 const char* vscan_last_error(void) { return g_last_error.c_str(); }
