@@ -185,6 +185,16 @@ vscan_status vscan_workspace_size(const vscan_route* route, const vscan_args* ar
 vscan_status vscan_plan_info(const vscan_route* route, const vscan_args* args, int32_t* kernels);
 
 /*
+ * Name of the kernel that runs the scan for these arguments (host only), as
+ * a static NUL-terminated string owned by the library: "stream_scan_kernel<R>"
+ * (streaming scan), "resident_scan_kernel<R>" (chunked parallel scan of a
+ * shared-memory-resident tile; R = BIDIR, CROSS4 or ATROUS2), "pool_scan_kernel"
+ * (pooled routes) or "none" (empty batch). Same argument checks and errors
+ * as vscan_plan_info; *name is untouched on error.
+ */
+vscan_status vscan_plan_kernel(const vscan_route* route, const vscan_args* args, const char** name);
+
+/*
  * Run the fused routed scan on the device. Enqueued on stream; allocates
  * nothing; never synchronizes. The output y is fully overwritten. Concurrent
  * calls on different streams must use different workspaces.

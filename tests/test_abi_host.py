@@ -143,6 +143,28 @@ def test_plan_info_counts_launches():
     assert abi.lib.vscan_plan_info(r.handle, ctypes.byref(_args(batch=0)), ctypes.byref(n)) == 0 and n.value == 0
 
 
+def test_plan_kernel_names_the_scan_kernel():
+    name = ctypes.c_char_p()
+    for kind, h, w, cls, batch, D, chunks, expect in (
+            ("atrous2", 56, 56, -1, 8, 192, 0, "stream_scan_kernel<ATROUS2>"),
+            ("cross4", 56, 56, -1, 16, 192, 0, "stream_scan_kernel<CROSS4>"),
+            ("bidir", 64, 64, 2048, 64, 768, 0, "stream_scan_kernel<BIDIR>"),
+            ("bidir", 14, 14, 98, 1, 384, 0, "resident_scan_kernel<BIDIR>"),  # few sequences
+            ("cross4", 14, 14, -1, 1, 64, 4, "resident_scan_kernel<CROSS4>"),
+            ("atrous2", 9, 13, -1, 1, 64, 2, "resident_scan_kernel<ATROUS2>"),
+            ("atrous2", 9, 13, -1, 1, 64, 1, "stream_scan_kernel<ATROUS2>"),
+            ("pool_w", 8, 8, -1, 2, 64, 0, "pool_scan_kernel"),
+            ("pool_h", 8, 8, -1, 2, 64, 0, "pool_scan_kernel"),
+            ("atrous2", 4, 4, -1, 0, 64, 0, "none")):
+        r = vs.Route(kind, h, w, cls)
+        a = _args(batch=batch, channels=D, seq_chunks=chunks)
+        assert abi.lib.vscan_plan_kernel(r.handle, ctypes.byref(a), ctypes.byref(name)) == 0
+        assert name.value.decode() == expect, (kind, h, w, batch, chunks)
+    r = vs.Route("atrous2", 4, 4)
+    assert abi.lib.vscan_plan_kernel(r.handle, ctypes.byref(_args()), None) == -1
+    assert abi.lib.vscan_plan_kernel(r.handle, ctypes.byref(_args(d_state=0)), ctypes.byref(name)) != 0
+
+
 def test_chunked_scan_needs_the_tile_on_chip():
     big = vs.Route("cross4", 56, 56)
     assert abi.lib.vscan_forward(big.handle, ctypes.byref(_args(seq_chunks=4)), None) == -4

@@ -201,6 +201,18 @@ class Plan:
         """Enqueue the forward pass on a torch.cuda.Stream."""
         check(lib.vscan_forward(self.route.handle, self._ref, ctypes.c_void_p(stream.cuda_stream)))
 
+    def kernels(self):
+        """Number of kernel launches one run() makes (vscan_plan_info)."""
+        n = ctypes.c_int32()
+        check(lib.vscan_plan_info(self.route.handle, self._ref, ctypes.byref(n)))
+        return n.value
+
+    def kernel_name(self):
+        """Name of the kernel that runs the scan (vscan_plan_kernel)."""
+        name = ctypes.c_char_p()
+        check(lib.vscan_plan_kernel(self.route.handle, self._ref, ctypes.byref(name)))
+        return name.value.decode()
+
 
 __all__.append("Plan")
 

@@ -74,6 +74,7 @@ def _load():
         "vscan_workspace_size": ([p, pa, ctypes.POINTER(u64)], i32),
         "vscan_forward": ([p, pa, p], i32),
         "vscan_plan_info": ([p, pa, ctypes.POINTER(i32)], i32),
+        "vscan_plan_kernel": ([p, pa, ctypes.POINTER(ctypes.c_char_p)], i32),
         "vscan_forward_pooled_noalloc": ([p, pa, p], i32),
         "vscan_host_buffer_size": ([p, pa, ctypes.POINTER(u64)], i32),
         "vscan_forward_host": ([p, pa, p, u64, p], i32),

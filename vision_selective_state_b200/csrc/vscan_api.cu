@@ -448,6 +448,23 @@ vscan_status vscan_plan_info(const vscan_route* r, const vscan_args* a, int32_t*
     return VSCAN_OK;
 }
 
+vscan_status vscan_plan_kernel(const vscan_route* r, const vscan_args* a, const char** name)
+{
+    if (!name) return fail(VSCAN_ERR_INVALID_ARGUMENT, "name is NULL");
+    vscan_status st = check_shape(r, a);
+    if (st != VSCAN_OK) return st;
+    static const char* const stream_names[] = {"stream_scan_kernel<BIDIR>", "stream_scan_kernel<CROSS4>",
+                                               "stream_scan_kernel<ATROUS2>"};
+    static const char* const resident_names[] = {"resident_scan_kernel<BIDIR>",
+                                                 "resident_scan_kernel<CROSS4>",
+                                                 "resident_scan_kernel<ATROUS2>"};
+    if (a->batch == 0) *name = "none";
+    else if (is_pool(r->g.kind)) *name = "pool_scan_kernel";
+    else if (choose_chunks(r, a) > 1) *name = resident_names[r->g.kind];
+    else *name = stream_names[r->g.kind];
+    return VSCAN_OK;
+}
+
 vscan_status vscan_host_buffer_size(const vscan_route* r, const vscan_args* a, uint64_t* bytes)
 {
     if (!bytes) return fail(VSCAN_ERR_INVALID_ARGUMENT, "bytes is NULL");
