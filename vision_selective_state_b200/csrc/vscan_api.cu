@@ -142,17 +142,17 @@ uint64_t workspace_need(const vscan_route* r, const vscan_args* a)
     return 0;
 }
 
-template <int RK, typename T, bool N16, int KC, int MODE>
+template <int RK, typename T, bool N16, int KC, int MODE, int PW>
 cudaError_t launch_stream_mode(vscan::ScanParams p, int k_base, int grid_z, cudaStream_t s)
 {
     const size_t smem = vscan::stream_smem_bytes<T, KC, MODE>();
-    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16, KC, MODE>,
+    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     p.k_base = k_base;
     const dim3 grid((p.D + vscan::ST_CH - 1) / vscan::ST_CH, p.batch, grid_z);
-    vscan::stream_scan_kernel<RK, T, N16, KC, MODE>
-        <<<grid, vscan::StreamShape<T, KC, MODE>::THREADS, smem, s>>>(p);
+    vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW>
+        <<<grid, vscan::StreamShape<T, KC, MODE, PW>::THREADS, smem, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -164,12 +164,12 @@ cudaError_t launch_stream_n(const vscan::ScanParams& p, cudaStream_t s)
 {
     using namespace vscan;
     if constexpr (RK == RK_ATROUS2) {
-        if constexpr (sizeof(T) == 4) return launch_stream_mode<RK, T, N16, 1, MODE_OWNER>(p, 0, 4, s);
-        else return launch_stream_mode<RK, T, N16, 4, MODE_OWNER>(p, 0, 1, s);
+        if constexpr (sizeof(T) == 4) return launch_stream_mode<RK, T, N16, 1, MODE_OWNER, 1>(p, 0, 4, s);
+        else return launch_stream_mode<RK, T, N16, 4, MODE_OWNER, 1>(p, 0, 1, s);
     } else if constexpr (RK == RK_BIDIR) {
-        return launch_stream_mode<RK, T, N16, 2, MODE_PARK>(p, 0, 1, s);
+        return launch_stream_mode<RK, T, N16, 2, MODE_PARK, 1>(p, 0, 1, s);
     } else {
-        return launch_stream_mode<RK, T, N16, 4, MODE_PARK>(p, 0, 1, s);
+        return launch_stream_mode<RK, T, N16, 4, MODE_PARK, 1>(p, 0, 1, s);
     }
 }
 

@@ -13,8 +13,9 @@
 //         h  = dA * h + (Delta * u) * B      (FMUL + FFMA)
 //         y += C * h                         (FFMA)
 //
-//   producer warp (one per direction) does everything that happens once per
-//     (step, channel): it gathers the route's tokens for chunk tau+1+LOOK with
+//   producer warps (PW per direction, each owning 16/PW steps of every chunk)
+//     do everything that happens once per (step, channel): they gather the
+//     route's tokens for chunk tau+1+LOOK with
 //     cp.async into a shared-memory ring (zero fill for ATROUS2 padding;
 //     channels-last rows make every gathered token one contiguous segment),
 //     discretizes chunk tau+1 (Delta = softplus(raw + bias), Delta*u, B and C
@@ -114,7 +115,7 @@ struct __align__(16) PrepStage<false> {
     float2 dd[ST_TOK][ST_CH];
 };
 
-template <typename T, int KC, int MODE>
+template <typename T, int KC, int MODE, int PW = 1>
 struct StreamShape {
     static constexpr bool F32 = sizeof(T) == 4;
     static constexpr bool PARK = MODE == MODE_PARK;
@@ -124,7 +125,10 @@ struct StreamShape {
     // B/C slot: until discretized at tau = c-1 (bf16) or consumed at tau = c (f32)
     static constexpr int NBC = ST_LOOK + (F32 ? 2 : 1);
     static constexpr int NY = PARK ? 3 : 2;  // output ring
-    static constexpr int THREADS = 64 * KC;  // a consumer and a producer per direction
+    static constexpr int THREADS = 32 * KC * (1 + PW);  // a consumer and PW producers per direction
+    static constexpr int SPW = ST_TOK / PW;             // steps of a chunk per producer warp
+    static constexpr int RPL = SPW / 4;                 // (step, channel) items per producer lane
+    static_assert(PW == 1 || PW == 2, "one or two producer warps per direction");
 };
 
 template <typename T, int KC, int MODE>
@@ -156,10 +160,11 @@ __device__ __forceinline__ int finalizer(const RouteGeom& g, int p)
     return best_k;
 }
 
-template <int RK, typename T, bool N16, int KC, int MODE>
-__global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan_kernel(const ScanParams p)
+template <int RK, typename T, bool N16, int KC, int MODE, int PW>
+__global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_scan_kernel(const ScanParams p)
 {
-    using S = StreamShape<T, KC, MODE>;
+    using S = StreamShape<T, KC, MODE, PW>;
+    constexpr int SPW = S::SPW, RPL = S::RPL;
     constexpr int NR = S::NR, NBC = S::NBC, NY = S::NY;
     constexpr bool PARK = S::PARK;
     constexpr bool F32 = S::F32;
@@ -198,6 +203,32 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan
                 const auto& pr = sm.prep[kl][tau & 1];
                 const BCStage<T>& bcs = sm.bc[kl][tau % NBC];
                 float* yo = &sm.yout[kl][tau % NY][0][0];
+                // Software pipeline over the chunk's 16 steps: the loads, the SFU
+                // exponentials and the input terms of step j + 2 are issued before
+                // the state update of step j, which is the only serial dependency.
+                float2 e01[ST_TOK], e23[ST_TOK], w01[ST_TOK], w23[ST_TOK];
+                float4 cq[ST_TOK];
+                auto front = [&](int j) {
+                    const float2 dd = pr.dd[j][cc];
+                    float4 Bv;
+                    if constexpr (F32) {
+                        Bv = *reinterpret_cast<const float4*>(&bcs.B[j][4 * grp]);
+                        cq[j] = *reinterpret_cast<const float4*>(&bcs.C[j][4 * grp]);
+                    } else {
+                        Bv = pr.B[j][grp];
+                        cq[j] = pr.C[j][grp];
+                    }
+                    const float2 dsp2 = make_float2(dd.x, dd.x);
+                    const float2 du2 = make_float2(dd.y, dd.y);
+                    const float2 x01 = __fmul2_rn(dsp2, a01);
+                    const float2 x23 = __fmul2_rn(dsp2, a23);
+                    e01[j] = make_float2(fast_exp2(x01.x), fast_exp2(x01.y));
+                    e23[j] = make_float2(fast_exp2(x23.x), fast_exp2(x23.y));
+                    w01[j] = __fmul2_rn(du2, make_float2(Bv.x, Bv.y));
+                    w23[j] = __fmul2_rn(du2, make_float2(Bv.z, Bv.w));
+                };
+                front(0);
+                front(1);
                 float yv[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -205,25 +236,11 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                         const int j = 4 * q + jj;
-                        const float2 dd = pr.dd[j][cc];
-                        float4 Bv, Cv;
-                        if constexpr (F32) {
-                            Bv = *reinterpret_cast<const float4*>(&bcs.B[j][4 * grp]);
-                            Cv = *reinterpret_cast<const float4*>(&bcs.C[j][4 * grp]);
-                        } else {
-                            Bv = pr.B[j][grp];
-                            Cv = pr.C[j][grp];
-                        }
-                        const float2 dsp2 = make_float2(dd.x, dd.x);
-                        const float2 du2 = make_float2(dd.y, dd.y);
-                        const float2 x01 = __fmul2_rn(dsp2, a01);
-                        const float2 x23 = __fmul2_rn(dsp2, a23);
-                        const float2 e01 = make_float2(fast_exp2(x01.x), fast_exp2(x01.y));
-                        const float2 e23 = make_float2(fast_exp2(x23.x), fast_exp2(x23.y));
-                        h01 = __ffma2_rn(e01, h01, __fmul2_rn(du2, make_float2(Bv.x, Bv.y)));
-                        h23 = __ffma2_rn(e23, h23, __fmul2_rn(du2, make_float2(Bv.z, Bv.w)));
-                        float2 acc = __fmul2_rn(make_float2(Cv.x, Cv.y), h01);
-                        acc = __ffma2_rn(make_float2(Cv.z, Cv.w), h23, acc);
+                        if (j + 2 < ST_TOK) front(j + 2);
+                        h01 = __ffma2_rn(e01[j], h01, w01[j]);
+                        h23 = __ffma2_rn(e23[j], h23, w23[j]);
+                        float2 acc = __fmul2_rn(make_float2(cq[j].x, cq[j].y), h01);
+                        acc = __ffma2_rn(make_float2(cq[j].z, cq[j].w), h23, acc);
                         yp[jj] = acc.x + acc.y;
                     }
                     // Reduce-scatter over the 4 state-group lanes: lane grp keeps step 4q+grp.
@@ -250,7 +267,8 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan
     }
 
     // ================================= producer ===================================
-    const int kl = warp - KC;
+    const int kl = (warp - KC) / PW;
+    const int j0 = ((warp - KC) % PW) * SPW;        // first step of a chunk this warp owns
     const int k = p.k_base + blockIdx.z * KC + kl;  // direction this producer serves
     const int ce = lane & 7;  // channel of the tile this lane discretizes / stores
     const int dch = c0 + ce;
@@ -262,7 +280,8 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan
     // parked contributions of direction kk for this image and channel: + token * D
     auto park = [&](int kk) { return p.scratch + ((long long)kk * p.batch + b) * tokens * D + dch; };
 
-    // Gather chunk `chunk` into token slot chunk % NR and B/C slot chunk % NBC.
+    // Gather this warp's steps of chunk `chunk` into token slot chunk % NR and
+    // B/C slot chunk % NBC.
     auto issue = [&](int chunk) {
         if (chunk < nchunks) {
             auto& st = sm.tok[kl][chunk % NR];
@@ -271,13 +290,14 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan
             const T* d_base = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + c0;
             const T* B_base = static_cast<const T*>(p.B) + k * p.bc_dir + img * N;
             const T* C_base = static_cast<const T*>(p.C) + k * p.bc_dir + img * N;
-            const int t = chunk * ST_TOK + (lane & 15);
+            // lane i < SPW computes the route position of step j0 + i
+            const int t = chunk * ST_TOK + j0 + (lane & (SPW - 1));
             const int mypos = (t < L) ? route_token<RK>(p.g, k, t) : -2;
-            if (lane < 16) {
-                st.pos[lane] = mypos;
-                if constexpr (PARK) st.fin[lane] = (mypos >= 0 && finalizer<RK>(p.g, mypos) == k) ? 1 : 0;
+            if (lane < SPW) {
+                st.pos[j0 + lane] = mypos;
+                if constexpr (PARK) st.fin[j0 + lane] = (mypos >= 0 && finalizer<RK>(p.g, mypos) == k) ? 1 : 0;
             }
-            if (F32) {
+            if (F32 && PW == 1) {
                 // u, Delta, z: 16 steps x 32 bytes; lane -> (step lane>>1, 4-channel half lane&1)
                 const int j = lane >> 1, hf = lane & 1;
                 const int pj = __shfl_sync(FULL_MASK, mypos, j);
@@ -286,32 +306,53 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan
                 cp_async16(&st.u[j][4 * hf], u_base + off, ok);
                 cp_async16(&st.d[j][4 * hf], d_base + off, ok);
                 if (z_base) cp_async16(&st.z[j][4 * hf], z_base + off, ok);
+            } else if (F32) {
+                // 8 steps x 32 bytes per tensor: lanes 0-15 take u and z, lanes 16-31 take Delta;
+                // lane -> (step (lane&15)>>1, 4-channel half lane&1)
+                const int i = (lane & 15) >> 1, hf = lane & 1, j = j0 + i;
+                const int pj = __shfl_sync(FULL_MASK, mypos, i);
+                const bool ok = pj >= 0 && (c0 + 4 * hf) < D;
+                const long long off = (long long)(ok ? pj : 0) * D + 4 * hf;
+                if (lane < 16) {
+                    cp_async16(&st.u[j][4 * hf], u_base + off, ok);
+                    if (z_base) cp_async16(&st.z[j][4 * hf], z_base + off, ok);
+                } else {
+                    cp_async16(&st.d[j][4 * hf], d_base + off, ok);
+                }
             } else {
-                // 16 steps x 16 bytes: lanes 0-15 take u and z, lanes 16-31 take Delta
-                const int j = lane & 15;
-                const int pj = __shfl_sync(FULL_MASK, mypos, j);
+                // SPW steps x 16 bytes per tensor: lane -> (tensor lane / SPW, step lane % SPW)
+                const int i = lane & (SPW - 1), j = j0 + i, which = lane / SPW;
+                const int pj = __shfl_sync(FULL_MASK, mypos, i);
                 const bool ok = pj >= 0;
                 const long long off = (long long)(ok ? pj : 0) * D;
-                if (lane < 16) {
+                if (PW == 1) {
+                    if (lane < 16) {
+                        cp_async16(&st.u[j][0], u_base + off, ok);
+                        if (z_base) cp_async16(&st.z[j][0], z_base + off, ok);
+                    } else {
+                        cp_async16(&st.d[j][0], d_base + off, ok);
+                    }
+                } else if (which == 0) {
                     cp_async16(&st.u[j][0], u_base + off, ok);
-                    if (z_base) cp_async16(&st.z[j][0], z_base + off, ok);
-                } else {
+                } else if (which == 1) {
                     cp_async16(&st.d[j][0], d_base + off, ok);
+                } else if (which == 2 && z_base) {
+                    cp_async16(&st.z[j][0], z_base + off, ok);
                 }
             }
             if (N16) {
                 if (F32) {
-                    // 16 steps x 4 quads x 16 bytes per tensor: f = lane + 32i -> (step f>>2, quad f&3)
+                    // SPW steps x 4 quads x 16 bytes per tensor: f = lane + 32i -> (step f>>2, quad f&3)
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) {
+                    for (int i = 0; i < SPW / 8; ++i) {
                         const int f = lane + 32 * i;
                         const int pj = __shfl_sync(FULL_MASK, mypos, f >> 2);
                         const bool ok = pj >= 0;
                         const long long off = (long long)(ok ? pj : 0) * 16 + 4 * (f & 3);
-                        cp_async16(&sb.B[f >> 2][4 * (f & 3)], B_base + off, ok);
-                        cp_async16(&sb.C[f >> 2][4 * (f & 3)], C_base + off, ok);
+                        cp_async16(&sb.B[j0 + (f >> 2)][4 * (f & 3)], B_base + off, ok);
+                        cp_async16(&sb.C[j0 + (f >> 2)][4 * (f & 3)], C_base + off, ok);
                     }
-                } else {
+                } else if (PW == 1) {
                     // 16 steps x 2 halves x 16 bytes: lane -> (step lane>>1, half lane&1)
                     const int j = lane >> 1, hf = lane & 1;
                     const int pj = __shfl_sync(FULL_MASK, mypos, j);
@@ -319,14 +360,22 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan
                     const long long off = (long long)(ok ? pj : 0) * 16 + 8 * hf;
                     cp_async16(&sb.B[j][8 * hf], B_base + off, ok);
                     cp_async16(&sb.C[j][8 * hf], C_base + off, ok);
+                } else {
+                    // 8 steps x 2 halves x 16 bytes per tensor: lanes 0-15 take B, 16-31 take C
+                    const int i = (lane & 15) >> 1, hf = lane & 1;
+                    const int pj = __shfl_sync(FULL_MASK, mypos, i);
+                    const bool ok = pj >= 0;
+                    const long long off = (long long)(ok ? pj : 0) * 16 + 8 * hf;
+                    if (lane < 16) cp_async16(&sb.B[j0 + i][8 * hf], B_base + off, ok);
+                    else cp_async16(&sb.C[j0 + i][8 * hf], C_base + off, ok);
                 }
             } else {
                 // Any N <= 16: element loads (the 16-byte path needs rows of 16 states).
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
+                for (int i = 0; i < SPW / 2; ++i) {
                     const int e = lane + 32 * i;
-                    const int n = e & 15, j = e >> 4;
-                    const int pj = __shfl_sync(FULL_MASK, mypos, j);
+                    const int n = e & 15, j = j0 + (e >> 4);
+                    const int pj = __shfl_sync(FULL_MASK, mypos, e >> 4);
                     T vb = T(0.f), vc = T(0.f);
                     if (pj >= 0 && n < N) {
                         vb = B_base[(long long)pj * N + n];
@@ -344,43 +393,43 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan
     auto prepare = [&](int c) {
         const auto& st = sm.tok[kl][c % NR];
         auto& pr = sm.prep[kl][c & 1];
-        float xd[4], xu[4];
-        bool live[4];
+        float xd[RPL], xu[RPL];
+        bool live[RPL];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int j = (lane >> 3) + 4 * r;
+        for (int r = 0; r < RPL; ++r) {
+            const int j = j0 + (lane >> 3) + 4 * r;
             xd[r] = to_float(st.d[j][ce]);
             xu[r] = to_float(st.u[j][ce]);
             live[r] = st.pos[j] != -2 && evalid;  // past the end: a no-op step
         }
-        float4 cb[2], cv[2];
+        float4 cb[RPL / 2], cv[RPL / 2];
         if constexpr (!F32) {
             const BCStage<T>& sb = sm.bc[kl][c % NBC];
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int f = lane + 32 * r;  // (step f>>2, quad f&3)
-                const int j = f >> 2, q = f & 3;
+            for (int r = 0; r < RPL / 2; ++r) {
+                const int f = lane + 32 * r;  // (step j0 + f>>2, quad f&3)
+                const int j = j0 + (f >> 2), q = f & 3;
                 cb[r] = make_float4(to_float(sb.B[j][4 * q]), to_float(sb.B[j][4 * q + 1]),
                                     to_float(sb.B[j][4 * q + 2]), to_float(sb.B[j][4 * q + 3]));
                 cv[r] = make_float4(to_float(sb.C[j][4 * q]), to_float(sb.C[j][4 * q + 1]),
                                     to_float(sb.C[j][4 * q + 2]), to_float(sb.C[j][4 * q + 3]));
             }
         }
-        float2 out[4];
+        float2 out[RPL];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < RPL; ++r) {
             const float x = xd[r] + bias_k;
             const float dsp = live[r] ? (p.softplus ? softplus_f(x) : x) : 0.f;
             out[r] = make_float2(dsp, live[r] ? dsp * xu[r] : 0.f);
         }
 #pragma unroll
-        for (int r = 0; r < 4; ++r) pr.dd[(lane >> 3) + 4 * r][ce] = out[r];
+        for (int r = 0; r < RPL; ++r) pr.dd[j0 + (lane >> 3) + 4 * r][ce] = out[r];
         if constexpr (!F32) {
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
+            for (int r = 0; r < RPL / 2; ++r) {
                 const int f = lane + 32 * r;
-                pr.B[f >> 2][f & 3] = cb[r];
-                pr.C[f >> 2][f & 3] = cv[r];
+                pr.B[j0 + (f >> 2)][f & 3] = cb[r];
+                pr.C[j0 + (f >> 2)][f & 3] = cv[r];
             }
         }
     };
@@ -389,19 +438,19 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan
     auto finish_a = [&](int c) {
         const auto& st = sm.tok[kl][c % NR];
         float* yo = &sm.yout[kl][c % NY][0][0];
-        int pj[4], fin[4];
-        float yk[4], zz[4];
+        int pj[RPL], fin[RPL];
+        float yk[RPL], zz[RPL];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int j = (lane >> 3) + 4 * r;
+        for (int r = 0; r < RPL; ++r) {
+            const int j = j0 + (lane >> 3) + 4 * r;
             pj[r] = evalid ? st.pos[j] : -1;
             fin[r] = PARK ? st.fin[j] : 1;
             yk[r] = fmaf(Dk, to_float(st.u[j][ce]), yo[j * ST_CH + ce]);
             zz[r] = z_base ? to_float(st.z[j][ce]) : 0.f;
         }
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int j = (lane >> 3) + 4 * r;
+        for (int r = 0; r < RPL; ++r) {
+            const int j = j0 + (lane >> 3) + 4 * r;
             if (pj[r] < 0) continue;
             if constexpr (MODE == MODE_OWNER) {
                 float o = yk[r] * p.merge_scale;
@@ -418,12 +467,12 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan
     // MODE_PARK, second half (chunk c, one barrier after finish_a): the finalizer
     // adds the parked contributions, scales, gates and stores. The parked values
     // are loaded at the top of the iteration (fetch_b) and used at its end.
-    float parked[4];
+    float parked[RPL];
     auto fetch_b = [&](int c) {
         const auto& st = sm.tok[kl][c % NR];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int j = (lane >> 3) + 4 * r;
+        for (int r = 0; r < RPL; ++r) {
+            const int j = j0 + (lane >> 3) + 4 * r;
             const int pj = st.pos[j];
             float acc = 0.f;
             if (evalid && pj >= 0 && st.fin[j]) {
@@ -440,8 +489,8 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE>::THREADS) stream_scan
         const auto& st = sm.tok[kl][c % NR];
         const float* yo = &sm.yout[kl][c % NY][0][0];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int j = (lane >> 3) + 4 * r;
+        for (int r = 0; r < RPL; ++r) {
+            const int j = j0 + (lane >> 3) + 4 * r;
             const int pj = st.pos[j];
             if (!evalid || pj < 0 || !st.fin[j]) continue;
             float o = (yo[j * ST_CH + ce] + parked[r]) * p.merge_scale;
