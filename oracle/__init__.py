@@ -33,10 +33,10 @@ def _load():
         lib.oracle_geometry.restype = i
         lib.oracle_route.argtypes = [i, i, i, i, p]
         lib.oracle_route.restype = i
-        lib.oracle_scan_sequence.argtypes = [i, i, p, p, p, p, p, ctypes.c_double, p, p]
+        lib.oracle_scan_sequence.argtypes = [i, i, p, p, p, p, p, ctypes.c_double, i, p, p]
         lib.oracle_scan_sequence.restype = None
         lib.oracle_forward.argtypes = [i, i, i, i, i, i, i, p, p, p, p, p, p, p, p, i,
-                                       ctypes.c_double, i, i, p, i]
+                                       ctypes.c_double, i, i, p, p, i, p, i]
         lib.oracle_forward.restype = i
         lib.oracle_default_threads.argtypes = []
         lib.oracle_default_threads.restype = i
@@ -80,10 +80,11 @@ def route(kind, h, w, cls_pos=-1):
     return out
 
 
-def scan_sequence(u, dt, A, B, C, D=0.0):
+def scan_sequence(u, dt, A, B, C, D=0.0, zoh=False):
     """One channel, one sequence: h_t = e^{dt_t A} h + dt_t B_t u_t, y_t = C_t.h_t + D u_t.
 
     u, dt: [L]; A: [N]; B, C: [L, N]. dt is already discretized. Returns y [L].
+    zoh=True writes expm1(dt A) / A * B_t u_t (zero-order hold) instead of dt B_t u_t.
     """
     u, dt, A, B, C = map(_f64, (u, dt, A, B, C))
     L = u.shape[0]
@@ -92,18 +93,22 @@ def scan_sequence(u, dt, A, B, C, D=0.0):
     y = np.empty(L, dtype=np.float64)
     h = np.empty(N, dtype=np.float64)
     _load().oracle_scan_sequence(L, N, _ptr(u), _ptr(dt), _ptr(A), _ptr(B), _ptr(C),
-                                 float(D), _ptr(h), _ptr(y))
+                                 float(D), int(bool(zoh)), _ptr(h), _ptr(y))
     return y
 
 
 def forward(kind, h, w, u, delta, A, B, C, Dskip=None, bias=None, z=None, *,
             cls_pos=-1, delta_softplus=True, merge_scale=1.0,
-            per_dir_inputs=False, per_dir_params=False, threads=0):
+            per_dir_inputs=False, per_dir_params=False, conv_w=None, conv_b=None,
+            zoh=False, threads=0):
     """Routed forward pass in fp64.
 
     Shapes: u, delta [b, tokens, D] (or [K, b, tokens, D] with per_dir_inputs);
     B, C [b, tokens, N] (or [K, ...]); A [D, N] (or [K, D, N] with per_dir_params);
     Dskip, bias [D] (or [K, D]); z [b, tokens, D]. Returns y [b, tokens, D] float64.
+    conv_w [D, 4] (or [K, D, 4]) and conv_b [D] (or [K, D]) fuse the causal
+    kernel-four convolution + SiLU into u (BIDIR and pooled routes only);
+    zoh=True uses the zero-order-hold write term.
     """
     K, L, T = geometry(kind, h, w, cls_pos)
     u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
@@ -123,11 +128,18 @@ def forward(kind, h, w, u, delta, A, B, C, Dskip=None, bias=None, z=None, *,
         assert A.shape[0] == K
     if z is not None:
         assert z.shape == (b, T, D)
+    conv_w = None if conv_w is None else _f64(conv_w)
+    conv_b = None if conv_b is None else _f64(conv_b)
+    if conv_w is not None:
+        assert conv_w.shape == ((K, D, 4) if per_dir_params else (D, 4))
+        if conv_b is not None:
+            assert conv_b.shape == ((K, D) if per_dir_params else (D,))
     y = np.empty((b, T, D), dtype=np.float64)
     rc = _load().oracle_forward(_kind(kind), h, w, cls_pos, b, D, N, _ptr(u), _ptr(delta),
                                 _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip), _ptr(bias), _ptr(z),
                                 int(bool(delta_softplus)), float(merge_scale),
                                 int(bool(per_dir_inputs)), int(bool(per_dir_params)),
+                                _ptr(conv_w), _ptr(conv_b), int(bool(zoh)),
                                 _ptr(y), int(threads))
     if rc != 0:
         raise RuntimeError(f"oracle_forward failed (rc={rc})")

@@ -35,8 +35,14 @@
  *     before the bias and softplus; the whole scan (including D*u) runs on the
  *     pooled tokens; the result is repeated over the pooled axis and then gated
  *     with the un-pooled z of every grid token;
- *   - input write is Delta*B*u (the released convention), not exact ZOH;
- *   - softplus is the exact log(1 + e^x), evaluated without a threshold.
+ *   - input write is Delta*B*u (the released convention) unless the zero-order
+ *     hold flag asks for the exact integral of [NoD] Eq. 2;
+ *   - softplus is the exact log(1 + e^x), evaluated without a threshold;
+ *   - fused convolution: u holds the convolution input; each direction applies
+ *     its own kernel-four causal Conv1d + SiLU along its own sequence order
+ *     (BIDIR: the route; pooled routes: the row-major (POOL_W) or column-major
+ *     (POOL_H) token order, reversed for the backward direction) before any
+ *     pooling; the skip term D*u uses the convolved (and pooled) u.
  */
 #include <math.h>
 #include <omp.h>
@@ -182,21 +188,46 @@ static double silu(double z)
  *     y_t = sum_n C_{t,n} h_{t,n} + D * u_t
  * dt is the already-discretized step (after bias and softplus).
  * B and C are [L][N]; A is [N]; u, dt, y are [L]. h is caller scratch [N].
+ *
+ * zoh != 0 replaces the write term by the exact zero-order-hold input
+ * integral of [NoD] Eq. (2) (also the "discretization detail" paragraph of
+ * [Vim] sec. 4): for the diagonal A of the scan,
+ *     Bbar_n = (dt A_n)^-1 (exp(dt A_n) - 1) dt B_n = expm1(dt A_n) / A_n * B_n,
+ * whose limit for A_n = 0 is dt B_n.
  */
 void oracle_scan_sequence(int L, int N, const double* u, const double* dt, const double* A,
-                          const double* B, const double* C, double D, double* h, double* y)
+                          const double* B, const double* C, double D, int zoh, double* h,
+                          double* y)
 {
     for (int n = 0; n < N; ++n) h[n] = 0.0;
     for (int t = 0; t < L; ++t) {
         double read = 0.0;
         for (int n = 0; n < N; ++n) {
             double retention = exp(dt[t] * A[n]);
-            double write = dt[t] * B[(int64_t)t * N + n] * u[t];
+            double gain = dt[t];
+            if (zoh && A[n] != 0.0) gain = expm1(dt[t] * A[n]) / A[n];
+            double write = gain * B[(int64_t)t * N + n] * u[t];
             h[n] = retention * h[n] + write;
             read += C[(int64_t)t * N + n] * h[n];
         }
         y[t] = read + D * u[t];
     }
+}
+
+/*
+ * Causal depthwise convolution of kernel size 4 followed by SiLU, at step s of
+ * a sequence seq[0..]: SiLU(cb + sum_i cw[i] * seq[s - 3 + i]), with seq[<0] = 0
+ * ([Vim] "Inside the released Vim block": kernel-four causal Conv1d, then SiLU;
+ * "CPU backend substitutions": a grouped conv1d with left padding, then SiLU).
+ */
+static double causal_conv_silu(const double* seq, int64_t s, const double* cw, double cb)
+{
+    double acc = cb;
+    for (int i = 0; i < 4; ++i) {
+        int64_t j = s - 3 + i;
+        if (j >= 0) acc += cw[i] * seq[j];
+    }
+    return silu(acc);
 }
 
 /*
@@ -211,6 +242,19 @@ void oracle_scan_sequence(int L, int N, const double* u, const double* dt, const
  *   z        : [batch][tokens][D] (nullable: no gate); the gate is shared by all
  *              directions ([Vim] "Inside the released Vim block").
  *   y        : [batch][tokens][D]   output
+ *   conv_w   : [Kp][D][4]   (nullable: no convolution) -- with it, u holds the
+ *              convolution's input x and every direction k runs
+ *              u_k = SiLU(conv_k(x)) along its own sequence order before the
+ *              scan ([Vim] "Inside the released Vim block": each branch has its
+ *              own kernel-four causal Conv1d, the backward one on the reversed
+ *              sequence; it crosses row boundaries as the sequence does). BIDIR
+ *              convolves along the route; POOL_W / POOL_H convolve along the
+ *              row-major / column-major token order (forward and reversed) and
+ *              then pool the convolved values ([FVim] Methodology: Conv1D, then
+ *              mean-pool one axis). ATROUS2 and CROSS4 take no convolution
+ *              (OR_EINVAL): their pages convolve on the 2-D grid before routing.
+ *   conv_b   : [Kp][D]      (nullable: zero)
+ *   zoh      : 0 = dt * B * u write term; 1 = zero-order hold (oracle_scan_sequence)
  * Ki = K when per_dir_inputs, else 1; Kp = K when per_dir_params, else 1.
  * Every (batch, channel) pair is independent; channels and batches are
  * processed by OpenMP threads (nthreads <= 0: the OpenMP default).
@@ -220,12 +264,14 @@ int oracle_forward(int kind, int h, int w, int cls_pos, int batch, int D, int N,
                    const double* B, const double* C, const double* Dskip,
                    const double* bias, const double* z, int delta_softplus,
                    double merge_scale, int per_dir_inputs, int per_dir_params,
+                   const double* conv_w, const double* conv_b, int zoh,
                    double* y, int nthreads)
 {
     int K, L, tokens;
     int rc = oracle_geometry(kind, h, w, cls_pos, &K, &L, &tokens);
     if (rc != OR_OK) return rc;
     if (batch < 0 || D <= 0 || N <= 0) return OR_EINVAL;
+    if (conv_w && (kind == OR_ATROUS2 || kind == OR_CROSS4)) return OR_EINVAL;
     if (batch == 0) return OR_OK;
 
     int64_t* route = (int64_t*)malloc(sizeof(int64_t) * (size_t)K * L);
@@ -254,7 +300,9 @@ int oracle_forward(int kind, int h, int w, int cls_pos, int batch, int D, int N,
         double* hs = (double*)malloc(sizeof(double) * N);
         double* acc = (double*)malloc(sizeof(double) * (pooled ? L : tokens));
         int* owners = (int*)malloc(sizeof(int) * tokens);
-        int bad = (!su || !sdt || !sB || !sC || !sy || !hs || !acc || !owners);
+        double* xs = (double*)malloc(sizeof(double) * tokens); /* sequence-ordered conv input */
+        double* cu = (double*)malloc(sizeof(double) * tokens); /* conv output per token */
+        int bad = (!su || !sdt || !sB || !sC || !sy || !hs || !acc || !owners || !xs || !cu);
         if (bad) failed |= 1;
 
 #pragma omp for schedule(static)
@@ -274,6 +322,31 @@ int oracle_forward(int kind, int h, int w, int cls_pos, int batch, int D, int N,
                 const double* Ak = A + k * a_dir + (int64_t)d * N;
                 double Dk = Dskip ? Dskip[k * v_dir + d] : 0.0;
                 double bk = bias ? bias[k * v_dir + d] : 0.0;
+                const double* cw = conv_w ? conv_w + (k * v_dir + d) * 4 : 0;
+                double cb = (conv_w && conv_b) ? conv_b[k * v_dir + d] : 0.0;
+
+                if (conv_w && !pooled) {
+                    /* BIDIR: the convolution runs along this direction's route. */
+                    for (int t = 0; t < L; ++t) {
+                        int64_t q = route[(int64_t)k * L + t];
+                        xs[t] = q >= 0 ? uk[q * D + d] : 0.0;
+                    }
+                }
+                if (conv_w && pooled) {
+                    /* Token order of the convolution: row-major for POOL_W,
+                     * column-major for POOL_H; direction 1 runs it reversed. */
+                    int64_t g = (int64_t)h * w;
+                    for (int64_t s = 0; s < g; ++s) {
+                        int64_t q = k == 0 ? s : g - 1 - s;
+                        int64_t tok = (kind == OR_POOL_W) ? q : (q % h) * w + q / h;
+                        xs[s] = uk[tok * D + d];
+                    }
+                    for (int64_t s = 0; s < g; ++s) {
+                        int64_t q = k == 0 ? s : g - 1 - s;
+                        int64_t tok = (kind == OR_POOL_W) ? q : (q % h) * w + q / h;
+                        cu[tok] = causal_conv_silu(xs, s, cw, cb);
+                    }
+                }
 
                 /* Gather: one sequence step per route step. */
                 for (int t = 0; t < L; ++t) {
@@ -281,7 +354,7 @@ int oracle_forward(int kind, int h, int w, int cls_pos, int batch, int D, int N,
                     double uu = 0.0, dd = 0.0;
                     if (!pooled) {
                         if (q >= 0) { /* a real token */
-                            uu = uk[q * D + d];
+                            uu = conv_w ? causal_conv_silu(xs, t, cw, cb) : uk[q * D + d];
                             dd = dk[q * D + d];
                             for (int n = 0; n < N; ++n) {
                                 sB[(int64_t)t * N + n] = Bk[q * N + n];
@@ -306,7 +379,7 @@ int oracle_forward(int kind, int h, int w, int cls_pos, int batch, int D, int N,
                         }
                         for (int j = 0; j < cnt; ++j) {
                             int64_t tok = (kind == OR_POOL_W) ? q * w + j : (int64_t)j * w + q;
-                            su_ += uk[tok * D + d];
+                            su_ += conv_w ? cu[tok] : uk[tok * D + d];
                             sd_ += dk[tok * D + d];
                             for (int n = 0; n < N; ++n) {
                                 sB[(int64_t)t * N + n] += Bk[tok * N + n];
@@ -326,7 +399,7 @@ int oracle_forward(int kind, int h, int w, int cls_pos, int batch, int D, int N,
                     sdt[t] = delta_softplus ? softplus(x) : x;
                 }
 
-                oracle_scan_sequence(L, N, su, sdt, Ak, sB, sC, Dk, hs, sy);
+                oracle_scan_sequence(L, N, su, sdt, Ak, sB, sC, Dk, zoh, hs, sy);
 
                 /* Scatter back to the original coordinates. */
                 for (int t = 0; t < L; ++t) {
@@ -365,6 +438,7 @@ int oracle_forward(int kind, int h, int w, int cls_pos, int batch, int D, int N,
             }
         }
         free(su); free(sdt); free(sB); free(sC); free(sy); free(hs); free(acc); free(owners);
+        free(xs); free(cu);
     }
     free(route);
     if (failed & 1) return OR_ENOMEM;
