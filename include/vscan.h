@@ -93,6 +93,16 @@ typedef enum vscan_dtype {
     VSCAN_BF16 = 1 /* bfloat16; state and accumulation stay float32 */
 } vscan_dtype;
 
+/* Bits of vscan_args.flags. */
+typedef enum vscan_flag {
+    /* Exact zero-order-hold write term instead of Delta*B*u: for the diagonal A
+     * of the scan, Bbar = (Delta A)^-1 (exp(Delta A) - 1) Delta B =
+     * expm1(Delta A_n) / A_n * B_n, equal to Delta B_n for A_n = 0.
+     * "Norm or Direction? ...", sec. 3, Eq. 2; "Vision Mamba ...", sec. 4 (the
+     * released kernels keep Delta*B*u, the default). */
+    VSCAN_FLAG_ZOH = 1
+} vscan_flag;
+
 /* Opaque, immutable route description (host memory only). */
 typedef struct vscan_route vscan_route;
 
@@ -128,7 +138,23 @@ typedef struct vscan_args {
                                scan of affine pairs (BIDIR, CROSS4 and ATROUS2 when
                                the image's token tile fits on chip, else
                                VSCAN_ERR_UNSUPPORTED); ignored by the pooled routes */
-    int32_t reserved;       /* must be 0                                             */
+    int32_t flags;          /* OR of vscan_flag bits; other bits are rejected        */
+    const float* conv_w;    /* device, [Kp][D][4] float32, or NULL: no convolution.
+                               With it, u holds the convolution INPUT x and every
+                               direction k uses u_k = SiLU(conv_b + sum_i
+                               conv_w[i] * x[t - 3 + i]) along its own sequence
+                               order (x before the first step = 0) as the scan
+                               input, in the write term and in the skip term
+                               ("Vision Mamba ...", "Inside the released Vim
+                               block": each branch's kernel-four causal Conv1d,
+                               then SiLU; the backward branch on the reversed
+                               sequence). BIDIR: along the route. POOL_W / POOL_H:
+                               along the row-major / column-major token order
+                               (reversed for k = 1), before pooling ("Fast Vision
+                               Mamba ...", Methodology). CROSS4 and ATROUS2:
+                               VSCAN_ERR_UNSUPPORTED (their pages convolve on the
+                               2-D grid before routing).                          */
+    const float* conv_b;    /* device, [Kp][D] float32, or NULL for no conv bias    */
 } vscan_args;
 
 /*
@@ -258,7 +284,8 @@ const char* vscan_last_error(void);
 /* Static name of a status code. */
 const char* vscan_status_string(int32_t status);
 
-/* Library ABI version; changes whenever vscan_args changes layout. */
+/* Library ABI version; changes whenever vscan_args changes layout (2: flags,
+ * conv_w and conv_b). */
 int32_t vscan_abi_version(void);
 
 #ifdef __cplusplus

@@ -36,9 +36,10 @@ def test_library_exports_every_declared_function():
 
 
 def test_struct_layout_matches_the_header():
-    # int32 x4, 6 pointers, 3 pointers, int32 x3, float, pointer, uint64, int32 x2
-    assert ctypes.sizeof(abi.VscanArgs) == 16 + 48 + 24 + 12 + 4 + 8 + 8 + 8
-    assert abi.lib.vscan_abi_version() == abi.ABI_VERSION
+    # int32 x4, 6 pointers, 3 pointers, int32 x3, float, pointer, uint64, int32 x2, 2 pointers
+    assert ctypes.sizeof(abi.VscanArgs) == 16 + 48 + 24 + 12 + 4 + 8 + 8 + 8 + 16
+    assert abi.VscanArgs.flags.offset == 124 and abi.VscanArgs.conv_w.offset == 128
+    assert abi.lib.vscan_abi_version() == abi.ABI_VERSION == 2
 
 
 def test_status_strings():
@@ -101,7 +102,7 @@ def test_workspace_sizes():
 
 @pytest.mark.parametrize("field,value,status", [
     ("channels", 6, -3), ("channels", 0, -1), ("d_state", 17, -4), ("d_state", 0, -1),
-    ("dtype", 5, -1), ("batch", -1, -1), ("reserved", 1, -1), ("seq_chunks", 9, -1),
+    ("dtype", 5, -1), ("batch", -1, -1), ("flags", 2, -1), ("flags", -1, -1), ("seq_chunks", 9, -1),
     ("seq_chunks", 3, -1), ("seq_chunks", -1, -1),
     ("per_dir_inputs", 2, -1), ("merge_scale", float("nan"), -1),
 ])
@@ -187,3 +188,33 @@ def test_noalloc_pooled_forward_rejects_before_any_cuda_call():
 def test_pooled_route_length_limit():
     r = vs.Route("pool_w", 4000, 2)
     assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args()), None) == -4
+
+
+def test_convolution_is_refused_on_grid_routes_and_conv_b_needs_conv_w():
+    fake = dict(u=0x1000, delta=0x2000, B=0x3000, C=0x4000, y=0x5000, A=0x6000)
+    for kind in ("cross4", "atrous2"):
+        r = vs.Route(kind, 4, 4)
+        assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, conv_w=0x7000)), None) == -4
+        assert "BIDIR and the pooled routes" in abi.lib.vscan_last_error().decode()
+    r = vs.Route("bidir", 4, 4)
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, conv_b=0x7000)), None) == -1
+    # accepted on BIDIR and the pooled routes: the next failure is the missing workspace
+    for kind in ("bidir", "pool_w", "pool_h"):
+        r = vs.Route(kind, 4, 4)
+        assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, conv_w=0x7000)), None) == -6
+
+
+def test_zoh_flag_is_accepted_and_unknown_flags_are_not():
+    fake = dict(u=0x1000, delta=0x2000, B=0x3000, C=0x4000, y=0x5000, A=0x6000)
+    r = vs.Route("atrous2", 4, 4)
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, flags=abi.FLAG_ZOH)), None) != -1
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, flags=4)), None) == -1
+
+
+def test_host_buffer_holds_the_convolution_parameters():
+    r = vs.Route("bidir", 6, 6, 18)
+    n0, n1 = ctypes.c_uint64(), ctypes.c_uint64()
+    assert abi.lib.vscan_host_buffer_size(r.handle, ctypes.byref(_args()), ctypes.byref(n0)) == 0
+    a = _args(conv_w=1, conv_b=1)
+    assert abi.lib.vscan_host_buffer_size(r.handle, ctypes.byref(a), ctypes.byref(n1)) == 0
+    assert n1.value - n0.value == 2 * 256  # [D][4] and [D] floats, 256-byte rounded (D = 16)

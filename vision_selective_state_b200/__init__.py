@@ -8,6 +8,10 @@ kernels of the library. Tensors are channels-last:
     B, C           : [batch, tokens, N]   (leading K axis for per-direction B/C)
     A              : [D, N] float32        ([K, D, N] per direction)
     Dskip, bias    : [D] float32           ([K, D] per direction)
+    conv_w, conv_b : [D, 4], [D] float32   ([K, D, 4], [K, D] per direction), optional:
+                     fuse each direction's causal kernel-four Conv1d + SiLU into u
+                     (u then holds the convolution input); BIDIR and pooled routes
+    zoh=True       : zero-order-hold write term instead of Delta*B*u
 
 u, delta, B, C, z and y share one dtype: torch.float32 or torch.bfloat16.
 """
@@ -15,7 +19,7 @@ import ctypes
 
 import torch
 
-from ._abi import BF16, F32, ROUTES, VscanArgs, VscanError, check, lib
+from ._abi import BF16, F32, FLAG_ZOH, ROUTES, VscanArgs, VscanError, check, lib
 
 __all__ = ["Route", "forward", "forward_host", "workspace_size", "host_buffer_size", "VscanError",
            "ROUTES"]
@@ -82,12 +86,15 @@ def _ptr(t):
 
 
 def _args(route, u, delta, A, B, C, Dskip, delta_bias, z, y, delta_softplus, merge_scale,
-          per_dir_inputs, per_dir_params, workspace, seq_chunks):
+          per_dir_inputs, per_dir_params, workspace, seq_chunks, conv_w=None, conv_b=None,
+          zoh=False):
     for name, t in (("u", u), ("delta", delta), ("B", B), ("C", C), ("z", z), ("y", y),
-                    ("A", A), ("Dskip", Dskip), ("delta_bias", delta_bias)):
+                    ("A", A), ("Dskip", Dskip), ("delta_bias", delta_bias), ("conv_w", conv_w),
+                    ("conv_b", conv_b)):
         if t is not None and not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
-    for name, t in (("A", A), ("Dskip", Dskip), ("delta_bias", delta_bias)):
+    for name, t in (("A", A), ("Dskip", Dskip), ("delta_bias", delta_bias), ("conv_w", conv_w),
+                    ("conv_b", conv_b)):
         if t is not None and t.dtype != torch.float32:
             raise TypeError(f"{name} must be float32")
     lead = 1 if per_dir_inputs else 0
@@ -109,11 +116,12 @@ def _args(route, u, delta, A, B, C, Dskip, delta_bias, z, y, delta_softplus, mer
     if workspace is not None:
         a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
     a.seq_chunks = int(seq_chunks)
-    a.reserved = 0
+    a.flags = FLAG_ZOH if zoh else 0
+    a.conv_w, a.conv_b = _ptr(conv_w), _ptr(conv_b)
     return a
 
 
-def workspace_size(route, u, B, *, per_dir_inputs=False, per_dir_params=False):
+def workspace_size(route, u, B, *, per_dir_inputs=False, per_dir_params=False, **_):
     """Bytes of device scratch vscan_forward needs (host-only query)."""
     lead = 1 if per_dir_inputs else 0
     a = VscanArgs()
@@ -129,7 +137,7 @@ def workspace_size(route, u, B, *, per_dir_inputs=False, per_dir_params=False):
 
 def forward(route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, delta_softplus=True,
             merge_scale=1.0, per_dir_inputs=False, per_dir_params=False, out=None, workspace=None,
-            seq_chunks=0, stream=None):
+            seq_chunks=0, conv_w=None, conv_b=None, zoh=False, stream=None):
     """Routed selective scan on the GPU (vscan_forward). Returns y [batch, tokens, D]."""
     lead = 1 if per_dir_inputs else 0
     if out is None:
@@ -138,13 +146,13 @@ def forward(route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, de
         need = workspace_size(route, u, B, per_dir_inputs=per_dir_inputs, per_dir_params=per_dir_params)
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=u.device)
     a = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus, merge_scale,
-              per_dir_inputs, per_dir_params, workspace, seq_chunks)
+              per_dir_inputs, per_dir_params, workspace, seq_chunks, conv_w, conv_b, zoh)
     check(lib.vscan_forward(route.handle, ctypes.byref(a), _stream(stream, u.device)))
     return out
 
 
 def host_buffer_size(route, u, B, *, z=True, Dskip=True, delta_bias=True, per_dir_inputs=False,
-                     per_dir_params=False):
+                     per_dir_params=False, conv_w=False, conv_b=False):
     """Bytes of device memory forward_host needs (host-only query)."""
     lead = 1 if per_dir_inputs else 0
     a = VscanArgs()
@@ -157,6 +165,8 @@ def host_buffer_size(route, u, B, *, z=True, Dskip=True, delta_bias=True, per_di
     a.z = ctypes.c_void_p(1) if z else None
     a.Dskip = ctypes.c_void_p(1) if Dskip else None
     a.delta_bias = ctypes.c_void_p(1) if delta_bias else None
+    a.conv_w = ctypes.c_void_p(1) if conv_w else None
+    a.conv_b = ctypes.c_void_p(1) if conv_b else None
     n = ctypes.c_uint64()
     check(lib.vscan_host_buffer_size(route.handle, ctypes.byref(a), ctypes.byref(n)))
     return n.value
@@ -164,17 +174,17 @@ def host_buffer_size(route, u, B, *, z=True, Dskip=True, delta_bias=True, per_di
 
 def forward_host(route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, out,
                  device_buffer, delta_softplus=True, merge_scale=1.0, per_dir_inputs=False,
-                 per_dir_params=False, stream=None):
+                 per_dir_params=False, conv_w=None, conv_b=None, zoh=False, stream=None):
     """End-to-end call with host (CPU, ideally pinned) tensors (vscan_forward_host).
 
     Enqueues the host-to-device copies, the scan and the copy of y into `out`
     (a host tensor) on the stream; synchronize the stream before reading `out`.
     """
-    for t in (u, delta, A, B, C, Dskip, delta_bias, z, out):
+    for t in (u, delta, A, B, C, Dskip, delta_bias, z, out, conv_w, conv_b):
         if t is not None and t.is_cuda:
             raise ValueError("forward_host takes host tensors")
     a = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus, merge_scale,
-              per_dir_inputs, per_dir_params, None, 0)
+              per_dir_inputs, per_dir_params, None, 0, conv_w, conv_b, zoh)
     nbytes = device_buffer.numel() * device_buffer.element_size()
     check(lib.vscan_forward_host(route.handle, ctypes.byref(a), ctypes.c_void_p(device_buffer.data_ptr()),
                                  nbytes, _stream(stream, device_buffer.device)))
@@ -189,12 +199,13 @@ class Plan:
 
     def __init__(self, route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, out,
                  workspace, delta_softplus=True, merge_scale=1.0, per_dir_inputs=False,
-                 per_dir_params=False, seq_chunks=0):
+                 per_dir_params=False, seq_chunks=0, conv_w=None, conv_b=None, zoh=False):
         self.route = route
-        self._keep = (u, delta, A, B, C, Dskip, delta_bias, z, out, workspace)
+        self._keep = (u, delta, A, B, C, Dskip, delta_bias, z, out, workspace, conv_w, conv_b)
         self.out = out
         self.args = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus,
-                          merge_scale, per_dir_inputs, per_dir_params, workspace, seq_chunks)
+                          merge_scale, per_dir_inputs, per_dir_params, workspace, seq_chunks,
+                          conv_w, conv_b, zoh)
         self._ref = ctypes.byref(self.args)
 
     def run(self, stream):
@@ -222,15 +233,15 @@ class HostPlan:
 
     def __init__(self, route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, out,
                  device_buffer, delta_softplus=True, merge_scale=1.0, per_dir_inputs=False,
-                 per_dir_params=False):
-        for t in (u, delta, A, B, C, Dskip, delta_bias, z, out):
+                 per_dir_params=False, conv_w=None, conv_b=None, zoh=False):
+        for t in (u, delta, A, B, C, Dskip, delta_bias, z, out, conv_w, conv_b):
             if t is not None and t.is_cuda:
                 raise ValueError("HostPlan takes host tensors")
         self.route = route
-        self._keep = (u, delta, A, B, C, Dskip, delta_bias, z, out, device_buffer)
+        self._keep = (u, delta, A, B, C, Dskip, delta_bias, z, out, device_buffer, conv_w, conv_b)
         self.out = out
         self.args = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus,
-                          merge_scale, per_dir_inputs, per_dir_params, None, 0)
+                          merge_scale, per_dir_inputs, per_dir_params, None, 0, conv_w, conv_b, zoh)
         self._ref = ctypes.byref(self.args)
         self._buf = ctypes.c_void_p(device_buffer.data_ptr())
         self._nbytes = device_buffer.numel() * device_buffer.element_size()

@@ -21,7 +21,8 @@ STATUS = {
 }
 ROUTES = {"bidir": 0, "cross4": 1, "atrous2": 2, "pool_w": 3, "pool_h": 4}
 F32, BF16 = 0, 1
-ABI_VERSION = 1
+ABI_VERSION = 2
+FLAG_ZOH = 1
 
 
 class VscanArgs(ctypes.Structure):
@@ -48,7 +49,9 @@ class VscanArgs(ctypes.Structure):
         ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_uint64),
         ("seq_chunks", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("flags", ctypes.c_int32),
+        ("conv_w", ctypes.c_void_p),
+        ("conv_b", ctypes.c_void_p),
     ]
 
 

@@ -24,7 +24,7 @@ struct vscan_route {
 
 namespace {
 
-constexpr int32_t kAbiVersion = 1;
+constexpr int32_t kAbiVersion = 2;
 constexpr size_t kMaxSmem = 200 * 1024;  // dynamic shared memory the kernels may ask for
 thread_local std::string g_last_error;
 
@@ -56,7 +56,7 @@ size_t resident_bytes(const vscan_route* r, const vscan_args* a)
 {
     const int Ki = a->per_dir_inputs ? r->g.K : 1;
     const int Kd = (a->per_dir_inputs || a->per_dir_params) ? r->g.K : 1;
-    return vscan::resident_smem_bytes(r->g.kind, r->g.tokens, Ki, Kd);
+    return vscan::resident_smem_bytes(r->g.kind, r->g.tokens, Ki, Kd, a->conv_w != nullptr);
 }
 
 // Checks that do not depend on where the tensors live.
@@ -64,7 +64,11 @@ vscan_status check_shape(const vscan_route* r, const vscan_args* a)
 {
     if (!r) return fail(VSCAN_ERR_INVALID_ARGUMENT, "route is NULL");
     if (!a) return fail(VSCAN_ERR_INVALID_ARGUMENT, "args is NULL");
-    if (a->reserved != 0) return fail(VSCAN_ERR_INVALID_ARGUMENT, "args.reserved must be 0");
+    if (a->flags & ~int32_t(VSCAN_FLAG_ZOH))
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "unknown bits in args.flags 0x%x", (unsigned)a->flags);
+    if (a->conv_b && !a->conv_w) return fail(VSCAN_ERR_INVALID_ARGUMENT, "conv_b given without conv_w");
+    if (a->conv_w && (r->g.kind == vscan::RK_CROSS4 || r->g.kind == vscan::RK_ATROUS2))
+        return fail(VSCAN_ERR_UNSUPPORTED, "the fused convolution is defined for BIDIR and the pooled routes");
     if (a->dtype != VSCAN_F32 && a->dtype != VSCAN_BF16)
         return fail(VSCAN_ERR_INVALID_ARGUMENT, "unknown dtype %d", a->dtype);
     if (a->batch < 0) return fail(VSCAN_ERR_INVALID_ARGUMENT, "batch %d < 0", a->batch);
@@ -89,7 +93,7 @@ vscan_status check_shape(const vscan_route* r, const vscan_args* a)
         return fail(VSCAN_ERR_UNSUPPORTED, "tokens x channels of one image must be below 2^31");
     if (is_pool(r->g.kind)) {
         const int Ki = a->per_dir_inputs ? 2 : 1;
-        if (vscan::pool_scan_smem_bytes(Ki, r->g.L) > kMaxSmem)
+        if (vscan::pool_scan_smem_bytes(Ki, r->g.L, a->conv_w != nullptr) > kMaxSmem)
             return fail(VSCAN_ERR_UNSUPPORTED, "pooled length %d too long for the on-chip tile", r->g.L);
     } else if (a->seq_chunks > 1) {
         if (resident_bytes(r, a) > kMaxSmem)
@@ -142,16 +146,16 @@ uint64_t workspace_need(const vscan_route* r, const vscan_args* a)
     return 0;
 }
 
-template <int RK, typename T, bool N16, int KC, int MODE, int PW>
+template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL>
 cudaError_t launch_stream_mode(vscan::ScanParams p, int k_base, int grid_z, cudaStream_t s)
 {
-    const size_t smem = vscan::stream_smem_bytes<T, KC, MODE>();
-    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW>,
+    const size_t smem = vscan::stream_smem_bytes<T, KC, MODE, FL>();
+    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     p.k_base = k_base;
     const dim3 grid((p.D + vscan::ST_CH - 1) / vscan::ST_CH, p.batch, grid_z);
-    vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW>
+    vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL>
         <<<grid, vscan::StreamShape<T, KC, MODE, PW>::THREADS, smem, s>>>(p);
     return cudaGetLastError();
 }
@@ -159,63 +163,108 @@ cudaError_t launch_stream_mode(vscan::ScanParams p, int k_base, int grid_z, cuda
 // ATROUS2: every pixel has one owner; float32 I/O runs one direction per CTA
 //   (grid.z = 4), bf16 I/O all four directions per CTA.
 // BIDIR, CROSS4: all directions of an image tile in one CTA, merged by parking.
-template <int RK, typename T, bool N16>
+template <int RK, typename T, bool N16, int FL>
 cudaError_t launch_stream_n(const vscan::ScanParams& p, cudaStream_t s)
 {
     using namespace vscan;
     if constexpr (RK == RK_ATROUS2) {
-        if constexpr (sizeof(T) == 4) return launch_stream_mode<RK, T, N16, 1, MODE_OWNER, 1>(p, 0, 4, s);
-        else return launch_stream_mode<RK, T, N16, 4, MODE_OWNER, 1>(p, 0, 1, s);
+        if constexpr (sizeof(T) == 4) return launch_stream_mode<RK, T, N16, 1, MODE_OWNER, 1, FL>(p, 0, 4, s);
+        else return launch_stream_mode<RK, T, N16, 4, MODE_OWNER, 1, FL>(p, 0, 1, s);
     } else if constexpr (RK == RK_BIDIR) {
-        return launch_stream_mode<RK, T, N16, 2, MODE_PARK, 1>(p, 0, 1, s);
+        return launch_stream_mode<RK, T, N16, 2, MODE_PARK, 1, FL>(p, 0, 1, s);
     } else {
-        return launch_stream_mode<RK, T, N16, 4, MODE_PARK, 1>(p, 0, 1, s);
+        return launch_stream_mode<RK, T, N16, 4, MODE_PARK, 1, FL>(p, 0, 1, s);
     }
 }
 
-template <int RK, typename T>
-cudaError_t launch_stream(const vscan::ScanParams& p, cudaStream_t s)
+template <int RK, typename T, int FL>
+cudaError_t launch_stream_fl(const vscan::ScanParams& p, cudaStream_t s)
 {
-    return p.N == 16 ? launch_stream_n<RK, T, true>(p, s) : launch_stream_n<RK, T, false>(p, s);
+    return p.N == 16 ? launch_stream_n<RK, T, true, FL>(p, s) : launch_stream_n<RK, T, false, FL>(p, s);
 }
 
-template <int RK, typename T, int NC>
+// fl: OR of vscan::FL_ZOH and vscan::FL_CONV (the latter for BIDIR only).
+template <int RK, typename T>
+cudaError_t launch_stream(const vscan::ScanParams& p, int fl, cudaStream_t s)
+{
+    using namespace vscan;
+    if constexpr (RK == RK_BIDIR) {
+        switch (fl) {
+        case FL_ZOH: return launch_stream_fl<RK, T, FL_ZOH>(p, s);
+        case FL_CONV: return launch_stream_fl<RK, T, FL_CONV>(p, s);
+        case FL_ZOH | FL_CONV: return launch_stream_fl<RK, T, FL_ZOH | FL_CONV>(p, s);
+        default: return launch_stream_fl<RK, T, 0>(p, s);
+        }
+    } else {
+        return (fl & FL_ZOH) ? launch_stream_fl<RK, T, FL_ZOH>(p, s) : launch_stream_fl<RK, T, 0>(p, s);
+    }
+}
+
+template <int RK, typename T, int NC, int FL>
 cudaError_t launch_resident_nc(const vscan::ScanParams& p, size_t smem, cudaStream_t s)
 {
     constexpr int CH = vscan::ResidentShape<RK>::CH;
-    cudaError_t e = cudaFuncSetAttribute(vscan::resident_scan_kernel<RK, T, NC>,
+    cudaError_t e = cudaFuncSetAttribute(vscan::resident_scan_kernel<RK, T, NC, FL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem);
     if (e != cudaSuccess) return e;
     const dim3 grid((p.D + CH - 1) / CH, p.batch);
-    vscan::resident_scan_kernel<RK, T, NC><<<grid, 64 * NC, smem, s>>>(p);
+    vscan::resident_scan_kernel<RK, T, NC, FL><<<grid, 64 * NC, smem, s>>>(p);
     return cudaSuccess;
 }
 
-template <int RK, typename T>
-cudaError_t launch_resident(const vscan::ScanParams& p, int nc, cudaStream_t s)
+template <int RK, typename T, int FL>
+cudaError_t launch_resident_fl(const vscan::ScanParams& p, int nc, cudaStream_t s)
 {
     const int Ki = p.in_dir ? p.g.K : 1;
     const int Kd = (p.in_dir || p.v_dir) ? p.g.K : 1;
-    const size_t smem = vscan::resident_smem_bytes(RK, p.g.tokens, Ki, Kd);
+    const size_t smem = vscan::resident_smem_bytes(RK, p.g.tokens, Ki, Kd, (FL & vscan::FL_CONV) != 0);
     switch (nc) {
-    case 2: return launch_resident_nc<RK, T, 2>(p, smem, s);
-    case 4: return launch_resident_nc<RK, T, 4>(p, smem, s);
-    default: return launch_resident_nc<RK, T, 8>(p, smem, s);
+    case 2: return launch_resident_nc<RK, T, 2, FL>(p, smem, s);
+    case 4: return launch_resident_nc<RK, T, 4, FL>(p, smem, s);
+    default: return launch_resident_nc<RK, T, 8, FL>(p, smem, s);
     }
 }
 
-template <typename T>
-cudaError_t launch_pool(const vscan::PoolParams& p, cudaStream_t s)
+template <int RK, typename T>
+cudaError_t launch_resident(const vscan::ScanParams& p, int nc, int fl, cudaStream_t s)
+{
+    using namespace vscan;
+    if constexpr (RK == RK_BIDIR) {
+        switch (fl) {
+        case FL_ZOH: return launch_resident_fl<RK, T, FL_ZOH>(p, nc, s);
+        case FL_CONV: return launch_resident_fl<RK, T, FL_CONV>(p, nc, s);
+        case FL_ZOH | FL_CONV: return launch_resident_fl<RK, T, FL_ZOH | FL_CONV>(p, nc, s);
+        default: return launch_resident_fl<RK, T, 0>(p, nc, s);
+        }
+    } else {
+        return (fl & FL_ZOH) ? launch_resident_fl<RK, T, FL_ZOH>(p, nc, s) : launch_resident_fl<RK, T, 0>(p, nc, s);
+    }
+}
+
+template <typename T, int FL>
+cudaError_t launch_pool_fl(const vscan::PoolParams& p, cudaStream_t s)
 {
     const dim3 g1(p.g.L, p.batch, p.Ki);
     vscan::pool_bc_kernel<T><<<g1, 128, 0, s>>>(p);
-    const size_t smem = vscan::pool_scan_smem_bytes(p.Ki, p.g.L);
-    cudaError_t e = cudaFuncSetAttribute(vscan::pool_scan_kernel<T>,
+    const size_t smem = vscan::pool_scan_smem_bytes(p.Ki, p.g.L, (FL & vscan::FL_CONV) != 0);
+    cudaError_t e = cudaFuncSetAttribute(vscan::pool_scan_kernel<T, FL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (e != cudaSuccess) return e;
     const dim3 g2((p.D + vscan::PL_CH - 1) / vscan::PL_CH, p.batch);
-    vscan::pool_scan_kernel<T><<<g2, vscan::PL_THREADS, smem, s>>>(p);
+    vscan::pool_scan_kernel<T, FL><<<g2, vscan::PL_THREADS, smem, s>>>(p);
     return cudaSuccess;
+}
+
+template <typename T>
+cudaError_t launch_pool(const vscan::PoolParams& p, int fl, cudaStream_t s)
+{
+    using namespace vscan;
+    switch (fl) {
+    case FL_ZOH: return launch_pool_fl<T, FL_ZOH>(p, s);
+    case FL_CONV: return launch_pool_fl<T, FL_CONV>(p, s);
+    case FL_ZOH | FL_CONV: return launch_pool_fl<T, FL_ZOH | FL_CONV>(p, s);
+    default: return launch_pool_fl<T, 0>(p, s);
+    }
 }
 
 template <typename T>
@@ -223,6 +272,7 @@ vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s)
 {
     const vscan::RouteGeom& g = r->g;
     const long long plane = (long long)a->batch * g.tokens;
+    const int fl = ((a->flags & VSCAN_FLAG_ZOH) ? vscan::FL_ZOH : 0) | (a->conv_w ? vscan::FL_CONV : 0);
     if (is_pool(g.kind)) {
         vscan::PoolParams p{};
         p.g = g;
@@ -239,7 +289,8 @@ vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s)
         const uint64_t half = workspace_need(r, a) / 2;
         p.pB = static_cast<float*>(a->workspace);
         p.pC = reinterpret_cast<float*>(static_cast<char*>(a->workspace) + half);
-        cudaError_t e = launch_pool<T>(p, s);
+        p.conv_w = a->conv_w; p.conv_b = a->conv_b;
+        cudaError_t e = launch_pool<T>(p, fl, s);
         if (e != cudaSuccess) return cuda_fail(e, "configuring the pooled-scan kernel");
     } else {
         vscan::ScanParams p{};
@@ -254,21 +305,22 @@ vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s)
         p.softplus = a->delta_softplus;
         p.merge_scale = a->merge_scale;
         p.scratch = static_cast<float*>(a->workspace);
+        p.conv_w = a->conv_w; p.conv_b = a->conv_b;
         const int nc = choose_chunks(r, a);
         if (nc > 1) {
             cudaError_t e;
             switch (g.kind) {
-            case vscan::RK_BIDIR: e = launch_resident<vscan::RK_BIDIR, T>(p, nc, s); break;
-            case vscan::RK_CROSS4: e = launch_resident<vscan::RK_CROSS4, T>(p, nc, s); break;
-            default: e = launch_resident<vscan::RK_ATROUS2, T>(p, nc, s); break;
+            case vscan::RK_BIDIR: e = launch_resident<vscan::RK_BIDIR, T>(p, nc, fl, s); break;
+            case vscan::RK_CROSS4: e = launch_resident<vscan::RK_CROSS4, T>(p, nc, fl, s); break;
+            default: e = launch_resident<vscan::RK_ATROUS2, T>(p, nc, fl, s); break;
             }
             if (e != cudaSuccess) return cuda_fail(e, "configuring the resident scan kernel");
         } else {
             cudaError_t e;
             switch (g.kind) {
-            case vscan::RK_BIDIR: e = launch_stream<vscan::RK_BIDIR, T>(p, s); break;
-            case vscan::RK_CROSS4: e = launch_stream<vscan::RK_CROSS4, T>(p, s); break;
-            default: e = launch_stream<vscan::RK_ATROUS2, T>(p, s); break;
+            case vscan::RK_BIDIR: e = launch_stream<vscan::RK_BIDIR, T>(p, fl, s); break;
+            case vscan::RK_CROSS4: e = launch_stream<vscan::RK_CROSS4, T>(p, fl, s); break;
+            default: e = launch_stream<vscan::RK_ATROUS2, T>(p, fl, s); break;
             }
             if (e != cudaSuccess) return cuda_fail(e, "configuring the streaming scan kernel");
         }
@@ -302,7 +354,7 @@ __global__ void route_map_kernel(vscan::RouteGeom g, int32_t* out)
 }
 
 struct HostLayout {
-    size_t u, delta, B, C, z, y, A, Dskip, bias, ws, total;
+    size_t u, delta, B, C, z, y, A, Dskip, bias, conv_w, conv_b, ws, total;
 };
 
 HostLayout host_layout(const vscan_route* r, const vscan_args* a)
@@ -324,6 +376,8 @@ HostLayout host_layout(const vscan_route* r, const vscan_args* a)
     L.A = take(Kp * a->channels * a->d_state * sizeof(float));
     L.Dskip = take(a->Dskip ? Kp * a->channels * sizeof(float) : 0);
     L.bias = take(a->delta_bias ? Kp * a->channels * sizeof(float) : 0);
+    L.conv_w = take(a->conv_w ? Kp * a->channels * 4 * sizeof(float) : 0);
+    L.conv_b = take(a->conv_b ? Kp * a->channels * sizeof(float) : 0);
     L.ws = take(workspace_need(r, a));
     L.total = off;
     return L;
@@ -507,6 +561,8 @@ vscan_status vscan_forward_host(const vscan_route* r, const vscan_args* ha, void
     da.A = reinterpret_cast<const float*>(base + L.A);
     da.Dskip = ha->Dskip ? reinterpret_cast<const float*>(base + L.Dskip) : nullptr;
     da.delta_bias = ha->delta_bias ? reinterpret_cast<const float*>(base + L.bias) : nullptr;
+    da.conv_w = ha->conv_w ? reinterpret_cast<const float*>(base + L.conv_w) : nullptr;
+    da.conv_b = ha->conv_b ? reinterpret_cast<const float*>(base + L.conv_b) : nullptr;
     da.workspace = base + L.ws;
     da.workspace_bytes = workspace_need(r, ha);
 
@@ -520,6 +576,8 @@ vscan_status vscan_forward_host(const vscan_route* r, const vscan_args* ha, void
         {const_cast<float*>(da.A), ha->A, Kp * ha->channels * ha->d_state * sizeof(float)},
         {const_cast<float*>(da.Dskip), ha->Dskip, ha->Dskip ? Kp * ha->channels * sizeof(float) : 0},
         {const_cast<float*>(da.delta_bias), ha->delta_bias, ha->delta_bias ? Kp * ha->channels * sizeof(float) : 0},
+        {const_cast<float*>(da.conv_w), ha->conv_w, ha->conv_w ? Kp * ha->channels * 4 * sizeof(float) : 0},
+        {const_cast<float*>(da.conv_b), ha->conv_b, ha->conv_b ? Kp * ha->channels * sizeof(float) : 0},
     };
     for (const Copy& c : in) {
         if (c.bytes == 0) continue;

@@ -81,6 +81,10 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 v
     *reinterpret_cast<uint2*>(p) = raw;
 }
 
+// Optional steps of the scan, as kernel template flags: the zero-order-hold
+// write term and the fused causal convolution of u.
+enum ScanFlags : int { FL_ZOH = 1, FL_CONV = 2 };
+
 // ---- discretization ---------------------------------------------------------
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32). The retention
 // exp(Delta * A) is evaluated as 2^(Delta * A * log2 e), with A pre-scaled.
@@ -126,6 +130,26 @@ __device__ __forceinline__ float softplus_f(float x)
 __device__ __forceinline__ float silu_f(float z)
 {
     return z * fast_rcp(1.0f + fast_exp2(-z * LOG2E));
+}
+
+// Zero-order-hold gain ("Norm or Direction? ...", Eq. 2): for the diagonal A of
+// the scan, Bbar = (Delta A)^-1 (e^(Delta A) - 1) Delta B = phi(x) * Delta * B with
+//     phi(x) = (e^x - 1) / x,   x = Delta * A.
+// e = e^x is the retention the caller already has and rx = 1 / x. For |x| < 0.5
+// phi is a degree-6 least-squares polynomial with phi(0) = 1 made by
+// fit_expm1x.py (relative error 8e-8 in float32), which avoids the
+// cancellation in e - 1; elsewhere (e - 1) * rx. x = 0 (A = 0 or Delta = 0)
+// gives exactly 1, the Delta*B*u write.
+__device__ __forceinline__ float zoh_phi(float x, float e, float rx)
+{
+    float q = 1.986203570e-04f;
+    q = fmaf(q, x, 1.399721252e-03f);
+    q = fmaf(q, x, 8.333531208e-03f);
+    q = fmaf(q, x, 4.166532308e-02f);
+    q = fmaf(q, x, 1.666666418e-01f);
+    q = fmaf(q, x, 5.000000596e-01f);
+    q = fmaf(q, x, 1.0f);
+    return fabsf(x) < 0.5f ? q : (e - 1.0f) * rx;
 }
 
 }  // namespace vscan

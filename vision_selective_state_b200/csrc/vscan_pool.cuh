@@ -14,6 +14,16 @@
 //                     the repeated, gated output over every grid token.
 // The pooled-route memory traffic is the compulsory one: u, Delta and z read
 // once, y written once; B and C are read once by the small pre-pass.
+//
+// Optional steps (template flags FL, as for the streaming kernel):
+//   FL_ZOH   zero-order-hold write term (zoh_phi).
+//   FL_CONV  u holds the convolution input x. Each direction's kernel-four causal
+//            Conv1d + SiLU runs over the full token sequence before pooling
+//            ("Fast Vision Mamba ...", Methodology: Conv1D, then mean-pool one
+//            axis; "Vision Mamba ...", "Inside the released Vim block": the
+//            backward branch convolves the reversed sequence). The sequence is
+//            the row-major (POOL_W) or column-major (POOL_H) token order, so the
+//            members of one pooled index are consecutive in it.
 #pragma once
 
 #include "vscan_common.cuh"
@@ -41,6 +51,8 @@ struct PoolParams {
     float merge_scale;
     float* pB;  // [Ki][batch][Lp][N]
     float* pC;  // [Ki][batch][Lp][N]
+    const float* conv_w;  // FL_CONV: [Kp][D][4]
+    const float* conv_b;  // FL_CONV: [Kp][D] (nullable)
 };
 
 constexpr int PL_CH = 32;       // channels per CTA
@@ -90,21 +102,26 @@ __global__ void __launch_bounds__(128) pool_bc_kernel(const PoolParams p)
 }
 
 // Dynamic shared memory (floats): pd[Ki][Lp][32] (pooled raw Delta),
-// pu[Ki][Lp][32] (pooled u), Y[2][Lp][32] (per-direction outputs).
-inline size_t pool_scan_smem_bytes(int Ki, int Lp)
+// pu[Ku][Lp][32] (pooled u; Ku = 2 with the convolution, whose output differs
+// per direction, else Ki), Y[2][Lp][32] (per-direction outputs).
+inline size_t pool_scan_smem_bytes(int Ki, int Lp, bool conv = false)
 {
-    return sizeof(float) * (size_t)(2 * Ki + 2) * Lp * PL_CH;
+    const int Ku = conv ? 2 : Ki;
+    return sizeof(float) * (size_t)(Ki + Ku + 2) * Lp * PL_CH;
 }
 
-template <typename T>
+template <typename T, int FL>
 __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams p)
 {
+    constexpr bool ZOH = (FL & FL_ZOH) != 0;
+    constexpr bool CONV = (FL & FL_CONV) != 0;
     extern __shared__ __align__(16) float psm[];
     const int Lp = p.g.L;
     const int Ki = p.Ki;
+    const int Ku = CONV ? 2 : Ki;
     float* pd = psm;                          // [Ki][Lp][32]
-    float* pu = psm + (size_t)Ki * Lp * PL_CH;  // [Ki][Lp][32]
-    float* Y = pu + (size_t)Ki * Lp * PL_CH;    // [2][Lp][32]
+    float* pu = psm + (size_t)Ki * Lp * PL_CH;  // [Ku][Lp][32]
+    float* Y = pu + (size_t)Ku * Lp * PL_CH;    // [2][Lp][32]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = blockIdx.y;
@@ -115,8 +132,100 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
     const int cnt = (p.g.kind == RK_POOL_W) ? p.g.w : p.g.h;
     const float inv_cnt = 1.0f / (float)cnt;
 
+    // ---- phase 1 (FL_CONV): convolve along the token sequence, then pool -------
+    if constexpr (CONV) {
+        const int jl = lane >> 3;   // run of consecutive members 0..3
+        const int q = lane & 7;     // channel quad of the tile
+        const int ch = c0 + 4 * q;
+        const bool cval = ch < D;
+        const long long g_tok = (long long)p.g.h * p.g.w;
+        const int run = (cnt + 3) / 4;
+        const int jb = jl * run, je = min(cnt, jb + run);
+        for (int k = 0; k < Ki; ++k) {
+            // directions whose convolution reads this input plane
+            const int dlo = (Ki == 1) ? 0 : k, dhi = (Ki == 1) ? 1 : k;
+            float kw[2][4][4], kb[2][4];  // [direction][tap][channel of the quad]
+#pragma unroll
+            for (int dd = 0; dd < 2; ++dd)
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int dr = dd == 0 ? dlo : dhi;
+                    const long long o = (long long)dr * p.v_dir + ch + cc;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) kw[dd][i][cc] = cval ? __ldg(p.conv_w + o * 4 + i) : 0.f;
+                    kb[dd][cc] = (cval && p.conv_b) ? __ldg(p.conv_b + o) : 0.f;
+                }
+            const T* xb = static_cast<const T*>(p.u) + k * p.in_dir + img * D + ch;
+            const T* db = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + ch;
+            // x at sequence position sq (0 outside the sequence)
+            auto xat = [&](long long sq) {
+                if (!cval || sq < 0 || sq >= g_tok) return make_float4(0.f, 0.f, 0.f, 0.f);
+                const long long tok = pool_member(p.g, (int)(sq / cnt), (int)(sq % cnt));
+                return load4<T>(xb + tok * D);
+            };
+            for (int i = warp; i < Lp; i += PL_THREADS / 32) {
+                float4 au0 = make_float4(0.f, 0.f, 0.f, 0.f), au1 = au0, ad = au0;
+                const long long s0 = (long long)i * cnt + jb;
+                float4 win[7];  // x at s-3 .. s+3
+#pragma unroll
+                for (int m = 0; m < 6; ++m) win[m] = xat(s0 - 3 + m);
+                for (int j = jb; j < je; ++j) {
+                    const long long sq = (long long)i * cnt + j;
+                    win[6] = xat(sq + 3);
+                    const float4 dl = cval ? load4<T>(db + (long long)pool_member(p.g, i, j) * D)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                    ad.x += dl.x; ad.y += dl.y; ad.z += dl.z; ad.w += dl.w;
+                    const float* wv = reinterpret_cast<const float*>(win);  // [7][4]
+                    float f[4], bk[4];
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float a0 = kb[0][cc], a1 = kb[1][cc];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            a0 = fmaf(kw[0][t][cc], wv[4 * t + cc], a0);        // x[s - 3 + t]
+                            a1 = fmaf(kw[1][t][cc], wv[4 * (6 - t) + cc], a1);  // x[s + 3 - t]
+                        }
+                        f[cc] = silu_f(a0);
+                        bk[cc] = silu_f(a1);
+                    }
+                    if (Ki == 1 || k == 0) { au0.x += f[0]; au0.y += f[1]; au0.z += f[2]; au0.w += f[3]; }
+                    if (Ki == 1 || k == 1) { au1.x += bk[0]; au1.y += bk[1]; au1.z += bk[2]; au1.w += bk[3]; }
+#pragma unroll
+                    for (int m = 0; m < 6; ++m) win[m] = win[m + 1];
+                }
+#pragma unroll
+                for (int m = 8; m <= 16; m <<= 1) {
+                    au0.x += __shfl_xor_sync(FULL_MASK, au0.x, m);
+                    au0.y += __shfl_xor_sync(FULL_MASK, au0.y, m);
+                    au0.z += __shfl_xor_sync(FULL_MASK, au0.z, m);
+                    au0.w += __shfl_xor_sync(FULL_MASK, au0.w, m);
+                    au1.x += __shfl_xor_sync(FULL_MASK, au1.x, m);
+                    au1.y += __shfl_xor_sync(FULL_MASK, au1.y, m);
+                    au1.z += __shfl_xor_sync(FULL_MASK, au1.z, m);
+                    au1.w += __shfl_xor_sync(FULL_MASK, au1.w, m);
+                    ad.x += __shfl_xor_sync(FULL_MASK, ad.x, m);
+                    ad.y += __shfl_xor_sync(FULL_MASK, ad.y, m);
+                    ad.z += __shfl_xor_sync(FULL_MASK, ad.z, m);
+                    ad.w += __shfl_xor_sync(FULL_MASK, ad.w, m);
+                }
+                if (jl == 0) {
+                    float* dd_ = pd + ((size_t)k * Lp + i) * PL_CH + 4 * q;
+                    dd_[0] = ad.x * inv_cnt; dd_[1] = ad.y * inv_cnt; dd_[2] = ad.z * inv_cnt; dd_[3] = ad.w * inv_cnt;
+                    if (Ki == 1 || k == 0) {
+                        float* u0 = pu + ((size_t)0 * Lp + i) * PL_CH + 4 * q;
+                        u0[0] = au0.x * inv_cnt; u0[1] = au0.y * inv_cnt; u0[2] = au0.z * inv_cnt; u0[3] = au0.w * inv_cnt;
+                    }
+                    if (Ki == 1 || k == 1) {
+                        float* u1 = pu + ((size_t)1 * Lp + i) * PL_CH + 4 * q;
+                        u1[0] = au1.x * inv_cnt; u1[1] = au1.y * inv_cnt; u1[2] = au1.z * inv_cnt; u1[3] = au1.w * inv_cnt;
+                    }
+                }
+            }
+        }
+    }
+
     // ---- phase 1: mean-pool u and raw Delta of the channel tile ---------------
-    {
+    if constexpr (!CONV) {
         const int jl = lane >> 3;   // token sub-lane 0..3
         const int q = lane & 7;     // channel quad of the tile
         const int ch = c0 + 4 * q;
@@ -192,7 +301,10 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
         const float* pBk = p.pB + ((long long)ki * p.batch + b) * Lp * N;
         const float* pCk = p.pC + ((long long)ki * p.batch + b) * Lp * N;
         const float* pdk = pd + (size_t)ki * Lp * PL_CH;
-        const float* puk = pu + (size_t)ki * Lp * PL_CH;
+        const float* puk = pu + (size_t)(CONV ? kd : ki) * Lp * PL_CH;
+        float ia[4];  // ZOH: 1 / A per state (0 for A = 0)
+#pragma unroll
+        for (int s = 0; s < 4; ++s) ia[s] = (a2[s] != 0.f) ? LOG2E / a2[s] : 0.f;
         float* Yk = Y + (size_t)kd * Lp * PL_CH;
         float h[4] = {0.f, 0.f, 0.f, 0.f};
         for (int t0 = 0; t0 < Lp; t0 += 4) {
@@ -215,10 +327,13 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
                         bv[s] = n < N ? __ldg(pBk + (size_t)i * N + n) : 0.f;
                         cv[s] = n < N ? __ldg(pCk + (size_t)i * N + n) : 0.f;
                     }
+                    const float rd = ZOH ? fast_rcp(dsp) : 0.f;
 #pragma unroll
                     for (int s = 0; s < 4; ++s) {
                         const float e = fast_exp2(dsp * a2[s]);
-                        h[s] = fmaf(e, h[s], du * bv[s]);
+                        float w = du * bv[s];
+                        if constexpr (ZOH) w *= zoh_phi(dsp * a2[s] * LN2, e, rd * ia[s]);
+                        h[s] = fmaf(e, h[s], w);
                         acc = fmaf(cv[s], h[s], acc);
                     }
                 }

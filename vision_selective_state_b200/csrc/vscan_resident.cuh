@@ -21,6 +21,11 @@
 // The recurrence, discretization and merge follow "Vision Mamba ...", sec. 3-5,
 // and "EfficientVMamba ...", sec. 1-3, exactly as the streaming kernel does;
 // "Fast Vision Mamba ..." cites the log-depth parallel scan this realizes.
+//
+// Optional steps (template flags FL): FL_ZOH, the zero-order-hold write term;
+// FL_CONV (BIDIR), u holds the convolution input x and each direction's
+// kernel-four causal Conv1d + SiLU is applied along its route after staging,
+// into one convolved plane per direction.
 #pragma once
 
 #include "vscan_common.cuh"
@@ -41,7 +46,7 @@ struct ResidentShape {
 // Shared-memory bytes of the resident kernel, or 0 if RK is not supported.
 // Ki: input planes (u, B, C); Kd: planes of the discretized step (K when the
 // inputs or the bias differ per direction, else 1).
-inline size_t resident_smem_bytes(int kind, int tokens, int Ki, int Kd)
+inline size_t resident_smem_bytes(int kind, int tokens, int Ki, int Kd, bool conv = false)
 {
     int CH, PLANES;
     switch (kind) {
@@ -50,14 +55,19 @@ inline size_t resident_smem_bytes(int kind, int tokens, int Ki, int Kd)
     case RK_ATROUS2: CH = 4; PLANES = 1; break;
     default: return 0;
     }
-    const size_t per_token = (size_t)Ki * (CH + 32) + (size_t)Kd * CH + (size_t)PLANES * CH;
+    if (conv && kind != RK_BIDIR) return 0;
+    const size_t per_token = (size_t)Ki * (CH + 32) + (size_t)Kd * CH + (size_t)PLANES * CH +
+                             (conv ? (size_t)2 * CH : 0);
     return per_token * tokens * sizeof(float);
 }
 
-template <int RK, typename T, int NC>
+template <int RK, typename T, int NC, int FL>
 __global__ void __launch_bounds__(RS_THREADS) resident_scan_kernel(const ScanParams p)
 {
     using S = ResidentShape<RK>;
+    constexpr bool ZOH = (FL & FL_ZOH) != 0;
+    constexpr bool CONV = (FL & FL_CONV) != 0;
+    static_assert(!CONV || RK == RK_BIDIR, "the fused convolution is defined for the bidirectional route");
     constexpr int K = S::K, CH = S::CH, PLANES = S::PLANES;
     constexpr int LPC = 4 * NC;        // lanes per channel
     constexpr int CPW = 32 / LPC;      // channels per warp
@@ -73,6 +83,7 @@ __global__ void __launch_bounds__(RS_THREADS) resident_scan_kernel(const ScanPar
     float* sB = sp + (size_t)Kd * tokens * CH;        // [Ki][tokens][16]
     float* sC = sB + (size_t)Ki * tokens * 16;        // [Ki][tokens][16]
     float* sY = sC + (size_t)Ki * tokens * 16;        // [PLANES][tokens][CH]
+    float* sX = sY + (size_t)PLANES * tokens * CH;    // FL_CONV: [2][tokens][CH] convolved u
 
     const int tid = threadIdx.x;
     const int nthreads = K * WPD * 32;
@@ -151,6 +162,31 @@ __global__ void __launch_bounds__(RS_THREADS) resident_scan_kernel(const ScanPar
     }
     __syncthreads();
 
+    // ---- FL_CONV: u_k = SiLU(conv_k(x)) along each direction's route -------------
+    if constexpr (CONV) {
+        // BIDIR: direction 0 visits token t at step t, direction 1 at step tokens-1-t,
+        // so the causal taps of token t are x[t-3+i] (forward) and x[t+3-i] (backward).
+        for (int e = tid; e < 2 * tokens * CH; e += nthreads) {
+            const int kd = e / (tokens * CH);
+            const int rem = e - kd * tokens * CH;
+            const int tok = rem / CH, c = rem - tok * CH;
+            const int d = c0 + c;
+            float acc = 0.f;
+            if (d < D) {
+                const float* xk = su + (size_t)(Ki > 1 ? kd : 0) * tokens * CH;
+                const long long o = (long long)kd * p.v_dir + d;
+                acc = p.conv_b ? __ldg(p.conv_b + o) : 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int tt = kd == 0 ? tok - 3 + i : tok + 3 - i;
+                    if (tt >= 0 && tt < tokens) acc = fmaf(__ldg(p.conv_w + o * 4 + i), xk[(size_t)tt * CH + c], acc);
+                }
+            }
+            sX[e] = silu_f(acc);
+        }
+        __syncthreads();
+    }
+
     // ---- roles ------------------------------------------------------------------
     const int warp = tid >> 5, lane = tid & 31;
     const int k = warp / WPD;
@@ -172,7 +208,10 @@ __global__ void __launch_bounds__(RS_THREADS) resident_scan_kernel(const ScanPar
     const float Dd = (dvalid && p.Dskip) ? __ldg(p.Dskip + k * p.v_dir + d) : 0.f;
     const float bias = (dvalid && p.bias) ? __ldg(p.bias + k * p.v_dir + d) : 0.f;
     const float dsp_pad = p.softplus ? softplus_f(bias) : bias;  // ATROUS2 padding step
-    const float* suk = su + (size_t)ki * tokens * CH;
+    const float* suk = CONV ? sX + (size_t)k * tokens * CH : su + (size_t)ki * tokens * CH;
+    float ia[4];  // ZOH: 1 / A per state (0 for A = 0)
+#pragma unroll
+    for (int s = 0; s < 4; ++s) ia[s] = (a2[s] != 0.f) ? LOG2E / a2[s] : 0.f;
     const float* spk = sp + (size_t)(Kd > 1 ? k : 0) * tokens * CH;
     const float4* sBk = reinterpret_cast<const float4*>(sB + (size_t)ki * tokens * 16);
     const float4* sCk = reinterpret_cast<const float4*>(sC + (size_t)ki * tokens * 16);
@@ -207,11 +246,14 @@ __global__ void __launch_bounds__(RS_THREADS) resident_scan_kernel(const ScanPar
         int pos;
         step(t0 + i, dsp, du, uu, Bv, Cv, pos);
         const float bv[4] = {Bv.x, Bv.y, Bv.z, Bv.w};
+        const float rd = ZOH ? fast_rcp(dsp) : 0.f;
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
             const float e = fast_exp2(dsp * a2[s]);
+            float w = du * bv[s];
+            if constexpr (ZOH) w *= zoh_phi(dsp * a2[s] * LN2, e, rd * ia[s]);
             P[s] *= e;
-            H[s] = fmaf(e, H[s], du * bv[s]);
+            H[s] = fmaf(e, H[s], w);
         }
     }
 
@@ -244,11 +286,14 @@ __global__ void __launch_bounds__(RS_THREADS) resident_scan_kernel(const ScanPar
         step(t0 + i, dsp, du, uu, Bv, Cv, pos);
         const float bv[4] = {Bv.x, Bv.y, Bv.z, Bv.w};
         const float cv[4] = {Cv.x, Cv.y, Cv.z, Cv.w};
+        const float rd = ZOH ? fast_rcp(dsp) : 0.f;
         float acc = 0.f;
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
             const float e = fast_exp2(dsp * a2[s]);
-            h[s] = fmaf(e, h[s], du * bv[s]);
+            float w = du * bv[s];
+            if constexpr (ZOH) w *= zoh_phi(dsp * a2[s] * LN2, e, rd * ia[s]);
+            h[s] = fmaf(e, h[s], w);
             acc = fmaf(cv[s], h[s], acc);
         }
         acc += __shfl_xor_sync(FULL_MASK, acc, 1);

@@ -34,6 +34,14 @@
 //                 workspace; one barrier later the finalizer adds the parked
 //                 values to its own, scales, gates and stores.
 // Neither mode uses atomics or a separate pass over y.
+//
+// Optional steps (template flags FL):
+//   FL_ZOH   the write term uses the zero-order-hold gain phi(Delta A) (zoh_phi)
+//            instead of Delta*B*u ("Norm or Direction? ...", Eq. 2).
+//   FL_CONV  (BIDIR) u holds the convolution input x; the producer applies the
+//            direction's kernel-four causal Conv1d + SiLU along the route
+//            ("Vision Mamba ...", "Inside the released Vim block"), reading the
+//            three previous steps from the previous chunk's token slot.
 #pragma once
 
 #include "vscan_common.cuh"
@@ -63,6 +71,8 @@ struct ScanParams {
     float merge_scale;
     int k_base;        // first direction of this launch (direction = k_base + blockIdx.z*KC + local)
     float* scratch;    // PARK: [K][batch][tokens][D] float32
+    const float* conv_w;  // FL_CONV: [Kp][D][4]
+    const float* conv_b;  // FL_CONV: [Kp][D] (nullable)
 };
 
 constexpr int ST_TOK = 16;  // steps per chunk
@@ -99,20 +109,28 @@ struct __align__(16) BCStage {
     T C[ST_TOK][16];
 };
 
-// Discretized chunk of one direction; with CONV, float32 copies of B and C.
-template <bool CONV>
-struct PrepStage;
-
-template <>
-struct __align__(16) PrepStage<true> {
+// Discretized chunk of one direction: with BCF (bf16 I/O) float32 copies of B
+// and C, with ZOH the reciprocal of Delta.
+template <bool ON> struct PrepBC {};
+template <> struct PrepBC<true> {
     float4 B[ST_TOK][4];
     float4 C[ST_TOK][4];
+};
+template <bool ON> struct PrepRD {};
+template <> struct PrepRD<true> {
+    float rd[ST_TOK][ST_CH];  // 1 / Delta (inf for Delta = 0, where zoh_phi does not use it)
+};
+
+template <bool BCF, bool ZOH>
+struct __align__(16) PrepStage : PrepBC<BCF>, PrepRD<ZOH> {
     float2 dd[ST_TOK][ST_CH];  // {Delta after bias + softplus (0 past the end), Delta * u}
 };
 
-template <>
-struct __align__(16) PrepStage<false> {
-    float2 dd[ST_TOK][ST_CH];
+// FL_CONV: the convolved u of the last three chunks of each direction, for the
+// skip term D*u of the epilogue.
+template <bool ON, int KC> struct ConvRing {};
+template <int KC> struct ConvRing<true, KC> {
+    float uc[KC][3][ST_TOK][ST_CH];
 };
 
 template <typename T, int KC, int MODE, int PW = 1>
@@ -131,17 +149,17 @@ struct StreamShape {
     static_assert(PW == 1 || PW == 2, "one or two producer warps per direction");
 };
 
-template <typename T, int KC, int MODE>
-struct StreamSmem {
+template <typename T, int KC, int MODE, int FL = 0>
+struct StreamSmem : ConvRing<(FL & FL_CONV) != 0, KC> {
     using S = StreamShape<T, KC, MODE>;
     TokStage<T> tok[KC][S::NR];
     BCStage<T> bc[KC][S::NBC];
-    PrepStage<!S::F32> prep[KC][2];
+    PrepStage<!S::F32, (FL & FL_ZOH) != 0> prep[KC][2];
     float yout[KC][S::NY][ST_TOK][ST_CH];
 };
 
-template <typename T, int KC, int MODE>
-constexpr size_t stream_smem_bytes() { return sizeof(StreamSmem<T, KC, MODE>); }
+template <typename T, int KC, int MODE, int FL = 0>
+constexpr size_t stream_smem_bytes() { return sizeof(StreamSmem<T, KC, MODE, FL>); }
 
 // Direction that adds up token p: the one visiting p in the latest chunk.
 template <int RK>
@@ -160,17 +178,21 @@ __device__ __forceinline__ int finalizer(const RouteGeom& g, int p)
     return best_k;
 }
 
-template <int RK, typename T, bool N16, int KC, int MODE, int PW>
+template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL>
 __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_scan_kernel(const ScanParams p)
 {
     using S = StreamShape<T, KC, MODE, PW>;
     constexpr int SPW = S::SPW, RPL = S::RPL;
+    constexpr bool ZOH = (FL & FL_ZOH) != 0;
+    constexpr bool CONV = (FL & FL_CONV) != 0;
+    static_assert(!CONV || RK == RK_BIDIR, "the fused convolution is defined for the bidirectional route");
+    static_assert(!CONV || PW == 1, "the convolution reads steps gathered by the same producer warp");
     constexpr int NR = S::NR, NBC = S::NBC, NY = S::NY;
     constexpr bool PARK = S::PARK;
     constexpr bool F32 = S::F32;
     constexpr int KR = (RK == RK_BIDIR) ? 2 : 4;  // directions of the route
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    StreamSmem<T, KC, MODE>& sm = *reinterpret_cast<StreamSmem<T, KC, MODE>*>(smem_raw);
+    StreamSmem<T, KC, MODE, FL>& sm = *reinterpret_cast<StreamSmem<T, KC, MODE, FL>*>(smem_raw);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -195,6 +217,10 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
             a2[s] = (dvalid && n < N) ? __ldg(p.A + (long long)k * p.a_dir + (long long)d * N + n) * LOG2E : 0.f;
         }
         const float2 a01 = make_float2(a2[0], a2[1]), a23 = make_float2(a2[2], a2[3]);
+        // ZOH: 1 / A per state (0 for A = 0, where x = Delta A = 0 selects the polynomial)
+        float ia[4];
+#pragma unroll
+        for (int s = 0; s < 4; ++s) ia[s] = (a2[s] != 0.f) ? LOG2E / a2[s] : 0.f;
         float2 h01 = make_float2(0.f, 0.f), h23 = h01;
         __syncthreads();  // prologue: chunk 0 discretized
 
@@ -226,6 +252,16 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
                     e23[j] = make_float2(fast_exp2(x23.x), fast_exp2(x23.y));
                     w01[j] = __fmul2_rn(du2, make_float2(Bv.x, Bv.y));
                     w23[j] = __fmul2_rn(du2, make_float2(Bv.z, Bv.w));
+                    if constexpr (ZOH) {
+                        const float rd = pr.rd[j][cc];
+                        const float x[4] = {x01.x * LN2, x01.y * LN2, x23.x * LN2, x23.y * LN2};
+                        const float e[4] = {e01[j].x, e01[j].y, e23[j].x, e23[j].y};
+                        float g[4];
+#pragma unroll
+                        for (int s = 0; s < 4; ++s) g[s] = zoh_phi(x[s], e[s], rd * ia[s]);
+                        w01[j] = __fmul2_rn(w01[j], make_float2(g[0], g[1]));
+                        w23[j] = __fmul2_rn(w23[j], make_float2(g[2], g[3]));
+                    }
                 };
                 front(0);
                 front(1);
@@ -275,6 +311,15 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
     const bool evalid = dch < D;
     const float bias_k = (evalid && p.bias) ? __ldg(p.bias + k * p.v_dir + dch) : 0.f;
     const float Dk = (evalid && p.Dskip) ? __ldg(p.Dskip + k * p.v_dir + dch) : 0.f;
+    float kw[4] = {0.f, 0.f, 0.f, 0.f};  // FL_CONV: the direction's kernel and bias for channel dch
+    float kb = 0.f;
+    if constexpr (CONV) {
+        if (evalid) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) kw[i] = __ldg(p.conv_w + ((long long)k * p.v_dir + dch) * 4 + i);
+            kb = p.conv_b ? __ldg(p.conv_b + k * p.v_dir + dch) : 0.f;
+        }
+    }
     const T* z_base = p.z ? static_cast<const T*>(p.z) + img * D + c0 : nullptr;
     T* y_base = static_cast<T*>(p.y) + img * D + dch;  // + token * D (fits in int32)
     // parked contributions of direction kk for this image and channel: + token * D
@@ -402,6 +447,26 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
             xu[r] = to_float(st.u[j][ce]);
             live[r] = st.pos[j] != -2 && evalid;  // past the end: a no-op step
         }
+        if constexpr (CONV) {
+            // u = SiLU(kb + sum_i kw[i] x[t - 3 + i]) along the route: steps before
+            // the chunk come from the previous chunk's slot, before step 0 they are 0
+            const auto& prev = sm.tok[kl][(c + NR - 1) % NR];
+#pragma unroll
+            for (int r = 0; r < RPL; ++r) {
+                const int j = j0 + (lane >> 3) + 4 * r;
+                float acc = kb;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int jj = j - 3 + i;
+                    float xv;
+                    if (jj >= 0) xv = (i == 3) ? xu[r] : to_float(st.u[jj][ce]);
+                    else xv = (c > 0) ? to_float(prev.u[ST_TOK + jj][ce]) : 0.f;
+                    acc = fmaf(kw[i], xv, acc);
+                }
+                xu[r] = silu_f(acc);
+                sm.uc[kl][c % 3][j][ce] = xu[r];
+            }
+        }
         float4 cb[RPL / 2], cv[RPL / 2];
         if constexpr (!F32) {
             const BCStage<T>& sb = sm.bc[kl][c % NBC];
@@ -424,6 +489,10 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
         }
 #pragma unroll
         for (int r = 0; r < RPL; ++r) pr.dd[j0 + (lane >> 3) + 4 * r][ce] = out[r];
+        if constexpr (ZOH) {
+#pragma unroll
+            for (int r = 0; r < RPL; ++r) pr.rd[j0 + (lane >> 3) + 4 * r][ce] = fast_rcp(out[r].x);
+        }
         if constexpr (!F32) {
 #pragma unroll
             for (int r = 0; r < RPL / 2; ++r) {
@@ -445,7 +514,10 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
             const int j = j0 + (lane >> 3) + 4 * r;
             pj[r] = evalid ? st.pos[j] : -1;
             fin[r] = PARK ? st.fin[j] : 1;
-            yk[r] = fmaf(Dk, to_float(st.u[j][ce]), yo[j * ST_CH + ce]);
+            float uj;
+            if constexpr (CONV) uj = sm.uc[kl][c % 3][j][ce];
+            else uj = to_float(st.u[j][ce]);
+            yk[r] = fmaf(Dk, uj, yo[j * ST_CH + ce]);
             zz[r] = z_base ? to_float(st.z[j][ce]) : 0.f;
         }
 #pragma unroll

@@ -128,6 +128,19 @@ def draw(wl: Workload, *, per_dir_inputs: bool = False, per_dir_params: bool = F
     return out
 
 
+def draw_conv(wl: Workload, *, per_dir_params: bool = False) -> dict:
+    """Seeded kernel-four depthwise convolution weights and bias (float32):
+    conv_w [D, 4] (or [K, D, 4]) ~ 0.5 N(0, 1), conv_b [D] (or [K, D]) ~ 0.1 N(0, 1),
+    drawn from their own stream (seed + 7919) so the scan inputs stay unchanged."""
+    K = {"bidir": 2, "cross4": 4, "atrous2": 4, "pool_w": 2, "pool_h": 2}[wl.route]
+    rng = np.random.default_rng(wl.seed + 7919)
+    plead = (K,) if per_dir_params else ()
+    f32 = np.float32
+    conv_w = rng.standard_normal(plead + (wl.D, 4), dtype=f32) * f32(0.5)
+    conv_b = rng.standard_normal(plead + (wl.D,), dtype=f32) * f32(0.1)
+    return dict(conv_w=conv_w, conv_b=conv_b)
+
+
 def channel_slice(inputs: dict, channels, per_dir_params: bool = False) -> dict:
     """The inputs restricted to a subset of channels (channels are independent)."""
     ch = np.asarray(channels)
@@ -135,8 +148,11 @@ def channel_slice(inputs: dict, channels, per_dir_params: bool = False) -> dict:
     for key in ("u", "z", "delta"):
         out[key] = np.ascontiguousarray(inputs[key][..., ch])
     out["A"] = np.ascontiguousarray(inputs["A"][..., ch, :])
-    for key in ("Dskip", "bias"):
-        out[key] = np.ascontiguousarray(inputs[key][..., ch])
+    for key in ("Dskip", "bias", "conv_b"):
+        if inputs.get(key) is not None:
+            out[key] = np.ascontiguousarray(inputs[key][..., ch])
+    if inputs.get("conv_w") is not None:
+        out["conv_w"] = np.ascontiguousarray(inputs["conv_w"][..., ch, :])
     return out
 
 
