@@ -54,6 +54,9 @@ def parse():
                    help="override the workload's batch (small profiling captures only)")
     p.add_argument("--rotate", type=int, default=0,
                    help="device copies of the inputs cycled through (0: enough to exceed 3x L2)")
+    p.add_argument("--conv", action="store_true",
+                   help="fuse the causal kernel-four Conv1d + SiLU into u (BIDIR and pooled routes)")
+    p.add_argument("--zoh", action="store_true", help="zero-order-hold write term instead of Delta*B*u")
     return p.parse_args()
 
 
@@ -69,14 +72,15 @@ def workload_label(wls):
     w0 = wls[0]
     grids = "+".join(f"{w.h}x{w.w}" for w in wls)
     cls = "_cls" if w0.cls_pos >= 0 else ""
-    return f"{w0.route}_{grids}{cls}_b{w0.batch}_d{w0.D}_n{w0.N}_{w0.dtype}"
+    opt = ("_conv" if w0.conv else "") + ("_zoh" if w0.zoh else "")
+    return f"{w0.route}_{grids}{cls}_b{w0.batch}_d{w0.D}_n{w0.N}_{w0.dtype}{opt}"
 
 
 def algorithmic_bytes(wl):
     """Compulsory HBM bytes of one forward: read u, raw delta, z, B, C; write y."""
     eb = 2 if wl.dtype == "bf16" else 4
     per_token = (3 * wl.D + 2 * wl.N) * eb + wl.D * eb
-    params = (wl.D * wl.N + 2 * wl.D) * 4
+    params = (wl.D * wl.N + 2 * wl.D + (5 * wl.D if wl.conv else 0)) * 4
     return wl.batch * wl.tokens * per_token + params
 
 
@@ -240,10 +244,14 @@ def oracle_time(wls, channels, threads=0):
     import oracle
     total = 0.0
     for wl in wls:
-        x = workloads.channel_slice(workloads.draw(wl), channels)
+        x = workloads.draw(wl)
+        if wl.conv:
+            x.update(workloads.draw_conv(wl))
+        x = workloads.channel_slice(x, channels)
         t0 = time.perf_counter()
         oracle.forward(wl.route, wl.h, wl.w, x["u"], x["delta"], x["A"], x["B"], x["C"], x["Dskip"],
-                       x["bias"], x["z"] if wl.gate else None, cls_pos=wl.cls_pos, threads=threads)
+                       x["bias"], x["z"] if wl.gate else None, cls_pos=wl.cls_pos,
+                       conv_w=x.get("conv_w"), conv_b=x.get("conv_b"), zoh=wl.zoh, threads=threads)
         total += time.perf_counter() - t0
     return total
 
@@ -306,6 +314,7 @@ def config_block(wls, n):
     return {"workload": workload_label(wls), "route": w0.route,
             "grids": [f"{w.h}x{w.w}" for w in wls], "batch": w0.batch, "d_inner": w0.D,
             "d_state": w0.N, "io_dtype": w0.dtype, "gate": w0.gate, "merge_scale": w0.merge_scale,
+            "conv": w0.conv, "zoh": w0.zoh,
             "parallelism": f"replicas x{n} (one full workload per GPU, no collective)"}
 
 
@@ -336,8 +345,10 @@ def run_ours(args, wls):
         routes.append(route)
         dt = td[wl.dtype]
         host = {k: torch.from_numpy(x[k]).to(dt) for k in ("u", "delta", "B", "C", "z")}
+        if wl.conv:
+            x.update(workloads.draw_conv(wl))
         host.update({k: torch.from_numpy(np.ascontiguousarray(x[k], dtype=np.float32))
-                     for k in ("A", "Dskip", "bias")})
+                     for k in ("A", "Dskip", "bias") + (("conv_w", "conv_b") if wl.conv else ())})
         host_sets.append(host)
         ws_bytes = vs.workspace_size(route, host["u"], host["B"])
         per = []
@@ -347,7 +358,8 @@ def run_ours(args, wls):
             ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
             per.append(vs.Plan(route, d["u"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], d["bias"],
                                d["z"] if wl.gate else None, out=out, workspace=ws,
-                               merge_scale=wl.merge_scale))
+                               merge_scale=wl.merge_scale, conv_w=d.get("conv_w"),
+                               conv_b=d.get("conv_b"), zoh=wl.zoh))
         plans.append(per)
     launches_per_step = sum(per[0].kernels() for per in plans)
     knames = sorted({per[0].kernel_name() for per in plans})
@@ -435,13 +447,14 @@ def run_ours(args, wls):
         for wl, route, host in zip(wls, routes, host_sets):
             pin = {k: v.pin_memory() for k, v in host.items()}
             out = torch.empty_like(pin["u"]).pin_memory()
-            nbytes = vs.host_buffer_size(route, pin["u"], pin["B"], z=wl.gate)
+            nbytes = vs.host_buffer_size(route, pin["u"], pin["B"], z=wl.gate, conv_w=wl.conv,
+                                         conv_b=wl.conv)
             buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
             hplans.append(vs.HostPlan(route, pin["u"], pin["delta"], pin["A"], pin["B"], pin["C"],
                                       pin["Dskip"], pin["bias"], pin["z"] if wl.gate else None,
-                                      out=out, device_buffer=buf, merge_scale=wl.merge_scale))
-            h2d += sum(pin[k].numel() * pin[k].element_size()
-                       for k in ("u", "delta", "B", "C", "z", "A", "Dskip", "bias"))
+                                      out=out, device_buffer=buf, merge_scale=wl.merge_scale,
+                                      conv_w=pin.get("conv_w"), conv_b=pin.get("conv_b"), zoh=wl.zoh))
+            h2d += sum(v.numel() * v.element_size() for k, v in pin.items() if k != "z" or wl.gate)
             d2h += out.numel() * out.element_size()
         E = max(1, min(args.e2e_steps, K))
         with torch.cuda.stream(stream):
@@ -480,6 +493,10 @@ def main():
     wls = select(args.workload)
     if args.batch > 0:
         wls = [w.with_(batch=args.batch) for w in wls]
+    if args.conv or args.zoh:
+        wls = [w.with_(conv=args.conv, zoh=args.zoh) for w in wls]
+        if args.conv and wls[0].route in ("cross4", "atrous2"):
+            raise SystemExit("--conv applies to the bidir and pooled workloads (0, 3, 4)")
     if args.impl == "reference":
         run_reference(args, wls)
     else:

@@ -38,6 +38,9 @@ def _load():
         lib.oracle_forward.argtypes = [i, i, i, i, i, i, i, p, p, p, p, p, p, p, p, i,
                                        ctypes.c_double, i, i, p, p, i, p, i]
         lib.oracle_forward.restype = i
+        lib.oracle_forward_masked.argtypes = [i, i, i, i, i, p, i, i, p, p, p, p, p, p, p, p, i,
+                                              ctypes.c_double, i, i, i, p, i]
+        lib.oracle_forward_masked.restype = i
         lib.oracle_default_threads.argtypes = []
         lib.oracle_default_threads.restype = i
         _lib = lib
@@ -143,4 +146,34 @@ def forward(kind, h, w, u, delta, A, B, C, Dskip=None, bias=None, z=None, *,
                                 _ptr(y), int(threads))
     if rc != 0:
         raise RuntimeError(f"oracle_forward failed (rc={rc})")
+    return y
+
+
+def forward_masked(kind, h, w, pos, u, delta, A, B, C, Dskip=None, bias=None, z=None, *,
+                   delta_softplus=True, merge_scale=1.0, per_dir_inputs=False,
+                   per_dir_params=False, zoh=False, threads=0):
+    """Pooled route on a masked token set (FastMaskVim) in fp64.
+
+    pos [b, n] int grid positions (row * w + col) of the visible tokens; u, delta
+    [b, n, D] (or [2, b, n, D]); B, C [b, n, N] (or [2, ...]); z [b, n, D].
+    Pooled tokens are row (POOL_W) or column (POOL_H) sums over the visible
+    tokens divided by the nominal width (height). Returns y [b, n, D].
+    """
+    u, delta, A, B, C = map(_f64, (u, delta, A, B, C))
+    pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int32))
+    Dskip = None if Dskip is None else _f64(Dskip)
+    bias = None if bias is None else _f64(bias)
+    z = None if z is None else _f64(z)
+    lead = 1 if per_dir_inputs else 0
+    b, n, D = u.shape[lead:]
+    N = B.shape[-1]
+    assert pos.shape == (b, n) and delta.shape == u.shape and C.shape == B.shape
+    y = np.empty((b, n, D), dtype=np.float64)
+    rc = _load().oracle_forward_masked(_kind(kind), h, w, b, n, _ptr(pos), D, N, _ptr(u), _ptr(delta),
+                                       _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip), _ptr(bias), _ptr(z),
+                                       int(bool(delta_softplus)), float(merge_scale),
+                                       int(bool(per_dir_inputs)), int(bool(per_dir_params)),
+                                       int(bool(zoh)), _ptr(y), int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_forward_masked failed (rc={rc})")
     return y

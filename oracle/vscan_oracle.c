@@ -446,6 +446,123 @@ int oracle_forward(int kind, int h, int w, int cls_pos, int batch, int D, int N,
     return OR_OK;
 }
 
+/*
+ * Pooled route on a masked (sparse) token set, [FVim] "Innovation" and
+ * "Methodology": FastMaskVim keeps only the visible tokens, addresses them by
+ * their grid position (sparse indexing) and forms each pooled token as the sum
+ * of the visible tokens of that grid row (POOL_W) or column (POOL_H) divided by
+ * the nominal width w (or height h), not by the number of visible tokens. The
+ * pooled scan is the one of oracle_forward; its output is repeated onto every
+ * visible token of the row (column) and gated with that token's z.
+ *
+ * Layouts: pos [batch][n_tok] grid positions (row * w + col) in [0, h*w);
+ * u, delta [Ki][batch][n_tok][D]; B, C [Ki][batch][n_tok][N]; z, y
+ * [batch][n_tok][D]; A, Dskip, bias as in oracle_forward. A row (column) with
+ * no visible token pools to zeros. Returns OR_EINVAL for a position outside
+ * the grid.
+ */
+int oracle_forward_masked(int kind, int h, int w, int batch, int n_tok, const int32_t* pos,
+                          int D, int N, const double* u, const double* delta, const double* A,
+                          const double* B, const double* C, const double* Dskip,
+                          const double* bias, const double* z, int delta_softplus,
+                          double merge_scale, int per_dir_inputs, int per_dir_params, int zoh,
+                          double* y, int nthreads)
+{
+    if (kind != OR_POOL_W && kind != OR_POOL_H) return OR_EINVAL;
+    if (h < 1 || w < 1 || batch < 0 || n_tok < 0 || D <= 0 || N <= 0) return OR_EINVAL;
+    for (int64_t i = 0; i < (int64_t)batch * n_tok; ++i)
+        if (pos[i] < 0 || (int64_t)pos[i] >= (int64_t)h * w) return OR_EINVAL;
+    if (batch == 0 || n_tok == 0) return OR_OK;
+
+    const int K = 2;
+    const int L = (kind == OR_POOL_W) ? h : w;      /* pooled sequence length */
+    const double nominal = (kind == OR_POOL_W) ? w : h;
+    const int64_t in_dir = per_dir_inputs ? (int64_t)batch * n_tok * D : 0;
+    const int64_t bc_dir = per_dir_inputs ? (int64_t)batch * n_tok * N : 0;
+    const int64_t a_dir = per_dir_params ? (int64_t)D * N : 0;
+    const int64_t v_dir = per_dir_params ? (int64_t)D : 0;
+    int failed = 0;
+    int64_t pairs = (int64_t)batch * D;
+    int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+
+#pragma omp parallel num_threads(nt) reduction(| : failed)
+    {
+        double* pu = (double*)malloc(sizeof(double) * L);
+        double* pd = (double*)malloc(sizeof(double) * L);
+        double* pB = (double*)malloc(sizeof(double) * (size_t)L * N);
+        double* pC = (double*)malloc(sizeof(double) * (size_t)L * N);
+        double* su = (double*)malloc(sizeof(double) * L);
+        double* sdt = (double*)malloc(sizeof(double) * L);
+        double* sB = (double*)malloc(sizeof(double) * (size_t)L * N);
+        double* sC = (double*)malloc(sizeof(double) * (size_t)L * N);
+        double* sy = (double*)malloc(sizeof(double) * L);
+        double* hs = (double*)malloc(sizeof(double) * N);
+        double* acc = (double*)malloc(sizeof(double) * L);
+        int bad = (!pu || !pd || !pB || !pC || !su || !sdt || !sB || !sC || !sy || !hs || !acc);
+        if (bad) failed |= 1;
+
+#pragma omp for schedule(static)
+        for (int64_t pr = 0; pr < pairs; ++pr) {
+            if (bad) continue;
+            int bi = (int)(pr / D);
+            int d = (int)(pr % D);
+            const int32_t* pb = pos + (int64_t)bi * n_tok;
+            for (int i = 0; i < L; ++i) acc[i] = 0.0;
+            for (int k = 0; k < K; ++k) {
+                const double* uk = u + k * in_dir + (int64_t)bi * n_tok * D;
+                const double* dk = delta + k * in_dir + (int64_t)bi * n_tok * D;
+                const double* Bk = B + k * bc_dir + (int64_t)bi * n_tok * N;
+                const double* Ck = C + k * bc_dir + (int64_t)bi * n_tok * N;
+                const double* Ak = A + k * a_dir + (int64_t)d * N;
+                double Dk = Dskip ? Dskip[k * v_dir + d] : 0.0;
+                double bk = bias ? bias[k * v_dir + d] : 0.0;
+                /* mask-aware aggregation: sum the visible tokens of each row
+                 * (column), then divide by the nominal width (height) */
+                for (int i = 0; i < L; ++i) {
+                    pu[i] = 0.0; pd[i] = 0.0;
+                    for (int n = 0; n < N; ++n) { pB[(int64_t)i * N + n] = 0.0; pC[(int64_t)i * N + n] = 0.0; }
+                }
+                for (int t = 0; t < n_tok; ++t) {
+                    int row = pb[t] / w, col = pb[t] % w;
+                    int i = (kind == OR_POOL_W) ? row : col;
+                    pu[i] += uk[(int64_t)t * D + d];
+                    pd[i] += dk[(int64_t)t * D + d];
+                    for (int n = 0; n < N; ++n) {
+                        pB[(int64_t)i * N + n] += Bk[(int64_t)t * N + n];
+                        pC[(int64_t)i * N + n] += Ck[(int64_t)t * N + n];
+                    }
+                }
+                /* direction 0 walks the pooled sequence forward, 1 reversed */
+                for (int t = 0; t < L; ++t) {
+                    int i = (k == 0) ? t : L - 1 - t;
+                    su[t] = pu[i] / nominal;
+                    double x = pd[i] / nominal + bk;
+                    sdt[t] = delta_softplus ? softplus(x) : x;
+                    for (int n = 0; n < N; ++n) {
+                        sB[(int64_t)t * N + n] = pB[(int64_t)i * N + n] / nominal;
+                        sC[(int64_t)t * N + n] = pC[(int64_t)i * N + n] / nominal;
+                    }
+                }
+                oracle_scan_sequence(L, N, su, sdt, Ak, sB, sC, Dk, zoh, hs, sy);
+                for (int t = 0; t < L; ++t) acc[(k == 0) ? t : L - 1 - t] += sy[t];
+            }
+            /* repeat onto the visible tokens, merge scale, gate */
+            double* yb = y + (int64_t)bi * n_tok * D;
+            const double* zb = z ? z + (int64_t)bi * n_tok * D : 0;
+            for (int t = 0; t < n_tok; ++t) {
+                int row = pb[t] / w, col = pb[t] % w;
+                double v = acc[(kind == OR_POOL_W) ? row : col] * merge_scale;
+                if (zb) v *= silu(zb[(int64_t)t * D + d]);
+                yb[(int64_t)t * D + d] = v;
+            }
+        }
+        free(pu); free(pd); free(pB); free(pC); free(su); free(sdt); free(sB); free(sC);
+        free(sy); free(hs); free(acc);
+    }
+    if (failed & 1) return OR_ENOMEM;
+    return OR_OK;
+}
+
 /* Number of OpenMP threads oracle_forward uses when nthreads <= 0. */
 int oracle_default_threads(void)
 {

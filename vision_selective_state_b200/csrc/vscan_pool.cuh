@@ -157,21 +157,38 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
                 }
             const T* xb = static_cast<const T*>(p.u) + k * p.in_dir + img * D + ch;
             const T* db = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + ch;
-            // x at sequence position sq (0 outside the sequence)
-            auto xat = [&](long long sq) {
-                if (!cval || sq < 0 || sq >= g_tok) return make_float4(0.f, 0.f, 0.f, 0.f);
-                const long long tok = pool_member(p.g, (int)(sq / cnt), (int)(sq % cnt));
-                return load4<T>(xb + tok * D);
+            // Sequence position sq <-> token: POOL_W walks the tokens in order
+            // (sq = token); POOL_H walks the columns (sq = col * h + row). The
+            // loads of a run advance one position at a time, so the token index
+            // is carried along instead of divided out.
+            const bool colmajor = p.g.kind == RK_POOL_H;
+            auto xat = [&](int tok, bool in) {
+                return (cval && in) ? load4<T>(xb + (long long)tok * D) : make_float4(0.f, 0.f, 0.f, 0.f);
             };
             for (int i = warp; i < Lp; i += PL_THREADS / 32) {
                 float4 au0 = make_float4(0.f, 0.f, 0.f, 0.f), au1 = au0, ad = au0;
-                const long long s0 = (long long)i * cnt + jb;
+                // position of the first window entry, s0 - 3, as (sequence index, row, col)
+                int sq = i * cnt + jb - 3;
+                int row, col;
+                if (colmajor) { col = (sq + 3) / p.g.h; row = (sq + 3) - col * p.g.h - 3; }
+                else { row = (sq + 3) / p.g.w; col = (sq + 3) - row * p.g.w - 3; }
+                // normalize a negative offset within the row (POOL_W) or column (POOL_H)
+                if (colmajor) { while (row < 0) { row += p.g.h; --col; } }
+                else { while (col < 0) { col += p.g.w; --row; } }
+                auto advance = [&]() {
+                    ++sq;
+                    if (colmajor) { if (++row == p.g.h) { row = 0; ++col; } }
+                    else { if (++col == p.g.w) { col = 0; ++row; } }
+                };
                 float4 win[7];  // x at s-3 .. s+3
 #pragma unroll
-                for (int m = 0; m < 6; ++m) win[m] = xat(s0 - 3 + m);
+                for (int m = 0; m < 6; ++m) {
+                    win[m] = xat(row * p.g.w + col, sq >= 0 && sq < g_tok);
+                    advance();
+                }
                 for (int j = jb; j < je; ++j) {
-                    const long long sq = (long long)i * cnt + j;
-                    win[6] = xat(sq + 3);
+                    win[6] = xat(row * p.g.w + col, sq < g_tok);  // position s + 3 (>= 0 here)
+                    advance();
                     const float4 dl = cval ? load4<T>(db + (long long)pool_member(p.g, i, j) * D)
                                            : make_float4(0.f, 0.f, 0.f, 0.f);
                     ad.x += dl.x; ad.y += dl.y; ad.z += dl.z; ad.w += dl.w;

@@ -520,18 +520,24 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
             yk[r] = fmaf(Dk, uj, yo[j * ST_CH + ce]);
             zz[r] = z_base ? to_float(st.z[j][ce]) : 0.f;
         }
+        // every row computes its value; only the stores are predicated
+        float o[RPL];
+#pragma unroll
+        for (int r = 0; r < RPL; ++r) {
+            o[r] = yk[r];
+            if constexpr (MODE == MODE_OWNER) {
+                o[r] *= p.merge_scale;
+                if (z_base) o[r] *= silu_f(zz[r]);
+            }
+        }
 #pragma unroll
         for (int r = 0; r < RPL; ++r) {
             const int j = j0 + (lane >> 3) + 4 * r;
-            if (pj[r] < 0) continue;
             if constexpr (MODE == MODE_OWNER) {
-                float o = yk[r] * p.merge_scale;
-                if (z_base) o *= silu_f(zz[r]);
-                store_elem<T>(y_base + pj[r] * D, o);
-            } else if (fin[r]) {
-                yo[j * ST_CH + ce] = yk[r];
+                if (pj[r] >= 0) store_elem<T>(y_base + pj[r] * D, o[r]);
             } else {
-                park(k)[pj[r] * D] = yk[r];
+                if (pj[r] >= 0 && fin[r]) yo[j * ST_CH + ce] = o[r];
+                if (pj[r] >= 0 && !fin[r]) park(k)[pj[r] * D] = o[r];
             }
         }
     };

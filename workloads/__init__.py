@@ -32,6 +32,8 @@ class Workload:
     seed: int
     gate: bool = True
     merge_scale: float = 1.0
+    conv: bool = False  # fused kernel-four causal Conv1d + SiLU on u (BIDIR, pooled routes)
+    zoh: bool = False   # zero-order-hold write term instead of Delta*B*u
 
     @property
     def tokens(self) -> int:
