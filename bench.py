@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--conv", action="store_true",
                    help="fuse the causal kernel-four Conv1d + SiLU into u (BIDIR and pooled routes)")
     p.add_argument("--zoh", action="store_true", help="zero-order-hold write term instead of Delta*B*u")
+    p.add_argument("--mask-keep", type=float, default=1.0,
+                   help="pooled workloads: keep this fraction of tokens (random mask per image, FastMaskVim)")
     return p.parse_args()
 
 
@@ -72,7 +74,7 @@ def workload_label(wls):
     w0 = wls[0]
     grids = "+".join(f"{w.h}x{w.w}" for w in wls)
     cls = "_cls" if w0.cls_pos >= 0 else ""
-    opt = ("_conv" if w0.conv else "") + ("_zoh" if w0.zoh else "")
+    opt = ("_conv" if w0.conv else "") + ("_zoh" if w0.zoh else "") + (f"_keep{w0.keep:g}" if w0.keep < 1 else "")
     return f"{w0.route}_{grids}{cls}_b{w0.batch}_d{w0.D}_n{w0.N}_{w0.dtype}{opt}"
 
 
@@ -81,7 +83,8 @@ def algorithmic_bytes(wl):
     eb = 2 if wl.dtype == "bf16" else 4
     per_token = (3 * wl.D + 2 * wl.N) * eb + wl.D * eb
     params = (wl.D * wl.N + 2 * wl.D + (5 * wl.D if wl.conv else 0)) * 4
-    return wl.batch * wl.tokens * per_token + params
+    pos = 4 * wl.batch * wl.visible if wl.keep < 1 else 0  # grid positions of the visible tokens
+    return wl.batch * wl.visible * per_token + params + pos
 
 
 def seq_geometry(wl):
@@ -244,14 +247,19 @@ def oracle_time(wls, channels, threads=0):
     import oracle
     total = 0.0
     for wl in wls:
-        x = workloads.draw(wl)
+        x = workloads.draw_masked(wl) if wl.keep < 1 else workloads.draw(wl)
         if wl.conv:
             x.update(workloads.draw_conv(wl))
         x = workloads.channel_slice(x, channels)
         t0 = time.perf_counter()
-        oracle.forward(wl.route, wl.h, wl.w, x["u"], x["delta"], x["A"], x["B"], x["C"], x["Dskip"],
-                       x["bias"], x["z"] if wl.gate else None, cls_pos=wl.cls_pos,
-                       conv_w=x.get("conv_w"), conv_b=x.get("conv_b"), zoh=wl.zoh, threads=threads)
+        if wl.keep < 1:
+            oracle.forward_masked(wl.route, wl.h, wl.w, x["pos"], x["u"], x["delta"], x["A"], x["B"], x["C"],
+                                  x["Dskip"], x["bias"], x["z"] if wl.gate else None, zoh=wl.zoh,
+                                  threads=threads)
+        else:
+            oracle.forward(wl.route, wl.h, wl.w, x["u"], x["delta"], x["A"], x["B"], x["C"], x["Dskip"],
+                           x["bias"], x["z"] if wl.gate else None, cls_pos=wl.cls_pos,
+                           conv_w=x.get("conv_w"), conv_b=x.get("conv_b"), zoh=wl.zoh, threads=threads)
         total += time.perf_counter() - t0
     return total
 
@@ -270,7 +278,7 @@ def cpu_baseline(wls, budget_s):
     while passes == 0 or t < budget_s:
         t += oracle_time(wls, chans)
         passes += 1
-    units = sum(w.batch * w.tokens * nch for w in wls) * passes
+    units = sum(w.batch * w.visible * nch for w in wls) * passes
     return {"value": units / t, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"all images and tokens of every grid, {nch} of {D} channels, "
                       f"{passes} pass(es), fp64",
@@ -294,7 +302,7 @@ def run_reference(args, wls):
     t = 0.0
     for _ in range(args.steps):
         t += oracle_time(wls, chans)
-    units = sum(w.batch * w.tokens * nch for w in wls) * args.steps
+    units = sum(w.batch * w.visible * nch for w in wls) * args.steps
     value = units / t
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
@@ -314,7 +322,7 @@ def config_block(wls, n):
     return {"workload": workload_label(wls), "route": w0.route,
             "grids": [f"{w.h}x{w.w}" for w in wls], "batch": w0.batch, "d_inner": w0.D,
             "d_state": w0.N, "io_dtype": w0.dtype, "gate": w0.gate, "merge_scale": w0.merge_scale,
-            "conv": w0.conv, "zoh": w0.zoh,
+            "conv": w0.conv, "zoh": w0.zoh, "mask_keep": w0.keep,
             "parallelism": f"replicas x{n} (one full workload per GPU, no collective)"}
 
 
@@ -340,7 +348,7 @@ def run_ours(args, wls):
     rot = min(rot, 8) if args.rotate <= 0 else args.rotate
     plans, host_sets, routes = [], [], []
     for wi, wl in enumerate(wls):
-        x = workloads.draw(replica(wl, rank))
+        x = workloads.draw_masked(replica(wl, rank)) if wl.keep < 1 else workloads.draw(replica(wl, rank))
         route = vs.Route(wl.route, wl.h, wl.w, wl.cls_pos)
         routes.append(route)
         dt = td[wl.dtype]
@@ -349,6 +357,8 @@ def run_ours(args, wls):
             x.update(workloads.draw_conv(wl))
         host.update({k: torch.from_numpy(np.ascontiguousarray(x[k], dtype=np.float32))
                      for k in ("A", "Dskip", "bias") + (("conv_w", "conv_b") if wl.conv else ())})
+        if wl.keep < 1:
+            host["pos"] = torch.from_numpy(x["pos"])
         host_sets.append(host)
         ws_bytes = vs.workspace_size(route, host["u"], host["B"])
         per = []
@@ -359,7 +369,7 @@ def run_ours(args, wls):
             per.append(vs.Plan(route, d["u"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], d["bias"],
                                d["z"] if wl.gate else None, out=out, workspace=ws,
                                merge_scale=wl.merge_scale, conv_w=d.get("conv_w"),
-                               conv_b=d.get("conv_b"), zoh=wl.zoh))
+                               conv_b=d.get("conv_b"), zoh=wl.zoh, token_pos=d.get("pos")))
         plans.append(per)
     launches_per_step = sum(per[0].kernels() for per in plans)
     knames = sorted({per[0].kernel_name() for per in plans})
@@ -448,12 +458,13 @@ def run_ours(args, wls):
             pin = {k: v.pin_memory() for k, v in host.items()}
             out = torch.empty_like(pin["u"]).pin_memory()
             nbytes = vs.host_buffer_size(route, pin["u"], pin["B"], z=wl.gate, conv_w=wl.conv,
-                                         conv_b=wl.conv)
+                                         conv_b=wl.conv, token_pos=wl.keep < 1)
             buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
             hplans.append(vs.HostPlan(route, pin["u"], pin["delta"], pin["A"], pin["B"], pin["C"],
                                       pin["Dskip"], pin["bias"], pin["z"] if wl.gate else None,
                                       out=out, device_buffer=buf, merge_scale=wl.merge_scale,
-                                      conv_w=pin.get("conv_w"), conv_b=pin.get("conv_b"), zoh=wl.zoh))
+                                      conv_w=pin.get("conv_w"), conv_b=pin.get("conv_b"), zoh=wl.zoh,
+                                      token_pos=pin.get("pos")))
             h2d += sum(v.numel() * v.element_size() for k, v in pin.items() if k != "z" or wl.gate)
             d2h += out.numel() * out.element_size()
         E = max(1, min(args.e2e_steps, K))
@@ -493,8 +504,10 @@ def main():
     wls = select(args.workload)
     if args.batch > 0:
         wls = [w.with_(batch=args.batch) for w in wls]
-    if args.conv or args.zoh:
-        wls = [w.with_(conv=args.conv, zoh=args.zoh) for w in wls]
+    if args.conv or args.zoh or args.mask_keep < 1:
+        wls = [w.with_(conv=args.conv, zoh=args.zoh, keep=args.mask_keep) for w in wls]
+        if args.mask_keep < 1 and (wls[0].route not in ("pool_w", "pool_h") or args.conv):
+            raise SystemExit("--mask-keep applies to the pooled workload (3), without --conv")
         if args.conv and wls[0].route in ("cross4", "atrous2"):
             raise SystemExit("--conv applies to the bidir and pooled workloads (0, 3, 4)")
     if args.impl == "reference":

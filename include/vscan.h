@@ -155,6 +155,22 @@ typedef struct vscan_args {
                                VSCAN_ERR_UNSUPPORTED (their pages convolve on the
                                2-D grid before routing).                          */
     const float* conv_b;    /* device, [Kp][D] float32, or NULL for no conv bias    */
+    const int32_t* token_pos;/* device, [batch][n_tokens] int32, or NULL (dense grid).
+                               POOL_W / POOL_H on a masked or irregular token set
+                               (FastMaskVim: "Fast Vision Mamba ...", Innovation
+                               and Methodology): the token arrays hold n_tokens
+                               visible tokens per image instead of h*w, and
+                               token_pos gives each one's grid position
+                               row * w + col in [0, h*w). Every pooled token is the
+                               sum of the visible tokens of its row (POOL_W) or
+                               column (POOL_H) divided by the nominal w (h); the
+                               pooled output goes back to every visible token of
+                               that row (column). A position outside the grid is
+                               ignored and its y written as 0 (not checked on the
+                               host). Other routes, or together with conv_w:
+                               VSCAN_ERR_UNSUPPORTED.                             */
+    int32_t n_tokens;       /* visible tokens per image with token_pos, else 0     */
+    int32_t reserved2;      /* must be 0                                            */
 } vscan_args;
 
 /*
@@ -285,7 +301,7 @@ const char* vscan_last_error(void);
 const char* vscan_status_string(int32_t status);
 
 /* Library ABI version; changes whenever vscan_args changes layout (2: flags,
- * conv_w and conv_b). */
+ * conv_w and conv_b; 3: token_pos and n_tokens). */
 int32_t vscan_abi_version(void);
 
 #ifdef __cplusplus

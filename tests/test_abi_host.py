@@ -36,10 +36,11 @@ def test_library_exports_every_declared_function():
 
 
 def test_struct_layout_matches_the_header():
-    # int32 x4, 6 pointers, 3 pointers, int32 x3, float, pointer, uint64, int32 x2, 2 pointers
-    assert ctypes.sizeof(abi.VscanArgs) == 16 + 48 + 24 + 12 + 4 + 8 + 8 + 8 + 16
+    # int32 x4, 6 pointers, 3 pointers, int32 x3, float, pointer, uint64, int32 x2, 3 pointers, int32 x2
+    assert ctypes.sizeof(abi.VscanArgs) == 16 + 48 + 24 + 12 + 4 + 8 + 8 + 8 + 24 + 8
     assert abi.VscanArgs.flags.offset == 124 and abi.VscanArgs.conv_w.offset == 128
-    assert abi.lib.vscan_abi_version() == abi.ABI_VERSION == 2
+    assert abi.VscanArgs.token_pos.offset == 144 and abi.VscanArgs.n_tokens.offset == 152
+    assert abi.lib.vscan_abi_version() == abi.ABI_VERSION == 3
 
 
 def test_status_strings():
@@ -218,3 +219,25 @@ def test_host_buffer_holds_the_convolution_parameters():
     a = _args(conv_w=1, conv_b=1)
     assert abi.lib.vscan_host_buffer_size(r.handle, ctypes.byref(a), ctypes.byref(n1)) == 0
     assert n1.value - n0.value == 2 * 256  # [D][4] and [D] floats, 256-byte rounded (D = 16)
+
+
+def test_masked_token_sets_are_checked_on_the_host():
+    fake = dict(u=0x1000, delta=0x2000, B=0x3000, C=0x4000, y=0x5000, A=0x6000)
+    for kind in ("bidir", "cross4", "atrous2"):
+        r = vs.Route(kind, 4, 4, 8 if kind == "bidir" else -1)
+        assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, token_pos=0x7000, n_tokens=3)), None) == -4
+    r = vs.Route("pool_w", 4, 4)
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, n_tokens=3)), None) == -1
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, token_pos=0x7000, n_tokens=-1)), None) == -1
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, token_pos=0x7000, n_tokens=3,
+                                                              conv_w=0x8000)), None) == -4
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, reserved2=1)), None) == -1
+    # accepted: the next failure is the missing workspace
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, token_pos=0x7000, n_tokens=3)), None) == -6
+    # the host buffer holds the visible tokens and their positions, not the grid
+    n_dense, n_mask = ctypes.c_uint64(), ctypes.c_uint64()
+    big = vs.Route("pool_w", 64, 64)
+    assert abi.lib.vscan_host_buffer_size(big.handle, ctypes.byref(_args()), ctypes.byref(n_dense)) == 0
+    a = _args(token_pos=1, n_tokens=1024)
+    assert abi.lib.vscan_host_buffer_size(big.handle, ctypes.byref(a), ctypes.byref(n_mask)) == 0
+    assert n_mask.value < n_dense.value

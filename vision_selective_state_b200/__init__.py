@@ -12,6 +12,9 @@ kernels of the library. Tensors are channels-last:
                      fuse each direction's causal kernel-four Conv1d + SiLU into u
                      (u then holds the convolution input); BIDIR and pooled routes
     zoh=True       : zero-order-hold write term instead of Delta*B*u
+    token_pos      : [batch, n] int32, optional (POOL_W / POOL_H): a masked token set
+                     (FastMaskVim); u, delta, B, C, z, y then hold the n visible tokens
+                     and token_pos their grid positions row * w + col
 
 u, delta, B, C, z and y share one dtype: torch.float32 or torch.bfloat16.
 """
@@ -87,7 +90,7 @@ def _ptr(t):
 
 def _args(route, u, delta, A, B, C, Dskip, delta_bias, z, y, delta_softplus, merge_scale,
           per_dir_inputs, per_dir_params, workspace, seq_chunks, conv_w=None, conv_b=None,
-          zoh=False):
+          zoh=False, token_pos=None):
     for name, t in (("u", u), ("delta", delta), ("B", B), ("C", C), ("z", z), ("y", y),
                     ("A", A), ("Dskip", Dskip), ("delta_bias", delta_bias), ("conv_w", conv_w),
                     ("conv_b", conv_b)):
@@ -100,7 +103,12 @@ def _args(route, u, delta, A, B, C, Dskip, delta_bias, z, y, delta_softplus, mer
     lead = 1 if per_dir_inputs else 0
     batch, tokens, D = u.shape[lead:]
     N = B.shape[-1]
-    if tokens != route.tokens:
+    if token_pos is not None:
+        if token_pos.dtype != torch.int32 or not token_pos.is_contiguous():
+            raise TypeError("token_pos must be a contiguous int32 tensor")
+        if tuple(token_pos.shape) != (batch, tokens):
+            raise ValueError(f"token_pos shape {tuple(token_pos.shape)} != {(batch, tokens)}")
+    elif tokens != route.tokens:
         raise ValueError(f"u has {tokens} tokens per image, the route has {route.tokens}")
     code = _dtype_code(u)
     for name, t in (("delta", delta), ("B", B), ("C", C), ("z", z), ("y", y)):
@@ -118,6 +126,8 @@ def _args(route, u, delta, A, B, C, Dskip, delta_bias, z, y, delta_softplus, mer
     a.seq_chunks = int(seq_chunks)
     a.flags = FLAG_ZOH if zoh else 0
     a.conv_w, a.conv_b = _ptr(conv_w), _ptr(conv_b)
+    a.token_pos = _ptr(token_pos)
+    a.n_tokens = tokens if token_pos is not None else 0
     return a
 
 
@@ -137,22 +147,24 @@ def workspace_size(route, u, B, *, per_dir_inputs=False, per_dir_params=False, *
 
 def forward(route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, delta_softplus=True,
             merge_scale=1.0, per_dir_inputs=False, per_dir_params=False, out=None, workspace=None,
-            seq_chunks=0, conv_w=None, conv_b=None, zoh=False, stream=None):
+            seq_chunks=0, conv_w=None, conv_b=None, zoh=False, token_pos=None, stream=None):
     """Routed selective scan on the GPU (vscan_forward). Returns y [batch, tokens, D]."""
     lead = 1 if per_dir_inputs else 0
     if out is None:
         out = torch.empty(u.shape[lead:], dtype=u.dtype, device=u.device)
+    if token_pos is not None and token_pos.shape[-1] == 0:
+        return out  # an empty token set: nothing to compute (and no data pointers to pass)
     if workspace is None:
         need = workspace_size(route, u, B, per_dir_inputs=per_dir_inputs, per_dir_params=per_dir_params)
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=u.device)
     a = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus, merge_scale,
-              per_dir_inputs, per_dir_params, workspace, seq_chunks, conv_w, conv_b, zoh)
+              per_dir_inputs, per_dir_params, workspace, seq_chunks, conv_w, conv_b, zoh, token_pos)
     check(lib.vscan_forward(route.handle, ctypes.byref(a), _stream(stream, u.device)))
     return out
 
 
 def host_buffer_size(route, u, B, *, z=True, Dskip=True, delta_bias=True, per_dir_inputs=False,
-                     per_dir_params=False, conv_w=False, conv_b=False):
+                     per_dir_params=False, conv_w=False, conv_b=False, token_pos=False):
     """Bytes of device memory forward_host needs (host-only query)."""
     lead = 1 if per_dir_inputs else 0
     a = VscanArgs()
@@ -167,6 +179,9 @@ def host_buffer_size(route, u, B, *, z=True, Dskip=True, delta_bias=True, per_di
     a.delta_bias = ctypes.c_void_p(1) if delta_bias else None
     a.conv_w = ctypes.c_void_p(1) if conv_w else None
     a.conv_b = ctypes.c_void_p(1) if conv_b else None
+    if token_pos:
+        a.token_pos = ctypes.c_void_p(1)
+        a.n_tokens = u.shape[lead + 1]
     n = ctypes.c_uint64()
     check(lib.vscan_host_buffer_size(route.handle, ctypes.byref(a), ctypes.byref(n)))
     return n.value
@@ -174,17 +189,17 @@ def host_buffer_size(route, u, B, *, z=True, Dskip=True, delta_bias=True, per_di
 
 def forward_host(route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, out,
                  device_buffer, delta_softplus=True, merge_scale=1.0, per_dir_inputs=False,
-                 per_dir_params=False, conv_w=None, conv_b=None, zoh=False, stream=None):
+                 per_dir_params=False, conv_w=None, conv_b=None, zoh=False, token_pos=None, stream=None):
     """End-to-end call with host (CPU, ideally pinned) tensors (vscan_forward_host).
 
     Enqueues the host-to-device copies, the scan and the copy of y into `out`
     (a host tensor) on the stream; synchronize the stream before reading `out`.
     """
-    for t in (u, delta, A, B, C, Dskip, delta_bias, z, out, conv_w, conv_b):
+    for t in (u, delta, A, B, C, Dskip, delta_bias, z, out, conv_w, conv_b, token_pos):
         if t is not None and t.is_cuda:
             raise ValueError("forward_host takes host tensors")
     a = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus, merge_scale,
-              per_dir_inputs, per_dir_params, None, 0, conv_w, conv_b, zoh)
+              per_dir_inputs, per_dir_params, None, 0, conv_w, conv_b, zoh, token_pos)
     nbytes = device_buffer.numel() * device_buffer.element_size()
     check(lib.vscan_forward_host(route.handle, ctypes.byref(a), ctypes.c_void_p(device_buffer.data_ptr()),
                                  nbytes, _stream(stream, device_buffer.device)))
@@ -199,13 +214,14 @@ class Plan:
 
     def __init__(self, route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, out,
                  workspace, delta_softplus=True, merge_scale=1.0, per_dir_inputs=False,
-                 per_dir_params=False, seq_chunks=0, conv_w=None, conv_b=None, zoh=False):
+                 per_dir_params=False, seq_chunks=0, conv_w=None, conv_b=None, zoh=False,
+                 token_pos=None):
         self.route = route
-        self._keep = (u, delta, A, B, C, Dskip, delta_bias, z, out, workspace, conv_w, conv_b)
+        self._keep = (u, delta, A, B, C, Dskip, delta_bias, z, out, workspace, conv_w, conv_b, token_pos)
         self.out = out
         self.args = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus,
                           merge_scale, per_dir_inputs, per_dir_params, workspace, seq_chunks,
-                          conv_w, conv_b, zoh)
+                          conv_w, conv_b, zoh, token_pos)
         self._ref = ctypes.byref(self.args)
 
     def run(self, stream):
@@ -233,15 +249,16 @@ class HostPlan:
 
     def __init__(self, route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, out,
                  device_buffer, delta_softplus=True, merge_scale=1.0, per_dir_inputs=False,
-                 per_dir_params=False, conv_w=None, conv_b=None, zoh=False):
-        for t in (u, delta, A, B, C, Dskip, delta_bias, z, out, conv_w, conv_b):
+                 per_dir_params=False, conv_w=None, conv_b=None, zoh=False, token_pos=None):
+        for t in (u, delta, A, B, C, Dskip, delta_bias, z, out, conv_w, conv_b, token_pos):
             if t is not None and t.is_cuda:
                 raise ValueError("HostPlan takes host tensors")
         self.route = route
-        self._keep = (u, delta, A, B, C, Dskip, delta_bias, z, out, device_buffer, conv_w, conv_b)
+        self._keep = (u, delta, A, B, C, Dskip, delta_bias, z, out, device_buffer, conv_w, conv_b, token_pos)
         self.out = out
         self.args = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus,
-                          merge_scale, per_dir_inputs, per_dir_params, None, 0, conv_w, conv_b, zoh)
+                          merge_scale, per_dir_inputs, per_dir_params, None, 0, conv_w, conv_b, zoh,
+                          token_pos)
         self._ref = ctypes.byref(self.args)
         self._buf = ctypes.c_void_p(device_buffer.data_ptr())
         self._nbytes = device_buffer.numel() * device_buffer.element_size()

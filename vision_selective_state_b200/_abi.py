@@ -21,7 +21,7 @@ STATUS = {
 }
 ROUTES = {"bidir": 0, "cross4": 1, "atrous2": 2, "pool_w": 3, "pool_h": 4}
 F32, BF16 = 0, 1
-ABI_VERSION = 2
+ABI_VERSION = 3
 FLAG_ZOH = 1
 
 
@@ -52,6 +52,9 @@ class VscanArgs(ctypes.Structure):
         ("flags", ctypes.c_int32),
         ("conv_w", ctypes.c_void_p),
         ("conv_b", ctypes.c_void_p),
+        ("token_pos", ctypes.c_void_p),
+        ("n_tokens", ctypes.c_int32),
+        ("reserved2", ctypes.c_int32),
     ]
 
 

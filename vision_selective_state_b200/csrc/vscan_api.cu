@@ -24,7 +24,7 @@ struct vscan_route {
 
 namespace {
 
-constexpr int32_t kAbiVersion = 2;
+constexpr int32_t kAbiVersion = 3;
 constexpr size_t kMaxSmem = 200 * 1024;  // dynamic shared memory the kernels may ask for
 thread_local std::string g_last_error;
 
@@ -52,6 +52,10 @@ size_t elem_bytes(int32_t dtype) { return dtype == VSCAN_BF16 ? 2 : 4; }
 
 bool is_pool(int kind) { return kind == vscan::RK_POOL_W || kind == vscan::RK_POOL_H; }
 
+// Tokens per image in the token arrays: the visible ones of a masked set, else
+// the route's (grid, plus CLS for BIDIR).
+int tokens_of(const vscan_route* r, const vscan_args* a) { return a->token_pos ? a->n_tokens : r->g.tokens; }
+
 size_t resident_bytes(const vscan_route* r, const vscan_args* a)
 {
     const int Ki = a->per_dir_inputs ? r->g.K : 1;
@@ -67,6 +71,16 @@ vscan_status check_shape(const vscan_route* r, const vscan_args* a)
     if (a->flags & ~int32_t(VSCAN_FLAG_ZOH))
         return fail(VSCAN_ERR_INVALID_ARGUMENT, "unknown bits in args.flags 0x%x", (unsigned)a->flags);
     if (a->conv_b && !a->conv_w) return fail(VSCAN_ERR_INVALID_ARGUMENT, "conv_b given without conv_w");
+    if (a->reserved2 != 0) return fail(VSCAN_ERR_INVALID_ARGUMENT, "args.reserved2 must be 0");
+    if (a->token_pos) {
+        if (!is_pool(r->g.kind))
+            return fail(VSCAN_ERR_UNSUPPORTED, "a masked token set (token_pos) needs POOL_W or POOL_H");
+        if (a->conv_w)
+            return fail(VSCAN_ERR_UNSUPPORTED, "no convolution order is defined on a masked token set");
+        if (a->n_tokens < 0) return fail(VSCAN_ERR_INVALID_ARGUMENT, "n_tokens %d < 0", a->n_tokens);
+    } else if (a->n_tokens != 0) {
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "n_tokens is set without token_pos");
+    }
     if (a->conv_w && (r->g.kind == vscan::RK_CROSS4 || r->g.kind == vscan::RK_ATROUS2))
         return fail(VSCAN_ERR_UNSUPPORTED, "the fused convolution is defined for BIDIR and the pooled routes");
     if (a->dtype != VSCAN_F32 && a->dtype != VSCAN_BF16)
@@ -89,7 +103,7 @@ vscan_status check_shape(const vscan_route* r, const vscan_args* a)
         a->seq_chunks != 8)
         return fail(VSCAN_ERR_INVALID_ARGUMENT, "seq_chunks %d is not 0, 1, 2, 4 or 8", a->seq_chunks);
     if (a->batch > 65535) return fail(VSCAN_ERR_UNSUPPORTED, "batch %d > 65535", a->batch);
-    if ((long long)r->g.tokens * a->channels >= (1LL << 31))
+    if ((long long)tokens_of(r, a) * a->channels >= (1LL << 31))
         return fail(VSCAN_ERR_UNSUPPORTED, "tokens x channels of one image must be below 2^31");
     if (is_pool(r->g.kind)) {
         const int Ki = a->per_dir_inputs ? 2 : 1;
@@ -242,10 +256,20 @@ cudaError_t launch_resident(const vscan::ScanParams& p, int nc, int fl, cudaStre
 }
 
 template <typename T, int FL>
-cudaError_t launch_pool_fl(const vscan::PoolParams& p, cudaStream_t s)
+cudaError_t launch_pool_fl(const vscan::PoolParams& p, cudaStream_t s, size_t ws_bytes)
 {
-    const dim3 g1(p.g.L, p.batch, p.Ki);
-    vscan::pool_bc_kernel<T><<<g1, 128, 0, s>>>(p);
+    if constexpr ((FL & vscan::FL_MASK) != 0) {
+        // B and C sums are added into the zeroed workspace (pB and pC)
+        cudaError_t e = cudaMemsetAsync(p.pB, 0, ws_bytes, s);
+        if (e != cudaSuccess) return e;
+        if (p.n_tok > 0) {
+            const dim3 g1((unsigned)(((long long)p.n_tok * 16 + 255) / 256), p.batch, p.Ki);
+            vscan::pool_bc_masked_kernel<T><<<g1, 256, 0, s>>>(p);
+        }
+    } else {
+        const dim3 g1(p.g.L, p.batch, p.Ki);
+        vscan::pool_bc_kernel<T><<<g1, 128, 0, s>>>(p);
+    }
     const size_t smem = vscan::pool_scan_smem_bytes(p.Ki, p.g.L, (FL & vscan::FL_CONV) != 0);
     cudaError_t e = cudaFuncSetAttribute(vscan::pool_scan_kernel<T, FL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
@@ -256,14 +280,16 @@ cudaError_t launch_pool_fl(const vscan::PoolParams& p, cudaStream_t s)
 }
 
 template <typename T>
-cudaError_t launch_pool(const vscan::PoolParams& p, int fl, cudaStream_t s)
+cudaError_t launch_pool(const vscan::PoolParams& p, int fl, cudaStream_t s, size_t ws_bytes)
 {
     using namespace vscan;
     switch (fl) {
-    case FL_ZOH: return launch_pool_fl<T, FL_ZOH>(p, s);
-    case FL_CONV: return launch_pool_fl<T, FL_CONV>(p, s);
-    case FL_ZOH | FL_CONV: return launch_pool_fl<T, FL_ZOH | FL_CONV>(p, s);
-    default: return launch_pool_fl<T, 0>(p, s);
+    case FL_ZOH: return launch_pool_fl<T, FL_ZOH>(p, s, ws_bytes);
+    case FL_CONV: return launch_pool_fl<T, FL_CONV>(p, s, ws_bytes);
+    case FL_ZOH | FL_CONV: return launch_pool_fl<T, FL_ZOH | FL_CONV>(p, s, ws_bytes);
+    case FL_MASK: return launch_pool_fl<T, FL_MASK>(p, s, ws_bytes);
+    case FL_MASK | FL_ZOH: return launch_pool_fl<T, FL_MASK | FL_ZOH>(p, s, ws_bytes);
+    default: return launch_pool_fl<T, 0>(p, s, ws_bytes);
     }
 }
 
@@ -271,8 +297,9 @@ template <typename T>
 vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s)
 {
     const vscan::RouteGeom& g = r->g;
-    const long long plane = (long long)a->batch * g.tokens;
-    const int fl = ((a->flags & VSCAN_FLAG_ZOH) ? vscan::FL_ZOH : 0) | (a->conv_w ? vscan::FL_CONV : 0);
+    const long long plane = (long long)a->batch * tokens_of(r, a);
+    const int fl = ((a->flags & VSCAN_FLAG_ZOH) ? vscan::FL_ZOH : 0) | (a->conv_w ? vscan::FL_CONV : 0) |
+                   (a->token_pos ? vscan::FL_MASK : 0);
     if (is_pool(g.kind)) {
         vscan::PoolParams p{};
         p.g = g;
@@ -290,7 +317,9 @@ vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s)
         p.pB = static_cast<float*>(a->workspace);
         p.pC = reinterpret_cast<float*>(static_cast<char*>(a->workspace) + half);
         p.conv_w = a->conv_w; p.conv_b = a->conv_b;
-        cudaError_t e = launch_pool<T>(p, fl, s);
+        p.pos = a->token_pos;
+        p.n_tok = tokens_of(r, a);
+        cudaError_t e = launch_pool<T>(p, fl, s, workspace_need(r, a));
         if (e != cudaSuccess) return cuda_fail(e, "configuring the pooled-scan kernel");
     } else {
         vscan::ScanParams p{};
@@ -354,7 +383,7 @@ __global__ void route_map_kernel(vscan::RouteGeom g, int32_t* out)
 }
 
 struct HostLayout {
-    size_t u, delta, B, C, z, y, A, Dskip, bias, conv_w, conv_b, ws, total;
+    size_t u, delta, B, C, z, y, A, Dskip, bias, conv_w, conv_b, pos, ws, total;
 };
 
 HostLayout host_layout(const vscan_route* r, const vscan_args* a)
@@ -363,7 +392,7 @@ HostLayout host_layout(const vscan_route* r, const vscan_args* a)
     const size_t eb = elem_bytes(a->dtype);
     const size_t Ki = a->per_dir_inputs ? g.K : 1;
     const size_t Kp = a->per_dir_params ? g.K : 1;
-    const size_t plane = (size_t)a->batch * g.tokens;
+    const size_t plane = (size_t)a->batch * tokens_of(r, a);
     HostLayout L{};
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off += round256(bytes); return o; };
@@ -378,6 +407,7 @@ HostLayout host_layout(const vscan_route* r, const vscan_args* a)
     L.bias = take(a->delta_bias ? Kp * a->channels * sizeof(float) : 0);
     L.conv_w = take(a->conv_w ? Kp * a->channels * 4 * sizeof(float) : 0);
     L.conv_b = take(a->conv_b ? Kp * a->channels * sizeof(float) : 0);
+    L.pos = take(a->token_pos ? plane * sizeof(int32_t) : 0);
     L.ws = take(workspace_need(r, a));
     L.total = off;
     return L;
@@ -549,7 +579,7 @@ vscan_status vscan_forward_host(const vscan_route* r, const vscan_args* ha, void
     const size_t eb = elem_bytes(ha->dtype);
     const size_t Ki = ha->per_dir_inputs ? g.K : 1;
     const size_t Kp = ha->per_dir_params ? g.K : 1;
-    const size_t plane = (size_t)ha->batch * g.tokens;
+    const size_t plane = (size_t)ha->batch * tokens_of(r, ha);
 
     vscan_args da = *ha;
     da.u = base + L.u;
@@ -563,6 +593,7 @@ vscan_status vscan_forward_host(const vscan_route* r, const vscan_args* ha, void
     da.delta_bias = ha->delta_bias ? reinterpret_cast<const float*>(base + L.bias) : nullptr;
     da.conv_w = ha->conv_w ? reinterpret_cast<const float*>(base + L.conv_w) : nullptr;
     da.conv_b = ha->conv_b ? reinterpret_cast<const float*>(base + L.conv_b) : nullptr;
+    da.token_pos = ha->token_pos ? reinterpret_cast<const int32_t*>(base + L.pos) : nullptr;
     da.workspace = base + L.ws;
     da.workspace_bytes = workspace_need(r, ha);
 
@@ -578,6 +609,7 @@ vscan_status vscan_forward_host(const vscan_route* r, const vscan_args* ha, void
         {const_cast<float*>(da.delta_bias), ha->delta_bias, ha->delta_bias ? Kp * ha->channels * sizeof(float) : 0},
         {const_cast<float*>(da.conv_w), ha->conv_w, ha->conv_w ? Kp * ha->channels * 4 * sizeof(float) : 0},
         {const_cast<float*>(da.conv_b), ha->conv_b, ha->conv_b ? Kp * ha->channels * sizeof(float) : 0},
+        {const_cast<int32_t*>(da.token_pos), ha->token_pos, ha->token_pos ? plane * sizeof(int32_t) : 0},
     };
     for (const Copy& c : in) {
         if (c.bytes == 0) continue;

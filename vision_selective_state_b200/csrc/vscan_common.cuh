@@ -82,8 +82,9 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 v
 }
 
 // Optional steps of the scan, as kernel template flags: the zero-order-hold
-// write term and the fused causal convolution of u.
-enum ScanFlags : int { FL_ZOH = 1, FL_CONV = 2 };
+// write term, the fused causal convolution of u, and (pooled routes) a masked
+// token set addressed by grid position.
+enum ScanFlags : int { FL_ZOH = 1, FL_CONV = 2, FL_MASK = 4 };
 
 // ---- discretization ---------------------------------------------------------
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32). The retention

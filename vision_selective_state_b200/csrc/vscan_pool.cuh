@@ -24,6 +24,15 @@
 //            backward branch convolves the reversed sequence). The sequence is
 //            the row-major (POOL_W) or column-major (POOL_H) token order, so the
 //            members of one pooled index are consecutive in it.
+//   FL_MASK  masked token set (FastMaskVim, "Fast Vision Mamba ...", Innovation
+//            and Methodology: sparse indexing, mask-aware aggregation, row sums
+//            normalized by the nominal width). The token arrays hold n_tok
+//            visible tokens with their grid positions pos[]; pooling adds every
+//            visible token into its row (column) with shared-memory (u, Delta)
+//            and global (B, C; pool_bc_masked_kernel) float atomics, and the sums
+//            are divided by the nominal w (h). The repeat writes each visible
+//            token from its row (column). Positions outside the grid are skipped
+//            and their y written as 0.
 #pragma once
 
 #include "vscan_common.cuh"
@@ -53,7 +62,35 @@ struct PoolParams {
     float* pC;  // [Ki][batch][Lp][N]
     const float* conv_w;  // FL_CONV: [Kp][D][4]
     const float* conv_b;  // FL_CONV: [Kp][D] (nullable)
+    const int* pos;       // FL_MASK: [batch][n_tok] grid positions
+    int n_tok;            // tokens per image in the token arrays (h*w when dense)
 };
+
+// FL_MASK: pooled index of grid position q, or -1 outside the grid.
+__device__ __forceinline__ int pool_index(const RouteGeom& g, int q)
+{
+    if (q < 0 || q >= g.h * g.w) return -1;
+    const int r = q / g.w;
+    return (g.kind == RK_POOL_W) ? r : q - r * g.w;
+}
+
+// FL_MASK: sums of B and C over the visible tokens of every pooled index, added
+// with global float atomics into the zeroed workspace ([Ki][batch][Lp][N]); the
+// scan divides them by the nominal width. Grid (ceil(n_tok * 16 / 256), batch, Ki).
+template <typename T>
+__global__ void __launch_bounds__(256) pool_bc_masked_kernel(const PoolParams p)
+{
+    const int b = blockIdx.y, k = blockIdx.z;
+    const long long e = (long long)blockIdx.x * 256 + threadIdx.x;
+    const int t = (int)(e >> 4), n = (int)(e & 15);
+    if (t >= p.n_tok || n >= p.N) return;
+    const int i = pool_index(p.g, __ldg(p.pos + (long long)b * p.n_tok + t));
+    if (i < 0) return;
+    const long long src = k * p.bc_dir + ((long long)b * p.n_tok + t) * p.N + n;
+    const long long dst = (((long long)k * p.batch + b) * p.g.L + i) * p.N + n;
+    atomicAdd(p.pB + dst, load_elem<T>(static_cast<const T*>(p.B) + src));
+    atomicAdd(p.pC + dst, load_elem<T>(static_cast<const T*>(p.C) + src));
+}
 
 constexpr int PL_CH = 32;       // channels per CTA
 constexpr int PL_THREADS = 256;
@@ -115,6 +152,8 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
 {
     constexpr bool ZOH = (FL & FL_ZOH) != 0;
     constexpr bool CONV = (FL & FL_CONV) != 0;
+    constexpr bool MASK = (FL & FL_MASK) != 0;
+    static_assert(!(CONV && MASK), "no convolution order is defined on a masked token set");
     extern __shared__ __align__(16) float psm[];
     const int Lp = p.g.L;
     const int Ki = p.Ki;
@@ -127,7 +166,7 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
     const int b = blockIdx.y;
     const int c0 = blockIdx.x * PL_CH;
     const int D = p.D, N = p.N;
-    const int tokens = p.g.tokens;
+    const int tokens = p.n_tok;
     const long long img = (long long)b * tokens;
     const int cnt = (p.g.kind == RK_POOL_W) ? p.g.w : p.g.h;
     const float inv_cnt = 1.0f / (float)cnt;
@@ -241,8 +280,35 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
         }
     }
 
+    // ---- phase 1 (FL_MASK): add every visible token into its pooled index -----
+    if constexpr (MASK) {
+        for (int e = tid; e < (Ki + Ku) * Lp * PL_CH; e += PL_THREADS) psm[e] = 0.f;
+        __syncthreads();
+        const int q = lane & 7;        // channel quad of the tile
+        const int ch = c0 + 4 * q;
+        if (ch < D) {
+            const int* pb = p.pos + (long long)b * tokens;
+            for (int k = 0; k < Ki; ++k) {
+                const T* ub = static_cast<const T*>(p.u) + k * p.in_dir + img * D + ch;
+                const T* db = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + ch;
+                for (int t = tid >> 3; t < tokens; t += PL_THREADS / 8) {
+                    const int i = pool_index(p.g, __ldg(pb + t));
+                    if (i < 0) continue;
+                    const float4 u4 = load4<T>(ub + (long long)t * D);
+                    const float4 d4 = load4<T>(db + (long long)t * D);
+                    float* du_ = pu + ((size_t)k * Lp + i) * PL_CH + 4 * q;
+                    float* dd_ = pd + ((size_t)k * Lp + i) * PL_CH + 4 * q;
+                    atomicAdd(du_ + 0, u4.x); atomicAdd(du_ + 1, u4.y); atomicAdd(du_ + 2, u4.z); atomicAdd(du_ + 3, u4.w);
+                    atomicAdd(dd_ + 0, d4.x); atomicAdd(dd_ + 1, d4.y); atomicAdd(dd_ + 2, d4.z); atomicAdd(dd_ + 3, d4.w);
+                }
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < (Ki + Ku) * Lp * PL_CH; e += PL_THREADS) psm[e] *= inv_cnt;
+    }
+
     // ---- phase 1: mean-pool u and raw Delta of the channel tile ---------------
-    if constexpr (!CONV) {
+    if constexpr (!CONV && !MASK) {
         const int jl = lane >> 3;   // token sub-lane 0..3
         const int q = lane & 7;     // channel quad of the tile
         const int ch = c0 + 4 * q;
@@ -343,6 +409,7 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
                         const int n = 4 * grp + s;
                         bv[s] = n < N ? __ldg(pBk + (size_t)i * N + n) : 0.f;
                         cv[s] = n < N ? __ldg(pCk + (size_t)i * N + n) : 0.f;
+                        if constexpr (MASK) { bv[s] *= inv_cnt; cv[s] *= inv_cnt; }  // sums -> means
                     }
                     const float rd = ZOH ? fast_rcp(dsp) : 0.f;
 #pragma unroll
@@ -401,9 +468,18 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
                 for (int v = 0; v < U; ++v) {
                     const int tok = tok0 + 32 * v;
                     if (tok >= tokens) break;
-                    const int r = tok / p.g.w;
-                    const int col = tok - r * p.g.w;
-                    const int i = (p.g.kind == RK_POOL_W) ? r : col;
+                    int i;
+                    if constexpr (MASK) {
+                        i = pool_index(p.g, __ldg(p.pos + (long long)b * tokens + tok));
+                        if (i < 0) {  // outside the grid: written as 0
+                            store4<T>(yb + (long long)tok * D, make_float4(0.f, 0.f, 0.f, 0.f));
+                            continue;
+                        }
+                    } else {
+                        const int r = tok / p.g.w;
+                        const int col = tok - r * p.g.w;
+                        i = (p.g.kind == RK_POOL_W) ? r : col;
+                    }
                     const float4 f = *reinterpret_cast<const float4*>(Y0 + (size_t)i * PL_CH + 4 * q);
                     const float4 g = *reinterpret_cast<const float4*>(Y1 + (size_t)i * PL_CH + 4 * q);
                     float4 o = make_float4((f.x + g.x) * scale, (f.y + g.y) * scale,

@@ -34,6 +34,7 @@ class Workload:
     merge_scale: float = 1.0
     conv: bool = False  # fused kernel-four causal Conv1d + SiLU on u (BIDIR, pooled routes)
     zoh: bool = False   # zero-order-hold write term instead of Delta*B*u
+    keep: float = 1.0   # pooled routes: fraction of visible tokens (masked set) when < 1
 
     @property
     def tokens(self) -> int:
@@ -41,9 +42,14 @@ class Workload:
         return self.h * self.w + (1 if self.cls_pos >= 0 else 0)
 
     @property
+    def visible(self) -> int:
+        """Tokens per image in the token arrays: all of them, or the visible ones of a mask."""
+        return self.tokens if self.keep >= 1.0 else max(1, int(round(self.keep * self.h * self.w)))
+
+    @property
     def token_channels(self) -> int:
-        """Units of the throughput metric: batch * real tokens * channels."""
-        return self.batch * self.tokens * self.D
+        """Units of the throughput metric: batch * real (visible) tokens * channels."""
+        return self.batch * self.visible * self.D
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -141,6 +147,27 @@ def draw_conv(wl: Workload, *, per_dir_params: bool = False) -> dict:
     conv_w = rng.standard_normal(plead + (wl.D, 4), dtype=f32) * f32(0.5)
     conv_b = rng.standard_normal(plead + (wl.D,), dtype=f32) * f32(0.1)
     return dict(conv_w=conv_w, conv_b=conv_b)
+
+
+def mask_positions(wl: Workload) -> np.ndarray:
+    """[batch, visible] int32 sorted grid positions of a random mask per image
+    (MAE-style uniform sampling without replacement), from its own seed stream."""
+    rng = np.random.default_rng(wl.seed + 104729)
+    g = wl.h * wl.w
+    return np.stack([np.sort(rng.choice(g, wl.visible, replace=False))
+                     for _ in range(wl.batch)]).astype(np.int32)
+
+
+def draw_masked(wl: Workload) -> dict:
+    """Inputs of a masked pooled workload: draw() restricted to the visible tokens
+    of mask_positions(wl), plus "pos"."""
+    x = draw(wl)
+    pos = mask_positions(wl)
+    out = dict(x)
+    for key in ("u", "z", "delta", "B", "C"):
+        out[key] = np.ascontiguousarray(np.stack([x[key][i, pos[i]] for i in range(wl.batch)]))
+    out["pos"] = pos
+    return out
 
 
 def channel_slice(inputs: dict, channels, per_dir_params: bool = False) -> dict:
