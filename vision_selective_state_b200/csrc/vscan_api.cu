@@ -263,7 +263,8 @@ cudaError_t launch_pool_fl(const vscan::PoolParams& p, cudaStream_t s, size_t ws
         cudaError_t e = cudaMemsetAsync(p.pB, 0, ws_bytes, s);
         if (e != cudaSuccess) return e;
         if (p.n_tok > 0) {
-            const dim3 g1((unsigned)(((long long)p.n_tok * 16 + 255) / 256), p.batch, p.Ki);
+            constexpr int per_cta = 16 * vscan::PB_RUN;  // tokens of one CTA
+            const dim3 g1((unsigned)((p.n_tok + per_cta - 1) / per_cta), p.batch, p.Ki);
             vscan::pool_bc_masked_kernel<T><<<g1, 256, 0, s>>>(p);
         }
     } else {

@@ -75,21 +75,61 @@ __device__ __forceinline__ int pool_index(const RouteGeom& g, int q)
 }
 
 // FL_MASK: sums of B and C over the visible tokens of every pooled index, added
-// with global float atomics into the zeroed workspace ([Ki][batch][Lp][N]); the
-// scan divides them by the nominal width. Grid (ceil(n_tok * 16 / 256), batch, Ki).
+// into the zeroed workspace ([Ki][batch][Lp][N]) with global float atomics; the
+// scan divides them by the nominal width. Grid (splits, batch, Ki), 256
+// threads: thread (range r = tid >> 4, state n = tid & 15) walks a contiguous
+// range of PB_RUN tokens, sums consecutive tokens of one pooled index in
+// registers (one row of a sorted mask) and adds each run once.
+constexpr int PB_RUN = 16;
 template <typename T>
 __global__ void __launch_bounds__(256) pool_bc_masked_kernel(const PoolParams p)
 {
-    const int b = blockIdx.y, k = blockIdx.z;
-    const long long e = (long long)blockIdx.x * 256 + threadIdx.x;
-    const int t = (int)(e >> 4), n = (int)(e & 15);
-    if (t >= p.n_tok || n >= p.N) return;
-    const int i = pool_index(p.g, __ldg(p.pos + (long long)b * p.n_tok + t));
-    if (i < 0) return;
-    const long long src = k * p.bc_dir + ((long long)b * p.n_tok + t) * p.N + n;
-    const long long dst = (((long long)k * p.batch + b) * p.g.L + i) * p.N + n;
-    atomicAdd(p.pB + dst, load_elem<T>(static_cast<const T*>(p.B) + src));
-    atomicAdd(p.pC + dst, load_elem<T>(static_cast<const T*>(p.C) + src));
+    const int b = blockIdx.y, k = blockIdx.z, N = p.N;
+    const int n = threadIdx.x & 15;
+    const long long r = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
+    const long long tb = r * PB_RUN;
+    if (n >= N || tb >= p.n_tok) return;
+    const int te = (int)min((long long)p.n_tok, tb + PB_RUN);
+    const int* pb = p.pos + (long long)b * p.n_tok;
+    const T* Bb = static_cast<const T*>(p.B) + k * p.bc_dir + (long long)b * p.n_tok * N + n;
+    const T* Cb = static_cast<const T*>(p.C) + k * p.bc_dir + (long long)b * p.n_tok * N + n;
+    float* oB = p.pB + ((long long)k * p.batch + b) * p.g.L * N + n;
+    float* oC = p.pC + ((long long)k * p.batch + b) * p.g.L * N + n;
+    int cur = -1;
+    float sb = 0.f, sc = 0.f;
+    constexpr int U = 8;
+    for (int t0 = (int)tb; t0 < te; t0 += U) {
+        int ix[U];
+        float vb[U], vc[U];
+#pragma unroll
+        for (int v = 0; v < U; ++v) {  // loads first
+            const int t = t0 + v;
+            const bool in = t < te;
+            ix[v] = in ? __ldg(pb + t) : -1;
+            vb[v] = in ? load_elem<T>(Bb + (long long)t * N) : 0.f;
+            vc[v] = in ? load_elem<T>(Cb + (long long)t * N) : 0.f;
+        }
+#pragma unroll
+        for (int v = 0; v < U; ++v) {
+            const int i = pool_index(p.g, ix[v]);
+            if (i < 0) continue;
+            if (i != cur) {
+                if (cur >= 0) {
+                    atomicAdd(oB + (long long)cur * N, sb);
+                    atomicAdd(oC + (long long)cur * N, sc);
+                }
+                cur = i;
+                sb = 0.f;
+                sc = 0.f;
+            }
+            sb += vb[v];
+            sc += vc[v];
+        }
+    }
+    if (cur >= 0) {
+        atomicAdd(oB + (long long)cur * N, sb);
+        atomicAdd(oC + (long long)cur * N, sc);
+    }
 }
 
 constexpr int PL_CH = 32;       // channels per CTA
@@ -219,35 +259,45 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
                     if (colmajor) { if (++row == p.g.h) { row = 0; ++col; } }
                     else { if (++col == p.g.w) { col = 0; ++row; } }
                 };
-                float4 win[7];  // x at s-3 .. s+3
+                // x at s-3 .. s+6 for a group of four members s .. s+3
+                float4 win[10];
 #pragma unroll
                 for (int m = 0; m < 6; ++m) {
                     win[m] = xat(row * p.g.w + col, sq >= 0 && sq < g_tok);
                     advance();
                 }
-                for (int j = jb; j < je; ++j) {
-                    win[6] = xat(row * p.g.w + col, sq < g_tok);  // position s + 3 (>= 0 here)
-                    advance();
-                    const float4 dl = cval ? load4<T>(db + (long long)pool_member(p.g, i, j) * D)
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-                    ad.x += dl.x; ad.y += dl.y; ad.z += dl.z; ad.w += dl.w;
-                    const float* wv = reinterpret_cast<const float*>(win);  // [7][4]
-                    float f[4], bk[4];
+                for (int j = jb; j < je; j += 4) {
+                    // loads first: the next four window entries and four raw Deltas
+                    float4 dl[4];
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        float a0 = kb[0][cc], a1 = kb[1][cc];
-#pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            a0 = fmaf(kw[0][t][cc], wv[4 * t + cc], a0);        // x[s - 3 + t]
-                            a1 = fmaf(kw[1][t][cc], wv[4 * (6 - t) + cc], a1);  // x[s + 3 - t]
-                        }
-                        f[cc] = silu_f(a0);
-                        bk[cc] = silu_f(a1);
+                    for (int v = 0; v < 4; ++v) {
+                        win[6 + v] = xat(row * p.g.w + col, sq < g_tok);
+                        advance();
+                        dl[v] = (cval && j + v < je) ? load4<T>(db + (long long)pool_member(p.g, i, j + v) * D)
+                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
-                    if (Ki == 1 || k == 0) { au0.x += f[0]; au0.y += f[1]; au0.z += f[2]; au0.w += f[3]; }
-                    if (Ki == 1 || k == 1) { au1.x += bk[0]; au1.y += bk[1]; au1.z += bk[2]; au1.w += bk[3]; }
 #pragma unroll
-                    for (int m = 0; m < 6; ++m) win[m] = win[m + 1];
+                    for (int v = 0; v < 4; ++v) {
+                        if (j + v >= je) break;
+                        ad.x += dl[v].x; ad.y += dl[v].y; ad.z += dl[v].z; ad.w += dl[v].w;
+                        const float* wv = reinterpret_cast<const float*>(win + v);  // x[s + v - 3 ..]
+                        float f[4], bk[4];
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc) {
+                            float a0 = kb[0][cc], a1 = kb[1][cc];
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                a0 = fmaf(kw[0][t][cc], wv[4 * t + cc], a0);        // x[s - 3 + t]
+                                a1 = fmaf(kw[1][t][cc], wv[4 * (6 - t) + cc], a1);  // x[s + 3 - t]
+                            }
+                            f[cc] = silu_f(a0);
+                            bk[cc] = silu_f(a1);
+                        }
+                        if (Ki == 1 || k == 0) { au0.x += f[0]; au0.y += f[1]; au0.z += f[2]; au0.w += f[3]; }
+                        if (Ki == 1 || k == 1) { au1.x += bk[0]; au1.y += bk[1]; au1.z += bk[2]; au1.w += bk[3]; }
+                    }
+#pragma unroll
+                    for (int m = 0; m < 6; ++m) win[m] = win[m + 4];
                 }
 #pragma unroll
                 for (int m = 8; m <= 16; m <<= 1) {
@@ -291,16 +341,48 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
             for (int k = 0; k < Ki; ++k) {
                 const T* ub = static_cast<const T*>(p.u) + k * p.in_dir + img * D + ch;
                 const T* db = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + ch;
-                for (int t = tid >> 3; t < tokens; t += PL_THREADS / 8) {
-                    const int i = pool_index(p.g, __ldg(pb + t));
-                    if (i < 0) continue;
-                    const float4 u4 = load4<T>(ub + (long long)t * D);
-                    const float4 d4 = load4<T>(db + (long long)t * D);
-                    float* du_ = pu + ((size_t)k * Lp + i) * PL_CH + 4 * q;
-                    float* dd_ = pd + ((size_t)k * Lp + i) * PL_CH + 4 * q;
-                    atomicAdd(du_ + 0, u4.x); atomicAdd(du_ + 1, u4.y); atomicAdd(du_ + 2, u4.z); atomicAdd(du_ + 3, u4.w);
-                    atomicAdd(dd_ + 0, d4.x); atomicAdd(dd_ + 1, d4.y); atomicAdd(dd_ + 2, d4.z); atomicAdd(dd_ + 3, d4.w);
+                // Lane group g (tid >> 3, 32 groups) adds the contiguous token range
+                // [g*tokens/32, (g+1)*tokens/32): the four groups of a warp are far
+                // apart, so their atomics rarely meet, and consecutive tokens of one
+                // row (the usual sorted mask) are summed in registers and added once.
+                constexpr int G = PL_THREADS / 8, U = 8;
+                const int g = tid >> 3;
+                const int tb = (int)((long long)tokens * g / G), te = (int)((long long)tokens * (g + 1) / G);
+                int cur = -1;
+                float4 su = make_float4(0.f, 0.f, 0.f, 0.f), sd = su;
+                auto flush = [&]() {
+                    if (cur < 0) return;
+                    float* du_ = pu + ((size_t)k * Lp + cur) * PL_CH + 4 * q;
+                    float* dd_ = pd + ((size_t)k * Lp + cur) * PL_CH + 4 * q;
+                    atomicAdd(du_ + 0, su.x); atomicAdd(du_ + 1, su.y); atomicAdd(du_ + 2, su.z); atomicAdd(du_ + 3, su.w);
+                    atomicAdd(dd_ + 0, sd.x); atomicAdd(dd_ + 1, sd.y); atomicAdd(dd_ + 2, sd.z); atomicAdd(dd_ + 3, sd.w);
+                };
+                for (int t0 = tb; t0 < te; t0 += U) {
+                    int ix[U];
+                    float4 u4[U], d4[U];
+#pragma unroll
+                    for (int v = 0; v < U; ++v) {  // loads first
+                        const int t = t0 + v;
+                        const bool in = t < te;
+                        ix[v] = in ? __ldg(pb + t) : -1;
+                        u4[v] = in ? load4<T>(ub + (long long)t * D) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        d4[v] = in ? load4<T>(db + (long long)t * D) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int v = 0; v < U; ++v) {
+                        const int i = pool_index(p.g, ix[v]);
+                        if (i < 0) continue;
+                        if (i != cur) {
+                            flush();
+                            cur = i;
+                            su = make_float4(0.f, 0.f, 0.f, 0.f);
+                            sd = su;
+                        }
+                        su.x += u4[v].x; su.y += u4[v].y; su.z += u4[v].z; su.w += u4[v].w;
+                        sd.x += d4[v].x; sd.y += d4[v].y; sd.z += d4[v].z; sd.w += d4[v].w;
+                    }
                 }
+                flush();
             }
         }
         __syncthreads();
@@ -459,10 +541,12 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
             const float scale = p.merge_scale;
             for (int tok0 = tl; tok0 < tokens; tok0 += 32 * U) {
                 float4 zz[U];
+                int mp[U];  // FL_MASK: grid positions, loaded with z
 #pragma unroll
                 for (int v = 0; v < U; ++v) {
                     const int tok = tok0 + 32 * v;
                     zz[v] = (zb && tok < tokens) ? load4<T>(zb + (long long)tok * D) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    if constexpr (MASK) mp[v] = tok < tokens ? __ldg(p.pos + (long long)b * tokens + tok) : -1;
                 }
 #pragma unroll
                 for (int v = 0; v < U; ++v) {
@@ -470,7 +554,7 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
                     if (tok >= tokens) break;
                     int i;
                     if constexpr (MASK) {
-                        i = pool_index(p.g, __ldg(p.pos + (long long)b * tokens + tok));
+                        i = pool_index(p.g, mp[v]);
                         if (i < 0) {  // outside the grid: written as 0
                             store4<T>(yb + (long long)tok * D, make_float4(0.f, 0.f, 0.f, 0.f));
                             continue;
