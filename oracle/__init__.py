@@ -41,6 +41,9 @@ def _load():
         lib.oracle_forward_masked.argtypes = [i, i, i, i, i, p, i, i, p, p, p, p, p, p, p, p, i,
                                               ctypes.c_double, i, i, i, p, i]
         lib.oracle_forward_masked.restype = i
+        lib.oracle_backward.argtypes = [i, i, i, i, i, i, i, p, p, p, p, p, p, p, p, i, ctypes.c_double,
+                                        i, i, p, p, p, p, p, p, p, p, p, i]
+        lib.oracle_backward.restype = i
         lib.oracle_default_threads.argtypes = []
         lib.oracle_default_threads.restype = i
         _lib = lib
@@ -177,3 +180,37 @@ def forward_masked(kind, h, w, pos, u, delta, A, B, C, Dskip=None, bias=None, z=
     if rc != 0:
         raise RuntimeError(f"oracle_forward_masked failed (rc={rc})")
     return y
+
+
+def backward(kind, h, w, u, delta, A, B, C, Dskip=None, bias=None, z=None, *, dy, cls_pos=-1,
+             delta_softplus=True, merge_scale=1.0, per_dir_inputs=False, per_dir_params=False,
+             threads=0):
+    """Gradients of forward() w.r.t. every input, given dy = dL/dy, in fp64.
+
+    Returns a dict: du, ddelta (w.r.t. the raw step), dB, dC (shapes of the inputs),
+    dA, dDskip, dbias (shapes of the parameters) and dz (when z is given).
+    """
+    K, L, T = geometry(kind, h, w, cls_pos)
+    u, delta, A, B, C, dy = map(_f64, (u, delta, A, B, C, dy))
+    Dskip = None if Dskip is None else _f64(Dskip)
+    bias = None if bias is None else _f64(bias)
+    z = None if z is None else _f64(z)
+    lead = 1 if per_dir_inputs else 0
+    b, tok, D = u.shape[lead:]
+    N = B.shape[-1]
+    assert tok == T and dy.shape == (b, T, D)
+    Kp = K if per_dir_params else 1
+    out = dict(du=np.empty(u.shape), ddelta=np.empty(u.shape), dB=np.empty(B.shape), dC=np.empty(C.shape),
+               dA=np.empty(A.shape), dDskip=np.empty((Kp, D) if per_dir_params else (D,)),
+               dbias=np.empty((Kp, D) if per_dir_params else (D,)))
+    if z is not None:
+        out["dz"] = np.empty(z.shape)
+    rc = _load().oracle_backward(_kind(kind), h, w, cls_pos, b, D, N, _ptr(u), _ptr(delta), _ptr(A),
+                                 _ptr(B), _ptr(C), _ptr(Dskip), _ptr(bias), _ptr(z),
+                                 int(bool(delta_softplus)), float(merge_scale), int(bool(per_dir_inputs)),
+                                 int(bool(per_dir_params)), _ptr(dy), _ptr(out["du"]), _ptr(out["ddelta"]),
+                                 _ptr(out["dA"]), _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dDskip"]),
+                                 _ptr(out["dbias"]), _ptr(out.get("dz")), int(threads))
+    if rc != 0:
+        raise RuntimeError(f"oracle_backward failed (rc={rc})")
+    return out

@@ -563,6 +563,246 @@ int oracle_forward_masked(int kind, int h, int w, int batch, int n_tok, const in
     return OR_OK;
 }
 
+/*
+ * Gradient of oracle_forward by reverse-mode differentiation of its own loops:
+ * the gate, the merge (sum, or one owner for ATROUS2), the repeat and mean of
+ * the pooled routes, the recurrence run backwards in time, and the
+ * discretization. The released Delta*B*u write term only; no convolution.
+ * Steps of the recurrence ([Vim] sec. 4): with x = Delta, a = exp(x A),
+ *     h_t = a_t h_{t-1} + x_t B_t u_t,   y_t = C_t . h_t + D u_t,
+ * the adjoint g_t = dL/dh_t satisfies g_t = C_t dy_t + a_{t+1} g_{t+1}, and
+ *     dC_t = dy_t h_t,  dB_t = g_t x_t u_t,  du_t = D dy_t + sum_n g_t x_t B_t,
+ *     dx_t = sum_n g_t (A a_t h_{t-1} + B_t u_t),  dA += g_t x_t a_t h_{t-1},
+ *     dD += dy_t u_t,  draw_t = dx_t * sigmoid(raw_t + bias) (softplus' = sigmoid).
+ *
+ * dy: [batch][tokens][D]. Outputs (all overwritten; any may be NULL):
+ *   du, ddelta [Ki][batch][tokens][D] (ddelta: w.r.t. the raw step),
+ *   dB, dC [Ki][batch][tokens][N], dA [Kp][D][N], dDskip [Kp][D],
+ *   dbias [Kp][D], dz [batch][tokens][D].
+ */
+int oracle_backward(int kind, int h, int w, int cls_pos, int batch, int D, int N,
+                    const double* u, const double* delta, const double* A, const double* B,
+                    const double* C, const double* Dskip, const double* bias, const double* z,
+                    int delta_softplus, double merge_scale, int per_dir_inputs, int per_dir_params,
+                    const double* dy, double* du, double* ddelta, double* dA, double* dB,
+                    double* dC, double* dDskip, double* dbias, double* dz, int nthreads)
+{
+    int K, L, tokens;
+    int rc = oracle_geometry(kind, h, w, cls_pos, &K, &L, &tokens);
+    if (rc != OR_OK) return rc;
+    if (batch < 0 || D <= 0 || N <= 0) return OR_EINVAL;
+    const int pooled = (kind == OR_POOL_W || kind == OR_POOL_H);
+    const int Ki = per_dir_inputs ? K : 1, Kp = per_dir_params ? K : 1;
+    const int64_t in_dir = per_dir_inputs ? (int64_t)batch * tokens * D : 0;
+    const int64_t bc_dir = per_dir_inputs ? (int64_t)batch * tokens * N : 0;
+    const int64_t a_dir = per_dir_params ? (int64_t)D * N : 0;
+    const int64_t v_dir = per_dir_params ? (int64_t)D : 0;
+    if (du) memset(du, 0, sizeof(double) * (size_t)Ki * batch * tokens * D);
+    if (ddelta) memset(ddelta, 0, sizeof(double) * (size_t)Ki * batch * tokens * D);
+    if (dB) memset(dB, 0, sizeof(double) * (size_t)Ki * batch * tokens * N);
+    if (dC) memset(dC, 0, sizeof(double) * (size_t)Ki * batch * tokens * N);
+    if (dA) memset(dA, 0, sizeof(double) * (size_t)Kp * D * N);
+    if (dDskip) memset(dDskip, 0, sizeof(double) * (size_t)Kp * D);
+    if (dbias) memset(dbias, 0, sizeof(double) * (size_t)Kp * D);
+    if (batch == 0) return OR_OK;
+
+    int64_t* route = (int64_t*)malloc(sizeof(int64_t) * (size_t)K * L);
+    if (!route) return OR_ENOMEM;
+    rc = oracle_route(kind, h, w, cls_pos, route);
+    if (rc != OR_OK) { free(route); return rc; }
+    const int cnt = pooled ? ((kind == OR_POOL_W) ? w : h) : 1;
+    int failed = 0;
+    int nt = nthreads > 0 ? nthreads : omp_get_max_threads();
+
+    /* one image per thread: its token gradients are private; the parameter
+     * gradients are summed into thread-local arrays and added at the end */
+#pragma omp parallel num_threads(nt) reduction(| : failed)
+    {
+        double* su = (double*)malloc(sizeof(double) * L);
+        double* sraw = (double*)malloc(sizeof(double) * L);
+        double* sx = (double*)malloc(sizeof(double) * L);
+        double* sB = (double*)malloc(sizeof(double) * (size_t)L * N);
+        double* sC = (double*)malloc(sizeof(double) * (size_t)L * N);
+        double* hs = (double*)malloc(sizeof(double) * (size_t)(L + 1) * N); /* h_{-1} .. h_{L-1} */
+        double* ys = (double*)malloc(sizeof(double) * (size_t)K * L);
+        double* acc = (double*)malloc(sizeof(double) * tokens);
+        double* gacc = (double*)malloc(sizeof(double) * tokens);
+        double* dys = (double*)malloc(sizeof(double) * L);
+        double* g = (double*)malloc(sizeof(double) * N);
+        double* lA = (double*)calloc((size_t)Kp * D * N, sizeof(double));
+        double* lD = (double*)calloc((size_t)Kp * D, sizeof(double));
+        double* lb = (double*)calloc((size_t)Kp * D, sizeof(double));
+        int bad = (!su || !sraw || !sx || !sB || !sC || !hs || !ys || !acc || !gacc || !dys || !g ||
+                   !lA || !lD || !lb);
+        if (bad) failed |= 1;
+
+#pragma omp for schedule(static)
+        for (int bi = 0; bi < batch; ++bi) {
+            if (bad) continue;
+            for (int d = 0; d < D; ++d) {
+                /* gather direction kk's sequence from input plane pl */
+                #define GATHER(pl, kk)                                                          \
+                    do {                                                                        \
+                        const double* uk = u + (pl) * in_dir + (int64_t)bi * tokens * D;         \
+                        const double* dk = delta + (pl) * in_dir + (int64_t)bi * tokens * D;     \
+                        const double* Bk = B + (pl) * bc_dir + (int64_t)bi * tokens * N;         \
+                        const double* Ck = C + (pl) * bc_dir + (int64_t)bi * tokens * N;         \
+                        for (int t = 0; t < L; ++t) {                                           \
+                            int64_t q = route[(int64_t)(kk) * L + t];                           \
+                            su[t] = 0.0; sraw[t] = 0.0;                                         \
+                            for (int n = 0; n < N; ++n) { sB[(int64_t)t * N + n] = 0.0; sC[(int64_t)t * N + n] = 0.0; } \
+                            if (!pooled) {                                                      \
+                                if (q < 0) continue;                                            \
+                                su[t] = uk[q * D + d]; sraw[t] = dk[q * D + d];                 \
+                                for (int n = 0; n < N; ++n) {                                   \
+                                    sB[(int64_t)t * N + n] = Bk[q * N + n];                     \
+                                    sC[(int64_t)t * N + n] = Ck[q * N + n];                     \
+                                }                                                               \
+                            } else {                                                            \
+                                for (int j = 0; j < cnt; ++j) {                                 \
+                                    int64_t tok = (kind == OR_POOL_W) ? q * w + j : (int64_t)j * w + q; \
+                                    su[t] += uk[tok * D + d] / cnt; sraw[t] += dk[tok * D + d] / cnt; \
+                                    for (int n = 0; n < N; ++n) {                               \
+                                        sB[(int64_t)t * N + n] += Bk[tok * N + n] / cnt;        \
+                                        sC[(int64_t)t * N + n] += Ck[tok * N + n] / cnt;        \
+                                    }                                                           \
+                                }                                                               \
+                            }                                                                   \
+                        }                                                                       \
+                    } while (0)
+
+                /* forward: per-direction outputs and the merged pre-gate value */
+                for (int i = 0; i < tokens; ++i) acc[i] = 0.0;
+                for (int k = 0; k < K; ++k) {
+                    GATHER(per_dir_inputs ? k : 0, k);
+                    const double* Ak = A + k * a_dir + (int64_t)d * N;
+                    double Dk = Dskip ? Dskip[k * v_dir + d] : 0.0;
+                    double bk = bias ? bias[k * v_dir + d] : 0.0;
+                    for (int n = 0; n < N; ++n) hs[n] = 0.0;
+                    for (int t = 0; t < L; ++t) {
+                        double xr = sraw[t] + bk;
+                        double x = delta_softplus ? softplus(xr) : xr;
+                        double read = 0.0;
+                        for (int n = 0; n < N; ++n) {
+                            double hn = exp(x * Ak[n]) * hs[(int64_t)t * N + n] + x * sB[(int64_t)t * N + n] * su[t];
+                            hs[(int64_t)(t + 1) * N + n] = hn;
+                            read += sC[(int64_t)t * N + n] * hn;
+                        }
+                        ys[(int64_t)k * L + t] = read + Dk * su[t];
+                    }
+                    for (int t = 0; t < L; ++t) {
+                        int64_t q = route[(int64_t)k * L + t];
+                        if (q < 0) continue;
+                        if (kind == OR_ATROUS2) acc[q] = ys[(int64_t)k * L + t];
+                        else acc[q] += ys[(int64_t)k * L + t];
+                    }
+                }
+                /* gate and merge scale: Y = s * acc_repeated * silu(z) */
+                const double* zb = z ? z + (int64_t)bi * tokens * D : 0;
+                const double* dyb = dy + (int64_t)bi * tokens * D;
+                for (int i = 0; i < tokens; ++i) gacc[i] = 0.0;
+                for (int p = 0; p < tokens; ++p) {
+                    int pi = p;
+                    if (pooled) { int r = p / w, c = p % w; pi = (kind == OR_POOL_W) ? r : c; }
+                    double pre = merge_scale * acc[pi];
+                    double dyp = dyb[(int64_t)p * D + d];
+                    if (zb) {
+                        double zz = zb[(int64_t)p * D + d];
+                        double sg = 1.0 / (1.0 + exp(-zz));
+                        if (dz) dz[((int64_t)bi * tokens + p) * D + d] = dyp * pre * sg * (1.0 + zz * (1.0 - sg));
+                        gacc[pi] += dyp * merge_scale * zz * sg;
+                    } else {
+                        gacc[pi] += dyp * merge_scale;
+                    }
+                }
+                /* backward through each direction's recurrence */
+                for (int k = 0; k < K; ++k) {
+                    int ki = per_dir_inputs ? k : 0, kp = per_dir_params ? k : 0;
+                    GATHER(ki, k);
+                    const double* Ak = A + k * a_dir + (int64_t)d * N;
+                    double Dk = Dskip ? Dskip[k * v_dir + d] : 0.0;
+                    double bk = bias ? bias[k * v_dir + d] : 0.0;
+                    /* recompute the states h_t of this direction */
+                    for (int n = 0; n < N; ++n) hs[n] = 0.0;
+                    for (int t = 0; t < L; ++t) {
+                        double xr = sraw[t] + bk;
+                        sx[t] = delta_softplus ? softplus(xr) : xr;
+                        for (int n = 0; n < N; ++n)
+                            hs[(int64_t)(t + 1) * N + n] = exp(sx[t] * Ak[n]) * hs[(int64_t)t * N + n] +
+                                                           sx[t] * sB[(int64_t)t * N + n] * su[t];
+                    }
+                    for (int t = 0; t < L; ++t) {
+                        int64_t q = route[(int64_t)k * L + t];
+                        dys[t] = q >= 0 ? gacc[q] : 0.0;
+                    }
+                    for (int n = 0; n < N; ++n) g[n] = 0.0;
+                    for (int t = L - 1; t >= 0; --t) {
+                        double dyt = dys[t], dut = Dk * dyt, dxt = 0.0;
+                        lD[kp * D + d] += dyt * su[t];
+                        for (int n = 0; n < N; ++n) {
+                            double ht = hs[(int64_t)(t + 1) * N + n], hp = hs[(int64_t)t * N + n];
+                            double a = exp(sx[t] * Ak[n]);
+                            g[n] += sC[(int64_t)t * N + n] * dyt;
+                            double dCt = dyt * ht;
+                            double dBt = g[n] * sx[t] * su[t];
+                            dut += g[n] * sx[t] * sB[(int64_t)t * N + n];
+                            dxt += g[n] * (Ak[n] * a * hp + sB[(int64_t)t * N + n] * su[t]);
+                            lA[(kp * D + d) * N + n] += g[n] * sx[t] * a * hp;
+                            g[n] *= a;
+                            /* scatter the token gradients of B and C */
+                            int64_t q = route[(int64_t)k * L + t];
+                            if (q < 0) continue;
+                            double* dBk = dB ? dB + ki * bc_dir + (int64_t)bi * tokens * N : 0;
+                            double* dCk = dC ? dC + ki * bc_dir + (int64_t)bi * tokens * N : 0;
+                            if (!pooled) {
+                                if (dBk) dBk[q * N + n] += dBt;
+                                if (dCk) dCk[q * N + n] += dCt;
+                            } else {
+                                for (int j = 0; j < cnt; ++j) {
+                                    int64_t tok = (kind == OR_POOL_W) ? q * w + j : (int64_t)j * w + q;
+                                    if (dBk) dBk[tok * N + n] += dBt / cnt;
+                                    if (dCk) dCk[tok * N + n] += dCt / cnt;
+                                }
+                            }
+                        }
+                        double xr = sraw[t] + bk;
+                        double draw = delta_softplus ? dxt / (1.0 + exp(-xr)) : dxt;
+                        lb[kp * D + d] += draw;
+                        int64_t q = route[(int64_t)k * L + t];
+                        if (q < 0) continue; /* padding: only the bias gradient */
+                        double* duk = du ? du + ki * in_dir + (int64_t)bi * tokens * D : 0;
+                        double* ddk = ddelta ? ddelta + ki * in_dir + (int64_t)bi * tokens * D : 0;
+                        if (!pooled) {
+                            if (duk) duk[q * D + d] += dut;
+                            if (ddk) ddk[q * D + d] += draw;
+                        } else {
+                            for (int j = 0; j < cnt; ++j) {
+                                int64_t tok = (kind == OR_POOL_W) ? q * w + j : (int64_t)j * w + q;
+                                if (duk) duk[tok * D + d] += dut / cnt;
+                                if (ddk) ddk[tok * D + d] += draw / cnt;
+                            }
+                        }
+                    }
+                }
+                #undef GATHER
+            }
+        }
+#pragma omp critical
+        {
+            if (!bad) {
+                if (dA) for (int64_t i = 0; i < (int64_t)Kp * D * N; ++i) dA[i] += lA[i];
+                if (dDskip) for (int64_t i = 0; i < (int64_t)Kp * D; ++i) dDskip[i] += lD[i];
+                if (dbias) for (int64_t i = 0; i < (int64_t)Kp * D; ++i) dbias[i] += lb[i];
+            }
+        }
+        free(su); free(sraw); free(sx); free(sB); free(sC); free(hs); free(ys); free(acc); free(gacc);
+        free(dys); free(g); free(lA); free(lD); free(lb);
+    }
+    free(route);
+    if (failed & 1) return OR_ENOMEM;
+    return OR_OK;
+}
+
 /* Number of OpenMP threads oracle_forward uses when nthreads <= 0. */
 int oracle_default_threads(void)
 {
