@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--conv", action="store_true",
                    help="fuse the causal kernel-four Conv1d + SiLU into u (BIDIR and pooled routes)")
     p.add_argument("--zoh", action="store_true", help="zero-order-hold write term instead of Delta*B*u")
+    p.add_argument("--backward", action="store_true",
+                   help="time the backward pass (all gradients) instead of the forward")
     p.add_argument("--mask-keep", type=float, default=1.0,
                    help="pooled workloads: keep this fraction of tokens (random mask per image, FastMaskVim)")
     return p.parse_args()
@@ -76,6 +78,15 @@ def workload_label(wls):
     cls = "_cls" if w0.cls_pos >= 0 else ""
     opt = ("_conv" if w0.conv else "") + ("_zoh" if w0.zoh else "") + (f"_keep{w0.keep:g}" if w0.keep < 1 else "")
     return f"{w0.route}_{grids}{cls}_b{w0.batch}_d{w0.D}_n{w0.N}_{w0.dtype}{opt}"
+
+
+def algorithmic_bytes_bwd(wl):
+    """Compulsory HBM bytes of one backward: read u, raw delta, z, B, C and dy; write the
+    float32 gradients du, ddelta, dz (per token-channel) and dB, dC (per token-state)."""
+    eb = 2 if wl.dtype == "bf16" else 4
+    per_token = (4 * wl.D + 2 * wl.N) * eb + (3 * wl.D + 2 * wl.N) * 4
+    params = (wl.D * wl.N + 2 * wl.D) * 4 * 2
+    return wl.batch * wl.tokens * per_token + params
 
 
 def algorithmic_bytes(wl):
@@ -322,7 +333,7 @@ def config_block(wls, n):
     return {"workload": workload_label(wls), "route": w0.route,
             "grids": [f"{w.h}x{w.w}" for w in wls], "batch": w0.batch, "d_inner": w0.D,
             "d_state": w0.N, "io_dtype": w0.dtype, "gate": w0.gate, "merge_scale": w0.merge_scale,
-            "conv": w0.conv, "zoh": w0.zoh, "mask_keep": w0.keep,
+            "conv": w0.conv, "zoh": w0.zoh, "mask_keep": w0.keep, "pass": "forward",
             "parallelism": f"replicas x{n} (one full workload per GPU, no collective)"}
 
 
@@ -366,6 +377,13 @@ def run_ours(args, wls):
             d = {k: v.to(dev) for k, v in host.items()}
             out = torch.empty_like(d["u"])
             ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+            if args.backward:
+                dy = torch.randn(d["u"].shape[-3:], generator=torch.Generator().manual_seed(rank)).to(
+                    dev, d["u"].dtype)
+                per.append(vs.BackwardPlan(route, d["u"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"],
+                                           d["bias"], d["z"] if wl.gate else None, dy=dy,
+                                           merge_scale=wl.merge_scale))
+                continue
             per.append(vs.Plan(route, d["u"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], d["bias"],
                                d["z"] if wl.gate else None, out=out, workspace=ws,
                                merge_scale=wl.merge_scale, conv_w=d.get("conv_w"),
@@ -420,7 +438,8 @@ def run_ours(args, wls):
     # the streaming routes; for the pooled route the bracket also holds the small
     # B/C pooling pre-pass)
     hbm_peak, peak_src, sm_max = peaks()
-    bytes_all = sum(algorithmic_bytes(w) * K for w in wls)
+    ab = algorithmic_bytes_bwd if args.backward else algorithmic_bytes
+    bytes_all = sum(ab(w) * K for w in wls)
     ms_all = sum(sum(v) for v in per_launch_ms)
     achieved = bytes_all / (ms_all * 1e-3) / 1e9
     kname = "+".join(knames)
@@ -431,7 +450,7 @@ def run_ours(args, wls):
                 "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                 "kernel": kname, "launch_ms_avg": round(ms_all / (K * nfw), 5),
-                "algorithmic_bytes_per_launch": [algorithmic_bytes(w) for w in wls],
+                "algorithmic_bytes_per_launch": [ab(w) for w in wls],
                 "sfu": {"state_updates_per_s": upd_all / (ms_all * 1e-3), "peak": sfu_peak,
                         "frac": round(upd_all / (ms_all * 1e-3) / sfu_peak, 4),
                         "note": "one ex2 per state update, 16 SFU results/clk/SM x 148 SMs at max clock"}}
@@ -442,7 +461,7 @@ def run_ours(args, wls):
         "scaling": "weak", "vs_baseline": None,
         "dtype": "f32" if wls[0].dtype == "f32" else "bf16",
         "data": "synthetic, seeded (page-workload shapes and value recipe)",
-        "config": dict(config_block(wls, world),
+        "config": dict(config_block(wls, world), **({"pass": "backward (all gradients)"} if args.backward else {}),
                        l2=f"rotating {rot} device copies of the inputs ({rot * step_bytes / 2**20:.0f} MiB; "
                           f"each step's inputs were last touched {rot - 1} steps earlier)"),
         "roofline": roofline,
@@ -504,6 +523,10 @@ def main():
     wls = select(args.workload)
     if args.batch > 0:
         wls = [w.with_(batch=args.batch) for w in wls]
+    if args.backward and (args.conv or args.zoh or args.mask_keep < 1):
+        raise SystemExit("--backward covers the Delta*B*u scan without --conv, --zoh or --mask-keep")
+    if args.backward:
+        args.no_e2e = True  # the end-to-end leg times the forward entry point
     if args.conv or args.zoh or args.mask_keep < 1:
         wls = [w.with_(conv=args.conv, zoh=args.zoh, keep=args.mask_keep) for w in wls]
         if args.mask_keep < 1 and (wls[0].route not in ("pool_w", "pool_h") or args.conv):

@@ -294,6 +294,52 @@ vscan_status vscan_host_buffer_size(const vscan_route* route, const vscan_args* 
 vscan_status vscan_forward_host(const vscan_route* route, const vscan_args* host_args,
                                 void* device_buffer, uint64_t device_buffer_bytes, void* stream);
 
+/*
+ * Gradients of vscan_forward, all float32 and written (not accumulated):
+ * the reverse-mode derivative of the forward steps ("Vision Mamba ...",
+ * sec. 3-5; "EfficientVMamba ...", sec. 1-3; "Fast Vision Mamba ...",
+ * Methodology) for the Delta*B*u write term. Any pointer may be NULL when that
+ * gradient is not wanted (its work is then skipped where possible).
+ */
+typedef struct vscan_grads {
+    float* du;        /* device, [Ki][batch][tokens][D]                         */
+    float* ddelta;    /* device, [Ki][batch][tokens][D], w.r.t. the raw step     */
+    float* dB;        /* device, [Ki][batch][tokens][N]                         */
+    float* dC;        /* device, [Ki][batch][tokens][N]                         */
+    float* dA;        /* device, [Kp][D][N]                                     */
+    float* dDskip;    /* device, [Kp][D] (w.r.t. D even when args->Dskip is NULL)  */
+    float* dbias;     /* device, [Kp][D] (w.r.t. the bias, also when it is NULL) */
+    float* dz;        /* device, [batch][tokens][D]; needs args->z              */
+    void* workspace;  /* device scratch of >= vscan_backward_workspace_size()   */
+    uint64_t workspace_bytes;
+} vscan_grads;
+
+/*
+ * Device scratch bytes vscan_backward needs for these arguments (host only):
+ * the pre-gate forward output, the forward's own workspace, the gradient of the
+ * merged value, the state at every 16-step chunk boundary of every sequence
+ * ([K][batch][ceil(L/16)][D][16] float32), and for the pooled routes the
+ * pooled inputs and their gradients.
+ */
+vscan_status vscan_backward_workspace_size(const vscan_route* route, const vscan_args* args,
+                                           uint64_t* bytes);
+
+/*
+ * Backward pass. args are the forward's arguments (args->y and args->workspace
+ * are not used); dy is dL/dy, [batch][tokens][D] in args->dtype, device. The
+ * call enqueues on stream: zeroing of the requested gradients, the pre-gate
+ * forward pass, the gate's gradient, and the reverse-time adjoint scan of every
+ * direction (checkpointed every 16 steps), then the gradients. Token gradients
+ * shared by several directions, channel tiles or images are summed with float
+ * atomics, so their low-order bits can vary from run to run.
+ * Errors: as vscan_forward; VSCAN_ERR_UNSUPPORTED with the fused convolution,
+ * the zero-order-hold flag or a masked token set; VSCAN_ERR_WORKSPACE if
+ * grads->workspace is too small; VSCAN_ERR_INVALID_ARGUMENT for dy or grads
+ * NULL, or dz requested without args->z.
+ */
+vscan_status vscan_backward(const vscan_route* route, const vscan_args* args, const void* dy,
+                            const vscan_grads* grads, void* stream);
+
 /* Message for the last non-OK status on this thread ("" if none). */
 const char* vscan_last_error(void);
 

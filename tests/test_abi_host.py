@@ -241,3 +241,28 @@ def test_masked_token_sets_are_checked_on_the_host():
     a = _args(token_pos=1, n_tokens=1024)
     assert abi.lib.vscan_host_buffer_size(big.handle, ctypes.byref(a), ctypes.byref(n_mask)) == 0
     assert n_mask.value < n_dense.value
+
+
+def test_backward_argument_checks_run_before_any_cuda_call():
+    fake = dict(u=0x1000, delta=0x2000, B=0x3000, C=0x4000, y=0x5000, A=0x6000)
+    r = vs.Route("bidir", 4, 4)
+    n = ctypes.c_uint64()
+    for extra in (dict(conv_w=0x7000), dict(flags=abi.FLAG_ZOH)):
+        assert abi.lib.vscan_backward_workspace_size(r.handle, ctypes.byref(_args(**fake, **extra)),
+                                                     ctypes.byref(n)) == -4
+    pw = vs.Route("pool_w", 4, 4)
+    assert abi.lib.vscan_backward_workspace_size(pw.handle, ctypes.byref(_args(**fake, token_pos=0x7000, n_tokens=3)),
+                                                 ctypes.byref(n)) == -4
+    # size: forward workspace + pre-gate output + gy + checkpoints (batch 2, 16 tokens, D 16, N 16)
+    assert abi.lib.vscan_backward_workspace_size(r.handle, ctypes.byref(_args(**fake)), ctypes.byref(n)) == 0
+    fwd = 2 * 2 * 16 * 16 * 4
+    assert n.value == fwd + 2 * 16 * 16 * 4 + 2 * 16 * 16 * 4 + 2 * 2 * 1 * 16 * 16 * 4
+    g = abi.VscanGrads()
+    assert abi.lib.vscan_backward(r.handle, ctypes.byref(_args(**fake)), None, ctypes.byref(g), None) == -1
+    assert abi.lib.vscan_backward(r.handle, ctypes.byref(_args(**fake)), ctypes.c_void_p(0x8000), None, None) == -1
+    g.dz = 0x9000  # dz without z
+    assert abi.lib.vscan_backward(r.handle, ctypes.byref(_args(**fake)), ctypes.c_void_p(0x8000),
+                                  ctypes.byref(g), None) == -1
+    g.dz = None  # workspace missing
+    assert abi.lib.vscan_backward(r.handle, ctypes.byref(_args(**fake)), ctypes.c_void_p(0x8000),
+                                  ctypes.byref(g), None) == -6

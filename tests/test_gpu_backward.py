@@ -1,0 +1,89 @@
+"""CUDA backward pass vs the fp64 oracle's backward (itself pinned by finite
+differences): every gradient, every route, sequences spanning several 16-step
+chunks with ragged tails, per-direction inputs and parameters, the optional
+terms, and both I/O types. Gradients are float32 and summed with atomics, so
+they are compared with the tolerance metric, not bit for bit.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+import oracle as O
+import workloads
+from vscan_testlib import TOL, rel_err, small_workload, to_device
+
+import vision_selective_state_b200 as vs
+
+pytestmark = pytest.mark.gpu
+
+KEYS = ("du", "ddelta", "dB", "dC", "dA", "dDskip", "dbias", "dz")
+
+
+def _case(route, h, w, D, dtype, *, N=16, batch=2, seed=11, pdi=False, pdp=False, gate=True, skip=True,
+          bias=True, softplus=True, merge_scale=0.7, cls=None):
+    wl = small_workload(route, h, w, D, N, dtype, batch, seed, cls)
+    x = workloads.draw(wl, a_mode="random", per_dir_inputs=pdi, per_dir_params=pdp)
+    if not softplus:
+        x["delta"] = np.abs(x["delta"])
+        x["bias"] = np.full_like(x["bias"], 0.01)
+    rng = np.random.default_rng(seed + 3)
+    dy = rng.standard_normal((batch, wl.tokens, D)).astype(np.float32)
+    if dtype == "bf16":
+        dy = workloads.round_to_bf16(dy)
+    xd = to_device(x, dtype)
+    dyd = torch.from_numpy(dy).to("cuda", torch.bfloat16 if dtype == "bf16" else torch.float32)
+    r = vs.Route(route, h, w, wl.cls_pos)
+    g = vs.backward(r, xd["u"], xd["delta"], xd["A"], xd["B"], xd["C"], xd["Dskip"] if skip else None,
+                    xd["bias"] if bias else None, xd["z"] if gate else None, dy=dyd, delta_softplus=softplus,
+                    merge_scale=merge_scale, per_dir_inputs=pdi, per_dir_params=pdp)
+    torch.cuda.synchronize()
+    ref = O.backward(route, h, w, x["u"], x["delta"], x["A"], x["B"], x["C"], x["Dskip"] if skip else None,
+                     x["bias"] if bias else None, x["z"] if gate else None, dy=dy, cls_pos=wl.cls_pos,
+                     delta_softplus=softplus, merge_scale=merge_scale, per_dir_inputs=pdi, per_dir_params=pdp)
+    tol = TOL[dtype]
+    for k in KEYS:
+        if k not in ref or k not in g:
+            continue
+        err = rel_err(g[k].cpu().numpy(), ref[k])
+        assert err <= tol, (route, h, w, dtype, k, err)
+
+
+@pytest.mark.parametrize("route", ["bidir", "cross4", "atrous2", "pool_w", "pool_h"])
+@pytest.mark.parametrize("h,w", [(1, 1), (3, 5), (9, 13), (17, 19)])
+def test_backward_f32(route, h, w):
+    _case(route, h, w, 24, "f32")
+
+
+@pytest.mark.parametrize("route", ["bidir", "cross4", "atrous2", "pool_w"])
+def test_backward_bf16(route):
+    _case(route, 11, 14, 16, "bf16")
+
+
+@pytest.mark.parametrize("route", ["bidir", "cross4", "atrous2", "pool_w", "pool_h"])
+def test_backward_per_direction(route):
+    _case(route, 7, 9, 16, "f32", pdi=True, pdp=True)
+
+
+@pytest.mark.parametrize("route", ["bidir", "atrous2", "pool_h"])
+def test_backward_without_optional_terms_and_state_tail(route):
+    _case(route, 6, 7, 12, "f32", N=5, gate=False, skip=False, bias=False, softplus=False, merge_scale=1.0)
+
+
+def test_backward_bidir_with_middle_cls_and_long_sequence():
+    _case("bidir", 14, 14, 16, "f32", cls=98)
+    _case("bidir", 31, 33, 8, "f32", batch=1)
+
+
+def test_backward_refuses_unsupported_options():
+    r = vs.Route("bidir", 4, 4)
+    x = torch.zeros(1, 16, 8, device="cuda")
+    bc = torch.zeros(1, 16, 16, device="cuda")
+    A = -torch.ones(8, 16, device="cuda")
+    import ctypes
+    from vision_selective_state_b200 import _abi
+    a = vs._args(r, x, x, A, bc, bc, None, None, None, x, True, 1.0, False, False, None, 0, None, None, True)
+    n = ctypes.c_uint64()
+    assert _abi.lib.vscan_backward_workspace_size(r.handle, ctypes.byref(a), ctypes.byref(n)) == -4

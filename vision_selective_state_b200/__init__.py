@@ -22,10 +22,10 @@ import ctypes
 
 import torch
 
-from ._abi import BF16, F32, FLAG_ZOH, ROUTES, VscanArgs, VscanError, check, lib
+from ._abi import BF16, F32, FLAG_ZOH, ROUTES, VscanArgs, VscanError, VscanGrads, check, lib
 
-__all__ = ["Route", "forward", "forward_host", "workspace_size", "host_buffer_size", "VscanError",
-           "ROUTES"]
+__all__ = ["Route", "forward", "backward", "forward_host", "workspace_size", "host_buffer_size",
+           "VscanError", "ROUTES"]
 
 
 class Route:
@@ -269,3 +269,88 @@ class HostPlan:
 
 
 __all__.append("HostPlan")
+
+
+def backward(route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, dy, delta_softplus=True,
+             merge_scale=1.0, per_dir_inputs=False, per_dir_params=False, want=None, stream=None):
+    """Gradients of forward() (vscan_backward), float32 tensors in a dict.
+
+    dy: dL/dy, [batch, tokens, D] in the dtype of u. Keys: du, ddelta (w.r.t. the raw
+    step), dB, dC, dA, dDskip, dbias and dz (with z). `want` limits the keys computed.
+    """
+    lead = 1 if per_dir_inputs else 0
+    dev = u.device
+    K = route.K
+    Kp = K if per_dir_params else 1
+    D = u.shape[-1]
+    shapes = dict(du=u.shape, ddelta=u.shape, dB=B.shape, dC=C.shape, dA=A.shape,
+                  dDskip=(Kp, D) if per_dir_params else (D,), dbias=(Kp, D) if per_dir_params else (D,))
+    if z is not None:
+        shapes["dz"] = z.shape
+    keys = list(shapes) if want is None else [k for k in want if k in shapes]
+    out = {k: torch.empty(shapes[k], dtype=torch.float32, device=dev) for k in keys}
+    a = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, u[0] if lead else u, delta_softplus, merge_scale,
+              per_dir_inputs, per_dir_params, None, 0)
+    a.y = None
+    n = ctypes.c_uint64()
+    check(lib.vscan_backward_workspace_size(route.handle, ctypes.byref(a), ctypes.byref(n)))
+    ws = torch.empty(max(n.value, 256), dtype=torch.uint8, device=dev)
+    g = VscanGrads()
+    for k, t in out.items():
+        setattr(g, k, ctypes.c_void_p(t.data_ptr()))
+    g.workspace, g.workspace_bytes = ctypes.c_void_p(ws.data_ptr()), ws.numel()
+    if not dy.is_contiguous() or dy.dtype != u.dtype:
+        raise TypeError("dy must be contiguous with the dtype of u")
+    check(lib.vscan_backward(route.handle, ctypes.byref(a), ctypes.c_void_p(dy.data_ptr()), ctypes.byref(g),
+                             _stream(stream, dev)))
+    out["_workspace"] = ws  # keeps the scratch alive until the caller synchronizes
+    return out
+
+
+class BackwardPlan:
+    """A backward call with its arguments, gradients and scratch marshalled once."""
+
+    def __init__(self, route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, dy,
+                 delta_softplus=True, merge_scale=1.0, per_dir_inputs=False, per_dir_params=False):
+        self.route = route
+        dev = u.device
+        K = route.K
+        Kp = K if per_dir_params else 1
+        D = u.shape[-1]
+        shapes = dict(du=u.shape, ddelta=u.shape, dB=B.shape, dC=C.shape, dA=A.shape,
+                      dDskip=(Kp, D) if per_dir_params else (D,), dbias=(Kp, D) if per_dir_params else (D,))
+        if z is not None:
+            shapes["dz"] = z.shape
+        self.grads = {k: torch.empty(v, dtype=torch.float32, device=dev) for k, v in shapes.items()}
+        lead = 1 if per_dir_inputs else 0
+        self.args = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, u[0] if lead else u, delta_softplus,
+                          merge_scale, per_dir_inputs, per_dir_params, None, 0)
+        self.args.y = None
+        n = ctypes.c_uint64()
+        check(lib.vscan_backward_workspace_size(route.handle, ctypes.byref(self.args), ctypes.byref(n)))
+        self.workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=dev)
+        self.g = VscanGrads()
+        for k, t in self.grads.items():
+            setattr(self.g, k, ctypes.c_void_p(t.data_ptr()))
+        self.g.workspace, self.g.workspace_bytes = ctypes.c_void_p(self.workspace.data_ptr()), n.value
+        self._keep = (u, delta, A, B, C, Dskip, delta_bias, z, dy)
+        self._dy = ctypes.c_void_p(dy.data_ptr())
+        self._ra, self._rg = ctypes.byref(self.args), ctypes.byref(self.g)
+
+    def kernels(self):
+        """Kernel launches of one run(): the pre-gate forward, the gate gradient and the
+        adjoint scan, plus pooling and unpooling for the pooled routes."""
+        n = ctypes.c_int32()
+        check(lib.vscan_plan_info(self.route.handle, ctypes.byref(self.args), ctypes.byref(n)))
+        return n.value + (4 if self.route.kind_name in ("pool_w", "pool_h") else 2)
+
+    def kernel_name(self):
+        return "bwd_scan_kernel<" + ("BIDIR" if self.route.kind_name in ("pool_w", "pool_h")
+                                     else self.route.kind_name.upper()) + ">"
+
+    def run(self, stream):
+        """Enqueue the backward pass on a torch.cuda.Stream."""
+        check(lib.vscan_backward(self.route.handle, self._ra, self._dy, self._rg, ctypes.c_void_p(stream.cuda_stream)))
+
+
+__all__.append("BackwardPlan")

@@ -58,6 +58,14 @@ class VscanArgs(ctypes.Structure):
     ]
 
 
+class VscanGrads(ctypes.Structure):
+    """Mirror of struct vscan_grads (include/vscan.h)."""
+
+    _fields_ = [(name, ctypes.c_void_p) for name in
+                ("du", "ddelta", "dB", "dC", "dA", "dDskip", "dbias", "dz", "workspace")] + [
+        ("workspace_bytes", ctypes.c_uint64)]
+
+
 class VscanError(RuntimeError):
     def __init__(self, status, message):
         self.status = status
@@ -84,6 +92,8 @@ def _load():
         "vscan_forward_pooled_noalloc": ([p, pa, p], i32),
         "vscan_host_buffer_size": ([p, pa, ctypes.POINTER(u64)], i32),
         "vscan_forward_host": ([p, pa, p, u64, p], i32),
+        "vscan_backward_workspace_size": ([p, pa, ctypes.POINTER(u64)], i32),
+        "vscan_backward": ([p, pa, p, ctypes.POINTER(VscanGrads), p], i32),
         "vscan_last_error": ([], ctypes.c_char_p),
         "vscan_status_string": ([i32], ctypes.c_char_p),
         "vscan_abi_version": ([], i32),

@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -13,6 +14,7 @@
 #include <string>
 
 #include "vscan.h"
+#include "vscan_backward.cuh"
 #include "vscan_pool.cuh"
 #include "vscan_resident.cuh"
 #include "vscan_route.cuh"
@@ -444,6 +446,137 @@ vscan_status static_scratch_address(void** out)
     return VSCAN_OK;
 }
 
+// ---- backward ----------------------------------------------------------------------
+struct BwdLayout {
+    size_t fwd_ws, pre, gy, ckpt, pu, praw, pB, pC, pg, dpu, dpraw, dpB, dpC, total;
+};
+
+BwdLayout bwd_layout(const vscan_route* r, const vscan_args* a)
+{
+    const vscan::RouteGeom& g = r->g;
+    const size_t eb = elem_bytes(a->dtype);
+    const size_t Ki = a->per_dir_inputs ? g.K : 1;
+    const size_t b = a->batch, T = g.tokens, D = a->channels, N = a->d_state, L = g.L;
+    const size_t nch = (L + vscan::BW_TOK - 1) / vscan::BW_TOK;
+    BwdLayout Lo{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off += round256(bytes); return o; };
+    Lo.fwd_ws = take(workspace_need(r, a));
+    Lo.pre = take(b * T * D * eb);
+    Lo.gy = take(b * T * D * sizeof(float));
+    Lo.ckpt = take((size_t)g.K * b * nch * D * 16 * sizeof(float));
+    if (is_pool(g.kind)) {
+        Lo.pu = take(Ki * b * L * D * sizeof(float));
+        Lo.praw = take(Ki * b * L * D * sizeof(float));
+        Lo.pB = take(Ki * b * L * N * sizeof(float));
+        Lo.pC = take(Ki * b * L * N * sizeof(float));
+        Lo.pg = take(b * L * D * sizeof(float));
+        Lo.dpu = take(Ki * b * L * D * sizeof(float));
+        Lo.dpraw = take(Ki * b * L * D * sizeof(float));
+        Lo.dpB = take(Ki * b * L * N * sizeof(float));
+        Lo.dpC = take(Ki * b * L * N * sizeof(float));
+    }
+    Lo.total = off;
+    return Lo;
+}
+
+vscan_status check_backward(const vscan_route* r, const vscan_args* a)
+{
+    vscan_status st = check_shape(r, a);
+    if (st != VSCAN_OK) return st;
+    if (a->conv_w) return fail(VSCAN_ERR_UNSUPPORTED, "the backward pass does not take the fused convolution");
+    if (a->flags & VSCAN_FLAG_ZOH) return fail(VSCAN_ERR_UNSUPPORTED, "the backward pass is for the Delta*B*u write term");
+    if (a->token_pos) return fail(VSCAN_ERR_UNSUPPORTED, "the backward pass does not take a masked token set");
+    return VSCAN_OK;
+}
+
+template <typename T>
+vscan_status backward_device(const vscan_route* r, const vscan_args* a, const void* dy, const vscan_grads* gr,
+                             cudaStream_t s)
+{
+    const vscan::RouteGeom& g = r->g;
+    const BwdLayout Lo = bwd_layout(r, a);
+    char* ws = static_cast<char*>(gr->workspace);
+    const int K = g.K, Ki = a->per_dir_inputs ? K : 1, Kp = a->per_dir_params ? K : 1;
+    const long long b = a->batch, TK = g.tokens, D = a->channels, N = a->d_state, L = g.L;
+    const bool pooled = is_pool(g.kind);
+
+    struct Zero { void* p; size_t bytes; };
+    const Zero zeros[] = {
+        {gr->du, (size_t)Ki * b * TK * D * 4}, {gr->ddelta, (size_t)Ki * b * TK * D * 4},
+        {gr->dB, (size_t)Ki * b * TK * N * 4}, {gr->dC, (size_t)Ki * b * TK * N * 4},
+        {gr->dA, (size_t)Kp * D * N * 4}, {gr->dDskip, (size_t)Kp * D * 4}, {gr->dbias, (size_t)Kp * D * 4},
+        {pooled ? ws + Lo.dpu : nullptr, Lo.dpraw - Lo.dpu}, {pooled ? ws + Lo.dpraw : nullptr, Lo.dpB - Lo.dpraw},
+        {pooled ? ws + Lo.dpB : nullptr, Lo.dpC - Lo.dpB}, {pooled ? ws + Lo.dpC : nullptr, Lo.total - Lo.dpC},
+    };
+    for (const Zero& z : zeros) {
+        if (!z.p || z.bytes == 0) continue;
+        cudaError_t e = cudaMemsetAsync(z.p, 0, z.bytes, s);
+        if (e != cudaSuccess) return cuda_fail(e, "zeroing a gradient");
+    }
+    // forward without the gate: pre = s * merged scan output
+    vscan_args fa = *a;
+    fa.z = nullptr;
+    fa.y = ws + Lo.pre;
+    fa.workspace = ws + Lo.fwd_ws;
+    fa.workspace_bytes = Lo.pre - Lo.fwd_ws;
+    vscan_status st = forward_device(r, &fa, s);
+    if (st != VSCAN_OK) return st;
+    // gradient of the gate and of the merged value
+    float* gy = reinterpret_cast<float*>(ws + Lo.gy);
+    const long long n = b * TK * D;
+    const unsigned blocks = (unsigned)std::min<long long>((n + 255) / 256, 148LL * 16);
+    vscan::gate_grad_kernel<T><<<blocks, 256, 0, s>>>(static_cast<const T*>(dy), static_cast<const T*>(a->z),
+                                                      static_cast<const T*>(fa.y), a->merge_scale, n, gy, gr->dz);
+    vscan::BwdParams p{};
+    p.batch = a->batch; p.D = a->channels; p.N = a->d_state;
+    p.a_dir = a->per_dir_params ? a->channels * a->d_state : 0;
+    p.v_dir = a->per_dir_params ? a->channels : 0;
+    p.A = a->A; p.Dskip = a->Dskip; p.bias = a->delta_bias; p.softplus = a->delta_softplus;
+    p.ckpt = reinterpret_cast<float*>(ws + Lo.ckpt);
+    p.dA = gr->dA; p.dD = gr->dDskip; p.dbias = gr->dbias;
+    const dim3 grid((unsigned)((D + vscan::BW_CH - 1) / vscan::BW_CH), (unsigned)b, (unsigned)K);
+    if (!pooled) {
+        p.g = g;
+        p.u = a->u; p.delta = a->delta; p.B = a->B; p.C = a->C;
+        p.in_dir = a->per_dir_inputs ? b * TK * D : 0;
+        p.bc_dir = a->per_dir_inputs ? b * TK * N : 0;
+        p.gy = gy;
+        p.du = gr->du; p.ddelta = gr->ddelta; p.dB = gr->dB; p.dC = gr->dC;
+        switch (g.kind) {
+        case vscan::RK_BIDIR: vscan::bwd_scan_kernel<vscan::RK_BIDIR, T><<<grid, 32, 0, s>>>(p); break;
+        case vscan::RK_CROSS4: vscan::bwd_scan_kernel<vscan::RK_CROSS4, T><<<grid, 32, 0, s>>>(p); break;
+        default: vscan::bwd_scan_kernel<vscan::RK_ATROUS2, T><<<grid, 32, 0, s>>>(p); break;
+        }
+    } else {
+        float* pu = reinterpret_cast<float*>(ws + Lo.pu);
+        float* praw = reinterpret_cast<float*>(ws + Lo.praw);
+        float* pB = reinterpret_cast<float*>(ws + Lo.pB);
+        float* pC = reinterpret_cast<float*>(ws + Lo.pC);
+        float* pg = reinterpret_cast<float*>(ws + Lo.pg);
+        const long long in_dir = a->per_dir_inputs ? b * TK * D : 0, bc_dir = a->per_dir_inputs ? b * TK * N : 0;
+        vscan::bwd_pool_kernel<T><<<dim3((unsigned)L, (unsigned)b), 256, 0, s>>>(
+            g, (int)b, (int)D, (int)N, Ki, static_cast<const T*>(a->u), static_cast<const T*>(a->delta),
+            static_cast<const T*>(a->B), static_cast<const T*>(a->C), in_dir, bc_dir, gy, pu, praw, pB, pC, pg);
+        // the pooled sequence scanned forward and reversed: a bidirectional route of length L
+        vscan::make_geom(vscan::RK_BIDIR, 1, (int)L, -1, &p.g);
+        p.u = pu; p.delta = praw; p.B = pB; p.C = pC;
+        p.in_dir = a->per_dir_inputs ? b * L * D : 0;
+        p.bc_dir = a->per_dir_inputs ? b * L * N : 0;
+        p.gy = pg;
+        p.du = reinterpret_cast<float*>(ws + Lo.dpu);
+        p.ddelta = reinterpret_cast<float*>(ws + Lo.dpraw);
+        p.dB = reinterpret_cast<float*>(ws + Lo.dpB);
+        p.dC = reinterpret_cast<float*>(ws + Lo.dpC);
+        vscan::bwd_scan_kernel<vscan::RK_BIDIR, float><<<grid, 32, 0, s>>>(p);
+        vscan::bwd_unpool_kernel<<<dim3((unsigned)TK, (unsigned)b), 128, 0, s>>>(
+            g, (int)b, (int)D, (int)N, Ki, p.du, p.ddelta, p.dB, p.dC, gr->du, gr->ddelta, gr->dB, gr->dC);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
+    return VSCAN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -622,6 +755,40 @@ vscan_status vscan_forward_host(const vscan_route* r, const vscan_args* ha, void
     cudaError_t e = cudaMemcpyAsync(ha->y, da.y, plane * ha->channels * eb, cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
     return VSCAN_OK;
+}
+
+vscan_status vscan_backward_workspace_size(const vscan_route* r, const vscan_args* a, uint64_t* bytes)
+{
+    if (!bytes) return fail(VSCAN_ERR_INVALID_ARGUMENT, "bytes is NULL");
+    vscan_status st = check_backward(r, a);
+    if (st != VSCAN_OK) return st;
+    *bytes = a->batch == 0 ? 0 : bwd_layout(r, a).total;
+    return VSCAN_OK;
+}
+
+vscan_status vscan_backward(const vscan_route* r, const vscan_args* a, const void* dy, const vscan_grads* gr,
+                            void* stream)
+{
+    vscan_status st = check_backward(r, a);
+    if (st != VSCAN_OK) return st;
+    if (!gr) return fail(VSCAN_ERR_INVALID_ARGUMENT, "grads is NULL");
+    if (a->batch == 0) return VSCAN_OK;
+    if (!dy) return fail(VSCAN_ERR_INVALID_ARGUMENT, "dy is NULL");
+    if (!aligned16(dy)) return fail(VSCAN_ERR_ALIGNMENT, "dy is not 16-byte aligned");
+    if (gr->dz && !a->z) return fail(VSCAN_ERR_INVALID_ARGUMENT, "dz requested without z");
+    vscan_args chk = *a;
+    chk.y = const_cast<void*>(dy);  // y is not used by the backward pass
+    st = check_pointers(&chk, true);
+    if (st != VSCAN_OK) return st;
+    const uint64_t need = bwd_layout(r, a).total;
+    if (!gr->workspace || gr->workspace_bytes < need)
+        return fail(VSCAN_ERR_WORKSPACE, "backward workspace of %llu bytes needed, %llu given",
+                    (unsigned long long)need, (unsigned long long)(gr->workspace ? gr->workspace_bytes : 0));
+    if ((reinterpret_cast<uintptr_t>(gr->workspace) & 255u) != 0)
+        return fail(VSCAN_ERR_ALIGNMENT, "backward workspace is not 256-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return a->dtype == VSCAN_F32 ? backward_device<float>(r, a, dy, gr, s)
+                                 : backward_device<__nv_bfloat16>(r, a, dy, gr, s);
 }
 
 vscan_status vscan_forward_pooled_noalloc(const vscan_route* r, const vscan_args* a, void* stream)

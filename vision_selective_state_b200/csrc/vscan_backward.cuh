@@ -1,0 +1,324 @@
+// Backward pass of the routed selective scan (gradients of vscan_forward).
+//
+// Reverse-mode differentiation of the forward steps ("Vision Mamba ...",
+// sec. 3-5; "EfficientVMamba ...", sec. 1-3; "Fast Vision Mamba ...",
+// Methodology), for the released Delta*B*u write term. With x = Delta and
+// a = exp(x A), the recurrence h_t = a_t h_{t-1} + x_t B_t u_t, y_t = C_t.h_t +
+// D u_t has the adjoint g_t = dL/dh_t = C_t dy_t + a_{t+1} g_{t+1}, and
+//     dC_t = dy_t h_t,   dB_t = g_t x_t u_t,   du_t = D dy_t + sum_n g_t x_t B_t,
+//     dx_t = sum_n g_t (A a_t h_{t-1} + B_t u_t),   dA += g_t x_t a_t h_{t-1},
+//     dD += dy_t u_t,    draw_t = dx_t sigmoid(raw_t + bias).
+//
+// Kernels (launched by vscan_backward):
+//   gate_grad_kernel     dz and the gradient gy of the merged pre-gate value
+//                        (merge scale folded in), from dy, z and the pre-gate
+//                        forward output.
+//   bwd_pool_kernel      pooled routes: means of u, raw Delta, B, C and sums of
+//                        gy over each pooled index, so the scan below runs on the
+//                        pooled sequence exactly as the forward does.
+//   bwd_scan_kernel      one warp per (channel tile of 8, image, direction);
+//                        lane 4c + g holds channel c, states 4g..4g+3. Pass 1
+//                        runs the recurrence forward and saves the state at
+//                        every 16-step chunk boundary; pass 2 walks the chunks
+//                        backwards, recomputes the chunk's states from its
+//                        checkpoint and runs the adjoint recurrence. Token
+//                        gradients are summed over channels (B, C) or state
+//                        groups (u, Delta) with warp shuffles and added with
+//                        float atomics (directions, channel tiles and images
+//                        meet there); dA, D and bias gradients stay in
+//                        registers until the end.
+//   bwd_unpool_kernel    pooled routes: every member token receives its pooled
+//                        index's gradient divided by the member count.
+#pragma once
+
+#include "vscan_common.cuh"
+#include "vscan_route.cuh"
+
+namespace vscan {
+
+struct BwdParams {
+    RouteGeom g;       // route of the scan (pooled routes: BIDIR over the Lp pooled steps)
+    int batch, D, N;
+    const void* u;     // [Ki][batch][tokens][D] (TI)
+    const void* delta; // [Ki][batch][tokens][D] raw step (TI)
+    const void* B;     // [Ki][batch][tokens][N] (TI)
+    const void* C;     // [Ki][batch][tokens][N] (TI)
+    long long in_dir, bc_dir;
+    int a_dir, v_dir;
+    const float* A;
+    const float* Dskip;
+    const float* bias;
+    int softplus;
+    const float* gy;   // [batch][tokens][D]: dL / d(merged pre-gate value)
+    float* ckpt;       // [K][batch][nchunks][D][16]
+    float* du;         // [Ki][batch][tokens][D]
+    float* ddelta;     // [Ki][batch][tokens][D]
+    float* dB;         // [Ki][batch][tokens][N]
+    float* dC;         // [Ki][batch][tokens][N]
+    float* dA;         // [Kp][D][N]
+    float* dD;         // [Kp][D]
+    float* dbias;      // [Kp][D]
+};
+
+constexpr int BW_TOK = 16;  // steps per chunk
+constexpr int BW_CH = 8;    // channels per warp
+
+// dz = dy * pre * sigmoid(z) * (1 + z (1 - sigmoid(z))) and gy = dy * s * SiLU(z),
+// where pre = s * (merged scan output) is the forward output without the gate.
+template <typename T>
+__global__ void gate_grad_kernel(const T* __restrict__ dy, const T* __restrict__ z,
+                                 const T* __restrict__ pre, float scale, long long n,
+                                 float* __restrict__ gy, float* __restrict__ dz)
+{
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+         e += (long long)gridDim.x * blockDim.x) {
+        const float d = to_float(dy[e]);
+        if (z) {
+            const float zz = to_float(z[e]);
+            const float sg = 1.0f / (1.0f + __expf(-zz));
+            gy[e] = d * scale * zz * sg;
+            if (dz) dz[e] = d * to_float(pre[e]) * sg * (1.0f + zz * (1.0f - sg));
+        } else {
+            gy[e] = d * scale;
+        }
+    }
+}
+
+// Pooled routes: pu, praw [Ki][batch][Lp][D] and pB, pC [Ki][batch][Lp][N] are
+// the means over the members of each pooled index, pg [batch][Lp][D] the sum
+// of gy over them. Grid (Lp, batch); threads stride over channels and states.
+template <typename T>
+__global__ void bwd_pool_kernel(RouteGeom g, int batch, int D, int N, int Ki, const T* u, const T* delta,
+                                const T* B, const T* C, long long in_dir, long long bc_dir, const float* gy,
+                                float* pu, float* praw, float* pB, float* pC, float* pg)
+{
+    const int i = blockIdx.x, b = blockIdx.y, Lp = g.L;
+    const int cnt = (g.kind == RK_POOL_W) ? g.w : g.h;
+    const float inv = 1.0f / (float)cnt;
+    const long long img = (long long)b * g.tokens;
+    auto member = [&](int j) { return (long long)((g.kind == RK_POOL_W) ? i * g.w + j : j * g.w + i); };
+    for (int k = 0; k < Ki; ++k) {
+        for (int d = threadIdx.x; d < D; d += blockDim.x) {
+            float su = 0.f, sr = 0.f, sg = 0.f;
+            for (int j = 0; j < cnt; ++j) {
+                const long long o = (img + member(j)) * D + d;
+                su += to_float(u[k * in_dir + o]);
+                sr += to_float(delta[k * in_dir + o]);
+                if (k == 0) sg += gy[o];
+            }
+            const long long po = (((long long)k * batch + b) * Lp + i) * D + d;
+            pu[po] = su * inv;
+            praw[po] = sr * inv;
+            if (k == 0) pg[((long long)b * Lp + i) * D + d] = sg;
+        }
+        for (int n = threadIdx.x; n < N; n += blockDim.x) {
+            float sb = 0.f, sc = 0.f;
+            for (int j = 0; j < cnt; ++j) {
+                const long long o = (img + member(j)) * N + n;
+                sb += to_float(B[k * bc_dir + o]);
+                sc += to_float(C[k * bc_dir + o]);
+            }
+            const long long po = (((long long)k * batch + b) * Lp + i) * N + n;
+            pB[po] = sb * inv;
+            pC[po] = sc * inv;
+        }
+    }
+}
+
+// Pooled routes: token gradients from the pooled ones (the mean's adjoint).
+// Grid (tokens, batch).
+__global__ void bwd_unpool_kernel(RouteGeom g, int batch, int D, int N, int Ki, const float* dpu,
+                                  const float* dpraw, const float* dpB, const float* dpC, float* du,
+                                  float* ddelta, float* dB, float* dC)
+{
+    const int tok = blockIdx.x, b = blockIdx.y, Lp = g.L;
+    const int r = tok / g.w, c = tok - r * g.w;
+    const int i = (g.kind == RK_POOL_W) ? r : c;
+    const float inv = 1.0f / (float)((g.kind == RK_POOL_W) ? g.w : g.h);
+    for (int k = 0; k < Ki; ++k) {
+        const long long to = ((long long)k * batch + b) * g.tokens + tok;
+        const long long po = ((long long)k * batch + b) * Lp + i;
+        for (int d = threadIdx.x; d < D; d += blockDim.x) {
+            if (du) du[to * D + d] = dpu[po * D + d] * inv;
+            if (ddelta) ddelta[to * D + d] = dpraw[po * D + d] * inv;
+        }
+        for (int n = threadIdx.x; n < N; n += blockDim.x) {
+            if (dB) dB[to * N + n] = dpB[po * N + n] * inv;
+            if (dC) dC[to * N + n] = dpC[po * N + n] * inv;
+        }
+    }
+}
+
+// One 16-step chunk of one direction, staged in shared memory.
+struct BwdStage {
+    int pos[BW_TOK];           // token, -1 pad, -2 past the end
+    float x[BW_TOK][BW_CH];    // discretized step Delta
+    float sig[BW_TOK][BW_CH];  // d Delta / d raw
+    float u[BW_TOK][BW_CH];
+    float gy[BW_TOK][BW_CH];
+    float B[BW_TOK][16];
+    float C[BW_TOK][16];
+};
+
+template <int RK, typename TI>
+__global__ void __launch_bounds__(32) bwd_scan_kernel(const BwdParams p)
+{
+    __shared__ BwdStage st;
+    const int lane = threadIdx.x;
+    const int cc = lane >> 2, grp = lane & 3;
+    const int c0 = blockIdx.x * BW_CH, b = blockIdx.y, k = blockIdx.z;
+    const int D = p.D, N = p.N, L = p.g.L, tokens = p.g.tokens;
+    const int d = c0 + cc;
+    const bool dvalid = d < D;
+    const int ki = p.in_dir ? k : 0;
+    const long long img = (long long)b * tokens;
+    const int nch = (L + BW_TOK - 1) / BW_TOK;
+    float a2[4], An[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        const int n = 4 * grp + s;
+        An[s] = (dvalid && n < N) ? __ldg(p.A + (long long)k * p.a_dir + (long long)d * N + n) : 0.f;
+        a2[s] = An[s] * LOG2E;
+    }
+    const float Dd = (dvalid && p.Dskip) ? __ldg(p.Dskip + k * p.v_dir + d) : 0.f;
+    const float* gyb = p.gy + img * D;
+    const TI* ub = static_cast<const TI*>(p.u) + ki * p.in_dir + img * D;
+    const TI* rb = static_cast<const TI*>(p.delta) + ki * p.in_dir + img * D;
+    const TI* Bb = static_cast<const TI*>(p.B) + ki * p.bc_dir + img * N;
+    const TI* Cb = static_cast<const TI*>(p.C) + ki * p.bc_dir + img * N;
+    float* ck = p.ckpt + (((long long)k * p.batch + b) * nch) * D * 16;
+
+    // Stage chunk c: positions, Delta and its derivative, u, gy, B, C.
+    auto stage = [&](int c, bool with_grad) {
+        __syncwarp();
+        if (lane < BW_TOK) {
+            const int t = c * BW_TOK + lane;
+            st.pos[lane] = (t < L) ? route_token<RK>(p.g, k, t) : -2;
+        }
+        __syncwarp();
+        for (int e = lane; e < BW_TOK * BW_CH; e += 32) {
+            const int j = e / BW_CH, ch = e % BW_CH, dd = c0 + ch;
+            const int q = st.pos[j];
+            const float raw = (q >= 0 && dd < D) ? to_float(rb[(long long)q * D + dd]) : 0.f;
+            const float bias = (dd < D && p.bias) ? __ldg(p.bias + k * p.v_dir + dd) : 0.f;
+            const float xr = raw + bias;
+            float x = xr, sg = 1.f;
+            if (p.softplus) {
+                x = softplus_f(xr);
+                sg = 1.0f / (1.0f + __expf(-xr));
+            }
+            const bool live = q != -2 && dd < D;
+            st.x[j][ch] = live ? x : 0.f;
+            st.sig[j][ch] = sg;
+            st.u[j][ch] = (q >= 0 && dd < D) ? to_float(ub[(long long)q * D + dd]) : 0.f;
+            st.gy[j][ch] = (with_grad && q >= 0 && dd < D) ? gyb[(long long)q * D + dd] : 0.f;
+        }
+        for (int e = lane; e < BW_TOK * 16; e += 32) {
+            const int j = e >> 4, n = e & 15;
+            const int q = st.pos[j];
+            st.B[j][n] = (q >= 0 && n < N) ? to_float(Bb[(long long)q * N + n]) : 0.f;
+            st.C[j][n] = (q >= 0 && n < N) ? to_float(Cb[(long long)q * N + n]) : 0.f;
+        }
+        __syncwarp();
+    };
+
+    // ---- pass 1: forward recurrence, state saved at every chunk boundary --------
+    float h[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int c = 0; c < nch; ++c) {
+        if (dvalid) {
+#pragma unroll
+            for (int s = 0; s < 4; ++s) ck[((long long)c * D + d) * 16 + 4 * grp + s] = h[s];
+        }
+        stage(c, false);
+#pragma unroll 4
+        for (int j = 0; j < BW_TOK; ++j) {
+            const float x = st.x[j][cc], uu = st.u[j][cc];
+#pragma unroll
+            for (int s = 0; s < 4; ++s) h[s] = fmaf(fast_exp2(x * a2[s]), h[s], x * st.B[j][4 * grp + s] * uu);
+        }
+    }
+    __syncwarp();
+
+    // ---- pass 2: adjoint recurrence, chunks in reverse ------------------------------
+    float gs[4] = {0.f, 0.f, 0.f, 0.f}, dAs[4] = {0.f, 0.f, 0.f, 0.f};
+    float dDs = 0.f, dbs = 0.f;
+    for (int c = nch - 1; c >= 0; --c) {
+        stage(c, true);
+        float hs[BW_TOK + 1][4];  // hs[0] = state entering the chunk, hs[j + 1] after step j
+#pragma unroll
+        for (int s = 0; s < 4; ++s) hs[0][s] = dvalid ? ck[((long long)c * D + d) * 16 + 4 * grp + s] : 0.f;
+#pragma unroll
+        for (int j = 0; j < BW_TOK; ++j) {
+            const float x = st.x[j][cc], uu = st.u[j][cc];
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                hs[j + 1][s] = fmaf(fast_exp2(x * a2[s]), hs[j][s], x * st.B[j][4 * grp + s] * uu);
+        }
+#pragma unroll
+        for (int j = BW_TOK - 1; j >= 0; --j) {
+            const int q = st.pos[j];
+            if (q == -2) continue;  // past the end of the sequence (uniform over the warp)
+            const float x = st.x[j][cc], uu = st.u[j][cc], dy = st.gy[j][cc];
+            float dut = 0.f, dxt = 0.f, dBv[4], dCv[4];
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const float Bn = st.B[j][4 * grp + s], Cn = st.C[j][4 * grp + s];
+                const float a = fast_exp2(x * a2[s]);
+                gs[s] = fmaf(Cn, dy, gs[s]);
+                dCv[s] = dy * hs[j + 1][s];
+                dBv[s] = gs[s] * x * uu;
+                dut = fmaf(gs[s] * x, Bn, dut);
+                dxt = fmaf(gs[s], fmaf(An[s] * a, hs[j][s], Bn * uu), dxt);
+                dAs[s] = fmaf(gs[s] * x * a, hs[j][s], dAs[s]);
+                gs[s] *= a;
+            }
+            // sums over the four state groups of a channel (u, Delta) ...
+            dut += __shfl_xor_sync(FULL_MASK, dut, 1);
+            dut += __shfl_xor_sync(FULL_MASK, dut, 2);
+            dxt += __shfl_xor_sync(FULL_MASK, dxt, 1);
+            dxt += __shfl_xor_sync(FULL_MASK, dxt, 2);
+            // ... and over the eight channels of the warp (B, C)
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+#pragma unroll
+                for (int m = 4; m <= 16; m <<= 1) {
+                    dBv[s] += __shfl_xor_sync(FULL_MASK, dBv[s], m);
+                    dCv[s] += __shfl_xor_sync(FULL_MASK, dCv[s], m);
+                }
+            }
+            const float draw = dxt * st.sig[j][cc];
+            if (grp == 0 && dvalid) {
+                dbs += draw;
+                dDs = fmaf(dy, uu, dDs);
+                if (q >= 0) {
+                    const long long o = ki * p.in_dir + (img + q) * D + d;
+                    if (p.du) atomicAdd(p.du + o, fmaf(Dd, dy, dut));
+                    if (p.ddelta) atomicAdd(p.ddelta + o, draw);
+                }
+            }
+            if (cc == 0 && q >= 0) {
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const int n = 4 * grp + s;
+                    if (n >= N) continue;
+                    const long long o = ki * p.bc_dir + (img + q) * N + n;
+                    if (p.dB) atomicAdd(p.dB + o, dBv[s]);
+                    if (p.dC) atomicAdd(p.dC + o, dCv[s]);
+                }
+            }
+        }
+    }
+    if (dvalid) {
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const int n = 4 * grp + s;
+            if (n < N && p.dA) atomicAdd(p.dA + (long long)k * p.a_dir + (long long)d * N + n, dAs[s]);
+        }
+        if (grp == 0) {
+            if (p.dD) atomicAdd(p.dD + k * p.v_dir + d, dDs);
+            if (p.dbias) atomicAdd(p.dbias + k * p.v_dir + d, dbs);
+        }
+    }
+}
+
+}  // namespace vscan
