@@ -160,10 +160,19 @@ struct BwdStage {
     float C[BW_TOK][16];
 };
 
+// Per-chunk token-gradient partials of bwd_scan_kernel (summed after the chunk).
+struct BwdReduce {
+    float u[BW_TOK][BW_CH];       // du per (step, channel), state groups already summed
+    float x[BW_TOK][BW_CH];       // d raw Delta per (step, channel)
+    float B[BW_TOK][BW_CH][16];   // dB per (step, channel, state): summed over channels
+    float C[BW_TOK][BW_CH][16];   // dC likewise
+};
+
 template <int RK, typename TI>
 __global__ void __launch_bounds__(32) bwd_scan_kernel(const BwdParams p)
 {
     __shared__ BwdStage st;
+    __shared__ __align__(16) BwdReduce rd;
     const int lane = threadIdx.x;
     const int cc = lane >> 2, grp = lane & 3;
     const int c0 = blockIdx.x * BW_CH, b = blockIdx.y, k = blockIdx.z;
@@ -188,7 +197,13 @@ __global__ void __launch_bounds__(32) bwd_scan_kernel(const BwdParams p)
     const TI* Cb = static_cast<const TI*>(p.C) + ki * p.bc_dir + img * N;
     float* ck = p.ckpt + (((long long)k * p.batch + b) * nch) * D * 16;
 
-    // Stage chunk c: positions, Delta and its derivative, u, gy, B, C.
+    // Stage chunk c: positions, Delta and its derivative, u, gy, B, C. Every
+    // global load of the chunk is issued before any of them is used, so a chunk
+    // costs one memory latency, not one per element.
+    constexpr int NE = BW_TOK * BW_CH / 32;  // (step, channel) elements per lane: 4
+    constexpr int NS = BW_TOK * 16 / 32;     // (step, state) elements per lane: 8
+    // the channel of every staged (step, channel) element of a lane is lane % 8
+    const float bias_l = (c0 + (lane % BW_CH) < D && p.bias) ? __ldg(p.bias + k * p.v_dir + c0 + (lane % BW_CH)) : 0.f;
     auto stage = [&](int c, bool with_grad) {
         __syncwarp();
         if (lane < BW_TOK) {
@@ -196,28 +211,47 @@ __global__ void __launch_bounds__(32) bwd_scan_kernel(const BwdParams p)
             st.pos[lane] = (t < L) ? route_token<RK>(p.g, k, t) : -2;
         }
         __syncwarp();
-        for (int e = lane; e < BW_TOK * BW_CH; e += 32) {
-            const int j = e / BW_CH, ch = e % BW_CH, dd = c0 + ch;
+        float vr[NE], vu[NE], vg[NE], vb[NS], vc[NS];
+#pragma unroll
+        for (int r = 0; r < NE; ++r) {  // element e = lane + 32 r: step e / 8, channel e % 8 (= lane % 8)
+            const int e = lane + 32 * r;
+            const int j = e / BW_CH, dd = c0 + e % BW_CH;
             const int q = st.pos[j];
-            const float raw = (q >= 0 && dd < D) ? to_float(rb[(long long)q * D + dd]) : 0.f;
-            const float bias = (dd < D && p.bias) ? __ldg(p.bias + k * p.v_dir + dd) : 0.f;
-            const float xr = raw + bias;
+            const bool ok = q >= 0 && dd < D;
+            vr[r] = ok ? to_float(rb[(long long)q * D + dd]) : 0.f;
+            vu[r] = ok ? to_float(ub[(long long)q * D + dd]) : 0.f;
+            vg[r] = (ok && with_grad) ? gyb[(long long)q * D + dd] : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < NS; ++r) {  // element e = lane + 32 r: step e / 16, state e % 16
+            const int e = lane + 32 * r;
+            const int j = e >> 4, n = e & 15;
+            const int q = st.pos[j];
+            const bool ok = q >= 0 && n < N;
+            vb[r] = ok ? to_float(Bb[(long long)q * N + n]) : 0.f;
+            vc[r] = ok ? to_float(Cb[(long long)q * N + n]) : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < NE; ++r) {
+            const int e = lane + 32 * r;
+            const int j = e / BW_CH, ch = e % BW_CH, dd = c0 + ch;
+            const float xr = vr[r] + bias_l;
             float x = xr, sg = 1.f;
             if (p.softplus) {
                 x = softplus_f(xr);
                 sg = 1.0f / (1.0f + __expf(-xr));
             }
-            const bool live = q != -2 && dd < D;
+            const bool live = st.pos[j] != -2 && dd < D;
             st.x[j][ch] = live ? x : 0.f;
             st.sig[j][ch] = sg;
-            st.u[j][ch] = (q >= 0 && dd < D) ? to_float(ub[(long long)q * D + dd]) : 0.f;
-            st.gy[j][ch] = (with_grad && q >= 0 && dd < D) ? gyb[(long long)q * D + dd] : 0.f;
+            st.u[j][ch] = vu[r];
+            st.gy[j][ch] = vg[r];
         }
-        for (int e = lane; e < BW_TOK * 16; e += 32) {
-            const int j = e >> 4, n = e & 15;
-            const int q = st.pos[j];
-            st.B[j][n] = (q >= 0 && n < N) ? to_float(Bb[(long long)q * N + n]) : 0.f;
-            st.C[j][n] = (q >= 0 && n < N) ? to_float(Cb[(long long)q * N + n]) : 0.f;
+#pragma unroll
+        for (int r = 0; r < NS; ++r) {
+            const int e = lane + 32 * r;
+            st.B[e >> 4][e & 15] = vb[r];
+            st.C[e >> 4][e & 15] = vc[r];
         }
         __syncwarp();
     };
@@ -272,41 +306,54 @@ __global__ void __launch_bounds__(32) bwd_scan_kernel(const BwdParams p)
                 dAs[s] = fmaf(gs[s] * x * a, hs[j][s], dAs[s]);
                 gs[s] *= a;
             }
-            // sums over the four state groups of a channel (u, Delta) ...
+            // sums over the four state groups of a channel (u, Delta)
             dut += __shfl_xor_sync(FULL_MASK, dut, 1);
             dut += __shfl_xor_sync(FULL_MASK, dut, 2);
             dxt += __shfl_xor_sync(FULL_MASK, dxt, 1);
             dxt += __shfl_xor_sync(FULL_MASK, dxt, 2);
-            // ... and over the eight channels of the warp (B, C)
-#pragma unroll
-            for (int s = 0; s < 4; ++s) {
-#pragma unroll
-                for (int m = 4; m <= 16; m <<= 1) {
-                    dBv[s] += __shfl_xor_sync(FULL_MASK, dBv[s], m);
-                    dCv[s] += __shfl_xor_sync(FULL_MASK, dCv[s], m);
-                }
-            }
             const float draw = dxt * st.sig[j][cc];
-            if (grp == 0 && dvalid) {
-                dbs += draw;
-                dDs = fmaf(dy, uu, dDs);
-                if (q >= 0) {
-                    const long long o = ki * p.in_dir + (img + q) * D + d;
-                    if (p.du) atomicAdd(p.du + o, fmaf(Dd, dy, dut));
-                    if (p.ddelta) atomicAdd(p.ddelta + o, draw);
+            if (grp == 0) {
+                if (dvalid) {
+                    dbs += draw;
+                    dDs = fmaf(dy, uu, dDs);
                 }
+                rd.u[j][cc] = fmaf(Dd, dy, dut);
+                rd.x[j][cc] = draw;
             }
-            if (cc == 0 && q >= 0) {
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const int n = 4 * grp + s;
-                    if (n >= N) continue;
-                    const long long o = ki * p.bc_dir + (img + q) * N + n;
-                    if (p.dB) atomicAdd(p.dB + o, dBv[s]);
-                    if (p.dC) atomicAdd(p.dC + o, dCv[s]);
-                }
-            }
+            // per-channel partials of dB and dC, summed over the channels after the chunk
+            *reinterpret_cast<float4*>(&rd.B[j][cc][4 * grp]) = make_float4(dBv[0], dBv[1], dBv[2], dBv[3]);
+            *reinterpret_cast<float4*>(&rd.C[j][cc][4 * grp]) = make_float4(dCv[0], dCv[1], dCv[2], dCv[3]);
         }
+        // add the chunk's token gradients: one atomic per (step, channel) and per
+        // (step, state), every lane taking its share
+        __syncwarp();
+#pragma unroll
+        for (int r = 0; r < BW_TOK * BW_CH / 32; ++r) {
+            const int e = lane + 32 * r;
+            const int j = e / BW_CH, ch = e % BW_CH, dd = c0 + ch;
+            const int q = st.pos[j];
+            if (q < 0 || dd >= D) continue;
+            const long long o = ki * p.in_dir + (img + q) * D + dd;
+            if (p.du) atomicAdd(p.du + o, rd.u[j][ch]);
+            if (p.ddelta) atomicAdd(p.ddelta + o, rd.x[j][ch]);
+        }
+#pragma unroll
+        for (int r = 0; r < BW_TOK * 16 / 32; ++r) {
+            const int e = lane + 32 * r;
+            const int j = e >> 4, n = e & 15;
+            const int q = st.pos[j];
+            if (q < 0 || n >= N) continue;
+            float sb = 0.f, sc = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < BW_CH; ++ch) {
+                sb += rd.B[j][ch][n];
+                sc += rd.C[j][ch][n];
+            }
+            const long long o = ki * p.bc_dir + (img + q) * N + n;
+            if (p.dB) atomicAdd(p.dB + o, sb);
+            if (p.dC) atomicAdd(p.dC + o, sc);
+        }
+        __syncwarp();
     }
     if (dvalid) {
 #pragma unroll
