@@ -127,14 +127,27 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback", 1965.0
 
 
-def source_digest():
+# device-code files each timed kernel is compiled from (host-side API code excluded)
+KERNEL_SOURCES = {
+    "stream_scan_kernel": ("vscan_stream.cuh", "vscan_common.cuh", "vscan_route.cuh"),
+    "resident_scan_kernel": ("vscan_resident.cuh", "vscan_stream.cuh", "vscan_common.cuh", "vscan_route.cuh"),
+    "pool_scan_kernel": ("vscan_pool.cuh", "vscan_common.cuh", "vscan_route.cuh"),
+    "bwd_scan_kernel": ("vscan_backward.cuh", "vscan_common.cuh", "vscan_route.cuh"),
+}
+
+
+def source_digest(kernel=None):
+    """Digest of the device code a kernel is built from (all kernel headers if None)."""
     csrc = os.path.join(ROOT, "vision_selective_state_b200", "csrc")
+    if kernel is None:
+        names = sorted(n for n in os.listdir(csrc) if n.endswith(".cuh"))
+    else:
+        names = sorted(KERNEL_SOURCES[kernel.split("<")[0]])
     h = hashlib.sha256()
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith(".cuh"):  # the kernels' device code; host-side API code excluded
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in names:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -144,7 +157,7 @@ def recorded_traffic(kernel, workload):
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
-    digest = source_digest()
+    digest = source_digest(kernel)
     with open(path) as f:
         for ln in f:
             if ln.startswith("#") or not ln.strip():
