@@ -187,7 +187,10 @@ cudaError_t launch_stream_n(const vscan::ScanParams& p, cudaStream_t s)
         if constexpr (sizeof(T) == 4) return launch_stream_mode<RK, T, N16, 1, MODE_OWNER, 1, FL>(p, 0, 4, s);
         else return launch_stream_mode<RK, T, N16, 4, MODE_OWNER, 1, FL>(p, 0, 1, s);
     } else if constexpr (RK == RK_BIDIR) {
-        return launch_stream_mode<RK, T, N16, 2, MODE_PARK, 1, FL>(p, 0, 1, s);
+        // two producer warps per direction (measured faster on Vim-Small); the fused
+        // convolution reads steps gathered by one producer warp and keeps one
+        constexpr int PW = (FL & FL_CONV) ? 1 : 2;
+        return launch_stream_mode<RK, T, N16, 2, MODE_PARK, PW, FL>(p, 0, 1, s);
     } else {
         return launch_stream_mode<RK, T, N16, 4, MODE_PARK, 1, FL>(p, 0, 1, s);
     }
