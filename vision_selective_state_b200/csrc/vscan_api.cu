@@ -162,17 +162,17 @@ uint64_t workspace_need(const vscan_route* r, const vscan_args* a)
     return 0;
 }
 
-template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL>
+template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL, int CH = vscan::ST_CH>
 cudaError_t launch_stream_mode(vscan::ScanParams p, int k_base, int grid_z, cudaStream_t s)
 {
-    const size_t smem = vscan::stream_smem_bytes<T, KC, MODE, FL>();
-    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL>,
+    const size_t smem = vscan::stream_smem_bytes<T, KC, MODE, FL, CH>();
+    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     p.k_base = k_base;
-    const dim3 grid((p.D + vscan::ST_CH - 1) / vscan::ST_CH, p.batch, grid_z);
-    vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL>
-        <<<grid, vscan::StreamShape<T, KC, MODE, PW>::THREADS, smem, s>>>(p);
+    const dim3 grid((p.D + CH - 1) / CH, p.batch, grid_z);
+    vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH>
+        <<<grid, vscan::StreamShape<T, KC, MODE, PW, CH>::THREADS, smem, s>>>(p);
     return cudaGetLastError();
 }
 

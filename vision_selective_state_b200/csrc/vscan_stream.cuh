@@ -1,10 +1,11 @@
 // Streaming routed selective scan: BIDIR, CROSS4 and ATROUS2 routes.
 //
-// One CTA covers one image b, a tile of 8 channels and KC directions of the
-// route, and runs them as a software pipeline over 16-step chunks with two
-// kinds of warps:
+// One CTA covers one image b, a tile of CH = 8 or 16 channels and KC directions
+// of the route, and runs them as a software pipeline over 16-step chunks with
+// two kinds of warps:
 //
-//   consumer warp (one per direction) runs only the recurrence. Lane 4*c + g
+//   consumer warps (CH / 8 per direction) run only the recurrence, each for 8
+//     channels of the tile. Lane 4*c + g
 //     owns channel c of the tile and states 4g..4g+3, so the 16 states of a
 //     channel sit on 4 adjacent lanes and the read-out sum over n is a 4-lane
 //     reduction. Per step and state ("Vision Mamba ...", sec. 4;
@@ -76,7 +77,7 @@ struct ScanParams {
 };
 
 constexpr int ST_TOK = 16;  // steps per chunk
-constexpr int ST_CH = 8;    // channels per CTA
+constexpr int ST_CH = 8;    // channels per consumer warp (a CTA covers CH = 8 or 16 channels)
 constexpr int ST_LOOK = 3;  // chunks between a gather and its discretization
 
 // ---- cp.async (16-byte, L2 only) ------------------------------------------------
@@ -93,11 +94,11 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
 // Gathered per-token rows of one direction's chunk, in the I/O type.
-template <typename T>
+template <typename T, int CH>
 struct __align__(16) TokStage {
-    T u[ST_TOK][ST_CH];
-    T d[ST_TOK][ST_CH];
-    T z[ST_TOK][ST_CH];
+    T u[ST_TOK][CH];
+    T d[ST_TOK][CH];
+    T z[ST_TOK][CH];
     int pos[ST_TOK];  // token index, -1 pad, -2 past the end
     int fin[ST_TOK];  // MODE_PARK: 1 if this direction adds up the token
 };
@@ -116,24 +117,24 @@ template <> struct PrepBC<true> {
     float4 B[ST_TOK][4];
     float4 C[ST_TOK][4];
 };
-template <bool ON> struct PrepRD {};
-template <> struct PrepRD<true> {
-    float rd[ST_TOK][ST_CH];  // 1 / Delta (inf for Delta = 0, where zoh_phi does not use it)
+template <bool ON, int CH> struct PrepRD {};
+template <int CH> struct PrepRD<true, CH> {
+    float rd[ST_TOK][CH];  // 1 / Delta (inf for Delta = 0, where zoh_phi does not use it)
 };
 
-template <bool BCF, bool ZOH>
-struct __align__(16) PrepStage : PrepBC<BCF>, PrepRD<ZOH> {
-    float2 dd[ST_TOK][ST_CH];  // {Delta after bias + softplus (0 past the end), Delta * u}
+template <bool BCF, bool ZOH, int CH>
+struct __align__(16) PrepStage : PrepBC<BCF>, PrepRD<ZOH, CH> {
+    float2 dd[ST_TOK][CH];  // {Delta after bias + softplus (0 past the end), Delta * u}
 };
 
 // FL_CONV: the convolved u of the last three chunks of each direction, for the
 // skip term D*u of the epilogue.
-template <bool ON, int KC> struct ConvRing {};
-template <int KC> struct ConvRing<true, KC> {
-    float uc[KC][3][ST_TOK][ST_CH];
+template <bool ON, int KC, int CH> struct ConvRing {};
+template <int KC, int CH> struct ConvRing<true, KC, CH> {
+    float uc[KC][3][ST_TOK][CH];
 };
 
-template <typename T, int KC, int MODE, int PW = 1>
+template <typename T, int KC, int MODE, int PW = 1, int CH = ST_CH>
 struct StreamShape {
     static constexpr bool F32 = sizeof(T) == 4;
     static constexpr bool PARK = MODE == MODE_PARK;
@@ -143,23 +144,26 @@ struct StreamShape {
     // B/C slot: until discretized at tau = c-1 (bf16) or consumed at tau = c (f32)
     static constexpr int NBC = ST_LOOK + (F32 ? 2 : 1);
     static constexpr int NY = PARK ? 3 : 2;  // output ring
-    static constexpr int THREADS = 32 * KC * (1 + PW);  // a consumer and PW producers per direction
-    static constexpr int SPW = ST_TOK / PW;             // steps of a chunk per producer warp
-    static constexpr int RPL = SPW / 4;                 // (step, channel) items per producer lane
+    static constexpr int CW = CH / ST_CH;                // consumer warps per direction
+    static constexpr int THREADS = 32 * KC * (CW + PW);  // CW consumers and PW producers per direction
+    static constexpr int SPW = ST_TOK / PW;              // steps of a chunk per producer warp
+    static constexpr int RPL = SPW * CH / 32;            // (step, channel) items per producer lane
+    static constexpr int NBCV = SPW / 8;                 // bf16 B/C quads converted per producer lane
     static_assert(PW == 1 || PW == 2, "one or two producer warps per direction");
+    static_assert(CH == 8 || CH == 16, "8 or 16 channels per CTA");
 };
 
-template <typename T, int KC, int MODE, int FL = 0>
-struct StreamSmem : ConvRing<(FL & FL_CONV) != 0, KC> {
+template <typename T, int KC, int MODE, int FL = 0, int CH = ST_CH>
+struct StreamSmem : ConvRing<(FL & FL_CONV) != 0, KC, CH> {
     using S = StreamShape<T, KC, MODE>;
-    TokStage<T> tok[KC][S::NR];
+    TokStage<T, CH> tok[KC][S::NR];
     BCStage<T> bc[KC][S::NBC];
-    PrepStage<!S::F32, (FL & FL_ZOH) != 0> prep[KC][2];
-    float yout[KC][S::NY][ST_TOK][ST_CH];
+    PrepStage<!S::F32, (FL & FL_ZOH) != 0, CH> prep[KC][2];
+    float yout[KC][S::NY][ST_TOK][CH];
 };
 
-template <typename T, int KC, int MODE, int FL = 0>
-constexpr size_t stream_smem_bytes() { return sizeof(StreamSmem<T, KC, MODE, FL>); }
+template <typename T, int KC, int MODE, int FL = 0, int CH = ST_CH>
+constexpr size_t stream_smem_bytes() { return sizeof(StreamSmem<T, KC, MODE, FL, CH>); }
 
 // Direction that adds up token p: the one visiting p in the latest chunk.
 template <int RK>
@@ -178,11 +182,12 @@ __device__ __forceinline__ int finalizer(const RouteGeom& g, int p)
     return best_k;
 }
 
-template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL>
-__global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_scan_kernel(const ScanParams p)
+template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL, int CH>
+__global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) stream_scan_kernel(const ScanParams p)
 {
-    using S = StreamShape<T, KC, MODE, PW>;
-    constexpr int SPW = S::SPW, RPL = S::RPL;
+    using S = StreamShape<T, KC, MODE, PW, CH>;
+    constexpr int SPW = S::SPW, RPL = S::RPL, CW = S::CW, NBCV = S::NBCV;
+    constexpr int RSTEP = 32 / CH;  // rows between a producer lane's items
     constexpr bool ZOH = (FL & FL_ZOH) != 0;
     constexpr bool CONV = (FL & FL_CONV) != 0;
     static_assert(!CONV || RK == RK_BIDIR, "the fused convolution is defined for the bidirectional route");
@@ -192,22 +197,22 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
     constexpr bool F32 = S::F32;
     constexpr int KR = (RK == RK_BIDIR) ? 2 : 4;  // directions of the route
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    StreamSmem<T, KC, MODE, FL>& sm = *reinterpret_cast<StreamSmem<T, KC, MODE, FL>*>(smem_raw);
+    StreamSmem<T, KC, MODE, FL, CH>& sm = *reinterpret_cast<StreamSmem<T, KC, MODE, FL, CH>*>(smem_raw);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int b = blockIdx.y;
-    const int c0 = blockIdx.x * ST_CH;
+    const int c0 = blockIdx.x * CH;
     const int D = p.D, N = p.N, L = p.g.L, tokens = p.g.tokens;
     const int nchunks = (L + ST_TOK - 1) / ST_TOK;
     const int last_tau = nchunks + (PARK ? 1 : 0);
     const long long img = (long long)b * tokens;
 
-    if (warp < KC) {
+    if (warp < KC * CW) {
         // =============================== consumer =================================
-        const int kl = warp;
+        const int kl = warp / CW;
         const int k = p.k_base + blockIdx.z * KC + kl;
-        const int cc = lane >> 2, grp = lane & 3;
+        const int cc = (warp % CW) * ST_CH + (lane >> 2), grp = lane & 3;  // channel of the tile
         const int d = c0 + cc;
         const bool dvalid = d < D;
         float a2[4];
@@ -295,7 +300,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
                 }
                 // stores after every load of the chunk, so none of them waits on a store
 #pragma unroll
-                for (int q = 0; q < 4; ++q) yo[(4 * q + grp) * ST_CH + cc] = yv[q];
+                for (int q = 0; q < 4; ++q) yo[(4 * q + grp) * CH + cc] = yv[q];
             }
             __syncthreads();
         }
@@ -303,10 +308,11 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
     }
 
     // ================================= producer ===================================
-    const int kl = (warp - KC) / PW;
-    const int j0 = ((warp - KC) % PW) * SPW;        // first step of a chunk this warp owns
+    const int kl = (warp - KC * CW) / PW;
+    const int j0 = ((warp - KC * CW) % PW) * SPW;   // first step of a chunk this warp owns
     const int k = p.k_base + blockIdx.z * KC + kl;  // direction this producer serves
-    const int ce = lane & 7;  // channel of the tile this lane discretizes / stores
+    const int ce = lane % CH;  // channel of the tile this lane discretizes / stores
+    const int jl = j0 + lane / CH;  // first row of this lane's items; then every RSTEP rows
     const int dch = c0 + ce;
     const bool evalid = dch < D;
     const float bias_k = (evalid && p.bias) ? __ldg(p.bias + k * p.v_dir + dch) : 0.f;
@@ -342,47 +348,26 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
                 st.pos[j0 + lane] = mypos;
                 if constexpr (PARK) st.fin[j0 + lane] = (mypos >= 0 && finalizer<RK>(p.g, mypos) == k) ? 1 : 0;
             }
-            if (F32 && PW == 1) {
-                // u, Delta, z: 16 steps x 32 bytes; lane -> (step lane>>1, 4-channel half lane&1)
-                const int j = lane >> 1, hf = lane & 1;
-                const int pj = __shfl_sync(FULL_MASK, mypos, j);
-                const bool ok = pj >= 0 && (c0 + 4 * hf) < D;
-                const long long off = (long long)(ok ? pj : 0) * D + 4 * hf;
-                cp_async16(&st.u[j][4 * hf], u_base + off, ok);
-                cp_async16(&st.d[j][4 * hf], d_base + off, ok);
-                if (z_base) cp_async16(&st.z[j][4 * hf], z_base + off, ok);
-            } else if (F32) {
-                // 8 steps x 32 bytes per tensor: lanes 0-15 take u and z, lanes 16-31 take Delta;
-                // lane -> (step (lane&15)>>1, 4-channel half lane&1)
-                const int i = (lane & 15) >> 1, hf = lane & 1, j = j0 + i;
-                const int pj = __shfl_sync(FULL_MASK, mypos, i);
-                const bool ok = pj >= 0 && (c0 + 4 * hf) < D;
-                const long long off = (long long)(ok ? pj : 0) * D + 4 * hf;
-                if (lane < 16) {
-                    cp_async16(&st.u[j][4 * hf], u_base + off, ok);
-                    if (z_base) cp_async16(&st.z[j][4 * hf], z_base + off, ok);
-                } else {
-                    cp_async16(&st.d[j][4 * hf], d_base + off, ok);
-                }
-            } else {
-                // SPW steps x 16 bytes per tensor: lane -> (tensor lane / SPW, step lane % SPW)
-                const int i = lane & (SPW - 1), j = j0 + i, which = lane / SPW;
-                const int pj = __shfl_sync(FULL_MASK, mypos, i);
-                const bool ok = pj >= 0;
-                const long long off = (long long)(ok ? pj : 0) * D;
-                if (PW == 1) {
-                    if (lane < 16) {
-                        cp_async16(&st.u[j][0], u_base + off, ok);
-                        if (z_base) cp_async16(&st.z[j][0], z_base + off, ok);
-                    } else {
-                        cp_async16(&st.d[j][0], d_base + off, ok);
+            {
+                // u, Delta, z: SPW steps x CH channels per tensor, in 16-byte pieces;
+                // copy f -> (tensor, step, piece). Every lane runs every round (the
+                // position shuffle needs the whole warp); copies past the count skip.
+                constexpr int EL = 16 / sizeof(T);          // channels per piece
+                constexpr int PCS = CH / EL;                // pieces per step and tensor
+                constexpr int NT = 3 * SPW * PCS;           // copies of the three tensors
+#pragma unroll
+                for (int it = 0; it < (NT + 31) / 32; ++it) {
+                    const int f = lane + 32 * it;
+                    const int tsr = f / (SPW * PCS), rem = f % (SPW * PCS);
+                    const int i = rem / PCS, cel = (rem % PCS) * EL;
+                    const int pj = __shfl_sync(FULL_MASK, mypos, i);
+                    if (f < NT && (tsr < 2 || z_base)) {
+                        const bool ok = pj >= 0 && (c0 + cel) < D;
+                        const long long off = (long long)(ok ? pj : 0) * D + cel;
+                        T* dst = tsr == 0 ? &st.u[j0 + i][cel] : (tsr == 1 ? &st.d[j0 + i][cel] : &st.z[j0 + i][cel]);
+                        const T* src = (tsr == 0 ? u_base : (tsr == 1 ? d_base : z_base)) + off;
+                        cp_async16(dst, src, ok);
                     }
-                } else if (which == 0) {
-                    cp_async16(&st.u[j][0], u_base + off, ok);
-                } else if (which == 1) {
-                    cp_async16(&st.d[j][0], d_base + off, ok);
-                } else if (which == 2 && z_base) {
-                    cp_async16(&st.z[j][0], z_base + off, ok);
                 }
             }
             if (N16) {
@@ -442,7 +427,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
         bool live[RPL];
 #pragma unroll
         for (int r = 0; r < RPL; ++r) {
-            const int j = j0 + (lane >> 3) + 4 * r;
+            const int j = jl + RSTEP * r;
             xd[r] = to_float(st.d[j][ce]);
             xu[r] = to_float(st.u[j][ce]);
             live[r] = st.pos[j] != -2 && evalid;  // past the end: a no-op step
@@ -453,7 +438,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
             const auto& prev = sm.tok[kl][(c + NR - 1) % NR];
 #pragma unroll
             for (int r = 0; r < RPL; ++r) {
-                const int j = j0 + (lane >> 3) + 4 * r;
+                const int j = jl + RSTEP * r;
                 float acc = kb;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -467,11 +452,11 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
                 sm.uc[kl][c % 3][j][ce] = xu[r];
             }
         }
-        float4 cb[RPL / 2], cv[RPL / 2];
+        float4 cb[NBCV], cv[NBCV];
         if constexpr (!F32) {
             const BCStage<T>& sb = sm.bc[kl][c % NBC];
 #pragma unroll
-            for (int r = 0; r < RPL / 2; ++r) {
+            for (int r = 0; r < NBCV; ++r) {
                 const int f = lane + 32 * r;  // (step j0 + f>>2, quad f&3)
                 const int j = j0 + (f >> 2), q = f & 3;
                 cb[r] = make_float4(to_float(sb.B[j][4 * q]), to_float(sb.B[j][4 * q + 1]),
@@ -488,14 +473,14 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
             out[r] = make_float2(dsp, live[r] ? dsp * xu[r] : 0.f);
         }
 #pragma unroll
-        for (int r = 0; r < RPL; ++r) pr.dd[j0 + (lane >> 3) + 4 * r][ce] = out[r];
+        for (int r = 0; r < RPL; ++r) pr.dd[jl + RSTEP * r][ce] = out[r];
         if constexpr (ZOH) {
 #pragma unroll
-            for (int r = 0; r < RPL; ++r) pr.rd[j0 + (lane >> 3) + 4 * r][ce] = fast_rcp(out[r].x);
+            for (int r = 0; r < RPL; ++r) pr.rd[jl + RSTEP * r][ce] = fast_rcp(out[r].x);
         }
         if constexpr (!F32) {
 #pragma unroll
-            for (int r = 0; r < RPL / 2; ++r) {
+            for (int r = 0; r < NBCV; ++r) {
                 const int f = lane + 32 * r;
                 pr.B[j0 + (f >> 2)][f & 3] = cb[r];
                 pr.C[j0 + (f >> 2)][f & 3] = cv[r];
@@ -511,13 +496,13 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
         float yk[RPL], zz[RPL];
 #pragma unroll
         for (int r = 0; r < RPL; ++r) {
-            const int j = j0 + (lane >> 3) + 4 * r;
+            const int j = jl + RSTEP * r;
             pj[r] = evalid ? st.pos[j] : -1;
             fin[r] = PARK ? st.fin[j] : 1;
             float uj;
             if constexpr (CONV) uj = sm.uc[kl][c % 3][j][ce];
             else uj = to_float(st.u[j][ce]);
-            yk[r] = fmaf(Dk, uj, yo[j * ST_CH + ce]);
+            yk[r] = fmaf(Dk, uj, yo[j * CH + ce]);
             zz[r] = z_base ? to_float(st.z[j][ce]) : 0.f;
         }
         // every row computes its value; only the stores are predicated
@@ -532,11 +517,11 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
         }
 #pragma unroll
         for (int r = 0; r < RPL; ++r) {
-            const int j = j0 + (lane >> 3) + 4 * r;
+            const int j = jl + RSTEP * r;
             if constexpr (MODE == MODE_OWNER) {
                 if (pj[r] >= 0) store_elem<T>(y_base + pj[r] * D, o[r]);
             } else {
-                if (pj[r] >= 0 && fin[r]) yo[j * ST_CH + ce] = o[r];
+                if (pj[r] >= 0 && fin[r]) yo[j * CH + ce] = o[r];
                 if (pj[r] >= 0 && !fin[r]) park(k)[pj[r] * D] = o[r];
             }
         }
@@ -550,7 +535,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
         const auto& st = sm.tok[kl][c % NR];
 #pragma unroll
         for (int r = 0; r < RPL; ++r) {
-            const int j = j0 + (lane >> 3) + 4 * r;
+            const int j = jl + RSTEP * r;
             const int pj = st.pos[j];
             float acc = 0.f;
             if (evalid && pj >= 0 && st.fin[j]) {
@@ -568,10 +553,10 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW>::THREADS) stream_
         const float* yo = &sm.yout[kl][c % NY][0][0];
 #pragma unroll
         for (int r = 0; r < RPL; ++r) {
-            const int j = j0 + (lane >> 3) + 4 * r;
+            const int j = jl + RSTEP * r;
             const int pj = st.pos[j];
             if (!evalid || pj < 0 || !st.fin[j]) continue;
-            float o = (yo[j * ST_CH + ce] + parked[r]) * p.merge_scale;
+            float o = (yo[j * CH + ce] + parked[r]) * p.merge_scale;
             if (z_base) o *= silu_f(to_float(st.z[j][ce]));
             store_elem<T>(y_base + pj * D, o);
         }
