@@ -300,7 +300,7 @@ cudaError_t launch_pool(const vscan::PoolParams& p, int fl, cudaStream_t s, size
 }
 
 template <typename T>
-vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s)
+vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s, float* ckpt = nullptr)
 {
     const vscan::RouteGeom& g = r->g;
     const long long plane = (long long)a->batch * tokens_of(r, a);
@@ -341,7 +341,8 @@ vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s)
         p.merge_scale = a->merge_scale;
         p.scratch = static_cast<float*>(a->workspace);
         p.conv_w = a->conv_w; p.conv_b = a->conv_b;
-        const int nc = choose_chunks(r, a);
+        p.ckpt = ckpt;
+        const int nc = ckpt ? 1 : choose_chunks(r, a);  // checkpoints come from the streaming kernel
         if (nc > 1) {
             cudaError_t e;
             switch (g.kind) {
@@ -365,7 +366,7 @@ vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s)
     return VSCAN_OK;
 }
 
-vscan_status forward_device(const vscan_route* r, const vscan_args* a, cudaStream_t s)
+vscan_status forward_device(const vscan_route* r, const vscan_args* a, cudaStream_t s, float* ckpt = nullptr)
 {
     const uint64_t need = workspace_need(r, a);
     if (need > 0) {
@@ -375,7 +376,7 @@ vscan_status forward_device(const vscan_route* r, const vscan_args* a, cudaStrea
         if (!aligned16(a->workspace)) return fail(VSCAN_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
     }
     if (a->batch == 0) return VSCAN_OK;
-    return a->dtype == VSCAN_F32 ? dispatch<float>(r, a, s) : dispatch<__nv_bfloat16>(r, a, s);
+    return a->dtype == VSCAN_F32 ? dispatch<float>(r, a, s, ckpt) : dispatch<__nv_bfloat16>(r, a, s, ckpt);
 }
 
 __global__ void route_map_kernel(vscan::RouteGeom g, int32_t* out)
@@ -523,7 +524,10 @@ vscan_status backward_device(const vscan_route* r, const vscan_args* a, const vo
     fa.y = ws + Lo.pre;
     fa.workspace = ws + Lo.fwd_ws;
     fa.workspace_bytes = Lo.pre - Lo.fwd_ws;
-    vscan_status st = forward_device(r, &fa, s);
+    // grid routes: the forward's streaming kernel also saves the state at every
+    // chunk boundary, so the adjoint scan needs no forward pass of its own
+    float* ckpt = reinterpret_cast<float*>(ws + Lo.ckpt);
+    vscan_status st = forward_device(r, &fa, s, pooled ? nullptr : ckpt);
     if (st != VSCAN_OK) return st;
     // gradient of the gate and of the merged value
     float* gy = reinterpret_cast<float*>(ws + Lo.gy);
@@ -536,7 +540,8 @@ vscan_status backward_device(const vscan_route* r, const vscan_args* a, const vo
     p.a_dir = a->per_dir_params ? a->channels * a->d_state : 0;
     p.v_dir = a->per_dir_params ? a->channels : 0;
     p.A = a->A; p.Dskip = a->Dskip; p.bias = a->delta_bias; p.softplus = a->delta_softplus;
-    p.ckpt = reinterpret_cast<float*>(ws + Lo.ckpt);
+    p.ckpt = ckpt;
+    p.ckpt_ready = pooled ? 0 : 1;
     p.dA = gr->dA; p.dD = gr->dDskip; p.dbias = gr->dbias;
     const dim3 grid((unsigned)((D + vscan::BW_CH - 1) / vscan::BW_CH), (unsigned)b, (unsigned)K);
     if (!pooled) {

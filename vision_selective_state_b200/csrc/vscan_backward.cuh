@@ -51,6 +51,7 @@ struct BwdParams {
     int softplus;
     const float* gy;   // [batch][tokens][D]: dL / d(merged pre-gate value)
     float* ckpt;       // [K][batch][nchunks][D][16]
+    int ckpt_ready;    // 1: the forward pass already saved the checkpoints (skip pass 1)
     float* du;         // [Ki][batch][tokens][D]
     float* ddelta;     // [Ki][batch][tokens][D]
     float* dB;         // [Ki][batch][tokens][N]
@@ -100,11 +101,23 @@ __global__ void bwd_pool_kernel(RouteGeom g, int batch, int D, int N, int Ki, co
     for (int k = 0; k < Ki; ++k) {
         for (int d = threadIdx.x; d < D; d += blockDim.x) {
             float su = 0.f, sr = 0.f, sg = 0.f;
-            for (int j = 0; j < cnt; ++j) {
-                const long long o = (img + member(j)) * D + d;
-                su += to_float(u[k * in_dir + o]);
-                sr += to_float(delta[k * in_dir + o]);
-                if (k == 0) sg += gy[o];
+            constexpr int U = 8;  // members per round, all loads issued before the sums
+            for (int j0 = 0; j0 < cnt; j0 += U) {
+                float vu[U], vr[U], vg[U];
+#pragma unroll
+                for (int v = 0; v < U; ++v) {
+                    const bool in = j0 + v < cnt;
+                    const long long o = (img + member(in ? j0 + v : 0)) * D + d;
+                    vu[v] = in ? to_float(u[k * in_dir + o]) : 0.f;
+                    vr[v] = in ? to_float(delta[k * in_dir + o]) : 0.f;
+                    vg[v] = (in && k == 0) ? gy[o] : 0.f;
+                }
+#pragma unroll
+                for (int v = 0; v < U; ++v) {
+                    su += vu[v];
+                    sr += vr[v];
+                    sg += vg[v];
+                }
             }
             const long long po = (((long long)k * batch + b) * Lp + i) * D + d;
             pu[po] = su * inv;
@@ -113,10 +126,21 @@ __global__ void bwd_pool_kernel(RouteGeom g, int batch, int D, int N, int Ki, co
         }
         for (int n = threadIdx.x; n < N; n += blockDim.x) {
             float sb = 0.f, sc = 0.f;
-            for (int j = 0; j < cnt; ++j) {
-                const long long o = (img + member(j)) * N + n;
-                sb += to_float(B[k * bc_dir + o]);
-                sc += to_float(C[k * bc_dir + o]);
+            constexpr int U = 8;
+            for (int j0 = 0; j0 < cnt; j0 += U) {
+                float vb[U], vc[U];
+#pragma unroll
+                for (int v = 0; v < U; ++v) {
+                    const bool in = j0 + v < cnt;
+                    const long long o = (img + member(in ? j0 + v : 0)) * N + n;
+                    vb[v] = in ? to_float(B[k * bc_dir + o]) : 0.f;
+                    vc[v] = in ? to_float(C[k * bc_dir + o]) : 0.f;
+                }
+#pragma unroll
+                for (int v = 0; v < U; ++v) {
+                    sb += vb[v];
+                    sc += vc[v];
+                }
             }
             const long long po = (((long long)k * batch + b) * Lp + i) * N + n;
             pB[po] = sb * inv;
@@ -258,7 +282,7 @@ __global__ void __launch_bounds__(32) bwd_scan_kernel(const BwdParams p)
 
     // ---- pass 1: forward recurrence, state saved at every chunk boundary --------
     float h[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int c = 0; c < nch; ++c) {
+    for (int c = 0; c < (p.ckpt_ready ? 0 : nch); ++c) {
         if (dvalid) {
 #pragma unroll
             for (int s = 0; s < 4; ++s) ck[((long long)c * D + d) * 16 + 4 * grp + s] = h[s];

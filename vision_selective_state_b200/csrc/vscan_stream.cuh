@@ -74,6 +74,8 @@ struct ScanParams {
     float* scratch;    // PARK: [K][batch][tokens][D] float32
     const float* conv_w;  // FL_CONV: [Kp][D][4]
     const float* conv_b;  // FL_CONV: [Kp][D] (nullable)
+    float* ckpt;          // nullable: [K][batch][ceil(L/16)][D][16], the state entering every
+                          // 16-step chunk (saved for the backward pass)
 };
 
 constexpr int ST_TOK = 16;  // steps per chunk
@@ -229,8 +231,13 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
         float2 h01 = make_float2(0.f, 0.f), h23 = h01;
         __syncthreads();  // prologue: chunk 0 discretized
 
+        float* ck = (p.ckpt && dvalid)
+                        ? p.ckpt + (((long long)k * p.batch + b) * nchunks * D + d) * 16 + 4 * grp : nullptr;
         for (int tau = 0; tau <= last_tau; ++tau) {
             if (tau < nchunks) {
+                if (ck) {  // state entering chunk tau
+                    *reinterpret_cast<float4*>(ck + (long long)tau * D * 16) = make_float4(h01.x, h01.y, h23.x, h23.y);
+                }
                 const auto& pr = sm.prep[kl][tau & 1];
                 const BCStage<T>& bcs = sm.bc[kl][tau % NBC];
                 float* yo = &sm.yout[kl][tau % NY][0][0];
