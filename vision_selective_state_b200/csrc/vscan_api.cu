@@ -506,9 +506,13 @@ vscan_status backward_device(const vscan_route* r, const vscan_args* a, const vo
     const bool pooled = is_pool(g.kind);
 
     struct Zero { void* p; size_t bytes; };
+    // token gradients are accumulated with atomics on the grid routes; the pooled
+    // routes write them in full (bwd_unpool_kernel) and zero their pooled copies
     const Zero zeros[] = {
-        {gr->du, (size_t)Ki * b * TK * D * 4}, {gr->ddelta, (size_t)Ki * b * TK * D * 4},
-        {gr->dB, (size_t)Ki * b * TK * N * 4}, {gr->dC, (size_t)Ki * b * TK * N * 4},
+        {pooled ? nullptr : gr->du, (size_t)Ki * b * TK * D * 4},
+        {pooled ? nullptr : gr->ddelta, (size_t)Ki * b * TK * D * 4},
+        {pooled ? nullptr : gr->dB, (size_t)Ki * b * TK * N * 4},
+        {pooled ? nullptr : gr->dC, (size_t)Ki * b * TK * N * 4},
         {gr->dA, (size_t)Kp * D * N * 4}, {gr->dDskip, (size_t)Kp * D * 4}, {gr->dbias, (size_t)Kp * D * 4},
         {pooled ? ws + Lo.dpu : nullptr, Lo.dpraw - Lo.dpu}, {pooled ? ws + Lo.dpraw : nullptr, Lo.dpB - Lo.dpraw},
         {pooled ? ws + Lo.dpB : nullptr, Lo.dpC - Lo.dpB}, {pooled ? ws + Lo.dpC : nullptr, Lo.total - Lo.dpC},
