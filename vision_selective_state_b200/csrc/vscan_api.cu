@@ -207,6 +207,7 @@ template <int RK, typename T>
 cudaError_t launch_stream(const vscan::ScanParams& p, int fl, cudaStream_t s)
 {
     using namespace vscan;
+    if (fl & FL_CKPT) return launch_stream_fl<RK, T, FL_CKPT>(p, s);  // backward's forward run (plain scan)
     if constexpr (RK == RK_BIDIR) {
         switch (fl) {
         case FL_ZOH: return launch_stream_fl<RK, T, FL_ZOH>(p, s);
@@ -305,7 +306,7 @@ vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s,
     const vscan::RouteGeom& g = r->g;
     const long long plane = (long long)a->batch * tokens_of(r, a);
     const int fl = ((a->flags & VSCAN_FLAG_ZOH) ? vscan::FL_ZOH : 0) | (a->conv_w ? vscan::FL_CONV : 0) |
-                   (a->token_pos ? vscan::FL_MASK : 0);
+                   (a->token_pos ? vscan::FL_MASK : 0) | (ckpt ? vscan::FL_CKPT : 0);
     if (is_pool(g.kind)) {
         vscan::PoolParams p{};
         p.g = g;

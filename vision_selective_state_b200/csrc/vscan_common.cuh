@@ -82,9 +82,10 @@ __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 v
 }
 
 // Optional steps of the scan, as kernel template flags: the zero-order-hold
-// write term, the fused causal convolution of u, and (pooled routes) a masked
-// token set addressed by grid position.
-enum ScanFlags : int { FL_ZOH = 1, FL_CONV = 2, FL_MASK = 4 };
+// write term, the fused causal convolution of u, (pooled routes) a masked
+// token set addressed by grid position, and (streaming kernel) saving the state
+// at every chunk boundary for the backward pass.
+enum ScanFlags : int { FL_ZOH = 1, FL_CONV = 2, FL_MASK = 4, FL_CKPT = 8 };
 
 // ---- discretization ---------------------------------------------------------
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32). The retention

@@ -39,6 +39,8 @@
 // Optional steps (template flags FL):
 //   FL_ZOH   the write term uses the zero-order-hold gain phi(Delta A) (zoh_phi)
 //            instead of Delta*B*u ("Norm or Direction? ...", Eq. 2).
+//   FL_CKPT  the consumer also stores its state entering every chunk (ckpt),
+//            for the backward pass.
 //   FL_CONV  (BIDIR) u holds the convolution input x; the producer applies the
 //            direction's kernel-four causal Conv1d + SiLU along the route
 //            ("Vision Mamba ...", "Inside the released Vim block"), reading the
@@ -192,6 +194,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
     constexpr int RSTEP = 32 / CH;  // rows between a producer lane's items
     constexpr bool ZOH = (FL & FL_ZOH) != 0;
     constexpr bool CONV = (FL & FL_CONV) != 0;
+    constexpr bool CKPT = (FL & FL_CKPT) != 0;
     static_assert(!CONV || RK == RK_BIDIR, "the fused convolution is defined for the bidirectional route");
     static_assert(!CONV || PW == 1, "the convolution reads steps gathered by the same producer warp");
     constexpr int NR = S::NR, NBC = S::NBC, NY = S::NY;
@@ -231,12 +234,12 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
         float2 h01 = make_float2(0.f, 0.f), h23 = h01;
         __syncthreads();  // prologue: chunk 0 discretized
 
-        float* ck = (p.ckpt && dvalid)
+        float* ck = (CKPT && dvalid)
                         ? p.ckpt + (((long long)k * p.batch + b) * nchunks * D + d) * 16 + 4 * grp : nullptr;
         for (int tau = 0; tau <= last_tau; ++tau) {
             if (tau < nchunks) {
-                if (ck) {  // state entering chunk tau
-                    *reinterpret_cast<float4*>(ck + (long long)tau * D * 16) = make_float4(h01.x, h01.y, h23.x, h23.y);
+                if constexpr (CKPT) {  // state entering chunk tau
+                    if (ck) *reinterpret_cast<float4*>(ck + (long long)tau * D * 16) = make_float4(h01.x, h01.y, h23.x, h23.y);
                 }
                 const auto& pr = sm.prep[kl][tau & 1];
                 const BCStage<T>& bcs = sm.bc[kl][tau % NBC];
