@@ -358,6 +358,52 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
                 st.pos[j0 + lane] = mypos;
                 if constexpr (PARK) st.fin[j0 + lane] = (mypos >= 0 && finalizer<RK>(p.g, mypos) == k) ? 1 : 0;
             }
+            if constexpr (CH == ST_CH) {
+                // 8-channel tiles: one 16- or 32-byte row piece per lane and tensor
+                if (F32 && PW == 1) {
+                    // u, Delta, z: 16 steps x 32 bytes; lane -> (step lane>>1, 4-channel half lane&1)
+                    const int j = lane >> 1, hf = lane & 1;
+                    const int pj = __shfl_sync(FULL_MASK, mypos, j);
+                    const bool ok = pj >= 0 && (c0 + 4 * hf) < D;
+                    const long long off = (long long)(ok ? pj : 0) * D + 4 * hf;
+                    cp_async16(&st.u[j][4 * hf], u_base + off, ok);
+                    cp_async16(&st.d[j][4 * hf], d_base + off, ok);
+                    if (z_base) cp_async16(&st.z[j][4 * hf], z_base + off, ok);
+                } else if (F32) {
+                    // 8 steps x 32 bytes per tensor: lanes 0-15 take u and z, lanes 16-31 take Delta;
+                    // lane -> (step (lane&15)>>1, 4-channel half lane&1)
+                    const int i = (lane & 15) >> 1, hf = lane & 1, j = j0 + i;
+                    const int pj = __shfl_sync(FULL_MASK, mypos, i);
+                    const bool ok = pj >= 0 && (c0 + 4 * hf) < D;
+                    const long long off = (long long)(ok ? pj : 0) * D + 4 * hf;
+                    if (lane < 16) {
+                        cp_async16(&st.u[j][4 * hf], u_base + off, ok);
+                        if (z_base) cp_async16(&st.z[j][4 * hf], z_base + off, ok);
+                    } else {
+                        cp_async16(&st.d[j][4 * hf], d_base + off, ok);
+                    }
+                } else {
+                    // SPW steps x 16 bytes per tensor: lane -> (tensor lane / SPW, step lane % SPW)
+                    const int i = lane & (SPW - 1), j = j0 + i, which = lane / SPW;
+                    const int pj = __shfl_sync(FULL_MASK, mypos, i);
+                    const bool ok = pj >= 0;
+                    const long long off = (long long)(ok ? pj : 0) * D;
+                    if (PW == 1) {
+                        if (lane < 16) {
+                            cp_async16(&st.u[j][0], u_base + off, ok);
+                            if (z_base) cp_async16(&st.z[j][0], z_base + off, ok);
+                        } else {
+                            cp_async16(&st.d[j][0], d_base + off, ok);
+                        }
+                    } else if (which == 0) {
+                        cp_async16(&st.u[j][0], u_base + off, ok);
+                    } else if (which == 1) {
+                        cp_async16(&st.d[j][0], d_base + off, ok);
+                    } else if (which == 2 && z_base) {
+                        cp_async16(&st.z[j][0], z_base + off, ok);
+                    }
+                }
+            } else
             {
                 // u, Delta, z: SPW steps x CH channels per tensor, in 16-byte pieces;
                 // copy f -> (tensor, step, piece). Every lane runs every round (the
