@@ -452,6 +452,8 @@ vscan_status static_scratch_address(void** out)
 }
 
 // ---- backward ----------------------------------------------------------------------
+// the streaming kernel saves its state every ST_TOK steps for the adjoint scan's BW_TOK chunks
+static_assert(vscan::ST_TOK == vscan::BW_TOK, "checkpoint spacing of the forward and backward scans");
 struct BwdLayout {
     size_t fwd_ws, pre, gy, ckpt, pu, praw, pB, pC, pg, dpu, dpraw, dpB, dpC, total;
 };

@@ -280,9 +280,9 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
                 };
                 front(0);
                 front(1);
-                float yv[4];
+                float yv[ST_TOK / 4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < ST_TOK / 4; ++q) {
                     float yp[4];
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
                 }
                 // stores after every load of the chunk, so none of them waits on a store
 #pragma unroll
-                for (int q = 0; q < 4; ++q) yo[(4 * q + grp) * CH + cc] = yv[q];
+                for (int q = 0; q < ST_TOK / 4; ++q) yo[(4 * q + grp) * CH + cc] = yv[q];
             }
             __syncthreads();
         }
@@ -358,8 +358,8 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
                 st.pos[j0 + lane] = mypos;
                 if constexpr (PARK) st.fin[j0 + lane] = (mypos >= 0 && finalizer<RK>(p.g, mypos) == k) ? 1 : 0;
             }
-            if constexpr (CH == ST_CH) {
-                // 8-channel tiles: one 16- or 32-byte row piece per lane and tensor
+            if constexpr (CH == ST_CH && ST_TOK == 16) {
+                // 8-channel tiles of 16 steps: one 16- or 32-byte row piece per lane and tensor
                 if (F32 && PW == 1) {
                     // u, Delta, z: 16 steps x 32 bytes; lane -> (step lane>>1, 4-channel half lane&1)
                     const int j = lane >> 1, hf = lane & 1;
@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
                         cp_async16(&sb.B[j0 + (f >> 2)][4 * (f & 3)], B_base + off, ok);
                         cp_async16(&sb.C[j0 + (f >> 2)][4 * (f & 3)], C_base + off, ok);
                     }
-                } else if (PW == 1) {
+                } else if (PW == 1 && SPW == 16) {
                     // 16 steps x 2 halves x 16 bytes: lane -> (step lane>>1, half lane&1)
                     const int j = lane >> 1, hf = lane & 1;
                     const int pj = __shfl_sync(FULL_MASK, mypos, j);
@@ -446,7 +446,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
                     const long long off = (long long)(ok ? pj : 0) * 16 + 8 * hf;
                     cp_async16(&sb.B[j][8 * hf], B_base + off, ok);
                     cp_async16(&sb.C[j][8 * hf], C_base + off, ok);
-                } else {
+                } else if (SPW == 8) {
                     // 8 steps x 2 halves x 16 bytes per tensor: lanes 0-15 take B, 16-31 take C
                     const int i = (lane & 15) >> 1, hf = lane & 1;
                     const int pj = __shfl_sync(FULL_MASK, mypos, i);
@@ -454,6 +454,20 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
                     const long long off = (long long)(ok ? pj : 0) * 16 + 8 * hf;
                     if (lane < 16) cp_async16(&sb.B[j0 + i][8 * hf], B_base + off, ok);
                     else cp_async16(&sb.C[j0 + i][8 * hf], C_base + off, ok);
+                } else {
+                    // SPW steps x 2 halves x 16 bytes per tensor: copy f -> (tensor, step, half)
+#pragma unroll
+                    for (int it = 0; it < (4 * SPW + 31) / 32; ++it) {
+                        const int f = lane + 32 * it;
+                        const int tsr = f / (2 * SPW), i = (f % (2 * SPW)) >> 1, hf = f & 1;
+                        const int pj = __shfl_sync(FULL_MASK, mypos, i);
+                        if (f < 4 * SPW) {
+                            const bool ok = pj >= 0;
+                            const long long off = (long long)(ok ? pj : 0) * 16 + 8 * hf;
+                            if (tsr == 0) cp_async16(&sb.B[j0 + i][8 * hf], B_base + off, ok);
+                            else cp_async16(&sb.C[j0 + i][8 * hf], C_base + off, ok);
+                        }
+                    }
                 }
             } else {
                 // Any N <= 16: element loads (the 16-byte path needs rows of 16 states).
