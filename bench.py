@@ -356,10 +356,10 @@ def run_ours(args, wls):
     import torch.distributed as dist
 
     world, rank, local = dist_env()
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if world > 1:  # one process per GPU; the device is bound before the communicator
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
     import vision_selective_state_b200 as vs
 
