@@ -95,6 +95,15 @@ def test_bidirectional_without_cls_and_long_sequences():
     _case("cross4", 31, 33, 8, 16, "bf16", batch=1)      # L = 1023
 
 
+@pytest.mark.parametrize("h,w,cls", [(45, 46, 1035), (32, 64, -1), (47, 47, 1104)])
+def test_bidirectional_long_bf16_sequences_use_32_step_chunks(h, w, cls):
+    """bf16 BIDIR sequences of 2048 steps or more stream in 32-step chunks: ragged
+    last chunks (L = 2071, 2210) and an exact multiple (L = 2048, no CLS); N = 16 and
+    N < 16; shared and per-direction inputs; a channel tail (24 = 8-channel tiles x 3)."""
+    _case("bidir", h, w, 16, 16, "bf16", batch=1, cls=cls, seq_chunks=1)
+    _case("bidir", h, w, 24, 7, "bf16", batch=1, cls=cls, seq_chunks=1, pdi=True, pdp=True)
+
+
 def test_empty_batch_is_a_no_op():
     r = vs.Route("atrous2", 4, 4)
     wl = small_workload("atrous2", 4, 4, 8, 16, "f32", 1, 3)

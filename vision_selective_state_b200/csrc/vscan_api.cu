@@ -162,17 +162,22 @@ uint64_t workspace_need(const vscan_route* r, const vscan_args* a)
     return 0;
 }
 
-template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL, int CH = vscan::ST_CH>
+// BIDIR sequences at least this long run 32-step chunks (bf16 I/O, no options).
+constexpr int kLongChunkMinL = 2048;
+
+template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL, int TOK = vscan::ST_TOK,
+          int CH = vscan::ST_CH>
 cudaError_t launch_stream_mode(vscan::ScanParams p, int k_base, int grid_z, cudaStream_t s)
 {
-    const size_t smem = vscan::stream_smem_bytes<T, KC, MODE, FL, CH>();
-    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH>,
+    static_assert(!(FL & vscan::FL_CKPT) || TOK == vscan::BW_TOK, "checkpoints every BW_TOK steps");
+    const size_t smem = vscan::stream_smem_bytes<T, KC, MODE, FL, CH, TOK>();
+    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH, TOK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     p.k_base = k_base;
     const dim3 grid((p.D + CH - 1) / CH, p.batch, grid_z);
-    vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH>
-        <<<grid, vscan::StreamShape<T, KC, MODE, PW, CH>::THREADS, smem, s>>>(p);
+    vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH, TOK>
+        <<<grid, vscan::StreamShape<T, KC, MODE, PW, CH, TOK>::THREADS, smem, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -188,8 +193,15 @@ cudaError_t launch_stream_n(const vscan::ScanParams& p, cudaStream_t s)
         else return launch_stream_mode<RK, T, N16, 4, MODE_OWNER, 1, FL>(p, 0, 1, s);
     } else if constexpr (RK == RK_BIDIR) {
         // two producer warps per direction (measured faster on Vim-Small); the fused
-        // convolution reads steps gathered by one producer warp and keeps one
+        // convolution reads steps gathered by one producer warp and keeps one.
         constexpr int PW = (FL & FL_CONV) ? 1 : 2;
+        // 32-step chunks halve the barriers per token: measured 3-9 % faster for bf16
+        // sequences of 4097 steps, but slower for float32, for short sequences and with
+        // the ZOH or convolution options (which stay at 16, as does the checkpointing run
+        // the backward scan's 16-step chunks read).
+        if constexpr (FL == 0 && sizeof(T) == 2) {
+            if (p.g.L >= kLongChunkMinL) return launch_stream_mode<RK, T, N16, 2, MODE_PARK, PW, FL, 32>(p, 0, 1, s);
+        }
         return launch_stream_mode<RK, T, N16, 2, MODE_PARK, PW, FL>(p, 0, 1, s);
     } else {
         return launch_stream_mode<RK, T, N16, 4, MODE_PARK, 1, FL>(p, 0, 1, s);

@@ -1,8 +1,8 @@
 // Streaming routed selective scan: BIDIR, CROSS4 and ATROUS2 routes.
 //
 // One CTA covers one image b, a tile of CH = 8 or 16 channels and KC directions
-// of the route, and runs them as a software pipeline over 16-step chunks with
-// two kinds of warps:
+// of the route, and runs them as a software pipeline over chunks of TOK = 16
+// steps (32 for the long BIDIR sequences) with two kinds of warps:
 //
 //   consumer warps (CH / 8 per direction) run only the recurrence, each for 8
 //     channels of the tile. Lane 4*c + g
@@ -14,7 +14,7 @@
 //         h  = dA * h + (Delta * u) * B      (FMUL + FFMA)
 //         y += C * h                         (FFMA)
 //
-//   producer warps (PW per direction, each owning 16/PW steps of every chunk)
+//   producer warps (PW per direction, each owning TOK/PW steps of every chunk)
 //     do everything that happens once per (step, channel): they gather the
 //     route's tokens for chunk tau+1+LOOK with
 //     cp.async into a shared-memory ring (zero fill for ATROUS2 padding;
@@ -22,7 +22,7 @@
 //     discretizes chunk tau+1 (Delta = softplus(raw + bias), Delta*u, B and C
 //     as float32), and finishes chunk tau-1.
 //
-// All warps meet at one CTA barrier per chunk, so the gather of chunk tau+4,
+// All warps meet at one CTA barrier per chunk, so the gather of chunk tau+1+LOOK,
 // the discretization of tau+1, the recurrence of tau and the epilogue of tau-1
 // overlap.
 //
@@ -80,7 +80,7 @@ struct ScanParams {
                           // 16-step chunk (saved for the backward pass)
 };
 
-constexpr int ST_TOK = 16;  // steps per chunk
+constexpr int ST_TOK = 16;  // steps per chunk (default; the checkpointing run always uses 16)
 constexpr int ST_CH = 8;    // channels per consumer warp (a CTA covers CH = 8 or 16 channels)
 constexpr int ST_LOOK = 3;  // chunks between a gather and its discretization
 
@@ -98,86 +98,89 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
 // Gathered per-token rows of one direction's chunk, in the I/O type.
-template <typename T, int CH>
+template <typename T, int CH, int TOK>
 struct __align__(16) TokStage {
-    T u[ST_TOK][CH];
-    T d[ST_TOK][CH];
-    T z[ST_TOK][CH];
-    int pos[ST_TOK];  // token index, -1 pad, -2 past the end
-    int fin[ST_TOK];  // MODE_PARK: 1 if this direction adds up the token
+    T u[TOK][CH];
+    T d[TOK][CH];
+    T z[TOK][CH];
+    int pos[TOK];  // token index, -1 pad, -2 past the end
+    int fin[TOK];  // MODE_PARK: 1 if this direction adds up the token
 };
 
 // Gathered B and C rows of one direction's chunk, in the I/O type.
-template <typename T>
+template <typename T, int TOK>
 struct __align__(16) BCStage {
-    T B[ST_TOK][16];
-    T C[ST_TOK][16];
+    T B[TOK][16];
+    T C[TOK][16];
 };
 
 // Discretized chunk of one direction: with BCF (bf16 I/O) float32 copies of B
 // and C, with ZOH the reciprocal of Delta.
-template <bool ON> struct PrepBC {};
-template <> struct PrepBC<true> {
-    float4 B[ST_TOK][4];
-    float4 C[ST_TOK][4];
+template <bool ON, int TOK> struct PrepBC {};
+template <int TOK> struct PrepBC<true, TOK> {
+    float4 B[TOK][4];
+    float4 C[TOK][4];
 };
-template <bool ON, int CH> struct PrepRD {};
-template <int CH> struct PrepRD<true, CH> {
-    float rd[ST_TOK][CH];  // 1 / Delta (inf for Delta = 0, where zoh_phi does not use it)
+template <bool ON, int CH, int TOK> struct PrepRD {};
+template <int CH, int TOK> struct PrepRD<true, CH, TOK> {
+    float rd[TOK][CH];  // 1 / Delta (inf for Delta = 0, where zoh_phi does not use it)
 };
 
-template <bool BCF, bool ZOH, int CH>
-struct __align__(16) PrepStage : PrepBC<BCF>, PrepRD<ZOH, CH> {
-    float2 dd[ST_TOK][CH];  // {Delta after bias + softplus (0 past the end), Delta * u}
+template <bool BCF, bool ZOH, int CH, int TOK>
+struct __align__(16) PrepStage : PrepBC<BCF, TOK>, PrepRD<ZOH, CH, TOK> {
+    float2 dd[TOK][CH];  // {Delta after bias + softplus (0 past the end), Delta * u}
 };
 
 // FL_CONV: the convolved u of the last three chunks of each direction, for the
 // skip term D*u of the epilogue.
-template <bool ON, int KC, int CH> struct ConvRing {};
-template <int KC, int CH> struct ConvRing<true, KC, CH> {
-    float uc[KC][3][ST_TOK][CH];
+template <bool ON, int KC, int CH, int TOK> struct ConvRing {};
+template <int KC, int CH, int TOK> struct ConvRing<true, KC, CH, TOK> {
+    float uc[KC][3][TOK][CH];
 };
 
-template <typename T, int KC, int MODE, int PW = 1, int CH = ST_CH>
+template <typename T, int KC, int MODE, int PW = 1, int CH = ST_CH, int TOK = ST_TOK>
 struct StreamShape {
     static constexpr bool F32 = sizeof(T) == 4;
     static constexpr bool PARK = MODE == MODE_PARK;
     // token slot of chunk c lives from its gather (tau = c-1-LOOK) to its last
     // epilogue use (tau = c+1, or c+2 when parking)
-    static constexpr int NR = ST_LOOK + (PARK ? 4 : 3);
+    // chunks between a gather and its discretization: 3 for 16-step chunks, 1 for 32
+    static constexpr int LOOK = TOK >= 32 ? 1 : ST_LOOK;
+    static constexpr int NR = LOOK + (PARK ? 4 : 3);
     // B/C slot: until discretized at tau = c-1 (bf16) or consumed at tau = c (f32)
-    static constexpr int NBC = ST_LOOK + (F32 ? 2 : 1);
+    static constexpr int NBC = LOOK + (F32 ? 2 : 1);
     static constexpr int NY = PARK ? 3 : 2;  // output ring
     static constexpr int CW = CH / ST_CH;                // consumer warps per direction
     static constexpr int THREADS = 32 * KC * (CW + PW);  // CW consumers and PW producers per direction
-    static constexpr int SPW = ST_TOK / PW;              // steps of a chunk per producer warp
+    static constexpr int SPW = TOK / PW;                 // steps of a chunk per producer warp
     static constexpr int RPL = SPW * CH / 32;            // (step, channel) items per producer lane
     static constexpr int NBCV = SPW / 8;                 // bf16 B/C quads converted per producer lane
     static_assert(PW == 1 || PW == 2, "one or two producer warps per direction");
     static_assert(CH == 8 || CH == 16, "8 or 16 channels per CTA");
+    static_assert(TOK == 16 || TOK == 32, "16- or 32-step chunks");
 };
 
-template <typename T, int KC, int MODE, int FL = 0, int CH = ST_CH>
-struct StreamSmem : ConvRing<(FL & FL_CONV) != 0, KC, CH> {
-    using S = StreamShape<T, KC, MODE>;
-    TokStage<T, CH> tok[KC][S::NR];
-    BCStage<T> bc[KC][S::NBC];
-    PrepStage<!S::F32, (FL & FL_ZOH) != 0, CH> prep[KC][2];
-    float yout[KC][S::NY][ST_TOK][CH];
+template <typename T, int KC, int MODE, int FL = 0, int CH = ST_CH, int TOK = ST_TOK>
+struct StreamSmem : ConvRing<(FL & FL_CONV) != 0, KC, CH, TOK> {
+    using S = StreamShape<T, KC, MODE, 1, CH, TOK>;
+    TokStage<T, CH, TOK> tok[KC][S::NR];
+    BCStage<T, TOK> bc[KC][S::NBC];
+    PrepStage<!S::F32, (FL & FL_ZOH) != 0, CH, TOK> prep[KC][2];
+    float yout[KC][S::NY][TOK][CH];
 };
 
-template <typename T, int KC, int MODE, int FL = 0, int CH = ST_CH>
-constexpr size_t stream_smem_bytes() { return sizeof(StreamSmem<T, KC, MODE, FL, CH>); }
+template <typename T, int KC, int MODE, int FL = 0, int CH = ST_CH, int TOK = ST_TOK>
+constexpr size_t stream_smem_bytes() { return sizeof(StreamSmem<T, KC, MODE, FL, CH, TOK>); }
 
 // Direction that adds up token p: the one visiting p in the latest chunk.
-template <int RK>
+template <int RK, int TOK>
 __device__ __forceinline__ int finalizer(const RouteGeom& g, int p)
 {
     int best_k = 0;
-    int best_c = visit_step<RK>(g, 0, p) / ST_TOK;
+    int best_c = visit_step<RK>(g, 0, p) / TOK;
 #pragma unroll
     for (int kk = 1; kk < (RK == RK_CROSS4 ? 4 : 2); ++kk) {
-        const int c = visit_step<RK>(g, kk, p) / ST_TOK;
+        const int c = visit_step<RK>(g, kk, p) / TOK;
         if (c >= best_c) {
             best_c = c;
             best_k = kk;
@@ -186,10 +189,11 @@ __device__ __forceinline__ int finalizer(const RouteGeom& g, int p)
     return best_k;
 }
 
-template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL, int CH>
-__global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) stream_scan_kernel(const ScanParams p)
+template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL, int CH, int TOK>
+__global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH, TOK>::THREADS) stream_scan_kernel(const ScanParams p)
 {
-    using S = StreamShape<T, KC, MODE, PW, CH>;
+    using S = StreamShape<T, KC, MODE, PW, CH, TOK>;
+    constexpr int LOOK = S::LOOK;
     constexpr int SPW = S::SPW, RPL = S::RPL, CW = S::CW, NBCV = S::NBCV;
     constexpr int RSTEP = 32 / CH;  // rows between a producer lane's items
     constexpr bool ZOH = (FL & FL_ZOH) != 0;
@@ -202,14 +206,14 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
     constexpr bool F32 = S::F32;
     constexpr int KR = (RK == RK_BIDIR) ? 2 : 4;  // directions of the route
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    StreamSmem<T, KC, MODE, FL, CH>& sm = *reinterpret_cast<StreamSmem<T, KC, MODE, FL, CH>*>(smem_raw);
+    StreamSmem<T, KC, MODE, FL, CH, TOK>& sm = *reinterpret_cast<StreamSmem<T, KC, MODE, FL, CH, TOK>*>(smem_raw);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int b = blockIdx.y;
     const int c0 = blockIdx.x * CH;
     const int D = p.D, N = p.N, L = p.g.L, tokens = p.g.tokens;
-    const int nchunks = (L + ST_TOK - 1) / ST_TOK;
+    const int nchunks = (L + TOK - 1) / TOK;
     const int last_tau = nchunks + (PARK ? 1 : 0);
     const long long img = (long long)b * tokens;
 
@@ -242,13 +246,13 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
                     if (ck) *reinterpret_cast<float4*>(ck + (long long)tau * D * 16) = make_float4(h01.x, h01.y, h23.x, h23.y);
                 }
                 const auto& pr = sm.prep[kl][tau & 1];
-                const BCStage<T>& bcs = sm.bc[kl][tau % NBC];
+                const BCStage<T, TOK>& bcs = sm.bc[kl][tau % NBC];
                 float* yo = &sm.yout[kl][tau % NY][0][0];
-                // Software pipeline over the chunk's 16 steps: the loads, the SFU
+                // Software pipeline over the chunk's TOK steps: the loads, the SFU
                 // exponentials and the input terms of step j + 2 are issued before
                 // the state update of step j, which is the only serial dependency.
-                float2 e01[ST_TOK], e23[ST_TOK], w01[ST_TOK], w23[ST_TOK];
-                float4 cq[ST_TOK];
+                float2 e01[TOK], e23[TOK], w01[TOK], w23[TOK];
+                float4 cq[TOK];
                 auto front = [&](int j) {
                     const float2 dd = pr.dd[j][cc];
                     float4 Bv;
@@ -280,14 +284,14 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
                 };
                 front(0);
                 front(1);
-                float yv[ST_TOK / 4];
+                float yv[TOK / 4];
 #pragma unroll
-                for (int q = 0; q < ST_TOK / 4; ++q) {
+                for (int q = 0; q < TOK / 4; ++q) {
                     float yp[4];
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                         const int j = 4 * q + jj;
-                        if (j + 2 < ST_TOK) front(j + 2);
+                        if (j + 2 < TOK) front(j + 2);
                         h01 = __ffma2_rn(e01[j], h01, w01[j]);
                         h23 = __ffma2_rn(e23[j], h23, w23[j]);
                         float2 acc = __fmul2_rn(make_float2(cq[j].x, cq[j].y), h01);
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
                 }
                 // stores after every load of the chunk, so none of them waits on a store
 #pragma unroll
-                for (int q = 0; q < ST_TOK / 4; ++q) yo[(4 * q + grp) * CH + cc] = yv[q];
+                for (int q = 0; q < TOK / 4; ++q) yo[(4 * q + grp) * CH + cc] = yv[q];
             }
             __syncthreads();
         }
@@ -346,19 +350,19 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
     auto issue = [&](int chunk) {
         if (chunk < nchunks) {
             auto& st = sm.tok[kl][chunk % NR];
-            BCStage<T>& sb = sm.bc[kl][chunk % NBC];
+            BCStage<T, TOK>& sb = sm.bc[kl][chunk % NBC];
             const T* u_base = static_cast<const T*>(p.u) + k * p.in_dir + img * D + c0;
             const T* d_base = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + c0;
             const T* B_base = static_cast<const T*>(p.B) + k * p.bc_dir + img * N;
             const T* C_base = static_cast<const T*>(p.C) + k * p.bc_dir + img * N;
             // lane i < SPW computes the route position of step j0 + i
-            const int t = chunk * ST_TOK + j0 + (lane & (SPW - 1));
+            const int t = chunk * TOK + j0 + (lane & (SPW - 1));
             const int mypos = (t < L) ? route_token<RK>(p.g, k, t) : -2;
             if (lane < SPW) {
                 st.pos[j0 + lane] = mypos;
-                if constexpr (PARK) st.fin[j0 + lane] = (mypos >= 0 && finalizer<RK>(p.g, mypos) == k) ? 1 : 0;
+                if constexpr (PARK) st.fin[j0 + lane] = (mypos >= 0 && finalizer<RK, TOK>(p.g, mypos) == k) ? 1 : 0;
             }
-            if constexpr (CH == ST_CH && ST_TOK == 16) {
+            if constexpr (CH == ST_CH && TOK == 16) {
                 // 8-channel tiles of 16 steps: one 16- or 32-byte row piece per lane and tensor
                 if (F32 && PW == 1) {
                     // u, Delta, z: 16 steps x 32 bytes; lane -> (step lane>>1, 4-channel half lane&1)
@@ -515,7 +519,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
                     const int jj = j - 3 + i;
                     float xv;
                     if (jj >= 0) xv = (i == 3) ? xu[r] : to_float(st.u[jj][ce]);
-                    else xv = (c > 0) ? to_float(prev.u[ST_TOK + jj][ce]) : 0.f;
+                    else xv = (c > 0) ? to_float(prev.u[TOK + jj][ce]) : 0.f;
                     acc = fmaf(kw[i], xv, acc);
                 }
                 xu[r] = silu_f(acc);
@@ -524,7 +528,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
         }
         float4 cb[NBCV], cv[NBCV];
         if constexpr (!F32) {
-            const BCStage<T>& sb = sm.bc[kl][c % NBC];
+            const BCStage<T, TOK>& sb = sm.bc[kl][c % NBC];
 #pragma unroll
             for (int r = 0; r < NBCV; ++r) {
                 const int f = lane + 32 * r;  // (step j0 + f>>2, quad f&3)
@@ -634,8 +638,8 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
 
     // Prologue: gathers for chunks 0..LOOK in flight, chunk 0 discretized.
 #pragma unroll
-    for (int c = 0; c <= ST_LOOK; ++c) issue(c);
-    cp_async_wait<ST_LOOK>();
+    for (int c = 0; c <= LOOK; ++c) issue(c);
+    cp_async_wait<LOOK>();
     __syncwarp();
     if (nchunks > 0) prepare(0);
     __syncthreads();
@@ -643,9 +647,9 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH>::THREADS) str
     for (int tau = 0; tau <= last_tau; ++tau) {
         const bool do_b = PARK && tau >= 2 && tau - 2 < nchunks;
         if (do_b) fetch_b(tau - 2);
-        issue(tau + 1 + ST_LOOK);
+        issue(tau + 1 + LOOK);
         if (tau + 1 < nchunks) {
-            cp_async_wait<ST_LOOK>();  // chunk tau+1 has landed (this lane's copies)
+            cp_async_wait<LOOK>();  // chunk tau+1 has landed (this lane's copies)
             __syncwarp();              // ... and every lane's
             prepare(tau + 1);
         }
