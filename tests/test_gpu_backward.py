@@ -77,6 +77,19 @@ def test_backward_bidir_with_middle_cls_and_long_sequence():
     _case("bidir", 31, 33, 8, "f32", batch=1)
 
 
+@pytest.mark.parametrize("route,h,w,D,dtype,batch,kw", [
+    ("bidir", 5, 7, 196, "f32", 64, {}),                        # 25 tiles (channel tail) x 64 x 2
+    ("cross4", 5, 6, 64, "bf16", 96, {"N": 7}),                  # 8 x 96 x 4
+    ("atrous2", 5, 7, 24, "f32", 160, {"pdi": True, "pdp": True}),  # 3 x 160 x 4
+    ("pool_w", 6, 9, 104, "f32", 96, {}),                        # 13 x 96 x 2 over the pooled sequence
+])
+def test_backward_large_grids_take_the_register_capped_build(route, h, w, D, dtype, batch, kw):
+    """Grids of more than 8 warps per SM (here 1900-3200 warps) run the adjoint scan
+    built for 16 resident warps per SM, which sums dB and dC with a per-step shuffle
+    reduce-scatter instead of shared memory."""
+    _case(route, h, w, D, dtype, batch=batch, **kw)
+
+
 def test_backward_refuses_unsupported_options():
     r = vs.Route("bidir", 4, 4)
     x = torch.zeros(1, 16, 8, device="cuda")

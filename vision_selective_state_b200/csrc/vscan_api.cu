@@ -119,6 +119,18 @@ vscan_status check_shape(const vscan_route* r, const vscan_args* a)
     return VSCAN_OK;
 }
 
+// SMs of the current device (148 on B200), read once per process.
+int num_sms()
+{
+    static int n = [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+            v = 148;
+        return v;
+    }();
+    return n;
+}
+
 // Chunks per sequence for the streaming routes: 1 = streaming kernel, 2/4/8 =
 // resident chunked kernel. The library picks the resident kernel when the tile
 // fits on chip and the streaming kernel would leave most SMs idle.
@@ -509,6 +521,19 @@ vscan_status check_backward(const vscan_route* r, const vscan_args* a)
     return VSCAN_OK;
 }
 
+// The adjoint scan: one warp per (channel tile, image, direction). Grids of at most
+// 8 warps per SM take the variant with uncapped registers and the shared-memory dB/dC
+// sums (the faster one on the atrous b8 and Vim-Tiny b1 grids); larger grids the
+// one built for 16 resident warps per SM (22-28 % faster on Vim-Tiny b64, SS2D b16
+// and Vim-Small b64).
+template <int RK, typename T>
+void launch_bwd_scan(const vscan::BwdParams& p, dim3 grid, cudaStream_t s)
+{
+    const long long warps = (long long)grid.x * grid.y * grid.z;
+    if (warps <= 8LL * num_sms()) vscan::bwd_scan_kernel<RK, T, 1><<<grid, 32, 0, s>>>(p);
+    else vscan::bwd_scan_kernel<RK, T, vscan::BW_MIN_WARPS><<<grid, 32, 0, s>>>(p);
+}
+
 template <typename T>
 vscan_status backward_device(const vscan_route* r, const vscan_args* a, const void* dy, const vscan_grads* gr,
                              cudaStream_t s)
@@ -571,9 +596,9 @@ vscan_status backward_device(const vscan_route* r, const vscan_args* a, const vo
         p.gy = gy;
         p.du = gr->du; p.ddelta = gr->ddelta; p.dB = gr->dB; p.dC = gr->dC;
         switch (g.kind) {
-        case vscan::RK_BIDIR: vscan::bwd_scan_kernel<vscan::RK_BIDIR, T><<<grid, 32, 0, s>>>(p); break;
-        case vscan::RK_CROSS4: vscan::bwd_scan_kernel<vscan::RK_CROSS4, T><<<grid, 32, 0, s>>>(p); break;
-        default: vscan::bwd_scan_kernel<vscan::RK_ATROUS2, T><<<grid, 32, 0, s>>>(p); break;
+        case vscan::RK_BIDIR: launch_bwd_scan<vscan::RK_BIDIR, T>(p, grid, s); break;
+        case vscan::RK_CROSS4: launch_bwd_scan<vscan::RK_CROSS4, T>(p, grid, s); break;
+        default: launch_bwd_scan<vscan::RK_ATROUS2, T>(p, grid, s); break;
         }
     } else {
         float* pu = reinterpret_cast<float*>(ws + Lo.pu);
@@ -595,7 +620,7 @@ vscan_status backward_device(const vscan_route* r, const vscan_args* a, const vo
         p.ddelta = reinterpret_cast<float*>(ws + Lo.dpraw);
         p.dB = reinterpret_cast<float*>(ws + Lo.dpB);
         p.dC = reinterpret_cast<float*>(ws + Lo.dpC);
-        vscan::bwd_scan_kernel<vscan::RK_BIDIR, float><<<grid, 32, 0, s>>>(p);
+        launch_bwd_scan<vscan::RK_BIDIR, float>(p, grid, s);
         vscan::bwd_unpool_kernel<<<dim3((unsigned)TK, (unsigned)b), 128, 0, s>>>(
             g, (int)b, (int)D, (int)N, Ki, p.du, p.ddelta, p.dB, p.dC, gr->du, gr->ddelta, gr->dB, gr->dC);
     }

@@ -22,11 +22,13 @@
 //                        every 16-step chunk boundary; pass 2 walks the chunks
 //                        backwards, recomputes the chunk's states from its
 //                        checkpoint and runs the adjoint recurrence. Token
-//                        gradients are summed over channels (B, C) or state
-//                        groups (u, Delta) with warp shuffles and added with
-//                        float atomics (directions, channel tiles and images
-//                        meet there); dA, D and bias gradients stay in
-//                        registers until the end.
+//                        gradients are summed over channels (B, C: in shared
+//                        memory once per chunk on grids of few warps per SM,
+//                        one shuffle reduce-scatter per step on larger ones) or
+//                        state groups (u, Delta: shuffles) and added with float
+//                        atomics (directions, channel tiles and images meet
+//                        there); dA, D and bias gradients stay in registers
+//                        until the end.
 //   bwd_unpool_kernel    pooled routes: every member token receives its pooled
 //                        index's gradient divided by the member count.
 #pragma once
@@ -184,19 +186,34 @@ struct BwdStage {
     float C[BW_TOK][16];
 };
 
-// Per-chunk token-gradient partials of bwd_scan_kernel (summed after the chunk).
-struct BwdReduce {
-    float u[BW_TOK][BW_CH];       // du per (step, channel), state groups already summed
-    float x[BW_TOK][BW_CH];       // d raw Delta per (step, channel)
-    float B[BW_TOK][BW_CH][16];   // dB per (step, channel, state): summed over channels
-    float C[BW_TOK][BW_CH][16];   // dC likewise
+// Per-chunk gradient partials of bwd_scan_kernel, added to global memory after
+// the chunk. With SMEM_BC the per-channel dB and dC partials are staged too and
+// summed over the channels after the chunk; without it they are summed with
+// shuffles at every step.
+struct BwdReduceUX {
+    float u[BW_TOK][BW_CH];  // du per (step, channel), state groups already summed
+    float x[BW_TOK][BW_CH];  // d raw Delta per (step, channel)
+};
+template <bool SMEM_BC> struct BwdReduce : BwdReduceUX {};
+template <> struct BwdReduce<true> : BwdReduceUX {
+    float B[BW_TOK][BW_CH][16];  // dB per (step, channel, state)
+    float C[BW_TOK][BW_CH][16];  // dC likewise
 };
 
-template <int RK, typename TI>
-__global__ void __launch_bounds__(32) bwd_scan_kernel(const BwdParams p)
+// Warps per SM the backward scan is compiled for. MINW = BW_MIN_WARPS caps its
+// registers per thread and keeps its shared memory small (the kernel is
+// latency-bound, so on large grids resident warps matter more than scheduling
+// room) and sums dB and dC with shuffles. MINW = 1, for grids that put only a few
+// warps on each SM, leaves registers uncapped and sums dB and dC through shared
+// memory once per chunk, which keeps the shuffles off the steps' latency.
+constexpr int BW_MIN_WARPS = 16;
+
+template <int RK, typename TI, int MINW>
+__global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
 {
+    constexpr bool SMEM_BC = MINW == 1;
     __shared__ BwdStage st;
-    __shared__ __align__(16) BwdReduce rd;
+    __shared__ __align__(16) BwdReduce<SMEM_BC> rd;
     const int lane = threadIdx.x;
     const int cc = lane >> 2, grp = lane & 3;
     const int c0 = blockIdx.x * BW_CH, b = blockIdx.y, k = blockIdx.z;
@@ -344,12 +361,31 @@ __global__ void __launch_bounds__(32) bwd_scan_kernel(const BwdParams p)
                 rd.u[j][cc] = fmaf(Dd, dy, dut);
                 rd.x[j][cc] = draw;
             }
-            // per-channel partials of dB and dC, summed over the channels after the chunk
-            *reinterpret_cast<float4*>(&rd.B[j][cc][4 * grp]) = make_float4(dBv[0], dBv[1], dBv[2], dBv[3]);
-            *reinterpret_cast<float4*>(&rd.C[j][cc][4 * grp]) = make_float4(dCv[0], dCv[1], dCv[2], dCv[3]);
+            if constexpr (SMEM_BC) {
+                // per-channel partials of dB and dC, summed over the channels after the chunk
+                *reinterpret_cast<float4*>(&rd.B[j][cc][4 * grp]) = make_float4(dBv[0], dBv[1], dBv[2], dBv[3]);
+                *reinterpret_cast<float4*>(&rd.C[j][cc][4 * grp]) = make_float4(dCv[0], dCv[1], dCv[2], dCv[3]);
+            } else {
+                // dB and dC of the step, summed over the 8 channels (lanes 4c + grp, c = 0..7):
+                // a reduce-scatter over lane bits 4, 3, 2 leaves lane 4c + grp with value c of
+                // its group, i.e. tensor c >> 2 (0: B, 1: C) at state 4 grp + (c & 3).
+                const bool b4 = cc & 4, b2 = cc & 2, b1 = cc & 1;
+                float v4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    v4[i] = (b4 ? dCv[i] : dBv[i]) + __shfl_xor_sync(FULL_MASK, b4 ? dBv[i] : dCv[i], 16);
+                float v2[2];
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    v2[i] = (b2 ? v4[2 + i] : v4[i]) + __shfl_xor_sync(FULL_MASK, b2 ? v4[i] : v4[2 + i], 8);
+                const float v1 = (b1 ? v2[1] : v2[0]) + __shfl_xor_sync(FULL_MASK, b1 ? v2[0] : v2[1], 4);
+                const int n = 4 * grp + (cc & 3);
+                float* dst = b4 ? p.dC : p.dB;
+                if (q >= 0 && n < N && dst) atomicAdd(dst + ki * p.bc_dir + (img + q) * N + n, v1);
+            }
         }
-        // add the chunk's token gradients: one atomic per (step, channel) and per
-        // (step, state), every lane taking its share
+        // add the chunk's token gradients: one atomic per (step, channel) and, with
+        // SMEM_BC, per (step, state), every lane taking its share
         __syncwarp();
 #pragma unroll
         for (int r = 0; r < BW_TOK * BW_CH / 32; ++r) {
@@ -361,21 +397,23 @@ __global__ void __launch_bounds__(32) bwd_scan_kernel(const BwdParams p)
             if (p.du) atomicAdd(p.du + o, rd.u[j][ch]);
             if (p.ddelta) atomicAdd(p.ddelta + o, rd.x[j][ch]);
         }
+        if constexpr (SMEM_BC) {
 #pragma unroll
-        for (int r = 0; r < BW_TOK * 16 / 32; ++r) {
-            const int e = lane + 32 * r;
-            const int j = e >> 4, n = e & 15;
-            const int q = st.pos[j];
-            if (q < 0 || n >= N) continue;
-            float sb = 0.f, sc = 0.f;
+            for (int r = 0; r < BW_TOK * 16 / 32; ++r) {
+                const int e = lane + 32 * r;
+                const int j = e >> 4, n = e & 15;
+                const int q = st.pos[j];
+                if (q < 0 || n >= N) continue;
+                float sb = 0.f, sc = 0.f;
 #pragma unroll
-            for (int ch = 0; ch < BW_CH; ++ch) {
-                sb += rd.B[j][ch][n];
-                sc += rd.C[j][ch][n];
+                for (int ch = 0; ch < BW_CH; ++ch) {
+                    sb += rd.B[j][ch][n];
+                    sc += rd.C[j][ch][n];
+                }
+                const long long o = ki * p.bc_dir + (img + q) * N + n;
+                if (p.dB) atomicAdd(p.dB + o, sb);
+                if (p.dC) atomicAdd(p.dC + o, sc);
             }
-            const long long o = ki * p.bc_dir + (img + q) * N + n;
-            if (p.dB) atomicAdd(p.dB + o, sb);
-            if (p.dC) atomicAdd(p.dC + o, sc);
         }
         __syncwarp();
     }
