@@ -38,6 +38,8 @@ class Route:
         handle = ctypes.c_void_p()
         check(lib.vscan_create_route(ctypes.byref(handle), self.kind, self.h, self.w, self.cls_pos))
         self._handle = handle
+        # bound here: at interpreter exit the module global may be gone before __del__ runs
+        self._destroy = lib.vscan_destroy
         vals = [ctypes.c_int32() for _ in range(5)]
         check(lib.vscan_route_info(self._handle, *[ctypes.byref(v) for v in vals]))
         self.K, self.seq_len, self.tokens, self.padded_h, self.padded_w = (v.value for v in vals)
@@ -50,7 +52,7 @@ class Route:
 
     def close(self):
         if getattr(self, "_handle", None) is not None:
-            lib.vscan_destroy(self._handle)
+            self._destroy(self._handle)
             self._handle = None
 
     def __del__(self):
