@@ -12,6 +12,13 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
+    # a fresh checkout has no built library (it is not versioned): build it once, by
+    # the build script's path, before any test module imports the package
+    if not os.path.exists(os.path.join(ROOT, "vision_selective_state_b200", "libvscan.so")):
+        import __graft_entry__
+
+        __graft_entry__._load_build_script(os.path.join("vision_selective_state_b200", "build.py"),
+                                           "_vscan_build").build()
 
 
 def read_golden(name):
