@@ -325,3 +325,70 @@ def test_channels_and_images_are_independent():
     xs = workloads.batch_slice(workloads.channel_slice(x, [1, 6]), [1])
     part = O.forward(wl.route, wl.h, wl.w, xs["u"], xs["delta"], xs["A"], xs["B"], xs["C"], xs["Dskip"], xs["bias"], xs["z"])
     np.testing.assert_array_equal(part, full[1:2][..., [1, 6]])
+
+
+# ---------------------------------------------------------------- padding is a real step
+def _atrous_stream(h, w, k):
+    """Grid coordinates of atrous group k in visiting order, written out from the EfficientVMamba
+    review, sec. 1: offsets (m, n) = (0,0), (1,0), (0,1), (1,1) in (row, column); groups 0 and 2
+    row-major, 1 and 3 column-major, on the grid padded right/bottom to even size. A coordinate
+    outside h x w is a padding slot (None)."""
+    m, n = k & 1, k >> 1
+    rows, cols = (h + 1) // 2, (w + 1) // 2
+    order = [(r, c) for c in range(cols) for r in range(rows)] if k & 1 else \
+            [(r, c) for r in range(rows) for c in range(cols)]
+    out = []
+    for r, c in order:
+        y, x = 2 * r + m, 2 * c + n
+        out.append(y * w + x if (y < h and x < w) else None)
+    return out
+
+
+def _pad_runs(stream):
+    """(source token, pads skipped, next token) for every real token followed by padding and then
+    by another real token of the same stream."""
+    runs = []
+    for i, p in enumerate(stream):
+        if p is None or i + 1 >= len(stream) or stream[i + 1] is not None:
+            continue
+        j = i + 1
+        while j < len(stream) and stream[j] is None:
+            j += 1
+        if j < len(stream):
+            runs.append((p, j - i - 1, stream[j]))
+    return runs
+
+
+@pytest.mark.parametrize("h,w,samples", [(3, 5, None), (5, 3, None), (55, 57, 6)])
+def test_padding_slots_decay_the_state(h, w, samples):
+    """EfficientVMamba review, sec. 1-2: padding positions are zero-valued inputs to the scan, not
+    absent steps, so the state keeps decaying across them. With u an impulse at the last real token
+    before a run of k pads, the next real token of that stream reads
+        y = sum_n C_n exp(A_n (k softplus(bias) + softplus(raw_next + bias))) softplus(raw_src + bias) B_src,n.
+    Skipping the pads, or giving them Delta = 0, drops the k softplus(bias) term."""
+    r = _rng(31)
+    N = 3
+    A = -np.array([[0.7, 1.9, 3.1]])
+    bias = np.array([0.4])  # softplus(0.4) = 0.913: a pad decays exp(-0.64 .. -2.8) per step
+    sp = lambda v: np.logaddexp(0.0, v)  # noqa: E731  (numpy softplus)
+    checked = 0
+    for k in range(4):
+        runs = _pad_runs(_atrous_stream(h, w, k))
+        if samples is not None:
+            runs = runs[:: max(1, len(runs) // samples)][:samples]
+        for src, npad, nxt in runs:
+            raw = 0.5 * r.standard_normal((1, h * w, 1))
+            B = r.standard_normal((1, h * w, N))
+            C = r.standard_normal((1, h * w, N))
+            u = np.zeros((1, h * w, 1))
+            u[0, src, 0] = 1.0
+            y = O.forward("atrous2", h, w, u, raw, A, B, C, Dskip=np.zeros(1), bias=bias)
+            decay = np.exp(A[0] * (npad * sp(bias[0]) + sp(raw[0, nxt, 0] + bias[0])))
+            expect = np.dot(C[0, nxt], decay * sp(raw[0, src, 0] + bias[0]) * B[0, src])
+            assert y[0, nxt, 0] == pytest.approx(expect, rel=1e-12, abs=1e-15), (k, src, npad, nxt)
+            # the same impulse with the pads removed would read a visibly different value
+            no_pad = np.dot(C[0, nxt], np.exp(A[0] * sp(raw[0, nxt, 0] + bias[0]))
+                            * sp(raw[0, src, 0] + bias[0]) * B[0, src])
+            assert abs(no_pad - expect) > 1e-3 * max(abs(expect), 1e-3)
+            checked += 1
+    assert checked >= 3
