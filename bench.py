@@ -3,9 +3,12 @@
 
 A step is one pass of the whole fused path (gather, discretization,
 recurrence, read-out, merge, gate, store) over one batch of every grid of the
-selected workload. The default workload is the EfficientVMamba atrous p=2 scan:
-batch 8, d_inner 192, N 16, float32, on the 56x56 grid and on the odd 55x57
-grid (zero-padded to 56x58); one step runs both.
+selected workload. The default workload is the largest single-GPU one: the
+Vim-Small-shaped high-resolution bidirectional scan (1024^2 input, 16-pixel
+patches: 64x64 tokens + middle CLS = 4097 per image), batch 64, d_inner 768,
+N 16, bf16 I/O with float32 state, SiLU(z) gate. Workload 1 is the
+EfficientVMamba atrous p=2 scan (56x56 and the odd 55x57 grid, one step runs
+both).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -36,16 +39,18 @@ METRIC = "scan throughput tokens·ch/s at 1 B200; achieved HBM GB/s vs peak"
 UNIT = "tokens·ch/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+NORTH_STAR_HBM_GBS = 8000.0  # the HBM roofline the target is stated against (compulsory bytes / 8 TB/s)
 
 
 def parse():
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=4000)
-    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--steps", type=int, default=300)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="1",
-                   help="configuration index 0-4 or a workload name (default 1: atrous 56x56 + 55x57)")
+    p.add_argument("--workload", default="4",
+                   help="configuration index 0-4 or a workload name (default 4: Vim-Small 64x64+CLS, "
+                        "b64, D768, bf16)")
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -61,6 +66,9 @@ def parse():
                    help="time the backward pass (all gradients) instead of the forward")
     p.add_argument("--mask-keep", type=float, default=1.0,
                    help="pooled workloads: keep this fraction of tokens (random mask per image, FastMaskVim)")
+    p.add_argument("--per-dir", action="store_true",
+                   help="every direction its own u, raw Delta, B, C and A, D, bias planes (the Vim block's "
+                        "per-branch parameters)")
     return p.parse_args()
 
 
@@ -76,7 +84,8 @@ def workload_label(wls):
     w0 = wls[0]
     grids = "+".join(f"{w.h}x{w.w}" for w in wls)
     cls = "_cls" if w0.cls_pos >= 0 else ""
-    opt = ("_conv" if w0.conv else "") + ("_zoh" if w0.zoh else "") + (f"_keep{w0.keep:g}" if w0.keep < 1 else "")
+    opt = ("_conv" if w0.conv else "") + ("_zoh" if w0.zoh else "") + (f"_keep{w0.keep:g}" if w0.keep < 1 else "") \
+        + ("_perdir" if w0.per_dir else "")
     return f"{w0.route}_{grids}{cls}_b{w0.batch}_d{w0.D}_n{w0.N}_{w0.dtype}{opt}"
 
 
@@ -84,16 +93,19 @@ def algorithmic_bytes_bwd(wl):
     """Compulsory HBM bytes of one backward: read u, raw delta, z, B, C and dy; write the
     float32 gradients du, ddelta, dz (per token-channel) and dB, dC (per token-state)."""
     eb = 2 if wl.dtype == "bf16" else 4
-    per_token = (4 * wl.D + 2 * wl.N) * eb + (3 * wl.D + 2 * wl.N) * 4
-    params = (wl.D * wl.N + 2 * wl.D) * 4 * 2
+    ki = wl.K if wl.per_dir else 1
+    per_token = (ki * (2 * wl.D + 2 * wl.N) + 2 * wl.D) * eb + (ki * (2 * wl.D + 2 * wl.N) + wl.D) * 4
+    params = ki * (wl.D * wl.N + 2 * wl.D) * 4 * 2
     return wl.batch * wl.tokens * per_token + params
 
 
 def algorithmic_bytes(wl):
-    """Compulsory HBM bytes of one forward: read u, raw delta, z, B, C; write y."""
+    """Compulsory HBM bytes of one forward: read u, raw delta, B, C (one plane, or one per
+    direction with per-direction inputs) and z; write y."""
     eb = 2 if wl.dtype == "bf16" else 4
-    per_token = (3 * wl.D + 2 * wl.N) * eb + wl.D * eb
-    params = (wl.D * wl.N + 2 * wl.D + (5 * wl.D if wl.conv else 0)) * 4
+    ki = wl.K if wl.per_dir else 1
+    per_token = (ki * (2 * wl.D + 2 * wl.N) + wl.D) * eb + wl.D * eb
+    params = ki * (wl.D * wl.N + 2 * wl.D + (5 * wl.D if wl.conv else 0)) * 4
     pos = 4 * wl.batch * wl.visible if wl.keep < 1 else 0  # grid positions of the visible tokens
     return wl.batch * wl.visible * per_token + params + pos
 
@@ -178,21 +190,34 @@ class ClockSampler:
         0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, index, interval=0.02):
-        self.index, self.interval = index, interval
+    def __init__(self, device, interval=0.002):
+        self.interval = interval
         self.samples, self.reasons = [], set()
         self.max_mhz = None
+        self.pci_bus_id = None
         self._stop = threading.Event()
         self._thread = None
         try:
             import pynvml
             pynvml.nvmlInit()
             self.nvml = pynvml
-            self.handle = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.handle, self.pci_bus_id = self._nvml_handle(pynvml, device)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
         except Exception as e:  # noqa: BLE001
             self.nvml = None
             self.error = str(e)
+
+    @staticmethod
+    def _nvml_handle(pynvml, device):
+        """NVML handle of a torch CUDA device. CUDA and NVML number GPUs differently
+        (CUDA_VISIBLE_DEVICES, fastest-first ordering), so match by UUID, else by PCI bus id."""
+        import torch
+        prop = torch.cuda.get_device_properties(device)
+        bus = f"{prop.pci_domain_id:08x}:{prop.pci_bus_id:02x}:{prop.pci_device_id:02x}.0"
+        try:
+            return pynvml.nvmlDeviceGetHandleByUUID(f"GPU-{prop.uuid}"), bus
+        except Exception:  # noqa: BLE001
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus), bus
 
     def _reason_mask(self):
         fn = getattr(self.nvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
@@ -234,7 +259,9 @@ class ClockSampler:
         reasons = sorted(self.reasons - {"gpu_idle"})
         return {"sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples),
-                "source": "nvml, 20 ms interval, during the timed region"}
+                "pci_bus_id": self.pci_bus_id,
+                "source": f"nvml (device matched by UUID / PCI bus id), {1e3 * self.interval:g} ms "
+                          f"interval, during the timed region"}
 
 
 # ------------------------------------------------------------------ distributed
@@ -265,16 +292,35 @@ def job_throughput(units_per_rank_step, steps, world, elapsed_ms_max):
     return units_per_rank_step * steps * world / (elapsed_ms_max * 1e-3)
 
 
+# ------------------------------------------------------------------ inputs
+_DRAWN = {}
+
+
+def draw_inputs(wl):
+    """The seeded inputs of one workload (numpy, float32), drawn once per process."""
+    key = (wl.name, wl.seed, wl.batch, wl.keep, wl.conv, wl.per_dir)
+    if key not in _DRAWN:
+        if wl.keep < 1:
+            x = workloads.draw_masked(wl)
+        else:
+            x = workloads.draw(wl, per_dir_inputs=wl.per_dir, per_dir_params=wl.per_dir)
+        if wl.conv:
+            x.update(workloads.draw_conv(wl, per_dir_params=wl.per_dir))
+        _DRAWN[key] = x
+    return _DRAWN[key]
+
+
 # ------------------------------------------------------------------ CPU oracle
-def oracle_time(wls, channels, threads=0):
-    """Seconds the fp64 oracle takes for the given channel subset of every grid."""
+def oracle_inputs(wls, channels):
+    """Every grid's inputs restricted to a channel subset (channels are independent)."""
+    return [workloads.channel_slice(draw_inputs(wl), channels) for wl in wls]
+
+
+def oracle_time(wls, xs, threads=0):
+    """Seconds the fp64 oracle takes for the given (channel-sliced) inputs of every grid."""
     import oracle
     total = 0.0
-    for wl in wls:
-        x = workloads.draw_masked(wl) if wl.keep < 1 else workloads.draw(wl)
-        if wl.conv:
-            x.update(workloads.draw_conv(wl))
-        x = workloads.channel_slice(x, channels)
+    for wl, x in zip(wls, xs):
         t0 = time.perf_counter()
         if wl.keep < 1:
             oracle.forward_masked(wl.route, wl.h, wl.w, x["pos"], x["u"], x["delta"], x["A"], x["B"], x["C"],
@@ -283,7 +329,8 @@ def oracle_time(wls, channels, threads=0):
         else:
             oracle.forward(wl.route, wl.h, wl.w, x["u"], x["delta"], x["A"], x["B"], x["C"], x["Dskip"],
                            x["bias"], x["z"] if wl.gate else None, cls_pos=wl.cls_pos,
-                           conv_w=x.get("conv_w"), conv_b=x.get("conv_b"), zoh=wl.zoh, threads=threads)
+                           conv_w=x.get("conv_w"), conv_b=x.get("conv_b"), zoh=wl.zoh,
+                           per_dir_inputs=wl.per_dir, per_dir_params=wl.per_dir, threads=threads)
         total += time.perf_counter() - t0
     return total
 
@@ -293,14 +340,15 @@ def cpu_baseline(wls, budget_s):
     import oracle
     cores = oracle.default_threads()
     D = wls[0].D
-    t1 = oracle_time(wls, list(range(min(cores, D))))
-    per_channel = t1 / min(cores, D)
+    n1 = min(cores, D)
+    t1 = oracle_time(wls, oracle_inputs(wls, list(range(n1))))
+    per_channel = t1 / n1
     nch = int(max(1, min(D, budget_s / max(per_channel, 1e-9))))
-    chans = list(range(nch))
+    xs = oracle_inputs(wls, list(range(nch)))
     # repeat whole passes over the sample until the budget is spent (at least one)
     t, passes = 0.0, 0
     while passes == 0 or t < budget_s:
-        t += oracle_time(wls, chans)
+        t += oracle_time(wls, xs)
         passes += 1
     units = sum(w.batch * w.visible * nch for w in wls) * passes
     return {"value": units / t, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -316,16 +364,16 @@ def run_reference(args, wls):
     import oracle
     cores = oracle.default_threads()
     D = wls[0].D
-    probe = oracle_time(wls, [0])
+    probe = oracle_time(wls, oracle_inputs(wls, [0]))
     steps_total = args.steps + args.warmup
     budget = 150.0  # seconds for the whole run
     nch = int(max(1, min(D, budget / steps_total / max(probe, 1e-6))))
-    chans = list(range(nch))
+    xs = oracle_inputs(wls, list(range(nch)))
     for _ in range(args.warmup):
-        oracle_time(wls, chans)
+        oracle_time(wls, xs)
     t = 0.0
     for _ in range(args.steps):
-        t += oracle_time(wls, chans)
+        t += oracle_time(wls, xs)
     units = sum(w.batch * w.visible * nch for w in wls) * args.steps
     value = units / t
     line = {
@@ -346,7 +394,8 @@ def config_block(wls, n):
     return {"workload": workload_label(wls), "route": w0.route,
             "grids": [f"{w.h}x{w.w}" for w in wls], "batch": w0.batch, "d_inner": w0.D,
             "d_state": w0.N, "io_dtype": w0.dtype, "gate": w0.gate, "merge_scale": w0.merge_scale,
-            "conv": w0.conv, "zoh": w0.zoh, "mask_keep": w0.keep, "pass": "forward",
+            "conv": w0.conv, "zoh": w0.zoh, "mask_keep": w0.keep, "per_direction_planes": w0.per_dir,
+            "pass": "forward",
             "parallelism": f"replicas x{n} (one full workload per GPU, no collective)"}
 
 
@@ -372,35 +421,34 @@ def run_ours(args, wls):
     rot = min(rot, 8) if args.rotate <= 0 else args.rotate
     plans, host_sets, routes = [], [], []
     for wi, wl in enumerate(wls):
-        x = workloads.draw_masked(replica(wl, rank)) if wl.keep < 1 else workloads.draw(replica(wl, rank))
+        x = draw_inputs(replica(wl, rank))
         route = vs.Route(wl.route, wl.h, wl.w, wl.cls_pos)
         routes.append(route)
         dt = td[wl.dtype]
         host = {k: torch.from_numpy(x[k]).to(dt) for k in ("u", "delta", "B", "C", "z")}
-        if wl.conv:
-            x.update(workloads.draw_conv(wl))
         host.update({k: torch.from_numpy(np.ascontiguousarray(x[k], dtype=np.float32))
                      for k in ("A", "Dskip", "bias") + (("conv_w", "conv_b") if wl.conv else ())})
         if wl.keep < 1:
             host["pos"] = torch.from_numpy(x["pos"])
         host_sets.append(host)
-        ws_bytes = vs.workspace_size(route, host["u"], host["B"])
+        pd = dict(per_dir_inputs=wl.per_dir, per_dir_params=wl.per_dir)
+        ws_bytes = vs.workspace_size(route, host["u"], host["B"], **pd)
         per = []
         for r in range(rot):
             d = {k: v.to(dev) for k, v in host.items()}
-            out = torch.empty_like(d["u"])
             ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
             if args.backward:
                 dy = torch.randn(d["u"].shape[-3:], generator=torch.Generator().manual_seed(rank)).to(
                     dev, d["u"].dtype)
                 per.append(vs.BackwardPlan(route, d["u"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"],
                                            d["bias"], d["z"] if wl.gate else None, dy=dy,
-                                           merge_scale=wl.merge_scale))
+                                           merge_scale=wl.merge_scale, **pd))
                 continue
+            out = torch.empty(d["z"].shape, dtype=d["u"].dtype, device=dev)
             per.append(vs.Plan(route, d["u"], d["delta"], d["A"], d["B"], d["C"], d["Dskip"], d["bias"],
                                d["z"] if wl.gate else None, out=out, workspace=ws,
                                merge_scale=wl.merge_scale, conv_w=d.get("conv_w"),
-                               conv_b=d.get("conv_b"), zoh=wl.zoh, token_pos=d.get("pos")))
+                               conv_b=d.get("conv_b"), zoh=wl.zoh, token_pos=d.get("pos"), **pd))
         plans.append(per)
     launches_per_step = sum(per[0].kernels() for per in plans)
     knames = sorted({per[0].kernel_name() for per in plans})
@@ -419,7 +467,7 @@ def run_ours(args, wls):
            for _ in range(nfw)] for _ in range(K)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(dev.index if dev.index is not None else local)
+    sampler = ClockSampler(dev)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -459,14 +507,23 @@ def run_ours(args, wls):
     traffic = recorded_traffic(kname, workload_label(wls))
     upd_all = sum(updates(w) * K for w in wls)
     sfu_peak = 16 * 148 * sm_max * 1e6  # one exp per state update on the SFU
+    fma_peak = 128 * 148 * sm_max * 1e6  # FP32 lane-ops/s: 128 FP32 lanes per SM
+    upd_rate = upd_all / (ms_all * 1e-3)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "frac_vs_8TBs": round(achieved / NORTH_STAR_HBM_GBS, 4),
+                "frac_note": "frac divides by the measured copy bandwidth; frac_vs_8TBs by the 8 TB/s "
+                             "the >=60% HBM target is stated against",
                 "kernel": kname, "launch_ms_avg": round(ms_all / (K * nfw), 5),
                 "algorithmic_bytes_per_launch": [ab(w) for w in wls],
-                "sfu": {"state_updates_per_s": upd_all / (ms_all * 1e-3), "peak": sfu_peak,
-                        "frac": round(upd_all / (ms_all * 1e-3) / sfu_peak, 4),
-                        "note": "one ex2 per state update, 16 SFU results/clk/SM x 148 SMs at max clock"}}
+                "sfu": {"state_updates_per_s": upd_rate, "peak": sfu_peak,
+                        "frac": round(upd_rate / sfu_peak, 4),
+                        "note": "one ex2 per state update, 16 SFU results/clk/SM x 148 SMs at max clock"},
+                "fp32": {"lane_ops_per_s": 4 * upd_rate, "peak": fma_peak,
+                         "frac": round(4 * upd_rate / fma_peak, 4),
+                         "note": "4 FP32 ops per state update (Delta*A, Delta*u*B, the state FMA, the "
+                                 "read-out FMA), 128 FP32 lanes/clk/SM x 148 SMs at max clock"}}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -491,16 +548,17 @@ def run_ours(args, wls):
         hplans, h2d, d2h = [[], []], 0, 0
         for wl, route, host in zip(wls, routes, host_sets):
             pin = {k: v.pin_memory() for k, v in host.items()}
+            pd = dict(per_dir_inputs=wl.per_dir, per_dir_params=wl.per_dir)
             nbytes = vs.host_buffer_size(route, pin["u"], pin["B"], z=wl.gate, conv_w=wl.conv,
-                                         conv_b=wl.conv, token_pos=wl.keep < 1)
+                                         conv_b=wl.conv, token_pos=wl.keep < 1, **pd)
             for slot in range(2):
-                out = torch.empty_like(pin["u"]).pin_memory()
+                out = torch.empty(pin["z"].shape, dtype=pin["u"].dtype).pin_memory()
                 buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
                 hplans[slot].append(vs.HostPlan(route, pin["u"], pin["delta"], pin["A"], pin["B"], pin["C"],
                                                 pin["Dskip"], pin["bias"], pin["z"] if wl.gate else None,
                                                 out=out, device_buffer=buf, merge_scale=wl.merge_scale,
                                                 conv_w=pin.get("conv_w"), conv_b=pin.get("conv_b"),
-                                                zoh=wl.zoh, token_pos=pin.get("pos")))
+                                                zoh=wl.zoh, token_pos=pin.get("pos"), **pd))
             h2d += sum(v.numel() * v.element_size() for k, v in pin.items() if k != "z" or wl.gate)
             d2h += hplans[0][-1].out.numel() * hplans[0][-1].out.element_size()
         E = max(2, min(args.e2e_steps, K))
@@ -546,6 +604,10 @@ def main():
         wls = [w.with_(batch=args.batch) for w in wls]
     if args.backward and (args.conv or args.zoh or args.mask_keep < 1):
         raise SystemExit("--backward covers the Delta*B*u scan without --conv, --zoh or --mask-keep")
+    if args.per_dir:
+        if args.mask_keep < 1:
+            raise SystemExit("--per-dir does not combine with --mask-keep")
+        wls = [w.with_(per_dir=True) for w in wls]
     if args.backward:
         args.no_e2e = True  # the end-to-end leg times the forward entry point
     if args.conv or args.zoh or args.mask_keep < 1:

@@ -267,9 +267,12 @@ vscan_status vscan_forward(const vscan_route* route, const vscan_args* args, voi
  *     array's device address (cudaGetSymbolAddress) and keeps it; make that
  *     first call before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents.
- *     Nothing in it needs to start at zero (every element read is written
- *     first by the same call), but calls that overlap on the GPU (different
- *     streams, no ordering between them) race on it: order them.
+ *     On a dense grid every element the call reads is first written by the
+ *     same call. With a masked token set (token_pos) the pooled sums are
+ *     accumulated into the array, so the call first clears the bytes it uses
+ *     with an asynchronous memset on the caller's stream (no allocation).
+ *     Calls that overlap on the GPU (different streams, no ordering between
+ *     them) race on the array: order them.
  * Errors and the other conventions are those of vscan_forward.
  */
 vscan_status vscan_forward_pooled_noalloc(const vscan_route* route, const vscan_args* args, void* stream);

@@ -177,14 +177,34 @@ uint64_t workspace_need(const vscan_route* r, const vscan_args* a)
 // BIDIR sequences at least this long run 32-step chunks (bf16 I/O, no options).
 constexpr int kLongChunkMinL = 2048;
 
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute
+// stays set for the process), not on every launch: one flag per instantiation
+// of the calling template and device ordinal.
+template <typename Kernel>
+cudaError_t set_smem_once(Kernel* fn, int bytes, int* done_by_device, int max_devices)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < max_devices && __atomic_load_n(&done_by_device[dev], __ATOMIC_ACQUIRE) >= bytes)
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < max_devices)
+        __atomic_store_n(&done_by_device[dev], bytes, __ATOMIC_RELEASE);
+    return e;
+}
+
+constexpr int kAttrDevices = 64;
+
 template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL, int TOK = vscan::ST_TOK,
           int CH = vscan::ST_CH>
 cudaError_t launch_stream_mode(vscan::ScanParams p, int k_base, int grid_z, cudaStream_t s)
 {
     static_assert(!(FL & vscan::FL_CKPT) || TOK == vscan::BW_TOK, "checkpoints every BW_TOK steps");
     const size_t smem = vscan::stream_smem_bytes<T, KC, MODE, FL, CH, TOK>();
-    cudaError_t e = cudaFuncSetAttribute(vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH, TOK>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int attr_done[kAttrDevices] = {};
+    cudaError_t e = set_smem_once(vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH, TOK>, (int)smem,
+                                  attr_done, kAttrDevices);
     if (e != cudaSuccess) return e;
     p.k_base = k_base;
     const dim3 grid((p.D + CH - 1) / CH, p.batch, grid_z);
@@ -248,12 +268,13 @@ template <int RK, typename T, int NC, int FL>
 cudaError_t launch_resident_nc(const vscan::ScanParams& p, size_t smem, cudaStream_t s)
 {
     constexpr int CH = vscan::ResidentShape<RK>::CH;
-    cudaError_t e = cudaFuncSetAttribute(vscan::resident_scan_kernel<RK, T, NC, FL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem);
+    static int attr_done[kAttrDevices] = {};
+    cudaError_t e = set_smem_once(vscan::resident_scan_kernel<RK, T, NC, FL>, (int)kMaxSmem, attr_done,
+                                  kAttrDevices);
     if (e != cudaSuccess) return e;
     const dim3 grid((p.D + CH - 1) / CH, p.batch);
     vscan::resident_scan_kernel<RK, T, NC, FL><<<grid, 64 * NC, smem, s>>>(p);
-    return cudaSuccess;
+    return cudaGetLastError();
 }
 
 template <int RK, typename T, int FL>
@@ -285,33 +306,40 @@ cudaError_t launch_resident(const vscan::ScanParams& p, int nc, int fl, cudaStre
     }
 }
 
+// The pooled route's two launches; a failure names the step that failed.
 template <typename T, int FL>
-cudaError_t launch_pool_fl(const vscan::PoolParams& p, cudaStream_t s, size_t ws_bytes)
+vscan_status launch_pool_fl(const vscan::PoolParams& p, cudaStream_t s, size_t ws_bytes)
 {
     if constexpr ((FL & vscan::FL_MASK) != 0) {
         // B and C sums are added into the zeroed workspace (pB and pC)
         cudaError_t e = cudaMemsetAsync(p.pB, 0, ws_bytes, s);
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) return cuda_fail(e, "zeroing the pooled B/C sums");
         if (p.n_tok > 0) {
             constexpr int per_cta = 16 * vscan::PB_RUN;  // tokens of one CTA
             const dim3 g1((unsigned)((p.n_tok + per_cta - 1) / per_cta), p.batch, p.Ki);
             vscan::pool_bc_masked_kernel<T><<<g1, 256, 0, s>>>(p);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return cuda_fail(e, "launching pool_bc_masked_kernel");
         }
     } else {
         const dim3 g1(p.g.L, p.batch, p.Ki);
         vscan::pool_bc_kernel<T><<<g1, 128, 0, s>>>(p);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "launching pool_bc_kernel");
     }
     const size_t smem = vscan::pool_scan_smem_bytes(p.Ki, p.g.L, (FL & vscan::FL_CONV) != 0);
-    cudaError_t e = cudaFuncSetAttribute(vscan::pool_scan_kernel<T, FL>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    if (e != cudaSuccess) return e;
+    static int attr_done[kAttrDevices] = {};
+    cudaError_t e = set_smem_once(vscan::pool_scan_kernel<T, FL>, (int)kMaxSmem, attr_done, kAttrDevices);
+    if (e != cudaSuccess) return cuda_fail(e, "setting pool_scan_kernel's shared-memory limit");
     const dim3 g2((p.D + vscan::PL_CH - 1) / vscan::PL_CH, p.batch);
     vscan::pool_scan_kernel<T, FL><<<g2, vscan::PL_THREADS, smem, s>>>(p);
-    return cudaSuccess;
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launching pool_scan_kernel");
+    return VSCAN_OK;
 }
 
 template <typename T>
-cudaError_t launch_pool(const vscan::PoolParams& p, int fl, cudaStream_t s, size_t ws_bytes)
+vscan_status launch_pool(const vscan::PoolParams& p, int fl, cudaStream_t s, size_t ws_bytes)
 {
     using namespace vscan;
     switch (fl) {
@@ -350,8 +378,8 @@ vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s,
         p.conv_w = a->conv_w; p.conv_b = a->conv_b;
         p.pos = a->token_pos;
         p.n_tok = tokens_of(r, a);
-        cudaError_t e = launch_pool<T>(p, fl, s, workspace_need(r, a));
-        if (e != cudaSuccess) return cuda_fail(e, "configuring the pooled-scan kernel");
+        const vscan_status st = launch_pool<T>(p, fl, s, workspace_need(r, a));
+        if (st != VSCAN_OK) return st;
     } else {
         vscan::ScanParams p{};
         p.g = g;

@@ -35,6 +35,7 @@ class Workload:
     conv: bool = False  # fused kernel-four causal Conv1d + SiLU on u (BIDIR, pooled routes)
     zoh: bool = False   # zero-order-hold write term instead of Delta*B*u
     keep: float = 1.0   # pooled routes: fraction of visible tokens (masked set) when < 1
+    per_dir: bool = False  # every direction its own u, raw Delta, B, C and A, D, bias planes
 
     @property
     def tokens(self) -> int:
@@ -45,6 +46,11 @@ class Workload:
     def visible(self) -> int:
         """Tokens per image in the token arrays: all of them, or the visible ones of a mask."""
         return self.tokens if self.keep >= 1.0 else max(1, int(round(self.keep * self.h * self.w)))
+
+    @property
+    def K(self) -> int:
+        """Directions of the route."""
+        return {"bidir": 2, "cross4": 4, "atrous2": 4, "pool_w": 2, "pool_h": 2}[self.route]
 
     @property
     def token_channels(self) -> int:
