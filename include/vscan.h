@@ -58,7 +58,13 @@ typedef enum vscan_status {
     VSCAN_ERR_ALIGNMENT = -3,        /* pointer or channel count not 16-byte aligned */
     VSCAN_ERR_UNSUPPORTED = -4,      /* valid but not implemented (e.g. N > 16)    */
     VSCAN_ERR_CUDA = -5,             /* a CUDA runtime call failed                 */
-    VSCAN_ERR_WORKSPACE = -6         /* workspace missing or smaller than required */
+    VSCAN_ERR_WORKSPACE = -6,        /* workspace missing or smaller than required */
+    VSCAN_ERR_VALUE = -7,            /* device value check failed (see
+                                        VSCAN_FLAG_CHECK_VALUES); from
+                                        vscan_status_from_device_word only        */
+    VSCAN_ERR_DEVICE_TIMEOUT = -8    /* a kernel's internal pipeline wait gave up;
+                                        y is invalid; from
+                                        vscan_status_from_device_word only        */
 } vscan_status;
 
 /* Spatial routings. The token array of one image is row-major over the h x w
@@ -100,7 +106,15 @@ typedef enum vscan_flag {
      * expm1(Delta A_n) / A_n * B_n, equal to Delta B_n for A_n = 0.
      * "Norm or Direction? ...", sec. 3, Eq. 2; "Vision Mamba ...", sec. 4 (the
      * released kernels keep Delta*B*u, the default). */
-    VSCAN_FLAG_ZOH = 1
+    VSCAN_FLAG_ZOH = 1,
+    /* Opt-in value checks on the device before the scan, the conditions under
+     * which the scalar reference scan of "EfficientVMamba ...", sec. 2 ("Update
+     * an independent state inside each group") refuses its inputs: a
+     * non-finite value in any input or parameter, an unstable A (A > 0), or,
+     * with delta_softplus = 0, a negative time scale (raw Delta + bias < 0).
+     * A failure sets bit 1 of *args->status (which must then be non-NULL); the
+     * scan still runs. Costs one read of every input (bandwidth-bound). */
+    VSCAN_FLAG_CHECK_VALUES = 2
 } vscan_flag;
 
 /* Opaque, immutable route description (host memory only). */
@@ -171,6 +185,13 @@ typedef struct vscan_args {
                                VSCAN_ERR_UNSUPPORTED.                             */
     int32_t n_tokens;       /* visible tokens per image with token_pos, else 0     */
     int32_t reserved2;      /* must be 0                                            */
+    int32_t* status;        /* device int32 or NULL (also with vscan_forward_host).
+                               When given, kernels OR bits into it and never trap:
+                               1 = a value check failed (VSCAN_FLAG_CHECK_VALUES),
+                               2 = an internal pipeline wait gave up (y invalid).
+                               The caller zeroes it, synchronizes the stream and
+                               decodes it with vscan_status_from_device_word.
+                               Required with VSCAN_FLAG_CHECK_VALUES.             */
 } vscan_args;
 
 /*
@@ -220,19 +241,22 @@ vscan_status vscan_workspace_size(const vscan_route* route, const vscan_args* ar
 
 /*
  * Number of kernel launches vscan_forward makes for these arguments (host
- * only): 1 for BIDIR, CROSS4 and ATROUS2 (streaming or resident chunked
- * scan), 2 for the pooled routes (B/C pooling, then the fused
- * pool-scan-repeat), 0 for an empty batch.
+ * only): 1 for BIDIR, CROSS4 and ATROUS2 (pipelined, streaming or resident
+ * chunked scan), 2 for the pooled routes (B/C pooling, then the fused
+ * pool-scan-repeat), plus 1 with VSCAN_FLAG_CHECK_VALUES; 0 for an empty
+ * batch.
  */
 vscan_status vscan_plan_info(const vscan_route* route, const vscan_args* args, int32_t* kernels);
 
 /*
  * Name of the kernel that runs the scan for these arguments (host only), as
- * a static NUL-terminated string owned by the library: "stream_scan_kernel<R>"
- * (streaming scan), "resident_scan_kernel<R>" (chunked parallel scan of a
- * shared-memory-resident tile; R = BIDIR, CROSS4 or ATROUS2), "pool_scan_kernel"
- * (pooled routes) or "none" (empty batch). Same argument checks and errors
- * as vscan_plan_info; *name is untouched on error.
+ * a static NUL-terminated string owned by the library: "pipe_scan_kernel<R>"
+ * (mbarrier-pipelined scan, R = BIDIR or CROSS4, d_state 16 without the
+ * optional steps), "stream_scan_kernel<R>" (streaming scan),
+ * "resident_scan_kernel<R>" (chunked parallel scan of a shared-memory-resident
+ * tile; R = BIDIR, CROSS4 or ATROUS2), "pool_scan_kernel" (pooled routes) or
+ * "none" (empty batch). Same argument checks and errors as vscan_plan_info;
+ * *name is untouched on error.
  */
 vscan_status vscan_plan_kernel(const vscan_route* route, const vscan_args* args, const char** name);
 
@@ -343,6 +367,14 @@ vscan_status vscan_backward_workspace_size(const vscan_route* route, const vscan
 vscan_status vscan_backward(const vscan_route* route, const vscan_args* args, const void* dy,
                             const vscan_grads* grads, void* stream);
 
+/*
+ * Decode a device status word (vscan_args.status) after the stream has been
+ * synchronized: VSCAN_OK for 0, VSCAN_ERR_DEVICE_TIMEOUT if bit 2 is set, else
+ * VSCAN_ERR_VALUE if bit 1 is set. Host only; sets vscan_last_error() to a
+ * description when the result is not VSCAN_OK.
+ */
+vscan_status vscan_status_from_device_word(int32_t word);
+
 /* Message for the last non-OK status on this thread ("" if none). */
 const char* vscan_last_error(void);
 
@@ -350,7 +382,7 @@ const char* vscan_last_error(void);
 const char* vscan_status_string(int32_t status);
 
 /* Library ABI version; changes whenever vscan_args changes layout (2: flags,
- * conv_w and conv_b; 3: token_pos and n_tokens). */
+ * conv_w and conv_b; 3: token_pos and n_tokens; 4: status). */
 int32_t vscan_abi_version(void);
 
 #ifdef __cplusplus

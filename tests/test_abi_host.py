@@ -36,11 +36,13 @@ def test_library_exports_every_declared_function():
 
 
 def test_struct_layout_matches_the_header():
-    # int32 x4, 6 pointers, 3 pointers, int32 x3, float, pointer, uint64, int32 x2, 3 pointers, int32 x2
-    assert ctypes.sizeof(abi.VscanArgs) == 16 + 48 + 24 + 12 + 4 + 8 + 8 + 8 + 24 + 8
+    # int32 x4, 6 pointers, 3 pointers, int32 x3, float, pointer, uint64, int32 x2, 3 pointers, int32 x2,
+    # pointer
+    assert ctypes.sizeof(abi.VscanArgs) == 16 + 48 + 24 + 12 + 4 + 8 + 8 + 8 + 24 + 8 + 8
     assert abi.VscanArgs.flags.offset == 124 and abi.VscanArgs.conv_w.offset == 128
     assert abi.VscanArgs.token_pos.offset == 144 and abi.VscanArgs.n_tokens.offset == 152
-    assert abi.lib.vscan_abi_version() == abi.ABI_VERSION == 3
+    assert abi.VscanArgs.status.offset == 160
+    assert abi.lib.vscan_abi_version() == abi.ABI_VERSION == 4
 
 
 def test_status_strings():
@@ -149,8 +151,8 @@ def test_plan_kernel_names_the_scan_kernel():
     name = ctypes.c_char_p()
     for kind, h, w, cls, batch, D, chunks, expect in (
             ("atrous2", 56, 56, -1, 8, 192, 0, "stream_scan_kernel<ATROUS2>"),
-            ("cross4", 56, 56, -1, 16, 192, 0, "stream_scan_kernel<CROSS4>"),
-            ("bidir", 64, 64, 2048, 64, 768, 0, "stream_scan_kernel<BIDIR>"),
+            ("cross4", 56, 56, -1, 16, 192, 0, "pipe_scan_kernel<CROSS4>"),
+            ("bidir", 64, 64, 2048, 64, 768, 0, "pipe_scan_kernel<BIDIR>"),
             ("bidir", 14, 14, 98, 1, 384, 0, "resident_scan_kernel<BIDIR>"),  # few sequences
             ("cross4", 14, 14, -1, 1, 64, 4, "resident_scan_kernel<CROSS4>"),
             ("atrous2", 9, 13, -1, 1, 64, 2, "resident_scan_kernel<ATROUS2>"),
@@ -210,6 +212,46 @@ def test_zoh_flag_is_accepted_and_unknown_flags_are_not():
     r = vs.Route("atrous2", 4, 4)
     assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, flags=abi.FLAG_ZOH)), None) != -1
     assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, flags=4)), None) == -1
+
+
+def test_value_check_flag_needs_an_aligned_status_word():
+    fake = dict(u=0x1000, delta=0x2000, B=0x3000, C=0x4000, y=0x5000, A=0x6000)
+    r = vs.Route("cross4", 4, 4)
+    chk = abi.FLAG_CHECK_VALUES
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, flags=chk)), None) == -1
+    assert "status" in abi.lib.vscan_last_error().decode()
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, flags=chk, status=0x7002)), None) == -3
+    # accepted: the next failure is the missing workspace
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, flags=chk, status=0x7000)), None) == -6
+    assert abi.lib.vscan_forward(r.handle, ctypes.byref(_args(**fake, flags=chk | abi.FLAG_ZOH,
+                                                              status=0x7000)), None) == -6
+    n = ctypes.c_int32()
+    assert abi.lib.vscan_plan_info(r.handle, ctypes.byref(_args(**fake, flags=chk, status=0x7000)),
+                                   ctypes.byref(n)) == 0
+    assert n.value == 2
+
+
+def test_device_status_words_decode_on_the_host():
+    assert abi.lib.vscan_status_from_device_word(0) == 0
+    assert abi.lib.vscan_status_from_device_word(1) == -7
+    assert "value check" in abi.lib.vscan_last_error().decode()
+    assert abi.lib.vscan_status_from_device_word(2) == -8
+    assert abi.lib.vscan_status_from_device_word(3) == -8
+    assert abi.lib.vscan_status_from_device_word(8) == -1
+
+
+def test_plan_kernel_names_the_pipelined_kernel():
+    fake = dict(u=0x1000, delta=0x2000, B=0x3000, C=0x4000, y=0x5000, A=0x6000)
+    name = ctypes.c_char_p()
+    for kind, expect in (("bidir", "pipe_scan_kernel<BIDIR>"), ("cross4", "pipe_scan_kernel<CROSS4>"),
+                         ("atrous2", "stream_scan_kernel<ATROUS2>")):
+        r = vs.Route(kind, 8, 8)
+        for extra, exp in ((dict(seq_chunks=1), expect),
+                           (dict(seq_chunks=1, flags=abi.FLAG_ZOH), f"stream_scan_kernel<{kind.upper()}>"),
+                           (dict(seq_chunks=1, d_state=8), f"stream_scan_kernel<{kind.upper()}>")):
+            assert abi.lib.vscan_plan_kernel(r.handle, ctypes.byref(_args(**{**fake, **extra})),
+                                             ctypes.byref(name)) == 0
+            assert name.value.decode() == exp, (kind, extra)
 
 
 def test_host_buffer_holds_the_convolution_parameters():

@@ -22,10 +22,10 @@ import ctypes
 
 import torch
 
-from ._abi import BF16, F32, FLAG_ZOH, ROUTES, VscanArgs, VscanError, VscanGrads, check, lib
+from ._abi import BF16, F32, FLAG_CHECK_VALUES, FLAG_ZOH, ROUTES, VscanArgs, VscanError, VscanGrads, check, lib
 
 __all__ = ["Route", "forward", "backward", "forward_host", "workspace_size", "host_buffer_size",
-           "VscanError", "ROUTES"]
+           "status_from_device_word", "VscanError", "ROUTES"]
 
 
 class Route:
@@ -92,7 +92,7 @@ def _ptr(t):
 
 def _args(route, u, delta, A, B, C, Dskip, delta_bias, z, y, delta_softplus, merge_scale,
           per_dir_inputs, per_dir_params, workspace, seq_chunks, conv_w=None, conv_b=None,
-          zoh=False, token_pos=None):
+          zoh=False, token_pos=None, status=None, check_values=False):
     for name, t in (("u", u), ("delta", delta), ("B", B), ("C", C), ("z", z), ("y", y),
                     ("A", A), ("Dskip", Dskip), ("delta_bias", delta_bias), ("conv_w", conv_w),
                     ("conv_b", conv_b)):
@@ -126,7 +126,11 @@ def _args(route, u, delta, A, B, C, Dskip, delta_bias, z, y, delta_softplus, mer
     if workspace is not None:
         a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
     a.seq_chunks = int(seq_chunks)
-    a.flags = FLAG_ZOH if zoh else 0
+    a.flags = (FLAG_ZOH if zoh else 0) | (FLAG_CHECK_VALUES if check_values else 0)
+    if status is not None:
+        if status.dtype != torch.int32 or status.numel() < 1 or not status.is_cuda:
+            raise TypeError("status must be a CUDA int32 tensor")
+        a.status = _ptr(status)
     a.conv_w, a.conv_b = _ptr(conv_w), _ptr(conv_b)
     a.token_pos = _ptr(token_pos)
     a.n_tokens = tokens if token_pos is not None else 0
@@ -149,8 +153,15 @@ def workspace_size(route, u, B, *, per_dir_inputs=False, per_dir_params=False, *
 
 def forward(route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, delta_softplus=True,
             merge_scale=1.0, per_dir_inputs=False, per_dir_params=False, out=None, workspace=None,
-            seq_chunks=0, conv_w=None, conv_b=None, zoh=False, token_pos=None, stream=None):
-    """Routed selective scan on the GPU (vscan_forward). Returns y [batch, tokens, D]."""
+            seq_chunks=0, conv_w=None, conv_b=None, zoh=False, token_pos=None, stream=None,
+            status=None, check_values=False):
+    """Routed selective scan on the GPU (vscan_forward). Returns y [batch, tokens, D].
+
+    status: optional CUDA int32 tensor (one element, zeroed by the caller) into which the
+    kernels OR device-side findings; decode it with status_from_device_word after
+    synchronizing. check_values=True (needs status) first checks every input on the device:
+    non-finite values, A > 0, and (delta_softplus=False) a negative time scale.
+    """
     lead = 1 if per_dir_inputs else 0
     if out is None:
         out = torch.empty(u.shape[lead:], dtype=u.dtype, device=u.device)
@@ -160,9 +171,15 @@ def forward(route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, de
         need = workspace_size(route, u, B, per_dir_inputs=per_dir_inputs, per_dir_params=per_dir_params)
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=u.device)
     a = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus, merge_scale,
-              per_dir_inputs, per_dir_params, workspace, seq_chunks, conv_w, conv_b, zoh, token_pos)
+              per_dir_inputs, per_dir_params, workspace, seq_chunks, conv_w, conv_b, zoh, token_pos,
+              status, check_values)
     check(lib.vscan_forward(route.handle, ctypes.byref(a), _stream(stream, u.device)))
     return out
+
+
+def status_from_device_word(word):
+    """vscan_status_from_device_word: 0 (VSCAN_OK) or the negative status a device word encodes."""
+    return int(lib.vscan_status_from_device_word(int(word)))
 
 
 def host_buffer_size(route, u, B, *, z=True, Dskip=True, delta_bias=True, per_dir_inputs=False,

@@ -18,11 +18,14 @@ STATUS = {
     -4: "VSCAN_ERR_UNSUPPORTED",
     -5: "VSCAN_ERR_CUDA",
     -6: "VSCAN_ERR_WORKSPACE",
+    -7: "VSCAN_ERR_VALUE",
+    -8: "VSCAN_ERR_DEVICE_TIMEOUT",
 }
 ROUTES = {"bidir": 0, "cross4": 1, "atrous2": 2, "pool_w": 3, "pool_h": 4}
 F32, BF16 = 0, 1
-ABI_VERSION = 3
+ABI_VERSION = 4
 FLAG_ZOH = 1
+FLAG_CHECK_VALUES = 2
 
 
 class VscanArgs(ctypes.Structure):
@@ -55,6 +58,7 @@ class VscanArgs(ctypes.Structure):
         ("token_pos", ctypes.c_void_p),
         ("n_tokens", ctypes.c_int32),
         ("reserved2", ctypes.c_int32),
+        ("status", ctypes.c_void_p),
     ]
 
 
@@ -96,6 +100,7 @@ def _load():
         "vscan_backward": ([p, pa, p, ctypes.POINTER(VscanGrads), p], i32),
         "vscan_last_error": ([], ctypes.c_char_p),
         "vscan_status_string": ([i32], ctypes.c_char_p),
+        "vscan_status_from_device_word": ([i32], i32),
         "vscan_abi_version": ([], i32),
     }
     for name, (argtypes, restype) in sigs.items():

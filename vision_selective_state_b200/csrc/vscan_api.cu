@@ -15,6 +15,8 @@
 
 #include "vscan.h"
 #include "vscan_backward.cuh"
+#include "vscan_check.cuh"
+#include "vscan_pipe.cuh"
 #include "vscan_pool.cuh"
 #include "vscan_resident.cuh"
 #include "vscan_route.cuh"
@@ -26,7 +28,8 @@ struct vscan_route {
 
 namespace {
 
-constexpr int32_t kAbiVersion = 3;
+constexpr int32_t kAbiVersion = 4;
+constexpr int32_t kKnownFlags = VSCAN_FLAG_ZOH | VSCAN_FLAG_CHECK_VALUES;
 constexpr size_t kMaxSmem = 200 * 1024;  // dynamic shared memory the kernels may ask for
 thread_local std::string g_last_error;
 
@@ -70,8 +73,12 @@ vscan_status check_shape(const vscan_route* r, const vscan_args* a)
 {
     if (!r) return fail(VSCAN_ERR_INVALID_ARGUMENT, "route is NULL");
     if (!a) return fail(VSCAN_ERR_INVALID_ARGUMENT, "args is NULL");
-    if (a->flags & ~int32_t(VSCAN_FLAG_ZOH))
+    if (a->flags & ~kKnownFlags)
         return fail(VSCAN_ERR_INVALID_ARGUMENT, "unknown bits in args.flags 0x%x", (unsigned)a->flags);
+    if ((a->flags & VSCAN_FLAG_CHECK_VALUES) && !a->status)
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "VSCAN_FLAG_CHECK_VALUES needs a device status word (args.status)");
+    if ((reinterpret_cast<uintptr_t>(a->status) & 3u) != 0)
+        return fail(VSCAN_ERR_ALIGNMENT, "status is not 4-byte aligned");
     if (a->conv_b && !a->conv_w) return fail(VSCAN_ERR_INVALID_ARGUMENT, "conv_b given without conv_w");
     if (a->reserved2 != 0) return fail(VSCAN_ERR_INVALID_ARGUMENT, "args.reserved2 must be 0");
     if (a->token_pos) {
@@ -264,6 +271,41 @@ cudaError_t launch_stream(const vscan::ScanParams& p, int fl, cudaStream_t s)
     }
 }
 
+// The mbarrier-pipelined kernel (BIDIR, CROSS4; d_state 16; no optional step,
+// or the checkpoints of the backward's forward run).
+template <int RK, typename T, int LPC, int TOK, int NS, int MP, int MINB, int FL>
+cudaError_t launch_pipe_cfg(const vscan::ScanParams& p, cudaStream_t s)
+{
+    using Sh = vscan::PipeShape<RK, T, LPC, TOK, NS>;
+    const size_t smem = vscan::pipe_smem_bytes<RK, T, LPC, TOK, NS>();
+    static int attr_done[kAttrDevices] = {};
+    cudaError_t e = set_smem_once(vscan::pipe_scan_kernel<RK, T, LPC, TOK, NS, MP, MINB, FL>, (int)smem,
+                                  attr_done, kAttrDevices);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((p.D + Sh::CT - 1) / Sh::CT, p.batch);
+    vscan::pipe_scan_kernel<RK, T, LPC, TOK, NS, MP, MINB, FL><<<grid, Sh::THREADS, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+// Tile shape per route: BIDIR two lanes per channel (16-channel tiles, 3 CTAs
+// of 7 per SM at most); CROSS4 four lanes per channel (8-channel tiles), so that
+// the four-direction SS2D grids still put about ten consumer warps on every SM.
+template <int RK, typename T, int FL>
+cudaError_t launch_pipe(const vscan::ScanParams& p, cudaStream_t s)
+{
+    if constexpr (RK == vscan::RK_BIDIR) return launch_pipe_cfg<RK, T, 2, 16, 3, 0, 7, FL>(p, s);
+    else return launch_pipe_cfg<RK, T, 4, 16, 3, 0, 4, FL>(p, s);
+}
+
+// BIDIR and CROSS4 forwards with d_state 16 and none of the optional steps (the
+// backward's checkpointing run included) take the pipelined kernel when they
+// stream (the resident chunked kernel keeps the small grids).
+bool use_pipe(const vscan_route* r, const vscan_args* a, int fl)
+{
+    return (r->g.kind == vscan::RK_BIDIR || r->g.kind == vscan::RK_CROSS4) && (fl & ~vscan::FL_CKPT) == 0 &&
+           a->d_state == 16;
+}
+
 template <int RK, typename T, int NC, int FL>
 cudaError_t launch_resident_nc(const vscan::ScanParams& p, size_t smem, cudaStream_t s)
 {
@@ -395,8 +437,18 @@ vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s,
         p.scratch = static_cast<float*>(a->workspace);
         p.conv_w = a->conv_w; p.conv_b = a->conv_b;
         p.ckpt = ckpt;
+        p.status = a->status;
         const int nc = ckpt ? 1 : choose_chunks(r, a);  // checkpoints come from the streaming kernel
-        if (nc > 1) {
+        if (nc == 1 && use_pipe(r, a, fl)) {
+            cudaError_t e;
+            if (ckpt)
+                e = g.kind == vscan::RK_BIDIR ? launch_pipe<vscan::RK_BIDIR, T, vscan::FL_CKPT>(p, s)
+                                              : launch_pipe<vscan::RK_CROSS4, T, vscan::FL_CKPT>(p, s);
+            else
+                e = g.kind == vscan::RK_BIDIR ? launch_pipe<vscan::RK_BIDIR, T, 0>(p, s)
+                                              : launch_pipe<vscan::RK_CROSS4, T, 0>(p, s);
+            if (e != cudaSuccess) return cuda_fail(e, "launching pipe_scan_kernel");
+        } else if (nc > 1) {
             cudaError_t e;
             switch (g.kind) {
             case vscan::RK_BIDIR: e = launch_resident<vscan::RK_BIDIR, T>(p, nc, fl, s); break;
@@ -419,6 +471,43 @@ vscan_status dispatch(const vscan_route* r, const vscan_args* a, cudaStream_t s,
     return VSCAN_OK;
 }
 
+// VSCAN_FLAG_CHECK_VALUES: one bandwidth-bound pass over every input.
+vscan_status launch_value_checks(const vscan_route* r, const vscan_args* a, cudaStream_t s)
+{
+    vscan::CheckParams c{};
+    const int K = r->g.K;
+    const long long Ki = a->per_dir_inputs ? K : 1, Kp = a->per_dir_params ? K : 1;
+    const long long plane = (long long)a->batch * tokens_of(r, a);
+    const int bf = a->dtype == VSCAN_BF16;
+    auto add = [&](const void* ptr, long long n, int is_bf16, int nonpos, int vec) {
+        if (ptr && n > 0) c.seg[c.nseg++] = vscan::CheckSeg{ptr, n, is_bf16, nonpos, vec};
+    };
+    add(a->u, Ki * plane * a->channels, bf, 0, 1);
+    add(a->delta, Ki * plane * a->channels, bf, 0, 1);
+    add(a->B, Ki * plane * a->d_state, bf, 0, 0);
+    add(a->C, Ki * plane * a->d_state, bf, 0, 0);
+    add(a->z, plane * a->channels, bf, 0, 1);
+    add(a->A, Kp * a->channels * a->d_state, 0, 1, 0);
+    add(a->Dskip, Kp * a->channels, 0, 0, 0);
+    add(a->delta_bias, Kp * a->channels, 0, 0, 0);
+    add(a->conv_w, Kp * a->channels * 4, 0, 0, 0);
+    add(a->conv_b, Kp * a->channels, 0, 0, 0);
+    c.status = a->status;
+    c.dt_check = a->delta_softplus ? 0 : 1;
+    c.delta = a->delta;
+    c.delta_bf16 = bf;
+    c.bias = a->delta_bias;
+    c.plane = plane * a->channels;
+    c.D = a->channels;
+    c.Ki = (int)Ki;
+    c.Kp = (int)Kp;
+    const dim3 grid((unsigned)(4 * num_sms()), (unsigned)(c.nseg + c.dt_check));
+    vscan::check_values_kernel<<<grid, 256, 0, s>>>(c);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "launching check_values_kernel");
+    return VSCAN_OK;
+}
+
 vscan_status forward_device(const vscan_route* r, const vscan_args* a, cudaStream_t s, float* ckpt = nullptr)
 {
     const uint64_t need = workspace_need(r, a);
@@ -429,7 +518,17 @@ vscan_status forward_device(const vscan_route* r, const vscan_args* a, cudaStrea
         if (!aligned16(a->workspace)) return fail(VSCAN_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
     }
     if (a->batch == 0) return VSCAN_OK;
+    if (a->flags & VSCAN_FLAG_CHECK_VALUES) {
+        const vscan_status st = launch_value_checks(r, a, s);
+        if (st != VSCAN_OK) return st;
+    }
     return a->dtype == VSCAN_F32 ? dispatch<float>(r, a, s, ckpt) : dispatch<__nv_bfloat16>(r, a, s, ckpt);
+}
+
+int forward_flags(const vscan_args* a)
+{
+    return ((a->flags & VSCAN_FLAG_ZOH) ? vscan::FL_ZOH : 0) | (a->conv_w ? vscan::FL_CONV : 0) |
+           (a->token_pos ? vscan::FL_MASK : 0);
 }
 
 __global__ void route_map_kernel(vscan::RouteGeom g, int32_t* out)
@@ -554,12 +653,21 @@ vscan_status check_backward(const vscan_route* r, const vscan_args* a)
 // sums (the faster one on the atrous b8 and Vim-Tiny b1 grids); larger grids the
 // one built for 16 resident warps per SM (22-28 % faster on Vim-Tiny b64, SS2D b16
 // and Vim-Small b64).
+template <int RK, typename T, bool ASYNC>
+void launch_bwd_scan_async(const vscan::BwdParams& p, dim3 grid, cudaStream_t s)
+{
+    const long long warps = (long long)grid.x * grid.y * grid.z;
+    if (warps <= 8LL * num_sms()) vscan::bwd_scan_kernel<RK, T, 1, ASYNC><<<grid, 32, 0, s>>>(p);
+    else vscan::bwd_scan_kernel<RK, T, vscan::BW_MIN_WARPS, ASYNC><<<grid, 32, 0, s>>>(p);
+}
+
+// d_state 16 takes the build that gathers the next chunk with cp.async while the
+// current one runs (16-byte rows of B and C); other state counts load per element.
 template <int RK, typename T>
 void launch_bwd_scan(const vscan::BwdParams& p, dim3 grid, cudaStream_t s)
 {
-    const long long warps = (long long)grid.x * grid.y * grid.z;
-    if (warps <= 8LL * num_sms()) vscan::bwd_scan_kernel<RK, T, 1><<<grid, 32, 0, s>>>(p);
-    else vscan::bwd_scan_kernel<RK, T, vscan::BW_MIN_WARPS><<<grid, 32, 0, s>>>(p);
+    if (p.N == 16) launch_bwd_scan_async<RK, T, true>(p, grid, s);
+    else launch_bwd_scan_async<RK, T, false>(p, grid, s);
 }
 
 template <typename T>
@@ -740,9 +848,7 @@ vscan_status vscan_plan_info(const vscan_route* r, const vscan_args* a, int32_t*
     vscan_status st = check_shape(r, a);
     if (st != VSCAN_OK) return st;
     if (a->batch == 0) *kernels = 0;
-    else if (is_pool(r->g.kind)) *kernels = 2;
-    else if (choose_chunks(r, a) > 1) *kernels = 1;
-    else *kernels = 1;
+    else *kernels = (is_pool(r->g.kind) ? 2 : 1) + ((a->flags & VSCAN_FLAG_CHECK_VALUES) ? 1 : 0);
     return VSCAN_OK;
 }
 
@@ -756,9 +862,11 @@ vscan_status vscan_plan_kernel(const vscan_route* r, const vscan_args* a, const 
     static const char* const resident_names[] = {"resident_scan_kernel<BIDIR>",
                                                  "resident_scan_kernel<CROSS4>",
                                                  "resident_scan_kernel<ATROUS2>"};
+    static const char* const pipe_names[] = {"pipe_scan_kernel<BIDIR>", "pipe_scan_kernel<CROSS4>"};
     if (a->batch == 0) *name = "none";
     else if (is_pool(r->g.kind)) *name = "pool_scan_kernel";
     else if (choose_chunks(r, a) > 1) *name = resident_names[r->g.kind];
+    else if (use_pipe(r, a, forward_flags(a))) *name = pipe_names[r->g.kind];
     else *name = stream_names[r->g.kind];
     return VSCAN_OK;
 }
@@ -895,6 +1003,19 @@ vscan_status vscan_forward_pooled_noalloc(const vscan_route* r, const vscan_args
     return forward_device(r, &b, static_cast<cudaStream_t>(stream));
 }
 
+vscan_status vscan_status_from_device_word(int32_t word)
+{
+    if (word & vscan::DEV_STATUS_TIMEOUT)
+        return fail(VSCAN_ERR_DEVICE_TIMEOUT, "a kernel's pipeline wait gave up (device word 0x%x); y is invalid",
+                    (unsigned)word);
+    if (word & vscan::DEV_STATUS_VALUE)
+        return fail(VSCAN_ERR_VALUE,
+                    "value check failed (device word 0x%x): a non-finite input, A > 0, or a negative time scale",
+                    (unsigned)word);
+    if (word != 0) return fail(VSCAN_ERR_INVALID_ARGUMENT, "unknown bits in device word 0x%x", (unsigned)word);
+    return VSCAN_OK;
+}
+
 const char* vscan_last_error(void) { return g_last_error.c_str(); }
 
 const char* vscan_status_string(int32_t status)
@@ -907,6 +1028,8 @@ const char* vscan_status_string(int32_t status)
     case VSCAN_ERR_UNSUPPORTED: return "VSCAN_ERR_UNSUPPORTED";
     case VSCAN_ERR_CUDA: return "VSCAN_ERR_CUDA";
     case VSCAN_ERR_WORKSPACE: return "VSCAN_ERR_WORKSPACE";
+    case VSCAN_ERR_VALUE: return "VSCAN_ERR_VALUE";
+    case VSCAN_ERR_DEVICE_TIMEOUT: return "VSCAN_ERR_DEVICE_TIMEOUT";
     default: return "VSCAN_UNKNOWN_STATUS";
     }
 }

@@ -35,6 +35,7 @@
 
 #include "vscan_common.cuh"
 #include "vscan_route.cuh"
+#include "vscan_stream.cuh"
 
 namespace vscan {
 
@@ -175,6 +176,18 @@ __global__ void bwd_unpool_kernel(RouteGeom g, int batch, int D, int N, int Ki, 
     }
 }
 
+// Raw rows of one 16-step chunk as gathered by cp.async (ASYNC builds): the
+// next chunk's rows land here while the current chunk's adjoint runs.
+template <typename TI>
+struct __align__(16) BwdRaw {
+    TI d[BW_TOK][BW_CH];
+    TI u[BW_TOK][BW_CH];
+    float gy[BW_TOK][BW_CH];
+    TI B[BW_TOK][16];
+    TI C[BW_TOK][16];
+    int pos[BW_TOK];
+};
+
 // One 16-step chunk of one direction, staged in shared memory.
 struct BwdStage {
     int pos[BW_TOK];           // token, -1 pad, -2 past the end
@@ -208,12 +221,16 @@ template <> struct BwdReduce<true> : BwdReduceUX {
 // memory once per chunk, which keeps the shuffles off the steps' latency.
 constexpr int BW_MIN_WARPS = 16;
 
-template <int RK, typename TI, int MINW>
+// ASYNC (d_state 16): pass 2 gathers chunk c - 1 with cp.async while the
+// adjoint of chunk c runs, so a chunk's rows are waited for only once they have
+// had a whole chunk of compute to arrive.
+template <int RK, typename TI, int MINW, bool ASYNC>
 __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
 {
     constexpr bool SMEM_BC = MINW == 1;
     __shared__ BwdStage st;
     __shared__ __align__(16) BwdReduce<SMEM_BC> rd;
+    __shared__ BwdRaw<TI> raw[ASYNC ? 2 : 1];
     const int lane = threadIdx.x;
     const int cc = lane >> 2, grp = lane & 3;
     const int c0 = blockIdx.x * BW_CH, b = blockIdx.y, k = blockIdx.z;
@@ -297,6 +314,91 @@ __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
         __syncwarp();
     };
 
+    // ASYNC: gather chunk c's rows into raw[buf] (16-byte cp.async, zero fill for
+    // padding, past-the-end steps and channels beyond D), one commit group.
+    auto issue = [&](int c, int buf) {
+        BwdRaw<TI>& rw = raw[buf];
+        int q = -2;
+        if (lane < BW_TOK) {
+            const int t = c * BW_TOK + lane;
+            q = (t < L) ? route_token<RK>(p.g, k, t) : -2;
+            rw.pos[lane] = q;
+        }
+        constexpr int EL = 16 / (int)sizeof(TI);      // elements per 16-byte piece
+        constexpr int PR = BW_CH / EL;                 // pieces per u / Delta row
+        constexpr int PB = 16 / EL;                    // pieces per B / C row
+        constexpr int NPC = BW_TOK * (2 * PR + 2 + 2 * PB);  // + gy rows of 2 pieces
+#pragma unroll
+        for (int it = 0; it < (NPC + 31) / 32; ++it) {
+            const int f = lane + 32 * it;
+            int tsr, row, pc;  // 0 Delta, 1 u (PR pieces), 2 gy (2), 3 B, 4 C (PB)
+            if (f < 2 * BW_TOK * PR) {
+                tsr = f / (BW_TOK * PR);
+                const int r = f - tsr * BW_TOK * PR;
+                row = r / PR;
+                pc = r - row * PR;
+            } else if (f < 2 * BW_TOK * PR + 2 * BW_TOK) {
+                tsr = 2;
+                const int r = f - 2 * BW_TOK * PR;
+                row = r >> 1;
+                pc = r & 1;
+            } else {
+                const int r = f - 2 * BW_TOK * PR - 2 * BW_TOK;
+                tsr = 3 + r / (BW_TOK * PB);
+                const int r2 = r - (tsr - 3) * BW_TOK * PB;
+                row = r2 / PB;
+                pc = r2 - row * PB;
+            }
+            const int qj = __shfl_sync(FULL_MASK, q, row & (BW_TOK - 1));
+            if (f < NPC) {
+                const long long tok = qj >= 0 ? qj : 0;
+                if (tsr < 2) {
+                    const bool ok = qj >= 0 && c0 + pc * EL < D;
+                    const TI* src = (tsr == 0 ? rb : ub) + (ok ? tok * D + c0 + pc * EL : 0);
+                    cp_async16(tsr == 0 ? &rw.d[row][pc * EL] : &rw.u[row][pc * EL], src, ok);
+                } else if (tsr == 2) {
+                    const bool ok = qj >= 0 && c0 + 4 * pc < D;
+                    cp_async16(&rw.gy[row][4 * pc], gyb + (ok ? tok * D + c0 + 4 * pc : 0), ok);
+                } else {
+                    const bool ok = qj >= 0;
+                    const TI* src = (tsr == 3 ? Bb : Cb) + (ok ? tok * 16 + pc * EL : 0);
+                    cp_async16(tsr == 3 ? &rw.B[row][pc * EL] : &rw.C[row][pc * EL], src, ok);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+    // ASYNC: wait for raw[buf] and discretize it into st (as stage() does).
+    auto convert = [&](int buf) {
+        cp_async_wait<0>();
+        __syncwarp();
+        const BwdRaw<TI>& rw = raw[buf];
+        if (lane < BW_TOK) st.pos[lane] = rw.pos[lane];
+#pragma unroll
+        for (int r = 0; r < NE; ++r) {
+            const int e = lane + 32 * r;
+            const int j = e / BW_CH, ch = e % BW_CH, dd = c0 + ch;
+            const float xr = to_float(rw.d[j][ch]) + bias_l;
+            float x = xr, sg = 1.f;
+            if (p.softplus) {
+                x = softplus_f(xr);
+                sg = 1.0f / (1.0f + __expf(-xr));
+            }
+            const bool live = rw.pos[j] != -2 && dd < D;
+            st.x[j][ch] = live ? x : 0.f;
+            st.sig[j][ch] = sg;
+            st.u[j][ch] = to_float(rw.u[j][ch]);
+            st.gy[j][ch] = rw.gy[j][ch];
+        }
+#pragma unroll
+        for (int r = 0; r < NS; ++r) {
+            const int e = lane + 32 * r;
+            st.B[e >> 4][e & 15] = to_float(rw.B[e >> 4][e & 15]);
+            st.C[e >> 4][e & 15] = to_float(rw.C[e >> 4][e & 15]);
+        }
+        __syncwarp();
+    };
+
     // ---- pass 1: forward recurrence, state saved at every chunk boundary --------
     float h[4] = {0.f, 0.f, 0.f, 0.f};
     for (int c = 0; c < (p.ckpt_ready ? 0 : nch); ++c) {
@@ -317,8 +419,15 @@ __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
     // ---- pass 2: adjoint recurrence, chunks in reverse ------------------------------
     float gs[4] = {0.f, 0.f, 0.f, 0.f}, dAs[4] = {0.f, 0.f, 0.f, 0.f};
     float dDs = 0.f, dbs = 0.f;
+    if constexpr (ASYNC) issue(nch - 1, 0);
     for (int c = nch - 1; c >= 0; --c) {
-        stage(c, true);
+        if constexpr (ASYNC) {
+            const int buf = (nch - 1 - c) & 1;
+            convert(buf);
+            if (c > 0) issue(c - 1, buf ^ 1);  // lands while this chunk's adjoint runs
+        } else {
+            stage(c, true);
+        }
         float hs[BW_TOK + 1][4];  // hs[0] = state entering the chunk, hs[j + 1] after step j
 #pragma unroll
         for (int s = 0; s < 4; ++s) hs[0][s] = dvalid ? ck[((long long)c * D + d) * 16 + 4 * grp + s] : 0.f;
@@ -394,8 +503,14 @@ __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
             const int q = st.pos[j];
             if (q < 0 || dd >= D) continue;
             const long long o = ki * p.in_dir + (img + q) * D + dd;
-            if (p.du) atomicAdd(p.du + o, rd.u[j][ch]);
-            if (p.ddelta) atomicAdd(p.ddelta + o, rd.x[j][ch]);
+            if constexpr (RK == RK_ATROUS2) {
+                // one owner per pixel and channel: no other warp writes this element
+                if (p.du) p.du[o] = rd.u[j][ch];
+                if (p.ddelta) p.ddelta[o] = rd.x[j][ch];
+            } else {
+                if (p.du) atomicAdd(p.du + o, rd.u[j][ch]);
+                if (p.ddelta) atomicAdd(p.ddelta + o, rd.x[j][ch]);
+            }
         }
         if constexpr (SMEM_BC) {
 #pragma unroll

@@ -9,6 +9,11 @@
 namespace vscan {
 
 constexpr unsigned FULL_MASK = 0xffffffffu;
+
+// Bits of the caller's device status word (vscan_args.status), OR-ed in by the
+// kernels instead of trapping.
+constexpr int DEV_STATUS_VALUE = 1;    // a value check failed
+constexpr int DEV_STATUS_TIMEOUT = 2;  // a pipeline wait gave up (the output is invalid)
 constexpr float LOG2E = 1.4426950408889634f;
 
 // ---- element I/O -----------------------------------------------------------
@@ -95,6 +100,34 @@ __device__ __forceinline__ float fast_exp2(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x for a pair of x <= 0 on the FMA pipe instead of the SFU, so that a kernel
+// bound by the SFU's 16 results per clock and SM can move part of its
+// retentions to the 128-lane FP32 pipe. Range reduction of Cody and Waite
+// ("Software Manual for the Elementary Functions", 1980): k = round(x) by the
+// 1.5 * 2^23 shifter, f = x - k in [-1/2, 1/2], 2^f = 1 + f q(f) with q a
+// degree-5 least-squares fit of (2^f - 1)/f made by fit_exp2.py (relative
+// error 1e-7 in float32; 2^0 = 1 exactly), and 2^k added to the exponent
+// field. x is clamped at -126, where 2^x is below every normal float (the SFU
+// form flushes it to 0; this one returns 2^-126).
+__device__ __forceinline__ float2 exp2_fma2(float2 x)
+{
+    x.x = fmaxf(x.x, -126.f);
+    x.y = fmaxf(x.y, -126.f);
+    const float2 j = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+    const float2 k = __fadd2_rn(j, make_float2(-12582912.f, -12582912.f));
+    const float2 f = __ffma2_rn(k, make_float2(-1.f, -1.f), x);
+    float2 q = make_float2(1.537070493e-04f, 1.537070493e-04f);
+    q = __ffma2_rn(q, f, make_float2(1.339984825e-03f, 1.339984825e-03f));
+    q = __ffma2_rn(q, f, make_float2(9.618373588e-03f, 9.618373588e-03f));
+    q = __ffma2_rn(q, f, make_float2(5.550329015e-02f, 5.550329015e-02f));
+    q = __ffma2_rn(q, f, make_float2(2.402264774e-01f, 2.402264774e-01f));
+    q = __ffma2_rn(q, f, make_float2(6.931471825e-01f, 6.931471825e-01f));
+    const float2 p = __ffma2_rn(q, f, make_float2(1.f, 1.f));
+    // the low bits of j hold k (two's complement); k << 23 lands in the exponent
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
 }
 
 __device__ __forceinline__ float fast_rcp(float x)

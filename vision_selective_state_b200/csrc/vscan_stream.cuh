@@ -78,6 +78,7 @@ struct ScanParams {
     const float* conv_b;  // FL_CONV: [Kp][D] (nullable)
     float* ckpt;          // nullable: [K][batch][ceil(L/16)][D][16], the state entering every
                           // 16-step chunk (saved for the backward pass)
+    int* status;          // nullable device word: bits DEV_STATUS_* OR-ed in by the kernels
 };
 
 constexpr int ST_TOK = 16;  // steps per chunk (default; the checkpointing run always uses 16)
