@@ -287,14 +287,20 @@ cudaError_t launch_pipe_cfg(const vscan::ScanParams& p, cudaStream_t s)
     return cudaGetLastError();
 }
 
-// Tile shape per route: BIDIR two lanes per channel (16-channel tiles, 3 CTAs
-// of 7 per SM at most); CROSS4 four lanes per channel (8-channel tiles), so that
-// the four-direction SS2D grids still put about ten consumer warps on every SM.
+// Launch shape per route, measured on B200 (Vim-Small b64 bf16, SS2D b16 bf16):
+// BIDIR two lanes per channel (16-channel tiles), 16-step chunks, three slots,
+// launch bounds for 8 CTAs per SM (registers then allow 7 with this shared
+// memory); CROSS4 four lanes per channel (8-channel tiles: about ten consumer
+// warps per SM on the SS2D grid), 32-step chunks with two slots. The
+// checkpointing run of the backward pass takes 16-step chunks (the adjoint
+// scan's spacing).
 template <int RK, typename T, int FL>
 cudaError_t launch_pipe(const vscan::ScanParams& p, cudaStream_t s)
 {
-    if constexpr (RK == vscan::RK_BIDIR) return launch_pipe_cfg<RK, T, 2, 16, 3, 0, 7, FL>(p, s);
-    else return launch_pipe_cfg<RK, T, 4, 16, 3, 0, 4, FL>(p, s);
+    constexpr bool CK = (FL & vscan::FL_CKPT) != 0;
+    if constexpr (RK == vscan::RK_BIDIR) return launch_pipe_cfg<RK, T, 2, 16, 3, 0, 8, FL>(p, s);
+    else if constexpr (CK) return launch_pipe_cfg<RK, T, 4, 16, 3, 0, 4, FL>(p, s);
+    else return launch_pipe_cfg<RK, T, 4, 32, 2, 0, 3, FL>(p, s);
 }
 
 // BIDIR and CROSS4 forwards with d_state 16 and none of the optional steps (the

@@ -1,5 +1,5 @@
-// Pipelined routed selective scan: BIDIR (Vim, two directions), CROSS4 (SS2D,
-// four) and ATROUS2 (EfficientVMamba p = 2, four groups).
+// Pipelined routed selective scan for the routes whose directions all visit
+// every token: BIDIR (Vim, two directions) and CROSS4 (SS2D, four).
 //
 // One CTA covers one image b, a tile of CT channels and all KR directions of the
 // route, with one producer warp and one consumer warp per direction.
@@ -18,7 +18,8 @@
 //              cl * LPC + g owning channel cl of the tile and states
 //              g * SPL .. g * SPL + SPL - 1 (SPL = 16 / LPC). Per chunk:
 //                - discretize once per (step, channel) ("Vision Mamba ...",
-//                  sec. 3; "EfficientVMamba", sec. 2):
+//                  sec. 3; "EfficientVMamba", sec. 2), two items per packed
+//                  softplus:
 //                      Delta = softplus(raw + bias),  Delta * u
 //                  and, for bf16 I/O, widen the chunk's B and C to float32;
 //                - the recurrence and read-out per step and state (sec. 4),
@@ -28,12 +29,7 @@
 //                      h  = dA * h + (Delta * u) * B
 //                      y  = sum_n C * h              (butterfly reduce-scatter
 //                                                     over the LPC lanes)
-//                - ATROUS2 ("EfficientVMamba", sec. 3): every real pixel has
-//                  one owner, which scales, gates and stores y_k + D * u;
-//                  padding steps run (the state decays across them) and are
-//                  cropped. No merge, no barriers between the consumers.
-//                - BIDIR and CROSS4, the merge ("Vision Mamba ...", sec. 5;
-//                  SS2D): y_k + D * u
+//                - the merge ("Vision Mamba ...", sec. 5; SS2D): y_k + D * u
 //                  of every step goes to shared memory; the direction that
 //                  visits a token in the latest chunk (ties: larger k) is its
 //                  finalizer and adds the other directions' values, from
@@ -93,19 +89,20 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, unsigned parity)
 
 // Polls of a pipeline wait before it gives up (each poll may suspend the
 // thread for a short, hardware-defined time).
-constexpr int PIPE_WAIT_POLLS = 1 << 20;
+constexpr int PIPE_WAIT_POLLS = 1 << 18;
 
 // Wait until the phase with the given parity of an mbarrier has completed.
-// After PIPE_WAIT_POLLS polls it records the timeout and clears `live`; a warp
-// whose pipeline is no longer live skips every later wait, so a broken
-// pipeline costs one timeout, not one per chunk.
-__device__ __forceinline__ void mbar_wait(uint64_t* bar, unsigned parity, int* status, bool& live)
+// After PIPE_WAIT_POLLS polls it records the timeout and returns false; the
+// caller keeps that as its `live` flag and a warp whose pipeline is no longer
+// live skips every later wait, so a broken pipeline costs one timeout, not one
+// per chunk.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, int* status, bool live)
 {
-    if (!live) return;
+    if (!live) return false;
     for (int i = 0; i < PIPE_WAIT_POLLS; ++i)
-        if (mbar_test(bar, parity)) return;
+        if (mbar_test(bar, parity)) return true;
     if (status) atomicOr(status, DEV_STATUS_TIMEOUT);
-    live = false;
+    return false;
 }
 
 // Arrive on bar once all cp.async copies this thread issued before have landed
@@ -135,7 +132,8 @@ struct PipeShape {
     static constexpr int PC = CT / EL;                   // pieces per gathered row of u / Delta / z
     static constexpr int BCP = 16 / EL;                  // pieces per row of B (and of C)
     static constexpr int NP = TOK * (3 * PC + 2 * BCP);  // pieces per chunk and direction
-    static_assert(LPC == 1 || LPC == 2 || LPC == 4 || LPC == 8, "1, 2, 4 or 8 lanes per channel");
+    static_assert(LPC == 1 || LPC == 2 || LPC == 4, "1, 2 or 4 lanes per channel");
+    static_assert(RK == RK_BIDIR || RK == RK_CROSS4, "routes whose directions all visit every token");
     static_assert(PC >= 1, "a tile row must be at least 16 bytes");
     static_assert(TOK == 16 || TOK == 32, "16- or 32-step chunks");
     static_assert(TOK % LPC == 0, "whole groups of LPC steps per chunk");
@@ -214,25 +212,34 @@ __device__ __forceinline__ int4 pipe_meta(const RouteGeom& g, int k, int c, int 
     const int t = c * TOK + j;
     if (t >= g.L) return make_int4(-2, 0, 0, 0);
     const int p = route_token<RK>(g, k, t);
-    if constexpr (RK == RK_ATROUS2) return make_int4(p, 1, 0, 0);  // owner; -1 = padding
     int vs[KR];
 #pragma unroll
     for (int kk = 0; kk < KR; ++kk) vs[kk] = visit_step<RK>(g, kk, p);
-    int fk = 0;
+    // the finalizer and its chunk (kept alongside: indexing vs by a runtime value
+    // would put the array in local memory)
+    int fk = 0, fc = vs[0] / TOK;
 #pragma unroll
-    for (int kk = 1; kk < KR; ++kk)
-        if (vs[kk] / TOK >= vs[fk] / TOK) fk = kk;
+    for (int kk = 1; kk < KR; ++kk) {
+        const int ck = vs[kk] / TOK;
+        if (ck >= fc) {
+            fc = ck;
+            fk = kk;
+        }
+    }
     if (fk == k) {
-        int src = 0;
+        // byte o: the o-th other direction (constant array indices; the shift is
+        // the only runtime part)
+        int src = 0, o = 0;
 #pragma unroll
-        for (int o = 0; o < KR - 1; ++o) {
-            const int kk = o < k ? o : o + 1;
+        for (int kk = 0; kk < KR; ++kk) {
+            if (kk == k) continue;
             const int row = (vs[kk] / TOK == c) ? vs[kk] - c * TOK : 0xFF;
             src |= row << (8 * o);
+            ++o;
         }
         return make_int4(p, 1, src, 0);
     }
-    return make_int4(p, 0, (vs[fk] / TOK != c) ? 1 : 0, 0);
+    return make_int4(p, 0, (fc != c) ? 1 : 0, 0);
 }
 
 template <int RK, typename T, int LPC, int TOK, int NS, int MP, int MINB, int FL = 0>
@@ -244,7 +251,6 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
     using S = PipeShape<RK, T, LPC, TOK, NS>;
     constexpr int KR = S::KR, CT = S::CT, SPL = S::SPL, EPI = S::EPI, PC = S::PC, EL = S::EL;
     constexpr bool F32 = S::F32;
-    constexpr bool OWNER = RK == RK_ATROUS2;  // one owner per pixel: no merge between directions
     constexpr int NCONS = 32 * KR;            // threads in the consumers' named barriers
     static_assert(MP % 2 == 0 && MP <= SPL, "FMA-pipe retentions come in pairs");
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -274,15 +280,14 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NS;
             for (int k = 0; k < KR; ++k) {
-                if (c >= NS) mbar_wait(&sm.empty[k][s], ((c / NS) - 1) & 1, p.status, live);
+                if (c >= NS) live = mbar_wait(&sm.empty[k][s], ((c / NS) - 1) & 1, p.status, live);
                 PipeSlot<T, CT, TOK>& st = sm.slot[k][s];
                 int pos = -2, fin = 0;
                 if (lane < TOK) {
                     const int t = c * TOK + lane;
                     if (t < L) {
                         pos = route_token<RK>(p.g, k, t);
-                        if constexpr (OWNER) fin = pos >= 0;
-                        else fin = finalizer<RK, TOK>(p.g, pos) == k;
+                        fin = finalizer<RK, TOK>(p.g, pos) == k;
                     }
                 }
                 const T* u_base = static_cast<const T*>(p.u) + k * p.in_dir + img * D + c0;
@@ -362,17 +367,20 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % NS;
         const int mb = c & 1;
-        mbar_wait(&sm.full[k][s], (c / NS) & 1, p.status, live);
+        live = mbar_wait(&sm.full[k][s], (c / NS) & 1, p.status, live);
         const PipeSlot<T, CT, TOK>& st = sm.slot[k][s];
 
         // ---- discretize once per (step, channel); widen B and C (bf16)
+        static_assert(EPI % 2 == 0, "items come in pairs");
 #pragma unroll
-        for (int i = 0; i < EPI; ++i) {
-            const int j = g + LPC * i;
-            const bool live = ws.meta.m[mb][j].x != -2 && dvalid;
-            const float x = to_float(st.d[j][cl]) + bias_k;
-            const float dsp = live ? (p.softplus ? softplus_f(x) : x) : 0.f;
-            ws.dd[j][cl] = make_float2(dsp, live ? dsp * to_float(st.u[j][cl]) : 0.f);
+        for (int i = 0; i < EPI; i += 2) {
+            const int j0 = g + LPC * i, j1 = j0 + LPC;
+            const bool l0 = ws.meta.m[mb][j0].x != -2 && dvalid, l1 = ws.meta.m[mb][j1].x != -2 && dvalid;
+            const float2 x = make_float2(to_float(st.d[j0][cl]) + bias_k, to_float(st.d[j1][cl]) + bias_k);
+            const float2 sq = p.softplus ? softplus2(x) : x;
+            const float d0 = l0 ? sq.x : 0.f, d1 = l1 ? sq.y : 0.f;
+            ws.dd[j0][cl] = make_float2(d0, d0 * to_float(st.u[j0][cl]));
+            ws.dd[j1][cl] = make_float2(d1, d1 * to_float(st.u[j1][cl]));
         }
         if constexpr (!F32) {
 #pragma unroll
@@ -451,13 +459,9 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
             ws.yk[j][cl] = yv[i];
         }
         if (lane < TOK && c + 1 < nchunks) ws.meta.m[mb ^ 1][lane] = pipe_meta<RK, KR, TOK>(p.g, k, c + 1, lane);
-        if constexpr (OWNER) {
-            __syncwarp();
-        } else {
-            named_sync(1, NCONS);
-            cp_async_wait_all();  // this lane's prefetched parked values
-            __syncwarp();
-        }
+        named_sync(1, NCONS);
+        cp_async_wait_all();  // this lane's prefetched parked values
+        __syncwarp();
 
         // ---- merge, part 2: finalize (add the other directions, scale, gate, store) or park
 #pragma unroll
@@ -469,7 +473,7 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
             if (m.y) {
                 float acc = yown;
 #pragma unroll
-                for (int o = 0; o < (OWNER ? 0 : KR - 1); ++o) {
+                for (int o = 0; o < KR - 1; ++o) {
                     const int kk = o < k ? o : o + 1;
                     const int row = (m.z >> (8 * o)) & 0xFF;
                     acc += row == 0xFF ? ws.stg[o][j][cl] : sm.w[kk].yk[row][cl];
@@ -484,12 +488,7 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
         // the slot (u and z were its last readers) goes back to the producer
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[k][s]);
-        if constexpr (OWNER) {
-            __syncwarp();  // every lane's reads of dd, yk and meta come before the next chunk's writes
-            continue;
-        } else {
-            named_sync(2, NCONS);
-        }
+        named_sync(2, NCONS);
 
         // ---- prefetch the parked values the next chunk's finalizations need
         if (c + 1 < nchunks) {
