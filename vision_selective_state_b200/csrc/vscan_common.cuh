@@ -102,7 +102,7 @@ __device__ __forceinline__ float fast_exp2(float x)
     return y;
 }
 
-// 2^x for a pair of x <= 126 on the FMA pipe instead of the SFU, so that a kernel
+// 2^x for a pair of x <= 0 on the FMA pipe instead of the SFU, so that a kernel
 // bound by the SFU's 16 results per clock and SM can move part of its
 // retentions to the 128-lane FP32 pipe. Range reduction of Cody and Waite
 // ("Software Manual for the Elementary Functions", 1980): k = round(x) by the
@@ -175,50 +175,6 @@ __device__ __forceinline__ float2 softplus2(float2 x)
     p = __ffma2_rn(p, t, make_float2(1.442695022e+00f, 1.442695022e+00f));
     const float2 tp = __fmul2_rn(t, p);
     return make_float2(fmaxf(x.x, 0.f) + LN2 * tp.x, fmaxf(x.y, 0.f) + LN2 * tp.y);
-}
-
-// The same softplus with its exponential on the FMA pipe (exp2_fma2), for warps
-// that must not queue behind a kernel's SFU traffic.
-__device__ __forceinline__ float2 softplus2_fma(float2 x)
-{
-    const float2 t = exp2_fma2(make_float2(-fabsf(x.x) * LOG2E, -fabsf(x.y) * LOG2E));
-    float2 p = make_float2(7.366087753e-03f, 7.366087753e-03f);
-    p = __ffma2_rn(p, t, make_float2(-4.182628542e-02f, -4.182628542e-02f));
-    p = __ffma2_rn(p, t, make_float2(1.116363406e-01f, 1.116363406e-01f));
-    p = __ffma2_rn(p, t, make_float2(-1.960704774e-01f, -1.960704774e-01f));
-    p = __ffma2_rn(p, t, make_float2(2.751406133e-01f, 2.751406133e-01f));
-    p = __ffma2_rn(p, t, make_float2(-3.582780361e-01f, -3.582780361e-01f));
-    p = __ffma2_rn(p, t, make_float2(4.806761742e-01f, 4.806761742e-01f));
-    p = __ffma2_rn(p, t, make_float2(-7.213394046e-01f, -7.213394046e-01f));
-    p = __ffma2_rn(p, t, make_float2(1.442695022e+00f, 1.442695022e+00f));
-    const float2 tp = __fmul2_rn(t, p);
-    return make_float2(fmaxf(x.x, 0.f) + LN2 * tp.x, fmaxf(x.y, 0.f) + LN2 * tp.y);
-}
-
-// 1 / y for a pair of y in [1, 2^126] on the FMA pipe: the classic integer
-// first guess (subtracting the bits from 0x7EF311C3 mirrors the exponent,
-// relative error below 1/8), then three Newton steps r <- r (2 - y r), each
-// squaring the relative error (1.6e-2, 2.4e-4, 6e-8).
-__device__ __forceinline__ float2 rcp_fma2(float2 y)
-{
-    float2 r = make_float2(__int_as_float(0x7EF311C3 - __float_as_int(y.x)),
-                           __int_as_float(0x7EF311C3 - __float_as_int(y.y)));
-#pragma unroll
-    for (int i = 0; i < 3; ++i) {
-        const float2 e = __ffma2_rn(make_float2(-y.x, -y.y), r, make_float2(1.f, 1.f));  // 1 - y r
-        r = __ffma2_rn(r, e, r);                                                          // r + r (1 - y r)
-    }
-    return r;
-}
-
-// SiLU of a pair on the FMA pipe: z / (1 + 2^(-z log2 e)) with exp2_fma2 (the
-// exponent clamped to 126: below z = -87 the result is z * 2^-126, a signed
-// zero to within 1e-36) and rcp_fma2.
-__device__ __forceinline__ float2 silu2_fma(float2 z)
-{
-    const float2 e = exp2_fma2(make_float2(fminf(-z.x * LOG2E, 126.f), fminf(-z.y * LOG2E, 126.f)));
-    const float2 r = rcp_fma2(make_float2(1.f + e.x, 1.f + e.y));
-    return __fmul2_rn(z, r);
 }
 
 // SiLU(z) = z * sigma(z) = z / (1 + e^-z), signed and unbounded ("Vision
