@@ -288,17 +288,17 @@ cudaError_t launch_pipe_cfg(const vscan::ScanParams& p, cudaStream_t s)
 }
 
 // Launch shape per route, measured on B200 (Vim-Small b64 bf16, SS2D b16 bf16):
-// BIDIR two lanes per channel (16-channel tiles), 16-step chunks, three slots,
-// launch bounds for 8 CTAs per SM (registers then allow 7 with this shared
-// memory); CROSS4 four lanes per channel (8-channel tiles: about ten consumer
-// warps per SM on the SS2D grid), 32-step chunks with two slots. The
-// checkpointing run of the backward pass takes 16-step chunks (the adjoint
-// scan's spacing).
+// BIDIR two lanes per channel (16-channel tiles), 16-step chunks, two slots,
+// launch bounds for 8 CTAs per SM (80 registers; shared memory then also fits
+// 8, where three slots fit 7 and measured 6 % slower); CROSS4 four lanes per
+// channel (8-channel tiles: about ten consumer warps per SM on the SS2D grid),
+// 32-step chunks with two slots. The checkpointing run of the backward pass
+// takes 16-step chunks (the adjoint scan's spacing).
 template <int RK, typename T, int FL>
 cudaError_t launch_pipe(const vscan::ScanParams& p, cudaStream_t s)
 {
     constexpr bool CK = (FL & vscan::FL_CKPT) != 0;
-    if constexpr (RK == vscan::RK_BIDIR) return launch_pipe_cfg<RK, T, 2, 16, 3, 0, 8, FL>(p, s);
+    if constexpr (RK == vscan::RK_BIDIR) return launch_pipe_cfg<RK, T, 2, 16, 2, 0, 8, FL>(p, s);
     else if constexpr (CK) return launch_pipe_cfg<RK, T, 4, 16, 3, 0, 4, FL>(p, s);
     else return launch_pipe_cfg<RK, T, 4, 32, 2, 0, 3, FL>(p, s);
 }

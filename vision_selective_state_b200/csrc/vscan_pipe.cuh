@@ -140,23 +140,19 @@ struct PipeShape {
     static_assert(NS >= 2, "at least two slots per direction");
 };
 
-// Gathered rows of one direction's chunk, in the I/O type.
+// Gathered rows of one direction's chunk, in the I/O type, with the chunk's
+// merge plan. meta[j] for step j: x = token (-2 past the end), y = 1 if this
+// direction finalizes it, z = (finalizer) byte o = where the o-th other
+// direction's value is: its row in that direction's current chunk, or 0xFF =
+// parked in an earlier chunk; (non-finalizer) 1 if the value must be parked.
 template <typename T, int CT, int TOK>
 struct __align__(16) PipeSlot {
+    int4 meta[TOK];
     T u[TOK][CT];
     T d[TOK][CT];
     T z[TOK][CT];
     T B[TOK][16];
     T C[TOK][16];
-};
-
-// Per step of a chunk, for the merge: x = token (-2 past the end), y = 1 if this
-// direction finalizes it, z = (finalizer) byte o = where the o-th other
-// direction's value is: its row in that direction's current chunk, or 0xFF =
-// parked in an earlier chunk; (non-finalizer) 1 if the value must be parked.
-template <int KR, int TOK>
-struct __align__(16) PipeMeta {
-    int4 m[2][TOK];  // current and next chunk
 };
 
 template <int KR, int CT, int TOK, bool F32>
@@ -165,7 +161,6 @@ struct __align__(16) PipeWarpSmem {
     float yk[TOK][CT];            // y_k + D * u of the chunk (read by same-chunk finalizers)
     float stg[KR - 1][TOK][CT];   // parked values of the other directions (earlier chunks)
     float4 bcf[F32 ? 1 : TOK][8]; // bf16 I/O: the chunk's B (quads 0-3) and C (4-7) in float32
-    PipeMeta<KR, TOK> meta;
 };
 
 template <int RK, typename T, int LPC, int TOK, int NS>
@@ -267,7 +262,7 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
     if (threadIdx.x == 0) {
         for (int k = 0; k < KR; ++k)
             for (int s = 0; s < NS; ++s) {
-                mbar_init(&sm.full[k][s], 32);   // one cp.async arrival per producer lane
+                mbar_init(&sm.full[k][s], 64);   // per producer lane: its copies landed, its plan written
                 mbar_init(&sm.empty[k][s], 1);   // lane 0 of the consumer releases
             }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -282,14 +277,13 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
             for (int k = 0; k < KR; ++k) {
                 if (c >= NS) live = mbar_wait(&sm.empty[k][s], ((c / NS) - 1) & 1, p.status, live);
                 PipeSlot<T, CT, TOK>& st = sm.slot[k][s];
-                int pos = -2, fin = 0;
+                // the chunk's merge plan (route position, finalizer, sources or parking)
+                int4 plan = make_int4(-2, 0, 0, 0);
                 if (lane < TOK) {
-                    const int t = c * TOK + lane;
-                    if (t < L) {
-                        pos = route_token<RK>(p.g, k, t);
-                        fin = finalizer<RK, TOK>(p.g, pos) == k;
-                    }
+                    plan = pipe_meta<RK, KR, TOK>(p.g, k, c, lane);
+                    st.meta[lane] = plan;
                 }
+                const int pos = plan.x, fin = plan.y;
                 const T* u_base = static_cast<const T*>(p.u) + k * p.in_dir + img * D + c0;
                 const T* d_base = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + c0;
                 const T* z_base = p.z ? static_cast<const T*>(p.z) + img * D + c0 : nullptr;
@@ -331,6 +325,7 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
                     }
                 }
                 cp_async_mbar_arrive(&sm.full[k][s]);
+                mbar_arrive(&sm.full[k][s]);  // releases this lane's plan store
             }
         }
         cp_async_wait_all();
@@ -360,34 +355,47 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
     // FL_CKPT: this lane's SPL states of chunk c go to ck + c * D * 16
     float* ck = (CKPT && dvalid) ? p.ckpt + (((long long)k * p.batch + b) * nchunks * D + d) * 16 + g * SPL : nullptr;
 
-    if (lane < TOK) ws.meta.m[0][lane] = pipe_meta<RK, KR, TOK>(p.g, k, 0, lane);
-    __syncwarp();
-
-    bool live = true;
+    bool live = nchunks > 0 && mbar_wait(&sm.full[k][0], 0, p.status, true);
     for (int c = 0; c < nchunks; ++c) {
         const int s = c % NS;
-        const int mb = c & 1;
-        live = mbar_wait(&sm.full[k][s], (c / NS) & 1, p.status, live);
+        const int t0 = c * TOK;
         const PipeSlot<T, CT, TOK>& st = sm.slot[k][s];
 
-        // ---- discretize once per (step, channel); widen B and C (bf16)
+        // ---- discretize once per (step, channel); widen B and C (bf16). Every
+        // load comes before the first store: a store to the warp's buffers would
+        // otherwise hold back each later load (the compiler cannot tell the slot
+        // and the buffers apart), making one long chain of the chunk's items.
         static_assert(EPI % 2 == 0, "items come in pairs");
+        float dr[EPI], ur[EPI];
+#pragma unroll
+        for (int i = 0; i < EPI; ++i) {
+            const int j = g + LPC * i;
+            dr[i] = to_float(st.d[j][cl]) + bias_k;
+            ur[i] = to_float(st.u[j][cl]);
+        }
+        constexpr int NBC = F32 ? 1 : TOK / 4;
+        uint2 bcr[NBC];
+        if constexpr (!F32) {
+#pragma unroll
+            for (int i = 0; i < NBC; ++i) {
+                const int q = lane & 7, j = (lane >> 3) + 4 * i;
+                bcr[i] = *reinterpret_cast<const uint2*>(q < 4 ? &st.B[j][4 * q] : &st.C[j][4 * (q - 4)]);
+            }
+        }
 #pragma unroll
         for (int i = 0; i < EPI; i += 2) {
             const int j0 = g + LPC * i, j1 = j0 + LPC;
-            const bool l0 = ws.meta.m[mb][j0].x != -2 && dvalid, l1 = ws.meta.m[mb][j1].x != -2 && dvalid;
-            const float2 x = make_float2(to_float(st.d[j0][cl]) + bias_k, to_float(st.d[j1][cl]) + bias_k);
+            const float2 x = make_float2(dr[i], dr[i + 1]);
             const float2 sq = p.softplus ? softplus2(x) : x;
-            const float d0 = l0 ? sq.x : 0.f, d1 = l1 ? sq.y : 0.f;
-            ws.dd[j0][cl] = make_float2(d0, d0 * to_float(st.u[j0][cl]));
-            ws.dd[j1][cl] = make_float2(d1, d1 * to_float(st.u[j1][cl]));
+            const float d0 = (dvalid && t0 + j0 < L) ? sq.x : 0.f, d1 = (dvalid && t0 + j1 < L) ? sq.y : 0.f;
+            ws.dd[j0][cl] = make_float2(d0, d0 * ur[i]);
+            ws.dd[j1][cl] = make_float2(d1, d1 * ur[i + 1]);
         }
         if constexpr (!F32) {
 #pragma unroll
-            for (int i = 0; i < TOK / 4; ++i) {
+            for (int i = 0; i < NBC; ++i) {
                 const int q = lane & 7, j = (lane >> 3) + 4 * i;
-                const T* srcp = q < 4 ? &st.B[j][4 * q] : &st.C[j][4 * (q - 4)];
-                const uint2 raw = *reinterpret_cast<const uint2*>(srcp);
+                const uint2 raw = bcr[i];
                 ws.bcf[j][q] = make_float4(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u),
                                            __uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u));
             }
@@ -452,46 +460,74 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
             yv[gq] = reduce_scatter<LPC>(yp, g);  // this lane now holds step gq * LPC + g
         }
         // y_k + D * u of every step into shared memory (read by same-chunk finalizers)
+        float uy[EPI];
+#pragma unroll
+        for (int i = 0; i < EPI; ++i) uy[i] = to_float(st.u[g + LPC * i][cl]);
 #pragma unroll
         for (int i = 0; i < EPI; ++i) {
-            const int j = g + LPC * i;
-            yv[i] = fmaf(Dk, to_float(st.u[j][cl]), yv[i]);
-            ws.yk[j][cl] = yv[i];
+            yv[i] = fmaf(Dk, uy[i], yv[i]);
+            ws.yk[g + LPC * i][cl] = yv[i];
         }
-        if (lane < TOK && c + 1 < nchunks) ws.meta.m[mb ^ 1][lane] = pipe_meta<RK, KR, TOK>(p.g, k, c + 1, lane);
         named_sync(1, NCONS);
         cp_async_wait_all();  // this lane's prefetched parked values
         __syncwarp();
 
-        // ---- merge, part 2: finalize (add the other directions, scale, gate, store) or park
+        // ---- merge, part 2: finalize (add the other directions, scale, gate, store) or park.
+        // Loads first, then the arithmetic, then predicated stores; the two guards
+        // are warp-uniform (whole chunks finalize or park, but for the few where
+        // the directions cross).
+        int4 mt[EPI];
+        bool fin[EPI], park[EPI];
+        bool any_fin = false, any_park = false;
 #pragma unroll
         for (int i = 0; i < EPI; ++i) {
-            const int j = g + LPC * i;
-            const int4 m = ws.meta.m[mb][j];
-            if (m.x < 0 || !dvalid) continue;
-            const float yown = yv[i];
-            if (m.y) {
-                float acc = yown;
+            mt[i] = st.meta[g + LPC * i];
+            const bool ok = mt[i].x >= 0 && dvalid;
+            fin[i] = ok && mt[i].y;
+            park[i] = ok && !mt[i].y && mt[i].z;
+            any_fin |= fin[i];
+            any_park |= park[i];
+        }
+        if (__any_sync(FULL_MASK, any_fin)) {
+            // a non-finalizer's plan holds 0 or 1 in byte 0 and zeros above: every
+            // address below stays inside the buffers
+            float acc[EPI], zg[EPI];
+#pragma unroll
+            for (int i = 0; i < EPI; ++i) {
+                const int j = g + LPC * i;
+                acc[i] = yv[i];
 #pragma unroll
                 for (int o = 0; o < KR - 1; ++o) {
                     const int kk = o < k ? o : o + 1;
-                    const int row = (m.z >> (8 * o)) & 0xFF;
-                    acc += row == 0xFF ? ws.stg[o][j][cl] : sm.w[kk].yk[row][cl];
+                    const int row = (mt[i].z >> (8 * o)) & 0xFF;
+                    const float* src = row == 0xFF ? &ws.stg[o][j][cl] : &sm.w[kk].yk[row & (TOK - 1)][cl];
+                    acc[i] += *src;
                 }
-                float out = acc * p.merge_scale;
-                if (p.z) out *= silu_f(to_float(st.z[j][cl]));
-                store_elem<T>(y_base + (long long)m.x * D, out);
-            } else if (m.z) {
-                park_k[(long long)m.x * D] = yown;
+                zg[i] = p.z ? to_float(st.z[j][cl]) : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < EPI; ++i) {
+                float out = acc[i] * p.merge_scale;
+                if (p.z) out *= silu_f(zg[i]);
+                if (fin[i]) store_elem<T>(y_base + (long long)mt[i].x * D, out);
             }
         }
-        // the slot (u and z were its last readers) goes back to the producer
+        if (__any_sync(FULL_MASK, any_park)) {
+#pragma unroll
+            for (int i = 0; i < EPI; ++i)
+                if (park[i]) park_k[(long long)mt[i].x * D] = yv[i];
+        }
+        // the slot (u, z and the plan were its last readers) goes back to the producer
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[k][s]);
         named_sync(2, NCONS);
 
-        // ---- prefetch the parked values the next chunk's finalizations need
+        // ---- next chunk: wait for its slot, prefetch the parked values its
+        // finalizations need
         if (c + 1 < nchunks) {
+            const int s1 = (c + 1) % NS;
+            live = mbar_wait(&sm.full[k][s1], ((c + 1) / NS) & 1, p.status, live);
+            const PipeSlot<T, CT, TOK>& nx = sm.slot[k][s1];
             constexpr int PF = TOK * (KR - 1) * (CT / 4);  // 16-byte pieces of float32 rows
 #pragma unroll
             for (int it = 0; it < (PF + 31) / 32; ++it) {
@@ -500,7 +536,7 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
                     const int j = f / ((KR - 1) * (CT / 4));
                     const int r = f - j * (KR - 1) * (CT / 4);
                     const int o = r / (CT / 4), q = r - o * (CT / 4);
-                    const int4 m = ws.meta.m[mb ^ 1][j];
+                    const int4 m = nx.meta[j];
                     const bool ok = m.x >= 0 && m.y && ((m.z >> (8 * o)) & 0xFF) == 0xFF && (c0 + 4 * q) < D;
                     const int kk = o < k ? o : o + 1;
                     const float* src = p.scratch + ((long long)kk * p.batch + b) * tokens * D + c0 + 4 * q +
