@@ -131,7 +131,8 @@ struct PipeShape {
     static constexpr int EL = 16 / (int)sizeof(T);       // elements per 16-byte piece
     static constexpr int PC = CT / EL;                   // pieces per gathered row of u / Delta / z
     static constexpr int BCP = 16 / EL;                  // pieces per row of B (and of C)
-    static constexpr int NP = TOK * (3 * PC + 2 * BCP);  // pieces per chunk and direction
+    static constexpr int PPR = 3 * PC + 2 * BCP;         // pieces per step and direction
+    static constexpr int PARTS = 32 / TOK;               // producer lanes per step
     static_assert(LPC == 1 || LPC == 2 || LPC == 4, "1, 2 or 4 lanes per channel");
     static_assert(RK == RK_BIDIR || RK == RK_CROSS4, "routes whose directions all visit every token");
     static_assert(PC >= 1, "a tile row must be at least 16 bytes");
@@ -271,57 +272,39 @@ __global__ void __launch_bounds__(PipeShape<RK, T, LPC, TOK, NS>::THREADS, MINB)
 
     if (warp == KR) {
         // ================================ producer ==================================
+        const int r = lane % TOK, part = lane / TOK;
         bool live = true;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NS;
             for (int k = 0; k < KR; ++k) {
                 if (c >= NS) live = mbar_wait(&sm.empty[k][s], ((c / NS) - 1) & 1, p.status, live);
                 PipeSlot<T, CT, TOK>& st = sm.slot[k][s];
-                // the chunk's merge plan (route position, finalizer, sources or parking)
-                int4 plan = make_int4(-2, 0, 0, 0);
-                if (lane < TOK) {
-                    plan = pipe_meta<RK, KR, TOK>(p.g, k, c, lane);
-                    st.meta[lane] = plan;
-                }
-                const int pos = plan.x, fin = plan.y;
-                const T* u_base = static_cast<const T*>(p.u) + k * p.in_dir + img * D + c0;
-                const T* d_base = static_cast<const T*>(p.delta) + k * p.in_dir + img * D + c0;
-                const T* z_base = p.z ? static_cast<const T*>(p.z) + img * D + c0 : nullptr;
-                const T* B_base = static_cast<const T*>(p.B) + k * p.bc_dir + img * 16;
-                const T* C_base = static_cast<const T*>(p.C) + k * p.bc_dir + img * 16;
+                // lane -> (step r, part q of the step's 16-byte pieces): the lane's
+                // own plan gives the token, so no piece needs another lane's data
+                const int4 plan = pipe_meta<RK, KR, TOK>(p.g, k, c, r);
+                if (part == 0) st.meta[r] = plan;
+                const bool v = plan.x >= 0;
+                const long long tok = v ? plan.x : 0;
+                const T* u_row = static_cast<const T*>(p.u) + k * p.in_dir + (img + tok) * D + c0;
+                const T* d_row = static_cast<const T*>(p.delta) + k * p.in_dir + (img + tok) * D + c0;
+                const T* z_row = p.z ? static_cast<const T*>(p.z) + (img + tok) * D + c0 : u_row;
+                const bool zc = v && plan.y && p.z;
+                const T* B_row = static_cast<const T*>(p.B) + k * p.bc_dir + (img + tok) * 16;
+                const T* C_row = static_cast<const T*>(p.C) + k * p.bc_dir + (img + tok) * 16;
 #pragma unroll
-                for (int it = 0; it < (S::NP + 31) / 32; ++it) {
-                    const int f = lane + 32 * it;
-                    // f -> (tensor, row, piece): u, Delta, z rows of PC pieces, then B, C rows of BCP
-                    int tsr, row, pc;
-                    if (f < 3 * TOK * PC) {
-                        tsr = f / (TOK * PC);
-                        const int r = f - tsr * TOK * PC;
-                        row = r / PC;
-                        pc = r - row * PC;
-                    } else {
-                        const int r = f - 3 * TOK * PC;
-                        tsr = 3 + r / (TOK * S::BCP);
-                        const int r2 = r - (tsr - 3) * TOK * S::BCP;
-                        row = r2 / S::BCP;
-                        pc = r2 - row * S::BCP;
-                    }
-                    const int pj = __shfl_sync(FULL_MASK, pos, row & (TOK - 1));
-                    const int fj = __shfl_sync(FULL_MASK, fin, row & (TOK - 1));
-                    if (f < S::NP) {
-                        const long long tok = pj >= 0 ? pj : 0;
-                        if (tsr < 3) {
-                            const bool ok = pj >= 0 && (c0 + pc * EL) < D && (tsr < 2 || (fj && z_base));
-                            const T* src = (tsr == 0 ? u_base : (tsr == 1 ? d_base : (z_base ? z_base : u_base))) +
-                                           (ok ? tok * D + pc * EL : 0);
-                            T* dst = tsr == 0 ? &st.u[row][pc * EL] : (tsr == 1 ? &st.d[row][pc * EL] : &st.z[row][pc * EL]);
-                            cp_async16(dst, src, ok);
-                        } else {
-                            const bool ok = pj >= 0;
-                            const T* src = (tsr == 3 ? B_base : C_base) + (ok ? tok * 16 + pc * EL : 0);
-                            T* dst = tsr == 3 ? &st.B[row][pc * EL] : &st.C[row][pc * EL];
-                            cp_async16(dst, src, ok);
-                        }
+                for (int i = 0; i < S::PPR; ++i) {
+                    if (S::PARTS > 1 && i % S::PARTS != part) continue;
+                    if (i < 3 * PC) {  // u, Delta, z: PC pieces each
+                        const int t = i / PC, q = i % PC;
+                        const bool ok = (t == 2 ? zc : v) && (c0 + q * EL) < D;
+                        const T* src = (t == 0 ? u_row : (t == 1 ? d_row : z_row)) + (ok ? q * EL : 0);
+                        T* dst = (t == 0 ? &st.u[r][0] : (t == 1 ? &st.d[r][0] : &st.z[r][0])) + q * EL;
+                        cp_async16(dst, src, ok);
+                    } else {  // B, C: BCP pieces each
+                        const int t = (i - 3 * PC) / S::BCP, q = (i - 3 * PC) % S::BCP;
+                        const T* src = (t == 0 ? B_row : C_row) + (v ? q * EL : 0);
+                        T* dst = (t == 0 ? &st.B[r][0] : &st.C[r][0]) + q * EL;
+                        cp_async16(dst, src, v);
                     }
                 }
                 cp_async_mbar_arrive(&sm.full[k][s]);
