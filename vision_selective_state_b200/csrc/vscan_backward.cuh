@@ -188,8 +188,9 @@ struct __align__(16) BwdRaw {
     int pos[BW_TOK];
 };
 
-// One 16-step chunk of one direction, staged in shared memory.
-struct BwdStage {
+// One 16-step chunk of one direction, staged in shared memory (B and C rows are
+// read as 16-byte quads).
+struct __align__(16) BwdStage {
     int pos[BW_TOK];           // token, -1 pad, -2 past the end
     float x[BW_TOK][BW_CH];    // discretized step Delta
     float sig[BW_TOK][BW_CH];  // d Delta / d raw
@@ -240,12 +241,14 @@ __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
     const int ki = p.in_dir ? k : 0;
     const long long img = (long long)b * tokens;
     const int nch = (L + BW_TOK - 1) / BW_TOK;
-    float a2[4], An[4];
+    // this lane's four states as two pairs (packed f32x2 arithmetic)
+    float2 a2[2], An[2];
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        const int n = 4 * grp + s;
-        An[s] = (dvalid && n < N) ? __ldg(p.A + (long long)k * p.a_dir + (long long)d * N + n) : 0.f;
-        a2[s] = An[s] * LOG2E;
+    for (int q = 0; q < 2; ++q) {
+        const int n = 4 * grp + 2 * q;
+        const float* Ar = p.A + (long long)k * p.a_dir + (long long)d * N + n;
+        An[q] = make_float2((dvalid && n < N) ? __ldg(Ar) : 0.f, (dvalid && n + 1 < N) ? __ldg(Ar + 1) : 0.f);
+        a2[q] = make_float2(An[q].x * LOG2E, An[q].y * LOG2E);
     }
     const float Dd = (dvalid && p.Dskip) ? __ldg(p.Dskip + k * p.v_dir + d) : 0.f;
     const float* gyb = p.gy + img * D;
@@ -400,24 +403,34 @@ __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
     };
 
     // ---- pass 1: forward recurrence, state saved at every chunk boundary --------
-    float h[4] = {0.f, 0.f, 0.f, 0.f};
+    // one step of the recurrence for a pair of states: h = 2^(x A log2 e) h + (x B) u
+    auto step2 = [&](float2 hp, float x, float uu, float2 Bq, float2 a2q) {
+        const float2 xx = make_float2(x, x);
+        const float2 xa = __fmul2_rn(xx, a2q);
+        const float2 e = make_float2(fast_exp2(xa.x), fast_exp2(xa.y));
+        return __ffma2_rn(e, hp, __fmul2_rn(__fmul2_rn(xx, Bq), make_float2(uu, uu)));
+    };
+    float2 h[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
     for (int c = 0; c < (p.ckpt_ready ? 0 : nch); ++c) {
         if (dvalid) {
 #pragma unroll
-            for (int s = 0; s < 4; ++s) ck[((long long)c * D + d) * 16 + 4 * grp + s] = h[s];
+            for (int q = 0; q < 2; ++q)
+                *reinterpret_cast<float2*>(&ck[((long long)c * D + d) * 16 + 4 * grp + 2 * q]) = h[q];
         }
         stage(c, false);
 #pragma unroll 4
         for (int j = 0; j < BW_TOK; ++j) {
             const float x = st.x[j][cc], uu = st.u[j][cc];
-#pragma unroll
-            for (int s = 0; s < 4; ++s) h[s] = fmaf(fast_exp2(x * a2[s]), h[s], x * st.B[j][4 * grp + s] * uu);
+            const float4 Bv = *reinterpret_cast<const float4*>(&st.B[j][4 * grp]);
+            h[0] = step2(h[0], x, uu, make_float2(Bv.x, Bv.y), a2[0]);
+            h[1] = step2(h[1], x, uu, make_float2(Bv.z, Bv.w), a2[1]);
         }
     }
     __syncwarp();
 
     // ---- pass 2: adjoint recurrence, chunks in reverse ------------------------------
-    float gs[4] = {0.f, 0.f, 0.f, 0.f}, dAs[4] = {0.f, 0.f, 0.f, 0.f};
+    float2 gs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    float2 dAs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
     float dDs = 0.f, dbs = 0.f;
     if constexpr (ASYNC) issue(nch - 1, 0);
     for (int c = nch - 1; c >= 0; --c) {
@@ -428,34 +441,46 @@ __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
         } else {
             stage(c, true);
         }
-        float hs[BW_TOK + 1][4];  // hs[0] = state entering the chunk, hs[j + 1] after step j
+        float2 hs[BW_TOK + 1][2];  // hs[0] = state entering the chunk, hs[j + 1] after step j
 #pragma unroll
-        for (int s = 0; s < 4; ++s) hs[0][s] = dvalid ? ck[((long long)c * D + d) * 16 + 4 * grp + s] : 0.f;
+        for (int q = 0; q < 2; ++q)
+            hs[0][q] = dvalid ? *reinterpret_cast<const float2*>(&ck[((long long)c * D + d) * 16 + 4 * grp + 2 * q])
+                              : make_float2(0.f, 0.f);
 #pragma unroll
         for (int j = 0; j < BW_TOK; ++j) {
             const float x = st.x[j][cc], uu = st.u[j][cc];
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                hs[j + 1][s] = fmaf(fast_exp2(x * a2[s]), hs[j][s], x * st.B[j][4 * grp + s] * uu);
+            const float4 Bv = *reinterpret_cast<const float4*>(&st.B[j][4 * grp]);
+            hs[j + 1][0] = step2(hs[j][0], x, uu, make_float2(Bv.x, Bv.y), a2[0]);
+            hs[j + 1][1] = step2(hs[j][1], x, uu, make_float2(Bv.z, Bv.w), a2[1]);
         }
 #pragma unroll
         for (int j = BW_TOK - 1; j >= 0; --j) {
             const int q = st.pos[j];
             if (q == -2) continue;  // past the end of the sequence (uniform over the warp)
             const float x = st.x[j][cc], uu = st.u[j][cc], dy = st.gy[j][cc];
-            float dut = 0.f, dxt = 0.f, dBv[4], dCv[4];
+            const float2 xx = make_float2(x, x), uu2 = make_float2(uu, uu), dy2 = make_float2(dy, dy);
+            const float4 Bv = *reinterpret_cast<const float4*>(&st.B[j][4 * grp]);
+            const float4 Cv = *reinterpret_cast<const float4*>(&st.C[j][4 * grp]);
+            const float2 Bp[2] = {make_float2(Bv.x, Bv.y), make_float2(Bv.z, Bv.w)};
+            const float2 Cp[2] = {make_float2(Cv.x, Cv.y), make_float2(Cv.z, Cv.w)};
+            float2 dut2 = make_float2(0.f, 0.f), dxt2 = make_float2(0.f, 0.f), dB2[2], dC2[2];
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const float Bn = st.B[j][4 * grp + s], Cn = st.C[j][4 * grp + s];
-                const float a = fast_exp2(x * a2[s]);
-                gs[s] = fmaf(Cn, dy, gs[s]);
-                dCv[s] = dy * hs[j + 1][s];
-                dBv[s] = gs[s] * x * uu;
-                dut = fmaf(gs[s] * x, Bn, dut);
-                dxt = fmaf(gs[s], fmaf(An[s] * a, hs[j][s], Bn * uu), dxt);
-                dAs[s] = fmaf(gs[s] * x * a, hs[j][s], dAs[s]);
-                gs[s] *= a;
+            for (int q = 0; q < 2; ++q) {
+                const float2 xa = __fmul2_rn(xx, a2[q]);
+                const float2 a = make_float2(fast_exp2(xa.x), fast_exp2(xa.y));
+                gs[q] = __ffma2_rn(Cp[q], dy2, gs[q]);                   // g += C dy
+                dC2[q] = __fmul2_rn(dy2, hs[j + 1][q]);                  // dC = dy h
+                const float2 gx = __fmul2_rn(gs[q], xx);
+                dB2[q] = __fmul2_rn(gx, uu2);                             // dB = g x u
+                dut2 = __ffma2_rn(gx, Bp[q], dut2);                       // du += g x B
+                const float2 t = __ffma2_rn(__fmul2_rn(An[q], a), hs[j][q], __fmul2_rn(Bp[q], uu2));
+                dxt2 = __ffma2_rn(gs[q], t, dxt2);                        // dx += g (A a h' + B u)
+                dAs[q] = __ffma2_rn(__fmul2_rn(gx, a), hs[j][q], dAs[q]); // dA += g x a h'
+                gs[q] = __fmul2_rn(gs[q], a);                             // carried to step j - 1
             }
+            float dut = dut2.x + dut2.y, dxt = dxt2.x + dxt2.y;
+            const float dBv[4] = {dB2[0].x, dB2[0].y, dB2[1].x, dB2[1].y};
+            const float dCv[4] = {dC2[0].x, dC2[0].y, dC2[1].x, dC2[1].y};
             // sums over the four state groups of a channel (u, Delta)
             dut += __shfl_xor_sync(FULL_MASK, dut, 1);
             dut += __shfl_xor_sync(FULL_MASK, dut, 2);
@@ -536,7 +561,8 @@ __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
             const int n = 4 * grp + s;
-            if (n < N && p.dA) atomicAdd(p.dA + (long long)k * p.a_dir + (long long)d * N + n, dAs[s]);
+            const float v = (s & 1) ? dAs[s >> 1].y : dAs[s >> 1].x;
+            if (n < N && p.dA) atomicAdd(p.dA + (long long)k * p.a_dir + (long long)d * N + n, v);
         }
         if (grp == 0) {
             if (p.dD) atomicAdd(p.dD + k * p.v_dir + d, dDs);
