@@ -187,8 +187,10 @@ inline size_t pool_scan_smem_bytes(int Ki, int Lp, bool conv = false)
     return sizeof(float) * (size_t)(Ki + Ku + 2) * Lp * PL_CH;
 }
 
+// Three CTAs per SM (80 registers) where shared memory allows them; two for the
+// convolution and the mask (128 registers), whose phase 1 holds more state.
 template <typename T, int FL>
-__global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams p)
+__global__ void __launch_bounds__(PL_THREADS, (FL & (FL_CONV | FL_MASK)) ? 2 : 3) pool_scan_kernel(const PoolParams p)
 {
     constexpr bool ZOH = (FL & FL_ZOH) != 0;
     constexpr bool CONV = (FL & FL_CONV) != 0;
@@ -472,38 +474,63 @@ __global__ void __launch_bounds__(PL_THREADS) pool_scan_kernel(const PoolParams 
         for (int s = 0; s < 4; ++s) ia[s] = (a2[s] != 0.f) ? LOG2E / a2[s] : 0.f;
         float* Yk = Y + (size_t)kd * Lp * PL_CH;
         float h[4] = {0.f, 0.f, 0.f, 0.f};
+        // B and C of the lane's four states as 16-byte quads (N = 16), else per state
+        const bool quad = N == 16;
         for (int t0 = 0; t0 < Lp; t0 += 4) {
-            float yp[4];
+            // the four steps' loads first (a step past the end re-reads step
+            // Lp - 1 and is not applied): the pooled B and C come from L2, and a
+            // load per step behind the previous step's update would cost one L2
+            // round trip per step
+            float xs[4], us[4];
+            float4 bq[4], cq[4];
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
-                const int t = t0 + jj;
-                float acc = 0.f;
-                if (t < Lp) {
-                    const int i = kd == 0 ? t : Lp - 1 - t;
-                    // Delta = softplus(mean raw Delta + bias): the bias and
-                    // softplus act on the pooled token.
-                    const float x = pdk[(size_t)i * PL_CH + c] + bias;
-                    const float dsp = p.softplus ? softplus_f(x) : x;
-                    const float du = dsp * puk[(size_t)i * PL_CH + c];
-                    float bv[4], cv[4];
+                const int t = min(t0 + jj, Lp - 1);
+                const int i = kd == 0 ? t : Lp - 1 - t;
+                xs[jj] = pdk[(size_t)i * PL_CH + c];
+                us[jj] = puk[(size_t)i * PL_CH + c];
+                if (quad) {
+                    bq[jj] = __ldg(reinterpret_cast<const float4*>(pBk + (size_t)i * 16 + 4 * grp));
+                    cq[jj] = __ldg(reinterpret_cast<const float4*>(pCk + (size_t)i * 16 + 4 * grp));
+                } else {
+                    float bb[4], cc4[4];
 #pragma unroll
                     for (int s = 0; s < 4; ++s) {
                         const int n = 4 * grp + s;
-                        bv[s] = n < N ? __ldg(pBk + (size_t)i * N + n) : 0.f;
-                        cv[s] = n < N ? __ldg(pCk + (size_t)i * N + n) : 0.f;
-                        if constexpr (MASK) { bv[s] *= inv_cnt; cv[s] *= inv_cnt; }  // sums -> means
+                        bb[s] = n < N ? __ldg(pBk + (size_t)i * N + n) : 0.f;
+                        cc4[s] = n < N ? __ldg(pCk + (size_t)i * N + n) : 0.f;
                     }
-                    const float rd = ZOH ? fast_rcp(dsp) : 0.f;
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        const float e = fast_exp2(dsp * a2[s]);
-                        float w = du * bv[s];
-                        if constexpr (ZOH) w *= zoh_phi(dsp * a2[s] * LN2, e, rd * ia[s]);
-                        h[s] = fmaf(e, h[s], w);
-                        acc = fmaf(cv[s], h[s], acc);
-                    }
+                    bq[jj] = make_float4(bb[0], bb[1], bb[2], bb[3]);
+                    cq[jj] = make_float4(cc4[0], cc4[1], cc4[2], cc4[3]);
                 }
-                yp[jj] = acc;
+            }
+            float yp[4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const bool live = t0 + jj < Lp;
+                // Delta = softplus(mean raw Delta + bias): the bias and
+                // softplus act on the pooled token.
+                const float x = xs[jj] + bias;
+                const float dsp = p.softplus ? softplus_f(x) : x;
+                const float du = dsp * us[jj];
+                float bv[4] = {bq[jj].x, bq[jj].y, bq[jj].z, bq[jj].w};
+                float cv[4] = {cq[jj].x, cq[jj].y, cq[jj].z, cq[jj].w};
+                if constexpr (MASK) {
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) { bv[s] *= inv_cnt; cv[s] *= inv_cnt; }  // sums -> means
+                }
+                const float rd = ZOH ? fast_rcp(dsp) : 0.f;
+                float acc = 0.f;
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const float e = fast_exp2(dsp * a2[s]);
+                    float w = du * bv[s];
+                    if constexpr (ZOH) w *= zoh_phi(dsp * a2[s] * LN2, e, rd * ia[s]);
+                    const float hn = fmaf(e, h[s], w);
+                    h[s] = live ? hn : h[s];
+                    acc = fmaf(cv[s], h[s], acc);
+                }
+                yp[jj] = live ? acc : 0.f;
             }
             const bool hi = grp & 2;
             float x0 = hi ? yp[2] : yp[0];
