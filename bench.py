@@ -433,7 +433,7 @@ def run_ours(args, wls):
             host["pos"] = torch.from_numpy(x["pos"])
         host_sets.append(host)
         pd = dict(per_dir_inputs=wl.per_dir, per_dir_params=wl.per_dir)
-        ws_bytes = vs.workspace_size(route, host["u"], host["B"], **pd)
+        ws_bytes = vs.workspace_size(route, host["u"], host["B"], token_pos=host.get("pos"), **pd)
         per = []
         for r in range(rot):
             d = {k: v.to(dev) for k, v in host.items()}

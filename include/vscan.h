@@ -121,10 +121,12 @@ typedef enum vscan_flag {
 typedef struct vscan_route vscan_route;
 
 /*
- * Arguments of one forward pass. All tensors are dense, row-major, with the
- * channel (or state) axis contiguous. "tokens" is the route's token count per
- * image (vscan_route_info), Ki = K if per_dir_inputs else 1, Kp = K if
- * per_dir_params else 1.
+ * Arguments of one forward pass. All tensors are row-major with the channel
+ * (or state) axis contiguous; u, delta, z and y may step between tokens and
+ * images by tok_stride and batch_stride elements, B and C by bc_tok_stride and
+ * bc_batch_stride (0 = dense). "tokens" is the route's token count per image
+ * (vscan_route_info), Ki = K if per_dir_inputs else 1, Kp = K if
+ * per_dir_params else 1. The shapes below are the dense case.
  */
 typedef struct vscan_args {
     int32_t batch;          /* images, >= 0 (0 = nothing to do)                      */
@@ -192,6 +194,22 @@ typedef struct vscan_args {
                                The caller zeroes it, synchronizes the stream and
                                decodes it with vscan_status_from_device_word.
                                Required with VSCAN_FLAG_CHECK_VALUES.             */
+    /* Strides in elements (0 = dense). Token t of image b of direction plane k
+     * of u and delta sits at (k * batch + b) * batch_stride + t * tok_stride;
+     * z and y use the same strides with k = 0; B and C use the bc_ strides.
+     * tok_stride >= channels, a multiple of 4 (f32) or 8 (bf16);
+     * batch_stride >= tokens * tok_stride, the same multiple; bc_tok_stride >=
+     * d_state; bc_batch_stride >= tokens * bc_tok_stride. Strided tensors are
+     * packed into the workspace by a copy kernel before the scan (y: written
+     * there and copied out after it), one more read and write of each: an
+     * addition of this library for callers holding views of larger buffers
+     * (the pages' tensors are dense). vscan_forward only; vscan_forward_host,
+     * vscan_backward and vscan_forward_pooled_noalloc return
+     * VSCAN_ERR_UNSUPPORTED for non-dense strides.                          */
+    int64_t tok_stride;
+    int64_t batch_stride;
+    int64_t bc_tok_stride;
+    int64_t bc_batch_stride;
 } vscan_args;
 
 /*
@@ -382,7 +400,7 @@ const char* vscan_last_error(void);
 const char* vscan_status_string(int32_t status);
 
 /* Library ABI version; changes whenever vscan_args changes layout (2: flags,
- * conv_w and conv_b; 3: token_pos and n_tokens; 4: status). */
+ * conv_w and conv_b; 3: token_pos and n_tokens; 4: status; 5: strides). */
 int32_t vscan_abi_version(void);
 
 #ifdef __cplusplus

@@ -10,6 +10,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from conftest import ROOT, read_golden
 
@@ -37,12 +38,14 @@ def test_library_exports_every_declared_function():
 
 def test_struct_layout_matches_the_header():
     # int32 x4, 6 pointers, 3 pointers, int32 x3, float, pointer, uint64, int32 x2, 3 pointers, int32 x2,
-    # pointer
-    assert ctypes.sizeof(abi.VscanArgs) == 16 + 48 + 24 + 12 + 4 + 8 + 8 + 8 + 24 + 8 + 8
+    # pointer, int64 x4
+    assert ctypes.sizeof(abi.VscanArgs) == 16 + 48 + 24 + 12 + 4 + 8 + 8 + 8 + 24 + 8 + 8 + 32
     assert abi.VscanArgs.flags.offset == 124 and abi.VscanArgs.conv_w.offset == 128
     assert abi.VscanArgs.token_pos.offset == 144 and abi.VscanArgs.n_tokens.offset == 152
     assert abi.VscanArgs.status.offset == 160
-    assert abi.lib.vscan_abi_version() == abi.ABI_VERSION == 4
+    assert (abi.VscanArgs.tok_stride.offset, abi.VscanArgs.batch_stride.offset,
+            abi.VscanArgs.bc_tok_stride.offset, abi.VscanArgs.bc_batch_stride.offset) == (168, 176, 184, 192)
+    assert abi.lib.vscan_abi_version() == abi.ABI_VERSION == 5
 
 
 def test_status_strings():
@@ -308,3 +311,75 @@ def test_backward_argument_checks_run_before_any_cuda_call():
     g.dz = None  # workspace missing
     assert abi.lib.vscan_backward(r.handle, ctypes.byref(_args(**fake)), ctypes.c_void_p(0x8000),
                                   ctypes.byref(g), None) == -6
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("tok_stride", -4, -1), ("tok_stride", 8, -3), ("tok_stride", 18, -3), ("batch_stride", 16, -3),
+    ("batch_stride", 17 * 16 + 2, -3), ("bc_tok_stride", 8, -1), ("bc_batch_stride", 16, -1)])
+def test_stride_checks(field, value, status):
+    r = vs.Route("bidir", 4, 4, 8)  # 17 tokens; channels 16, d_state 16, float32 (multiples of 4)
+    n = ctypes.c_uint64()
+    assert abi.lib.vscan_workspace_size(r.handle, ctypes.byref(_args(**{field: value})), ctypes.byref(n)) == status
+
+
+def test_workspace_counts_packed_copies():
+    r = vs.Route("bidir", 4, 4, 8)
+    r256 = lambda x: (x + 255) // 256 * 256
+    path = r256(2 * 2 * 17 * 16 * 4)          # parking planes: K x batch x tokens x D float32
+    plane = r256(2 * 17 * 16 * 4)             # one packed batch x tokens x 16 float32 tensor
+    n = ctypes.c_uint64()
+
+    def ws(**kw):
+        assert abi.lib.vscan_workspace_size(r.handle, ctypes.byref(_args(**kw)), ctypes.byref(n)) == 0
+        return n.value
+    assert ws() == path
+    assert ws(tok_stride=16, batch_stride=17 * 16, bc_tok_stride=16, bc_batch_stride=17 * 16) == path  # dense
+    assert ws(tok_stride=32) == path + 3 * plane             # u, delta, y
+    assert ws(tok_stride=32, z=0x7000) == path + 4 * plane   # and z
+    assert ws(batch_stride=18 * 16) == path + 3 * plane      # padding between images only
+    assert ws(bc_tok_stride=20) == path + 2 * plane          # B, C
+    assert ws(tok_stride=32, bc_batch_stride=20 * 16) == path + 5 * plane
+
+
+def test_plan_info_counts_pack_launches():
+    r = vs.Route("bidir", 64, 64, 2048)
+    n = ctypes.c_int32()
+
+    def launches(**kw):
+        assert abi.lib.vscan_plan_info(r.handle, ctypes.byref(_args(seq_chunks=1, **kw)), ctypes.byref(n)) == 0
+        return n.value
+    assert launches() == 1
+    assert launches(tok_stride=32) == 4                 # pack u, delta; scan; copy y out
+    assert launches(tok_stride=32, z=0x7000) == 5
+    assert launches(bc_tok_stride=32) == 3
+    assert launches(tok_stride=32, bc_tok_stride=32) == 6
+
+
+def test_dense_only_entry_points_reject_strides():
+    fake = dict(u=0x1000, delta=0x2000, B=0x3000, C=0x4000, y=0x5000, A=0x6000)
+    n = ctypes.c_uint64()
+    for route in ("bidir", "pool_w"):
+        r = vs.Route(route, 4, 4, 8 if route == "bidir" else -1)
+        for kw in (dict(tok_stride=32), dict(bc_batch_stride=32 * 16)):
+            a = _args(**fake, **kw)
+            assert abi.lib.vscan_host_buffer_size(r.handle, ctypes.byref(a), ctypes.byref(n)) == -4
+            assert "dense" in abi.lib.vscan_last_error().decode()
+            assert abi.lib.vscan_backward_workspace_size(r.handle, ctypes.byref(a), ctypes.byref(n)) == -4
+            if route == "pool_w":
+                assert abi.lib.vscan_forward_pooled_noalloc(r.handle, ctypes.byref(a), None) == -4
+
+
+def test_binding_reads_strides_from_views():
+    u = torch.zeros(3, 17, 24)[:, :, :16]
+    B = torch.zeros(3, 20, 18)[:, :17, :16]
+    assert vs._layout(u, False) == (24, 17 * 24)
+    assert vs._strides(u, u, None, u, B, B, False) == (24, 17 * 24, 18, 20 * 18)
+    dense = torch.zeros(3, 17, 16)
+    with pytest.raises(ValueError, match="delta"):
+        vs._strides(u, dense, None, u, B, B, False)
+    with pytest.raises(ValueError, match="contiguous"):
+        vs._layout(torch.zeros(3, 17, 16).transpose(1, 2), False)
+    planes = torch.zeros(2, 3, 18, 16)[:, :, :17, :]      # per-direction planes, batch x image stride apart
+    assert vs._layout(planes, True) == (16, 18 * 16)
+    with pytest.raises(ValueError, match="planes"):
+        vs._layout(torch.zeros(2, 4, 17, 16)[:, :3], True)

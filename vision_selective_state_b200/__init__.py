@@ -90,11 +90,35 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _layout(t, per_dir):
+    """(token stride, image stride) in elements of a [(K,) batch, tokens, rows] tensor whose
+    last axis is contiguous; with a direction axis its planes must follow one another."""
+    if t.dim() < 3 or (t.stride(-1) != 1 and t.shape[-1] > 1):
+        raise ValueError("the channel (state) axis must be contiguous")
+    # a size-1 axis has no meaningful stride: take the dense value
+    ts = t.stride(-2) if t.shape[-2] > 1 else t.shape[-1]
+    bs = t.stride(-3) if t.shape[-3] > 1 else t.shape[-2] * ts
+    if per_dir and t.shape[0] > 1 and t.stride(0) != t.shape[1] * bs:
+        raise ValueError("direction planes must be spaced batch x image stride apart")
+    return ts, bs
+
+
+def _strides(u, delta, z, y, B, C, per_dir_inputs):
+    """The ABI's strides: one layout for u, delta, z, y and one for B, C."""
+    ts, bs = _layout(u, per_dir_inputs)
+    for name, t, pd in (("delta", delta, per_dir_inputs), ("z", z, False), ("y", y, False)):
+        if t is not None and _layout(t, pd) != (ts, bs):
+            raise ValueError(f"{name} must have u's token and image strides {(ts, bs)}")
+    bts, bbs = _layout(B, per_dir_inputs)
+    if _layout(C, per_dir_inputs) != (bts, bbs):
+        raise ValueError(f"C must have B's token and image strides {(bts, bbs)}")
+    return ts, bs, bts, bbs
+
+
 def _args(route, u, delta, A, B, C, Dskip, delta_bias, z, y, delta_softplus, merge_scale,
           per_dir_inputs, per_dir_params, workspace, seq_chunks, conv_w=None, conv_b=None,
           zoh=False, token_pos=None, status=None, check_values=False):
-    for name, t in (("u", u), ("delta", delta), ("B", B), ("C", C), ("z", z), ("y", y),
-                    ("A", A), ("Dskip", Dskip), ("delta_bias", delta_bias), ("conv_w", conv_w),
+    for name, t in (("A", A), ("Dskip", Dskip), ("delta_bias", delta_bias), ("conv_w", conv_w),
                     ("conv_b", conv_b)):
         if t is not None and not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
@@ -134,11 +158,15 @@ def _args(route, u, delta, A, B, C, Dskip, delta_bias, z, y, delta_softplus, mer
     a.conv_w, a.conv_b = _ptr(conv_w), _ptr(conv_b)
     a.token_pos = _ptr(token_pos)
     a.n_tokens = tokens if token_pos is not None else 0
+    a.tok_stride, a.batch_stride, a.bc_tok_stride, a.bc_batch_stride = _strides(u, delta, z, y, B, C,
+                                                                                per_dir_inputs)
     return a
 
 
-def workspace_size(route, u, B, *, per_dir_inputs=False, per_dir_params=False, **_):
-    """Bytes of device scratch vscan_forward needs (host-only query)."""
+def workspace_size(route, u, B, *, per_dir_inputs=False, per_dir_params=False, z=None, token_pos=None, **_):
+    """Bytes of device scratch vscan_forward needs (host-only query); u's and B's strides
+    (and whether z is given) count when the tensors are not dense, and a masked token set
+    (token_pos) sets the tokens per image."""
     lead = 1 if per_dir_inputs else 0
     a = VscanArgs()
     a.batch, _, a.channels = u.shape[lead:]
@@ -146,6 +174,12 @@ def workspace_size(route, u, B, *, per_dir_inputs=False, per_dir_params=False, *
     a.dtype = _dtype_code(u)
     a.per_dir_inputs, a.per_dir_params = int(bool(per_dir_inputs)), int(bool(per_dir_params))
     a.delta_softplus, a.merge_scale = 1, 1.0
+    a.z = ctypes.c_void_p(1) if z is not None else None  # only nullness matters here
+    if token_pos is not None:
+        a.token_pos = ctypes.c_void_p(1)
+        a.n_tokens = u.shape[lead + 1]
+    a.tok_stride, a.batch_stride = _layout(u, per_dir_inputs)
+    a.bc_tok_stride, a.bc_batch_stride = _layout(B, per_dir_inputs)
     n = ctypes.c_uint64()
     check(lib.vscan_workspace_size(route.handle, ctypes.byref(a), ctypes.byref(n)))
     return n.value
@@ -163,12 +197,14 @@ def forward(route, u, delta, A, B, C, Dskip=None, delta_bias=None, z=None, *, de
     non-finite values, A > 0, and (delta_softplus=False) a negative time scale.
     """
     lead = 1 if per_dir_inputs else 0
-    if out is None:
-        out = torch.empty(u.shape[lead:], dtype=u.dtype, device=u.device)
+    if out is None:  # in u's layout (the ABI has one layout for u, delta, z and y)
+        ts, bs = _layout(u, per_dir_inputs)
+        out = torch.empty_strided(u.shape[lead:], (bs, ts, 1), dtype=u.dtype, device=u.device)
     if token_pos is not None and token_pos.shape[-1] == 0:
         return out  # an empty token set: nothing to compute (and no data pointers to pass)
     if workspace is None:
-        need = workspace_size(route, u, B, per_dir_inputs=per_dir_inputs, per_dir_params=per_dir_params)
+        need = workspace_size(route, u, B, per_dir_inputs=per_dir_inputs, per_dir_params=per_dir_params, z=z,
+                              token_pos=token_pos)
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=u.device)
     a = _args(route, u, delta, A, B, C, Dskip, delta_bias, z, out, delta_softplus, merge_scale,
               per_dir_inputs, per_dir_params, workspace, seq_chunks, conv_w, conv_b, zoh, token_pos,

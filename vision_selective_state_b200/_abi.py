@@ -23,7 +23,7 @@ STATUS = {
 }
 ROUTES = {"bidir": 0, "cross4": 1, "atrous2": 2, "pool_w": 3, "pool_h": 4}
 F32, BF16 = 0, 1
-ABI_VERSION = 4
+ABI_VERSION = 5
 FLAG_ZOH = 1
 FLAG_CHECK_VALUES = 2
 
@@ -59,6 +59,10 @@ class VscanArgs(ctypes.Structure):
         ("n_tokens", ctypes.c_int32),
         ("reserved2", ctypes.c_int32),
         ("status", ctypes.c_void_p),
+        ("tok_stride", ctypes.c_int64),
+        ("batch_stride", ctypes.c_int64),
+        ("bc_tok_stride", ctypes.c_int64),
+        ("bc_batch_stride", ctypes.c_int64),
     ]
 
 

@@ -16,6 +16,7 @@
 #include "vscan.h"
 #include "vscan_backward.cuh"
 #include "vscan_check.cuh"
+#include "vscan_layout.cuh"
 #include "vscan_pipe.cuh"
 #include "vscan_pool.cuh"
 #include "vscan_resident.cuh"
@@ -28,7 +29,7 @@ struct vscan_route {
 
 namespace {
 
-constexpr int32_t kAbiVersion = 4;
+constexpr int32_t kAbiVersion = 5;
 constexpr int32_t kKnownFlags = VSCAN_FLAG_ZOH | VSCAN_FLAG_CHECK_VALUES;
 constexpr size_t kMaxSmem = 200 * 1024;  // dynamic shared memory the kernels may ask for
 thread_local std::string g_last_error;
@@ -60,6 +61,28 @@ bool is_pool(int kind) { return kind == vscan::RK_POOL_W || kind == vscan::RK_PO
 // Tokens per image in the token arrays: the visible ones of a masked set, else
 // the route's (grid, plus CLS for BIDIR).
 int tokens_of(const vscan_route* r, const vscan_args* a) { return a->token_pos ? a->n_tokens : r->g.tokens; }
+
+// Strides of the token arrays in elements, with 0 resolved to the dense value.
+long long tok_stride_of(const vscan_args* a) { return a->tok_stride ? a->tok_stride : a->channels; }
+long long batch_stride_of(const vscan_route* r, const vscan_args* a)
+{
+    return a->batch_stride ? a->batch_stride : (long long)tokens_of(r, a) * tok_stride_of(a);
+}
+long long bc_tok_stride_of(const vscan_args* a) { return a->bc_tok_stride ? a->bc_tok_stride : a->d_state; }
+long long bc_batch_stride_of(const vscan_route* r, const vscan_args* a)
+{
+    return a->bc_batch_stride ? a->bc_batch_stride : (long long)tokens_of(r, a) * bc_tok_stride_of(a);
+}
+// u, delta, z, y (main) or B, C not laid out densely
+bool strided_main(const vscan_route* r, const vscan_args* a)
+{
+    return tok_stride_of(a) != a->channels || batch_stride_of(r, a) != (long long)tokens_of(r, a) * a->channels;
+}
+bool strided_bc(const vscan_route* r, const vscan_args* a)
+{
+    return bc_tok_stride_of(a) != a->d_state ||
+           bc_batch_stride_of(r, a) != (long long)tokens_of(r, a) * a->d_state;
+}
 
 size_t resident_bytes(const vscan_route* r, const vscan_args* a)
 {
@@ -114,6 +137,19 @@ vscan_status check_shape(const vscan_route* r, const vscan_args* a)
     if (a->batch > 65535) return fail(VSCAN_ERR_UNSUPPORTED, "batch %d > 65535", a->batch);
     if ((long long)tokens_of(r, a) * a->channels >= (1LL << 31))
         return fail(VSCAN_ERR_UNSUPPORTED, "tokens x channels of one image must be below 2^31");
+    if (a->tok_stride < 0 || a->batch_stride < 0 || a->bc_tok_stride < 0 || a->bc_batch_stride < 0)
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "strides must be >= 0 (0 = dense)");
+    if (tok_stride_of(a) < a->channels || tok_stride_of(a) % vec != 0)
+        return fail(VSCAN_ERR_ALIGNMENT, "tok_stride %lld must be >= channels and a multiple of %d",
+                    (long long)a->tok_stride, vec);
+    if (batch_stride_of(r, a) < (long long)tokens_of(r, a) * tok_stride_of(a) || batch_stride_of(r, a) % vec != 0)
+        return fail(VSCAN_ERR_ALIGNMENT, "batch_stride %lld must be >= tokens x tok_stride and a multiple of %d",
+                    (long long)a->batch_stride, vec);
+    if (bc_tok_stride_of(a) < a->d_state)
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "bc_tok_stride %lld < d_state", (long long)a->bc_tok_stride);
+    if (bc_batch_stride_of(r, a) < (long long)tokens_of(r, a) * bc_tok_stride_of(a))
+        return fail(VSCAN_ERR_INVALID_ARGUMENT, "bc_batch_stride %lld < tokens x bc_tok_stride",
+                    (long long)a->bc_batch_stride);
     if (is_pool(r->g.kind)) {
         const int Ki = a->per_dir_inputs ? 2 : 1;
         if (vscan::pool_scan_smem_bytes(Ki, r->g.L, a->conv_w != nullptr) > kMaxSmem)
@@ -514,9 +550,91 @@ vscan_status launch_value_checks(const vscan_route* r, const vscan_args* a, cuda
     return VSCAN_OK;
 }
 
+// Packed copies of strided tensors, placed in the workspace after the path's
+// own scratch (offsets from its start; main: u, delta, z and y are packed; bc:
+// B and C are).
+struct PackLayout {
+    bool main, bc;
+    uint64_t u, d, z, y, B, C, total;
+};
+
+uint64_t pack_layout(const vscan_route* r, const vscan_args* a, PackLayout* L)
+{
+    *L = PackLayout{};
+    const bool mn = strided_main(r, a), bc = strided_bc(r, a);
+    if (!mn && !bc) return 0;
+    const int Ki = a->per_dir_inputs ? r->g.K : 1;
+    const uint64_t eb = a->dtype == VSCAN_F32 ? 4 : 2;
+    const uint64_t plane = (uint64_t)a->batch * tokens_of(r, a);
+    uint64_t off = round256(workspace_need(r, a));
+    auto take = [&](uint64_t bytes) { const uint64_t o = off; off += round256(bytes); return o; };
+    L->main = mn;
+    L->bc = bc;
+    if (mn) {
+        L->u = take(Ki * plane * a->channels * eb);
+        L->d = take(Ki * plane * a->channels * eb);
+        if (a->z) L->z = take(plane * a->channels * eb);
+        L->y = take(plane * a->channels * eb);
+    }
+    if (bc) {
+        L->B = take(Ki * plane * a->d_state * eb);
+        L->C = take(Ki * plane * a->d_state * eb);
+    }
+    L->total = off;
+    return off;
+}
+
+// Workspace bytes vscan_forward needs: the path's scratch, plus the packed copies
+// of strided tensors.
+uint64_t forward_workspace_need(const vscan_route* r, const vscan_args* a)
+{
+    PackLayout L;
+    const uint64_t packed = pack_layout(r, a, &L);
+    return packed ? packed : workspace_need(r, a);
+}
+
+// Copy nimg images of ntok rows of `row` elements between strided layouts (strides
+// in elements of size eb); 16-byte pieces where rows, strides and both bases allow.
+vscan_status copy_rows(const void* src, long long s_img, long long s_tok, void* dst, long long d_img,
+                       long long d_tok, int nimg, int ntok, int row, int eb, cudaStream_t s)
+{
+    if (nimg == 0 || ntok == 0) return VSCAN_OK;
+    const long long bytes = (long long)row * eb;
+    const bool v16 = bytes % 16 == 0 && (s_img * eb) % 16 == 0 && (s_tok * eb) % 16 == 0 &&
+                     (d_img * eb) % 16 == 0 && (d_tok * eb) % 16 == 0 && aligned16(src) && aligned16(dst);
+    const dim3 grid((unsigned)std::min(1024, (ntok + 7) / 8), (unsigned)std::min(nimg, 65535));
+    if (v16) {
+        const long long k = 16 / eb;
+        vscan::copy_rows_kernel<uint4><<<grid, 256, 0, s>>>(static_cast<const uint4*>(src), s_img / k, s_tok / k,
+                                                            static_cast<uint4*>(dst), d_img / k, d_tok / k, nimg,
+                                                            ntok, (int)(bytes / 16));
+    } else if (eb == 4) {
+        vscan::copy_rows_kernel<uint32_t><<<grid, 256, 0, s>>>(static_cast<const uint32_t*>(src), s_img, s_tok,
+                                                               static_cast<uint32_t*>(dst), d_img, d_tok, nimg,
+                                                               ntok, row);
+    } else {
+        vscan::copy_rows_kernel<uint16_t><<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(src), s_img, s_tok,
+                                                               static_cast<uint16_t*>(dst), d_img, d_tok, nimg,
+                                                               ntok, row);
+    }
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? VSCAN_OK : cuda_fail(e, "launching copy_rows_kernel");
+}
+
+vscan_status forward_dense(const vscan_route* r, const vscan_args* a, cudaStream_t s, float* ckpt)
+{
+    if (a->flags & VSCAN_FLAG_CHECK_VALUES) {
+        const vscan_status st = launch_value_checks(r, a, s);
+        if (st != VSCAN_OK) return st;
+    }
+    return a->dtype == VSCAN_F32 ? dispatch<float>(r, a, s, ckpt) : dispatch<__nv_bfloat16>(r, a, s, ckpt);
+}
+
 vscan_status forward_device(const vscan_route* r, const vscan_args* a, cudaStream_t s, float* ckpt = nullptr)
 {
-    const uint64_t need = workspace_need(r, a);
+    PackLayout L;
+    const uint64_t packed = pack_layout(r, a, &L);
+    const uint64_t need = packed ? packed : workspace_need(r, a);
     if (need > 0) {
         if (!a->workspace || a->workspace_bytes < need)
             return fail(VSCAN_ERR_WORKSPACE, "workspace of %llu bytes needed, %llu given",
@@ -524,11 +642,46 @@ vscan_status forward_device(const vscan_route* r, const vscan_args* a, cudaStrea
         if (!aligned16(a->workspace)) return fail(VSCAN_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
     }
     if (a->batch == 0) return VSCAN_OK;
-    if (a->flags & VSCAN_FLAG_CHECK_VALUES) {
-        const vscan_status st = launch_value_checks(r, a, s);
-        if (st != VSCAN_OK) return st;
+    if (!packed) return forward_dense(r, a, s, ckpt);
+
+    // strided tensors: pack them densely, scan, copy y out
+    char* ws = static_cast<char*>(a->workspace);
+    vscan_args b = *a;
+    b.tok_stride = b.batch_stride = b.bc_tok_stride = b.bc_batch_stride = 0;
+    b.workspace_bytes = workspace_need(r, a);
+    const int Ki = a->per_dir_inputs ? r->g.K : 1, T = tokens_of(r, a), D = a->channels, N = a->d_state;
+    const int eb = a->dtype == VSCAN_F32 ? 4 : 2;
+    const long long ts = tok_stride_of(a), bs = batch_stride_of(r, a);
+    const long long bts = bc_tok_stride_of(a), bbs = bc_batch_stride_of(r, a);
+    vscan_status st = VSCAN_OK;
+    if (L.main) {
+        b.u = ws + L.u;
+        b.delta = ws + L.d;
+        st = copy_rows(a->u, bs, ts, ws + L.u, (long long)T * D, D, Ki * a->batch, T, D, eb, s);
+        if (st == VSCAN_OK) st = copy_rows(a->delta, bs, ts, ws + L.d, (long long)T * D, D, Ki * a->batch, T, D, eb, s);
+        if (st == VSCAN_OK && a->z) {
+            b.z = ws + L.z;
+            st = copy_rows(a->z, bs, ts, ws + L.z, (long long)T * D, D, a->batch, T, D, eb, s);
+        }
+        b.y = ws + L.y;
     }
-    return a->dtype == VSCAN_F32 ? dispatch<float>(r, a, s, ckpt) : dispatch<__nv_bfloat16>(r, a, s, ckpt);
+    if (st == VSCAN_OK && L.bc) {
+        b.B = ws + L.B;
+        b.C = ws + L.C;
+        st = copy_rows(a->B, bbs, bts, ws + L.B, (long long)T * N, N, Ki * a->batch, T, N, eb, s);
+        if (st == VSCAN_OK) st = copy_rows(a->C, bbs, bts, ws + L.C, (long long)T * N, N, Ki * a->batch, T, N, eb, s);
+    }
+    if (st == VSCAN_OK) st = forward_dense(r, &b, s, ckpt);
+    if (st == VSCAN_OK && L.main) st = copy_rows(ws + L.y, (long long)T * D, D, a->y, bs, ts, a->batch, T, D, eb, s);
+    return st;
+}
+
+// Entry points that take dense tensors only.
+vscan_status require_dense(const vscan_route* r, const vscan_args* a, const char* what)
+{
+    if (strided_main(r, a) || strided_bc(r, a))
+        return fail(VSCAN_ERR_UNSUPPORTED, "%s takes dense tensors only (strides 0 or the dense values)", what);
+    return VSCAN_OK;
 }
 
 int forward_flags(const vscan_args* a)
@@ -651,6 +804,8 @@ vscan_status check_backward(const vscan_route* r, const vscan_args* a)
     if (a->conv_w) return fail(VSCAN_ERR_UNSUPPORTED, "the backward pass does not take the fused convolution");
     if (a->flags & VSCAN_FLAG_ZOH) return fail(VSCAN_ERR_UNSUPPORTED, "the backward pass is for the Delta*B*u write term");
     if (a->token_pos) return fail(VSCAN_ERR_UNSUPPORTED, "the backward pass does not take a masked token set");
+    st = require_dense(r, a, "vscan_backward");
+    if (st != VSCAN_OK) return st;
     return VSCAN_OK;
 }
 
@@ -835,7 +990,7 @@ vscan_status vscan_workspace_size(const vscan_route* r, const vscan_args* a, uin
     if (!bytes) return fail(VSCAN_ERR_INVALID_ARGUMENT, "bytes is NULL");
     vscan_status st = check_shape(r, a);
     if (st != VSCAN_OK) return st;
-    *bytes = workspace_need(r, a);
+    *bytes = forward_workspace_need(r, a);
     return VSCAN_OK;
 }
 
@@ -853,8 +1008,13 @@ vscan_status vscan_plan_info(const vscan_route* r, const vscan_args* a, int32_t*
     if (!kernels) return fail(VSCAN_ERR_INVALID_ARGUMENT, "kernels is NULL");
     vscan_status st = check_shape(r, a);
     if (st != VSCAN_OK) return st;
-    if (a->batch == 0) *kernels = 0;
-    else *kernels = (is_pool(r->g.kind) ? 2 : 1) + ((a->flags & VSCAN_FLAG_CHECK_VALUES) ? 1 : 0);
+    if (a->batch == 0) {
+        *kernels = 0;
+    } else {
+        *kernels = (is_pool(r->g.kind) ? 2 : 1) + ((a->flags & VSCAN_FLAG_CHECK_VALUES) ? 1 : 0);
+        if (strided_main(r, a)) *kernels += 3 + (a->z ? 1 : 0);  // pack u, delta (z), copy y out
+        if (strided_bc(r, a)) *kernels += 2;                      // pack B, C
+    }
     return VSCAN_OK;
 }
 
@@ -882,6 +1042,8 @@ vscan_status vscan_host_buffer_size(const vscan_route* r, const vscan_args* a, u
     if (!bytes) return fail(VSCAN_ERR_INVALID_ARGUMENT, "bytes is NULL");
     vscan_status st = check_shape(r, a);
     if (st != VSCAN_OK) return st;
+    st = require_dense(r, a, "vscan_forward_host");
+    if (st != VSCAN_OK) return st;
     *bytes = host_layout(r, a).total;
     return VSCAN_OK;
 }
@@ -890,6 +1052,8 @@ vscan_status vscan_forward_host(const vscan_route* r, const vscan_args* ha, void
                                 uint64_t device_buffer_bytes, void* stream)
 {
     vscan_status st = check_shape(r, ha);
+    if (st != VSCAN_OK) return st;
+    st = require_dense(r, ha, "vscan_forward_host");
     if (st != VSCAN_OK) return st;
     st = check_pointers(ha, false);
     if (st != VSCAN_OK) return st;
@@ -988,6 +1152,8 @@ vscan_status vscan_backward(const vscan_route* r, const vscan_args* a, const voi
 vscan_status vscan_forward_pooled_noalloc(const vscan_route* r, const vscan_args* a, void* stream)
 {
     vscan_status st = check_shape(r, a);
+    if (st != VSCAN_OK) return st;
+    st = require_dense(r, a, "vscan_forward_pooled_noalloc");
     if (st != VSCAN_OK) return st;
     st = check_pointers(a, true);
     if (st != VSCAN_OK) return st;
