@@ -347,8 +347,9 @@ vscan_status vscan_forward_host(const vscan_route* route, const vscan_args* host
  * gradient is not wanted (its work is then skipped where possible).
  */
 typedef struct vscan_grads {
-    float* du;        /* device, [Ki][batch][tokens][D]                         */
-    float* ddelta;    /* device, [Ki][batch][tokens][D], w.r.t. the raw step     */
+    float* du;        /* device, [Ki][batch][tokens][D], 16-byte aligned        */
+    float* ddelta;    /* device, [Ki][batch][tokens][D], w.r.t. the raw step,
+                         16-byte aligned                                        */
     float* dB;        /* device, [Ki][batch][tokens][N]                         */
     float* dC;        /* device, [Ki][batch][tokens][N]                         */
     float* dA;        /* device, [Kp][D][N]                                     */

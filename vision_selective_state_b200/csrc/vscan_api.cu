@@ -930,7 +930,9 @@ vscan_status backward_device(const vscan_route* r, const vscan_args* a, const vo
         p.dB = reinterpret_cast<float*>(ws + Lo.dpB);
         p.dC = reinterpret_cast<float*>(ws + Lo.dpC);
         launch_bwd_scan<vscan::RK_BIDIR, float>(p, grid, s);
-        vscan::bwd_unpool_kernel<<<dim3((unsigned)TK, (unsigned)b), 128, 0, s>>>(
+        // 8 token rows per CTA at a time, about 16 CTAs per SM over the batch
+        const unsigned ux = (unsigned)std::max(1LL, std::min<long long>((TK + 7) / 8, 16LL * 148 / std::max(1LL, (long long)b)));
+        vscan::bwd_unpool_kernel<<<dim3(ux, (unsigned)b), 256, 0, s>>>(
             g, (int)b, (int)D, (int)N, Ki, p.du, p.ddelta, p.dB, p.dC, gr->du, gr->ddelta, gr->dB, gr->dC);
     }
     cudaError_t e = cudaGetLastError();
@@ -1149,6 +1151,8 @@ vscan_status vscan_backward(const vscan_route* r, const vscan_args* a, const voi
     if (!dy) return fail(VSCAN_ERR_INVALID_ARGUMENT, "dy is NULL");
     if (!aligned16(dy)) return fail(VSCAN_ERR_ALIGNMENT, "dy is not 16-byte aligned");
     if (gr->dz && !a->z) return fail(VSCAN_ERR_INVALID_ARGUMENT, "dz requested without z");
+    if ((gr->du && !aligned16(gr->du)) || (gr->ddelta && !aligned16(gr->ddelta)))
+        return fail(VSCAN_ERR_ALIGNMENT, "du and ddelta must be 16-byte aligned");
     vscan_args chk = *a;
     chk.y = const_cast<void*>(dy);  // y is not used by the backward pass
     st = check_pointers(&chk, true);

@@ -153,25 +153,56 @@ __global__ void bwd_pool_kernel(RouteGeom g, int batch, int D, int N, int Ki, co
 }
 
 // Pooled routes: token gradients from the pooled ones (the mean's adjoint).
-// Grid (tokens, batch).
-__global__ void bwd_unpool_kernel(RouteGeom g, int batch, int D, int N, int Ki, const float* dpu,
-                                  const float* dpraw, const float* dpB, const float* dpC, float* du,
-                                  float* ddelta, float* dB, float* dC)
+// Grid (x, batch), 8 warps per CTA: each warp writes whole token rows (u and
+// raw Delta gradients in 16-byte pieces, D a multiple of 4), striding over the
+// image's tokens, so the stores stream at full width.
+__global__ void __launch_bounds__(256) bwd_unpool_kernel(RouteGeom g, int batch, int D, int N, int Ki,
+                                                         const float* dpu, const float* dpraw, const float* dpB,
+                                                         const float* dpC, float* du, float* ddelta, float* dB,
+                                                         float* dC)
 {
-    const int tok = blockIdx.x, b = blockIdx.y, Lp = g.L;
-    const int r = tok / g.w, c = tok - r * g.w;
-    const int i = (g.kind == RK_POOL_W) ? r : c;
+    const int b = blockIdx.y, Lp = g.L, lane = threadIdx.x & 31;
+    const int nw = gridDim.x * (blockDim.x >> 5);
     const float inv = 1.0f / (float)((g.kind == RK_POOL_W) ? g.w : g.h);
-    for (int k = 0; k < Ki; ++k) {
-        const long long to = ((long long)k * batch + b) * g.tokens + tok;
-        const long long po = ((long long)k * batch + b) * Lp + i;
-        for (int d = threadIdx.x; d < D; d += blockDim.x) {
-            if (du) du[to * D + d] = dpu[po * D + d] * inv;
-            if (ddelta) ddelta[to * D + d] = dpraw[po * D + d] * inv;
+    const int Q = D / 4;
+    constexpr int U = 2;  // token rows per warp per round, loads first
+    for (int t0 = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t0 < g.tokens; t0 += U * nw) {
+        int tk[U], ix[U];
+#pragma unroll
+        for (int v = 0; v < U; ++v) {
+            tk[v] = t0 + v * nw;
+            const int r = tk[v] / g.w, c = tk[v] - r * g.w;
+            ix[v] = tk[v] < g.tokens ? ((g.kind == RK_POOL_W) ? r : c) : -1;
         }
-        for (int n = threadIdx.x; n < N; n += blockDim.x) {
-            if (dB) dB[to * N + n] = dpB[po * N + n] * inv;
-            if (dC) dC[to * N + n] = dpC[po * N + n] * inv;
+        for (int k = 0; k < Ki; ++k) {
+            for (int q = lane; q < Q; q += 32) {
+                float4 vu[U], vd[U];
+#pragma unroll
+                for (int v = 0; v < U; ++v) {
+                    const long long po = (((long long)k * batch + b) * Lp + max(ix[v], 0)) * D + 4 * q;
+                    vu[v] = du ? *reinterpret_cast<const float4*>(dpu + po) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    vd[v] = ddelta ? *reinterpret_cast<const float4*>(dpraw + po) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int v = 0; v < U; ++v) {
+                    if (ix[v] < 0) continue;
+                    const long long to = (((long long)k * batch + b) * g.tokens + tk[v]) * D + 4 * q;
+                    if (du) *reinterpret_cast<float4*>(du + to) = make_float4(vu[v].x * inv, vu[v].y * inv, vu[v].z * inv, vu[v].w * inv);
+                    if (ddelta)
+                        *reinterpret_cast<float4*>(ddelta + to) =
+                            make_float4(vd[v].x * inv, vd[v].y * inv, vd[v].z * inv, vd[v].w * inv);
+                }
+            }
+            if (lane < N) {
+#pragma unroll
+                for (int v = 0; v < U; ++v) {
+                    if (ix[v] < 0) continue;
+                    const long long to = ((long long)k * batch + b) * g.tokens + tk[v];
+                    const long long po = ((long long)k * batch + b) * Lp + ix[v];
+                    if (dB) dB[to * N + lane] = dpB[po * N + lane] * inv;
+                    if (dC) dC[to * N + lane] = dpC[po * N + lane] * inv;
+                }
+            }
         }
     }
 }
