@@ -111,6 +111,14 @@ def test_zoh_all_routes(route, dtype, h, w):
     _case(route, h, w, D, dtype, zoh=True, seq_chunks=1 if route in ("cross4", "atrous2", "bidir") else 0)
 
 
+@pytest.mark.parametrize("zoh,conv", [(True, False), (False, True), (True, True)])
+def test_resident_wide_tile_with_optional_steps(zoh, conv):
+    """The 8-channel BIDIR resident tile (1188 channels, 149 tiles at batch 1) with the
+    zero-order-hold term and the fused convolution."""
+    _case("bidir", 7, 6, 1188, "f32", zoh=zoh, conv=conv, batch=1, seq_chunks=8)
+    _case("bidir", 7, 6, 1188, "f32", zoh=zoh, conv=conv, batch=2, seq_chunks=4, pdi=True, pdp=True)
+
+
 @pytest.mark.parametrize("route", ["bidir", "cross4", "atrous2"])
 @pytest.mark.parametrize("seq_chunks", [2, 8])
 def test_zoh_resident(route, seq_chunks):

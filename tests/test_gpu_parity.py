@@ -81,6 +81,20 @@ def test_resident_chunked_scan(route, nc, h, w):
     _case(route, h, w, 8, 16, "f32", seq_chunks=nc, merge_scale=0.5, gate=False)
 
 
+@pytest.mark.parametrize("nc", [2, 4, 8])
+def test_resident_tile_widths(nc):
+    """BIDIR resident tiles are 4 channels wide while 8-channel tiles would leave SMs
+    without a CTA, else 8: 1188 channels (149 eight-channel tiles, the last one half
+    past the end) at batch 1 and 2 take the wide tile, 384 channels at batch 1 the
+    narrow one; f32 with N = 16 stages by cp.async pieces, the others element-wise."""
+    _case("bidir", 5, 6, 1188, 16, "f32", batch=1, seq_chunks=nc)
+    _case("bidir", 5, 6, 1188, 16, "f32", batch=2, seq_chunks=nc, pdi=True, pdp=True)
+    _case("bidir", 5, 6, 1188, 16, "f32", batch=1, seq_chunks=nc, gate=False)
+    _case("bidir", 5, 6, 1192, 7, "bf16", batch=1, seq_chunks=nc, pdp=True)
+    _case("bidir", 6, 5, 1192, 16, "bf16", batch=1, seq_chunks=nc)
+    _case("bidir", 14, 14, 384, 16, "f32", batch=1, seq_chunks=nc, pdp=True)
+
+
 @pytest.mark.parametrize("route,h,w", [("bidir", 14, 14), ("cross4", 9, 13), ("atrous2", 9, 13),
                                        ("bidir", 31, 33), ("cross4", 31, 33), ("atrous2", 31, 33)])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])

@@ -360,29 +360,42 @@ bool use_pipe(const vscan_route* r, const vscan_args* a, int fl)
            a->d_state == 16;
 }
 
-template <int RK, typename T, int NC, int FL>
-cudaError_t launch_resident_nc(const vscan::ScanParams& p, size_t smem, cudaStream_t s)
+template <int RK, typename T, int NC, int FL, int CH>
+cudaError_t launch_resident_ch(const vscan::ScanParams& p, cudaStream_t s)
 {
-    constexpr int CH = vscan::ResidentShape<RK>::CH;
+    constexpr int threads = vscan::ResidentShape<RK>::K * CH * NC * 4;  // one channel-direction per 32 / (4 NC) lanes
+    const int Ki = p.in_dir ? p.g.K : 1;
+    const int Kd = (p.in_dir || p.v_dir) ? p.g.K : 1;
+    const size_t smem = vscan::resident_smem_bytes(RK, p.g.tokens, Ki, Kd, (FL & vscan::FL_CONV) != 0, CH);
     static int attr_done[kAttrDevices] = {};
-    cudaError_t e = set_smem_once(vscan::resident_scan_kernel<RK, T, NC, FL>, (int)kMaxSmem, attr_done,
+    cudaError_t e = set_smem_once(vscan::resident_scan_kernel<RK, T, NC, FL, CH>, (int)kMaxSmem, attr_done,
                                   kAttrDevices);
     if (e != cudaSuccess) return e;
     const dim3 grid((p.D + CH - 1) / CH, p.batch);
-    vscan::resident_scan_kernel<RK, T, NC, FL><<<grid, 64 * NC, smem, s>>>(p);
+    vscan::resident_scan_kernel<RK, T, NC, FL, CH><<<grid, threads, smem, s>>>(p);
     return cudaGetLastError();
+}
+
+// BIDIR takes 4-channel tiles when 8-channel ones would give fewer CTAs than SMs
+// (Vim-Tiny at batch 1: 96 CTAs instead of 48), so that twice as many SMs share the
+// latency-bound chains.
+template <int RK, typename T, int NC, int FL>
+cudaError_t launch_resident_nc(const vscan::ScanParams& p, cudaStream_t s)
+{
+    constexpr int CH = vscan::ResidentShape<RK>::CH;
+    if constexpr (CH == 8 && NC >= 2) {
+        if ((long long)p.batch * ((p.D + CH - 1) / CH) < num_sms()) return launch_resident_ch<RK, T, NC, FL, 4>(p, s);
+    }
+    return launch_resident_ch<RK, T, NC, FL, CH>(p, s);
 }
 
 template <int RK, typename T, int FL>
 cudaError_t launch_resident_fl(const vscan::ScanParams& p, int nc, cudaStream_t s)
 {
-    const int Ki = p.in_dir ? p.g.K : 1;
-    const int Kd = (p.in_dir || p.v_dir) ? p.g.K : 1;
-    const size_t smem = vscan::resident_smem_bytes(RK, p.g.tokens, Ki, Kd, (FL & vscan::FL_CONV) != 0);
     switch (nc) {
-    case 2: return launch_resident_nc<RK, T, 2, FL>(p, smem, s);
-    case 4: return launch_resident_nc<RK, T, 4, FL>(p, smem, s);
-    default: return launch_resident_nc<RK, T, 8, FL>(p, smem, s);
+    case 2: return launch_resident_nc<RK, T, 2, FL>(p, s);
+    case 4: return launch_resident_nc<RK, T, 4, FL>(p, s);
+    default: return launch_resident_nc<RK, T, 8, FL>(p, s);
     }
 }
 
