@@ -146,6 +146,7 @@ KERNEL_SOURCES = {
     "resident_scan_kernel": ("vscan_resident.cuh", "vscan_stream.cuh", "vscan_common.cuh", "vscan_route.cuh"),
     "pool_scan_kernel": ("vscan_pool.cuh", "vscan_common.cuh", "vscan_route.cuh"),
     "bwd_scan_kernel": ("vscan_backward.cuh", "vscan_common.cuh", "vscan_route.cuh"),
+    "bwd_scan_split_kernel": ("vscan_backward.cuh", "vscan_common.cuh", "vscan_route.cuh"),
 }
 
 

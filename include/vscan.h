@@ -371,6 +371,18 @@ vscan_status vscan_backward_workspace_size(const vscan_route* route, const vscan
                                            uint64_t* bytes);
 
 /*
+ * Name of the kernel that runs vscan_backward's adjoint scan for these arguments
+ * (host only), as a static NUL-terminated string owned by the library:
+ * "bwd_scan_split_kernel<R>" (each tile of 8 channels, one image and one
+ * direction on a CTA of two warps that split its 16 states; grids of at most 8
+ * tiles per SM) or "bwd_scan_kernel<R>" (one warp per tile), R = BIDIR, CROSS4 or
+ * ATROUS2, BIDIR for the pooled routes (their pooled sequence is scanned as a
+ * bidirectional route); "none" for an empty batch. Same argument checks and errors
+ * as vscan_backward_workspace_size; *name is untouched on error.
+ */
+vscan_status vscan_backward_plan_kernel(const vscan_route* route, const vscan_args* args, const char** name);
+
+/*
  * Backward pass. args are the forward's arguments (args->y and args->workspace
  * are not used); dy is dL/dy, [batch][tokens][D] in args->dtype, device. The
  * call enqueues on stream: zeroing of the requested gradients, the pre-gate

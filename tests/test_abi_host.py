@@ -172,6 +172,30 @@ def test_plan_kernel_names_the_scan_kernel():
     assert abi.lib.vscan_plan_kernel(r.handle, ctypes.byref(_args(d_state=0)), ctypes.byref(name)) != 0
 
 
+def test_backward_plan_kernel_names_the_adjoint_scan_kernel():
+    """Grids of at most 8 adjoint tiles (8 channels x image x direction) per SM take the
+    two-warp state split (148 SMs are assumed without a GPU)."""
+    name = ctypes.c_char_p()
+    for kind, h, w, cls, batch, D, expect in (
+            ("atrous2", 56, 56, -1, 8, 192, "bwd_scan_split_kernel<ATROUS2>"),    # 768 tiles
+            ("cross4", 56, 56, -1, 16, 192, "bwd_scan_kernel<CROSS4>"),           # 1536
+            ("cross4", 56, 56, -1, 8, 192, "bwd_scan_split_kernel<CROSS4>"),      # 768
+            ("bidir", 14, 14, 98, 1, 384, "bwd_scan_split_kernel<BIDIR>"),        # 96
+            ("bidir", 64, 64, 2048, 64, 768, "bwd_scan_kernel<BIDIR>"),           # 12288
+            ("pool_w", 128, 128, -1, 32, 384, "bwd_scan_kernel<BIDIR>"),          # 3072, pooled as BIDIR
+            ("pool_h", 8, 8, -1, 2, 64, "bwd_scan_split_kernel<BIDIR>"),          # 32
+            ("atrous2", 5, 5, -1, 296, 8, "bwd_scan_split_kernel<ATROUS2>"),      # 1184 = 8 x 148
+            ("atrous2", 5, 5, -1, 297, 8, "bwd_scan_kernel<ATROUS2>"),            # 1188
+            ("atrous2", 4, 4, -1, 0, 64, "none")):
+        r = vs.Route(kind, h, w, cls)
+        a = _args(batch=batch, channels=D)
+        assert abi.lib.vscan_backward_plan_kernel(r.handle, ctypes.byref(a), ctypes.byref(name)) == 0
+        assert name.value.decode() == expect, (kind, h, w, batch, D)
+    r = vs.Route("bidir", 4, 4)
+    assert abi.lib.vscan_backward_plan_kernel(r.handle, ctypes.byref(_args()), None) == -1
+    assert abi.lib.vscan_backward_plan_kernel(r.handle, ctypes.byref(_args(d_state=0)), ctypes.byref(name)) != 0
+
+
 def test_chunked_scan_needs_the_tile_on_chip():
     big = vs.Route("cross4", 56, 56)
     assert abi.lib.vscan_forward(big.handle, ctypes.byref(_args(seq_chunks=4)), None) == -4

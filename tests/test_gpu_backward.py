@@ -78,15 +78,24 @@ def test_backward_bidir_with_middle_cls_and_long_sequence():
 
 
 @pytest.mark.parametrize("route,h,w,D,dtype,batch,kw", [
-    ("bidir", 5, 7, 196, "f32", 64, {}),                        # 25 tiles (channel tail) x 64 x 2
-    ("cross4", 5, 6, 64, "bf16", 96, {"N": 7}),                  # 8 x 96 x 4
+    ("bidir", 5, 7, 196, "f32", 64, {}),                          # 25 tiles (channel tail) x 64 x 2
+    ("bidir", 6, 6, 64, "bf16", 96, {"pdi": True}),               # 8 x 96 x 2
+    ("bidir", 4, 6, 24, "f32", 256, {"gate": False, "skip": False, "bias": False, "softplus": False,
+                                     "merge_scale": 1.0}),       # 3 x 256 x 2
+    ("cross4", 5, 6, 64, "bf16", 96, {"N": 7}),                   # 8 x 96 x 4, plain loads
+    ("cross4", 5, 6, 64, "bf16", 48, {}),                         # 8 x 48 x 4
+    ("cross4", 5, 5, 24, "f32", 128, {"N": 7, "pdi": True, "pdp": True}),  # 3 x 128 x 4
     ("atrous2", 5, 7, 24, "f32", 160, {"pdi": True, "pdp": True}),  # 3 x 160 x 4
-    ("pool_w", 6, 9, 104, "f32", 96, {}),                        # 13 x 96 x 2 over the pooled sequence
+    ("atrous2", 7, 5, 16, "bf16", 192, {}),                       # 2 x 192 x 4
+    ("pool_w", 6, 9, 104, "f32", 96, {}),                         # 13 x 96 x 2 over the pooled sequence
+    ("pool_h", 5, 8, 48, "bf16", 128, {"N": 5, "pdp": True}),     # 6 x 128 x 2, plain loads
 ])
-def test_backward_large_grids_take_the_register_capped_build(route, h, w, D, dtype, batch, kw):
-    """Grids of more than 8 warps per SM (here 1900-3200 warps) run the adjoint scan
-    built for 16 resident warps per SM, which sums dB and dC with a per-step shuffle
-    reduce-scatter instead of shared memory."""
+def test_backward_large_grids_take_the_one_warp_register_capped_build(route, h, w, D, dtype, batch, kw):
+    """Grids of more than 8 tiles per SM (here 1536-3200 tiles) run the adjoint scan with
+    one warp per tile, built for 16 resident warps per SM, which sums dB and dC with a
+    per-step shuffle reduce-scatter; the pooled routes also run its forward pass (no
+    saved checkpoints). Smaller grids, every other case in this file, run the build that
+    splits a tile's states over two warps."""
     _case(route, h, w, D, dtype, batch=batch, **kw)
 
 

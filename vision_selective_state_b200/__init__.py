@@ -400,8 +400,10 @@ class BackwardPlan:
         return n.value + (4 if self.route.kind_name in ("pool_w", "pool_h") else 2)
 
     def kernel_name(self):
-        return "bwd_scan_kernel<" + ("BIDIR" if self.route.kind_name in ("pool_w", "pool_h")
-                                     else self.route.kind_name.upper()) + ">"
+        """Name of the kernel that runs the adjoint scan (vscan_backward_plan_kernel)."""
+        name = ctypes.c_char_p()
+        check(lib.vscan_backward_plan_kernel(self.route.handle, self._ra, ctypes.byref(name)))
+        return name.value.decode()
 
     def run(self, stream):
         """Enqueue the backward pass on a torch.cuda.Stream."""

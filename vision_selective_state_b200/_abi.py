@@ -101,6 +101,7 @@ def _load():
         "vscan_host_buffer_size": ([p, pa, ctypes.POINTER(u64)], i32),
         "vscan_forward_host": ([p, pa, p, u64, p], i32),
         "vscan_backward_workspace_size": ([p, pa, ctypes.POINTER(u64)], i32),
+        "vscan_backward_plan_kernel": ([p, pa, ctypes.POINTER(ctypes.c_char_p)], i32),
         "vscan_backward": ([p, pa, p, ctypes.POINTER(VscanGrads), p], i32),
         "vscan_last_error": ([], ctypes.c_char_p),
         "vscan_status_string": ([i32], ctypes.c_char_p),

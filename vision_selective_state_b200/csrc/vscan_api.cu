@@ -834,17 +834,29 @@ vscan_status check_backward(const vscan_route* r, const vscan_args* a)
     return VSCAN_OK;
 }
 
-// The adjoint scan: one warp per (channel tile, image, direction). Grids of at most
-// 8 warps per SM take the variant with uncapped registers and the shared-memory dB/dC
-// sums (the faster one on the atrous b8 and Vim-Tiny b1 grids); larger grids the
-// one built for 16 resident warps per SM (22-28 % faster on Vim-Tiny b64, SS2D b16
-// and Vim-Small b64).
+// The adjoint scan. Grids of at most 8 tiles (8 channels, one image, one direction)
+// per SM split every tile's states over a CTA of two warps: twice the warps, each with
+// half the per-step chain (measured 7-13 % faster than one warp per tile on Vim-Tiny
+// b1 and b8, the atrous b8 and SS2D b8 grids). Larger grids take one warp per tile,
+// built for 16 resident warps per SM, where the split's extra instructions cost more
+// than its latency hiding gains (SS2D b16 2.24 against 2.17 ms, Vim-Small b64 17.6
+// against 16.9 ms).
+bool bwd_split(long long tiles) { return tiles <= 8LL * num_sms(); }
+
+// Tiles of the adjoint scan's grid: channel tiles x images x directions (2 for the
+// pooled routes, whose pooled sequence is scanned as a bidirectional route).
+long long bwd_tiles(const vscan_route* r, const vscan_args* a)
+{
+    return (long long)((a->channels + vscan::BW_CH - 1) / vscan::BW_CH) * a->batch * r->g.K;
+}
+
 template <int RK, typename T, bool ASYNC>
 void launch_bwd_scan_async(const vscan::BwdParams& p, dim3 grid, cudaStream_t s)
 {
-    const long long warps = (long long)grid.x * grid.y * grid.z;
-    if (warps <= 8LL * num_sms()) vscan::bwd_scan_kernel<RK, T, 1, ASYNC><<<grid, 32, 0, s>>>(p);
-    else vscan::bwd_scan_kernel<RK, T, vscan::BW_MIN_WARPS, ASYNC><<<grid, 32, 0, s>>>(p);
+    if (bwd_split((long long)grid.x * grid.y * grid.z))
+        vscan::bwd_scan_split_kernel<RK, T, ASYNC><<<grid, vscan::BWS_THREADS, 0, s>>>(p);
+    else
+        vscan::bwd_scan_kernel<RK, T, ASYNC><<<grid, 32, 0, s>>>(p);
 }
 
 // d_state 16 takes the build that gathers the next chunk with cp.async while the
@@ -1150,6 +1162,24 @@ vscan_status vscan_backward_workspace_size(const vscan_route* r, const vscan_arg
     vscan_status st = check_backward(r, a);
     if (st != VSCAN_OK) return st;
     *bytes = a->batch == 0 ? 0 : bwd_layout(r, a).total;
+    return VSCAN_OK;
+}
+
+vscan_status vscan_backward_plan_kernel(const vscan_route* r, const vscan_args* a, const char** name)
+{
+    if (!name) return fail(VSCAN_ERR_INVALID_ARGUMENT, "name is NULL");
+    vscan_status st = check_backward(r, a);
+    if (st != VSCAN_OK) return st;
+    static const char* const split_names[] = {"bwd_scan_split_kernel<BIDIR>", "bwd_scan_split_kernel<CROSS4>",
+                                              "bwd_scan_split_kernel<ATROUS2>"};
+    static const char* const warp_names[] = {"bwd_scan_kernel<BIDIR>", "bwd_scan_kernel<CROSS4>",
+                                             "bwd_scan_kernel<ATROUS2>"};
+    if (a->batch == 0) {
+        *name = "none";
+        return VSCAN_OK;
+    }
+    const int kind = is_pool(r->g.kind) ? (int)vscan::RK_BIDIR : r->g.kind;
+    *name = bwd_split(bwd_tiles(r, a)) ? split_names[kind] : warp_names[kind];
     return VSCAN_OK;
 }
 

@@ -22,13 +22,13 @@
 //                        every 16-step chunk boundary; pass 2 walks the chunks
 //                        backwards, recomputes the chunk's states from its
 //                        checkpoint and runs the adjoint recurrence. Token
-//                        gradients are summed over channels (B, C: in shared
-//                        memory once per chunk on grids of few warps per SM,
-//                        one shuffle reduce-scatter per step on larger ones) or
-//                        state groups (u, Delta: shuffles) and added with float
-//                        atomics (directions, channel tiles and images meet
-//                        there); dA, D and bias gradients stay in registers
-//                        until the end.
+//                        gradients are summed over channels (B, C: one shuffle
+//                        reduce-scatter per step) or state groups (u, Delta:
+//                        shuffles) and added with float atomics (directions,
+//                        channel tiles and images meet there); dA, D and bias
+//                        gradients stay in registers until the end.
+//   bwd_scan_split_kernel  the same with each tile's 16 states split over a CTA
+//                        of two warps, for grids with few warps per SM.
 //   bwd_unpool_kernel    pooled routes: every member token receives its pooled
 //                        index's gradient divided by the member count.
 #pragma once
@@ -232,36 +232,25 @@ struct __align__(16) BwdStage {
 };
 
 // Per-chunk gradient partials of bwd_scan_kernel, added to global memory after
-// the chunk. With SMEM_BC the per-channel dB and dC partials are staged too and
-// summed over the channels after the chunk; without it they are summed with
-// shuffles at every step.
+// the chunk (dB and dC are summed over the channels with shuffles at every step).
 struct BwdReduceUX {
     float u[BW_TOK][BW_CH];  // du per (step, channel), state groups already summed
     float x[BW_TOK][BW_CH];  // d raw Delta per (step, channel)
 };
-template <bool SMEM_BC> struct BwdReduce : BwdReduceUX {};
-template <> struct BwdReduce<true> : BwdReduceUX {
-    float B[BW_TOK][BW_CH][16];  // dB per (step, channel, state)
-    float C[BW_TOK][BW_CH][16];  // dC likewise
-};
 
-// Warps per SM the backward scan is compiled for. MINW = BW_MIN_WARPS caps its
-// registers per thread and keeps its shared memory small (the kernel is
-// latency-bound, so on large grids resident warps matter more than scheduling
-// room) and sums dB and dC with shuffles. MINW = 1, for grids that put only a few
-// warps on each SM, leaves registers uncapped and sums dB and dC through shared
-// memory once per chunk, which keeps the shuffles off the steps' latency.
+// Warps per SM the one-warp backward scan is compiled for: capped registers per
+// thread and small shared memory (the kernel is latency-bound, so on large grids
+// resident warps matter more than scheduling room).
 constexpr int BW_MIN_WARPS = 16;
 
 // ASYNC (d_state 16): pass 2 gathers chunk c - 1 with cp.async while the
 // adjoint of chunk c runs, so a chunk's rows are waited for only once they have
 // had a whole chunk of compute to arrive.
-template <int RK, typename TI, int MINW, bool ASYNC>
-__global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
+template <int RK, typename TI, bool ASYNC>
+__global__ void __launch_bounds__(32, BW_MIN_WARPS) bwd_scan_kernel(const BwdParams p)
 {
-    constexpr bool SMEM_BC = MINW == 1;
     __shared__ BwdStage st;
-    __shared__ __align__(16) BwdReduce<SMEM_BC> rd;
+    __shared__ __align__(16) BwdReduceUX rd;
     __shared__ BwdRaw<TI> raw[ASYNC ? 2 : 1];
     const int lane = threadIdx.x;
     const int cc = lane >> 2, grp = lane & 3;
@@ -526,11 +515,7 @@ __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
                 rd.u[j][cc] = fmaf(Dd, dy, dut);
                 rd.x[j][cc] = draw;
             }
-            if constexpr (SMEM_BC) {
-                // per-channel partials of dB and dC, summed over the channels after the chunk
-                *reinterpret_cast<float4*>(&rd.B[j][cc][4 * grp]) = make_float4(dBv[0], dBv[1], dBv[2], dBv[3]);
-                *reinterpret_cast<float4*>(&rd.C[j][cc][4 * grp]) = make_float4(dCv[0], dCv[1], dCv[2], dCv[3]);
-            } else {
+            {
                 // dB and dC of the step, summed over the 8 channels (lanes 4c + grp, c = 0..7):
                 // a reduce-scatter over lane bits 4, 3, 2 leaves lane 4c + grp with value c of
                 // its group, i.e. tensor c >> 2 (0: B, 1: C) at state 4 grp + (c & 3).
@@ -549,8 +534,8 @@ __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
                 if (q >= 0 && n < N && dst) atomicAdd(dst + ki * p.bc_dir + (img + q) * N + n, v1);
             }
         }
-        // add the chunk's token gradients: one atomic per (step, channel) and, with
-        // SMEM_BC, per (step, state), every lane taking its share
+        // add the chunk's token gradients: one atomic per (step, channel), every lane
+        // taking its share
         __syncwarp();
 #pragma unroll
         for (int r = 0; r < BW_TOK * BW_CH / 32; ++r) {
@@ -568,24 +553,6 @@ __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
                 if (p.ddelta) atomicAdd(p.ddelta + o, rd.x[j][ch]);
             }
         }
-        if constexpr (SMEM_BC) {
-#pragma unroll
-            for (int r = 0; r < BW_TOK * 16 / 32; ++r) {
-                const int e = lane + 32 * r;
-                const int j = e >> 4, n = e & 15;
-                const int q = st.pos[j];
-                if (q < 0 || n >= N) continue;
-                float sb = 0.f, sc = 0.f;
-#pragma unroll
-                for (int ch = 0; ch < BW_CH; ++ch) {
-                    sb += rd.B[j][ch][n];
-                    sc += rd.C[j][ch][n];
-                }
-                const long long o = ki * p.bc_dir + (img + q) * N + n;
-                if (p.dB) atomicAdd(p.dB + o, sb);
-                if (p.dC) atomicAdd(p.dC + o, sc);
-            }
-        }
         __syncwarp();
     }
     if (dvalid) {
@@ -599,6 +566,315 @@ __global__ void __launch_bounds__(32, MINW) bwd_scan_kernel(const BwdParams p)
             if (p.dD) atomicAdd(p.dD + k * p.v_dir + d, dDs);
             if (p.dbias) atomicAdd(p.dbias + k * p.v_dir + d, dbs);
         }
+    }
+}
+
+// The adjoint scan with a tile's 16 states split over two warps, for grids that
+// leave SMs short of warps with one warp per tile (at most 8 tiles per SM): a CTA of two warps covers one
+// (8-channel tile, image, direction); warp h holds states 8h..8h+7, lane 4c + g
+// channel c and the state pair 8h + 2g, 8h + 2g + 1. Each warp's per-step chain is
+// one state pair instead of two, and twice as many warps share the SMs. The
+// chunk's rows are staged once for both warps. The du and dDelta partials of the
+// two state halves meet in shared memory after the chunk; dB and dC are summed
+// over the 8 channels inside each warp (4 shuffles per step), so the atomics per
+// step equal the one-warp kernel's.
+constexpr int BWS_THREADS = 64;
+constexpr int BWS_MIN_BLOCKS = 12;  // 24 warps per SM: at most 85 registers per thread
+
+struct __align__(16) BwdSplitPart {
+    float u[2][BW_TOK][BW_CH];  // du partial of each state half, per (step, channel)
+    float x[2][BW_TOK][BW_CH];  // dDelta partial likewise
+};
+
+template <int RK, typename TI, bool ASYNC>
+__global__ void __launch_bounds__(BWS_THREADS, BWS_MIN_BLOCKS) bwd_scan_split_kernel(const BwdParams p)
+{
+    __shared__ BwdStage st;
+    __shared__ BwdSplitPart part;
+    __shared__ BwdRaw<TI> raw[ASYNC ? 2 : 1];
+    const int tid = threadIdx.x, h = tid >> 5, lane = tid & 31;
+    const int cc = lane >> 2, grp = lane & 3;
+    const int n0 = 8 * h + 2 * grp;  // this lane's state pair
+    const int c0 = blockIdx.x * BW_CH, b = blockIdx.y, k = blockIdx.z;
+    const int D = p.D, N = p.N, L = p.g.L, tokens = p.g.tokens;
+    const int d = c0 + cc;
+    const bool dvalid = d < D;
+    const int ki = p.in_dir ? k : 0;
+    const long long img = (long long)b * tokens;
+    const int nch = (L + BW_TOK - 1) / BW_TOK;
+    float2 An, a2;
+    {
+        const float* Ar = p.A + (long long)k * p.a_dir + (long long)d * N + n0;
+        An = make_float2((dvalid && n0 < N) ? __ldg(Ar) : 0.f, (dvalid && n0 + 1 < N) ? __ldg(Ar + 1) : 0.f);
+        a2 = make_float2(An.x * LOG2E, An.y * LOG2E);
+    }
+    // (step, channel) items of the staging and of the after-chunk sums: e = tid + 64 r,
+    // step e / 8, channel e % 8 = tid % 8 for every r
+    const int ce = tid & (BW_CH - 1);
+    const bool cev = c0 + ce < D;
+    const float Dd_e = (cev && p.Dskip) ? __ldg(p.Dskip + k * p.v_dir + c0 + ce) : 0.f;
+    const float bias_e = (cev && p.bias) ? __ldg(p.bias + k * p.v_dir + c0 + ce) : 0.f;
+    const float* gyb = p.gy + img * D;
+    const TI* ub = static_cast<const TI*>(p.u) + ki * p.in_dir + img * D;
+    const TI* rb = static_cast<const TI*>(p.delta) + ki * p.in_dir + img * D;
+    const TI* Bb = static_cast<const TI*>(p.B) + ki * p.bc_dir + img * N;
+    const TI* Cb = static_cast<const TI*>(p.C) + ki * p.bc_dir + img * N;
+    float* ck = p.ckpt + (((long long)k * p.batch + b) * nch) * D * 16;
+    constexpr int NE = BW_TOK * BW_CH / BWS_THREADS;  // (step, channel) items per thread: 2
+    constexpr int NS = BW_TOK * 16 / BWS_THREADS;     // (step, state) items per thread: 4
+
+    // discretized step (0 past the end and beyond D) and its derivative of one
+    // (step, channel) item
+    auto disc = [&](float raw_d, bool live, float& x, float& sg) {
+        const float xr = raw_d + bias_e;
+        x = xr;
+        sg = 1.f;
+        if (p.softplus) {
+            x = softplus_f(xr);
+            sg = 1.0f / (1.0f + __expf(-xr));
+        }
+        if (!live) x = 0.f;
+    };
+
+    // Stage chunk c with plain loads, every load of a thread issued before any use.
+    auto stage = [&](int c, bool with_grad) {
+        __syncthreads();  // every thread is done with st and part
+        if (tid < BW_TOK) {
+            const int t = c * BW_TOK + tid;
+            st.pos[tid] = (t < L) ? route_token<RK>(p.g, k, t) : -2;
+        }
+        __syncthreads();
+        float vr[NE], vu[NE], vg[NE], vb[NS], vc[NS];
+#pragma unroll
+        for (int r = 0; r < NE; ++r) {
+            const int j = (tid + BWS_THREADS * r) / BW_CH, dd = c0 + ce;
+            const int q = st.pos[j];
+            const bool ok = q >= 0 && dd < D;
+            vr[r] = ok ? to_float(rb[(long long)q * D + dd]) : 0.f;
+            vu[r] = ok ? to_float(ub[(long long)q * D + dd]) : 0.f;
+            vg[r] = (ok && with_grad) ? gyb[(long long)q * D + dd] : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < NS; ++r) {
+            const int e = tid + BWS_THREADS * r;
+            const int j = e >> 4, n = e & 15;
+            const int q = st.pos[j];
+            const bool ok = q >= 0 && n < N;
+            vb[r] = ok ? to_float(Bb[(long long)q * N + n]) : 0.f;
+            vc[r] = ok ? to_float(Cb[(long long)q * N + n]) : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < NE; ++r) {
+            const int j = (tid + BWS_THREADS * r) / BW_CH;
+            float x, sg;
+            disc(vr[r], st.pos[j] != -2 && cev, x, sg);
+            st.x[j][ce] = x;
+            st.sig[j][ce] = sg;
+            st.u[j][ce] = vu[r];
+            st.gy[j][ce] = vg[r];
+        }
+#pragma unroll
+        for (int r = 0; r < NS; ++r) {
+            const int e = tid + BWS_THREADS * r;
+            st.B[e >> 4][e & 15] = vb[r];
+            st.C[e >> 4][e & 15] = vc[r];
+        }
+        __syncthreads();
+    };
+
+    // ASYNC: gather chunk c's rows into raw[buf] (16-byte cp.async, zero fill for
+    // padding, past-the-end steps and channels beyond D), one commit group per thread.
+    auto issue = [&](int c, int buf) {
+        BwdRaw<TI>& rw = raw[buf];
+        int q = -2;
+        if (lane < BW_TOK) {  // both warps compute the chunk's positions for their shuffles
+            const int t = c * BW_TOK + lane;
+            q = (t < L) ? route_token<RK>(p.g, k, t) : -2;
+            if (h == 0) rw.pos[lane] = q;
+        }
+        constexpr int EL = 16 / (int)sizeof(TI);             // elements per 16-byte piece
+        constexpr int PR = BW_CH / EL;                        // pieces per u / Delta row
+        constexpr int PB = 16 / EL;                           // pieces per B / C row
+        constexpr int NPC = BW_TOK * (2 * PR + 2 + 2 * PB);   // + gy rows of 2 pieces
+#pragma unroll
+        for (int it = 0; it < (NPC + BWS_THREADS - 1) / BWS_THREADS; ++it) {
+            const int f = tid + BWS_THREADS * it;
+            int tsr, row, pc;  // 0 Delta, 1 u (PR pieces), 2 gy (2), 3 B, 4 C (PB)
+            if (f < 2 * BW_TOK * PR) {
+                tsr = f / (BW_TOK * PR);
+                const int r = f - tsr * BW_TOK * PR;
+                row = r / PR;
+                pc = r - row * PR;
+            } else if (f < 2 * BW_TOK * PR + 2 * BW_TOK) {
+                tsr = 2;
+                const int r = f - 2 * BW_TOK * PR;
+                row = r >> 1;
+                pc = r & 1;
+            } else {
+                const int r = f - 2 * BW_TOK * PR - 2 * BW_TOK;
+                tsr = 3 + r / (BW_TOK * PB);
+                const int r2 = r - (tsr - 3) * BW_TOK * PB;
+                row = r2 / PB;
+                pc = r2 - row * PB;
+            }
+            const int qj = __shfl_sync(FULL_MASK, q, row & (BW_TOK - 1));
+            if (f < NPC) {
+                const long long tok = qj >= 0 ? qj : 0;
+                if (tsr < 2) {
+                    const bool ok = qj >= 0 && c0 + pc * EL < D;
+                    const TI* src = (tsr == 0 ? rb : ub) + (ok ? tok * D + c0 + pc * EL : 0);
+                    cp_async16(tsr == 0 ? &rw.d[row][pc * EL] : &rw.u[row][pc * EL], src, ok);
+                } else if (tsr == 2) {
+                    const bool ok = qj >= 0 && c0 + 4 * pc < D;
+                    cp_async16(&rw.gy[row][4 * pc], gyb + (ok ? tok * D + c0 + 4 * pc : 0), ok);
+                } else {
+                    const bool ok = qj >= 0;
+                    const TI* src = (tsr == 3 ? Bb : Cb) + (ok ? tok * 16 + pc * EL : 0);
+                    cp_async16(tsr == 3 ? &rw.B[row][pc * EL] : &rw.C[row][pc * EL], src, ok);
+                }
+            }
+        }
+        cp_async_commit();
+    };
+    // ASYNC: wait for raw[buf] and discretize it into st.
+    auto convert = [&](int buf) {
+        cp_async_wait<0>();
+        __syncthreads();  // all copies of raw[buf] landed; every thread is done with st and part
+        const BwdRaw<TI>& rw = raw[buf];
+        if (tid < BW_TOK) st.pos[tid] = rw.pos[tid];
+#pragma unroll
+        for (int r = 0; r < NE; ++r) {
+            const int j = (tid + BWS_THREADS * r) / BW_CH;
+            float x, sg;
+            disc(to_float(rw.d[j][ce]), rw.pos[j] != -2 && cev, x, sg);
+            st.x[j][ce] = x;
+            st.sig[j][ce] = sg;
+            st.u[j][ce] = to_float(rw.u[j][ce]);
+            st.gy[j][ce] = rw.gy[j][ce];
+        }
+#pragma unroll
+        for (int r = 0; r < NS; ++r) {
+            const int e = tid + BWS_THREADS * r;
+            st.B[e >> 4][e & 15] = to_float(rw.B[e >> 4][e & 15]);
+            st.C[e >> 4][e & 15] = to_float(rw.C[e >> 4][e & 15]);
+        }
+        __syncthreads();
+    };
+
+    // one step of the recurrence for the lane's pair: h = 2^(x A log2 e) h + (x B) u
+    auto step2 = [&](float2 hp, float x, float uu, float2 Bq) {
+        const float2 xx = make_float2(x, x);
+        const float2 xa = __fmul2_rn(xx, a2);
+        const float2 e = make_float2(fast_exp2(xa.x), fast_exp2(xa.y));
+        return __ffma2_rn(e, hp, __fmul2_rn(__fmul2_rn(xx, Bq), make_float2(uu, uu)));
+    };
+
+    // ---- pass 1: forward recurrence, state saved at every chunk boundary --------
+    float2 hh = make_float2(0.f, 0.f);
+    for (int c = 0; c < (p.ckpt_ready ? 0 : nch); ++c) {
+        if (dvalid) *reinterpret_cast<float2*>(&ck[((long long)c * D + d) * 16 + n0]) = hh;
+        stage(c, false);
+#pragma unroll 4
+        for (int j = 0; j < BW_TOK; ++j)
+            hh = step2(hh, st.x[j][cc], st.u[j][cc], *reinterpret_cast<const float2*>(&st.B[j][n0]));
+    }
+
+    // ---- pass 2: adjoint recurrence, chunks in reverse ------------------------------
+    float2 gs = make_float2(0.f, 0.f), dAs = make_float2(0.f, 0.f);
+    float dDs = 0.f, dbs = 0.f;  // channel ce, summed over this thread's items
+    const bool b4 = cc & 4, b2 = cc & 2, b1 = cc & 1;
+    if constexpr (ASYNC) issue(nch - 1, 0);
+    for (int c = nch - 1; c >= 0; --c) {
+        if constexpr (ASYNC) {
+            const int buf = (nch - 1 - c) & 1;
+            convert(buf);
+            if (c > 0) issue(c - 1, buf ^ 1);  // lands while this chunk's adjoint runs
+        } else {
+            stage(c, true);
+        }
+        float2 hs[BW_TOK + 1];  // hs[0] = state entering the chunk, hs[j + 1] after step j
+        hs[0] = dvalid ? *reinterpret_cast<const float2*>(&ck[((long long)c * D + d) * 16 + n0]) : make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < BW_TOK; ++j)
+            hs[j + 1] = step2(hs[j], st.x[j][cc], st.u[j][cc], *reinterpret_cast<const float2*>(&st.B[j][n0]));
+#pragma unroll
+        for (int j = BW_TOK - 1; j >= 0; --j) {
+            const int q = st.pos[j];
+            if (q == -2) continue;  // past the end of the sequence (uniform over the CTA)
+            const float x = st.x[j][cc], uu = st.u[j][cc], dy = st.gy[j][cc];
+            const float2 xx = make_float2(x, x), uu2 = make_float2(uu, uu), dy2 = make_float2(dy, dy);
+            const float2 Bp = *reinterpret_cast<const float2*>(&st.B[j][n0]);
+            const float2 Cp = *reinterpret_cast<const float2*>(&st.C[j][n0]);
+            const float2 xa = __fmul2_rn(xx, a2);
+            const float2 a = make_float2(fast_exp2(xa.x), fast_exp2(xa.y));
+            gs = __ffma2_rn(Cp, dy2, gs);                              // g += C dy
+            const float2 dC2 = __fmul2_rn(dy2, hs[j + 1]);             // dC = dy h
+            const float2 gx = __fmul2_rn(gs, xx);
+            const float2 dB2 = __fmul2_rn(gx, uu2);                    // dB = g x u
+            const float2 dut2 = __fmul2_rn(gx, Bp);                    // du = g x B
+            const float2 t = __ffma2_rn(__fmul2_rn(An, a), hs[j], __fmul2_rn(Bp, uu2));
+            const float2 dxt2 = __fmul2_rn(gs, t);                     // dx = g (A a h' + B u)
+            dAs = __ffma2_rn(__fmul2_rn(gx, a), hs[j], dAs);           // dA += g x a h'
+            gs = __fmul2_rn(gs, a);                                    // carried to step j - 1
+            // du and dDelta over the warp's 8 states of the channel (lanes 4c .. 4c + 3)
+            float dut = dut2.x + dut2.y, dxt = dxt2.x + dxt2.y;
+            dut += __shfl_xor_sync(FULL_MASK, dut, 1);
+            dut += __shfl_xor_sync(FULL_MASK, dut, 2);
+            dxt += __shfl_xor_sync(FULL_MASK, dxt, 1);
+            dxt += __shfl_xor_sync(FULL_MASK, dxt, 2);
+            if (grp == 0) {
+                part.u[h][j][cc] = dut;
+                part.x[h][j][cc] = dxt;
+            }
+            // dB and dC of the step summed over the 8 channels (lane bits 4, 3, 2): lane
+            // 4c + g ends with tensor c >> 2 (0: B, 1: C) at state n0 + ((c >> 1) & 1);
+            // lanes 4c + g and 4(c ^ 1) + g hold the same sum and the even c adds it.
+            const float o0 = b4 ? dC2.x : dB2.x, o1 = b4 ? dC2.y : dB2.y;
+            const float s0 = b4 ? dB2.x : dC2.x, s1 = b4 ? dB2.y : dC2.y;
+            const float v0 = o0 + __shfl_xor_sync(FULL_MASK, s0, 16);
+            const float v1 = o1 + __shfl_xor_sync(FULL_MASK, s1, 16);
+            float w = (b2 ? v1 : v0) + __shfl_xor_sync(FULL_MASK, b2 ? v0 : v1, 8);
+            w += __shfl_xor_sync(FULL_MASK, w, 4);
+            const int n = n0 + (b2 ? 1 : 0);
+            float* dst = b4 ? p.dC : p.dB;
+            if (!b1 && q >= 0 && n < N && dst) atomicAdd(dst + ki * p.bc_dir + (img + q) * N + n, w);
+        }
+        __syncthreads();  // both state halves' partials are in part
+        // the chunk's token gradients: one store or atomic per (step, channel)
+#pragma unroll
+        for (int r = 0; r < NE; ++r) {
+            const int j = (tid + BWS_THREADS * r) / BW_CH;
+            const int q = st.pos[j];
+            if (q == -2 || !cev) continue;
+            const float gyv = st.gy[j][ce];
+            const float draw = (part.x[0][j][ce] + part.x[1][j][ce]) * st.sig[j][ce];
+            dbs += draw;
+            dDs = fmaf(gyv, st.u[j][ce], dDs);
+            if (q < 0) continue;
+            const float duv = fmaf(Dd_e, gyv, part.u[0][j][ce] + part.u[1][j][ce]);
+            const long long o = ki * p.in_dir + (img + q) * D + c0 + ce;
+            if constexpr (RK == RK_ATROUS2) {
+                // one owner per pixel and channel: no other CTA writes this element
+                if (p.du) p.du[o] = duv;
+                if (p.ddelta) p.ddelta[o] = draw;
+            } else {
+                if (p.du) atomicAdd(p.du + o, duv);
+                if (p.ddelta) atomicAdd(p.ddelta + o, draw);
+            }
+        }
+    }
+    if (dvalid) {
+        if (n0 < N && p.dA) atomicAdd(p.dA + (long long)k * p.a_dir + (long long)d * N + n0, dAs.x);
+        if (n0 + 1 < N && p.dA) atomicAdd(p.dA + (long long)k * p.a_dir + (long long)d * N + n0 + 1, dAs.y);
+    }
+    // D and bias gradients: lanes l, l ^ 8, l ^ 16, l ^ 24 of a warp share channel ce
+    dDs += __shfl_xor_sync(FULL_MASK, dDs, 8);
+    dDs += __shfl_xor_sync(FULL_MASK, dDs, 16);
+    dbs += __shfl_xor_sync(FULL_MASK, dbs, 8);
+    dbs += __shfl_xor_sync(FULL_MASK, dbs, 16);
+    if (lane < BW_CH && cev) {
+        if (p.dD) atomicAdd(p.dD + k * p.v_dir + c0 + ce, dDs);
+        if (p.dbias) atomicAdd(p.dbias + k * p.v_dir + c0 + ce, dbs);
     }
 }
 
