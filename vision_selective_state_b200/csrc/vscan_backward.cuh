@@ -67,6 +67,10 @@ struct BwdParams {
 constexpr int BW_TOK = 16;  // steps per chunk
 constexpr int BW_CH = 8;    // channels per warp
 
+// d softplus(x) / dx = sigma(x) = 1 / (1 + e^-x), on the SFU (2^x and the
+// reciprocal): 0 for x below about -88, where e^-x overflows, and 1 for large x.
+__device__ __forceinline__ float sigmoid_f(float x) { return fast_rcp(1.0f + fast_exp2(-x * LOG2E)); }
+
 // dz = dy * pre * sigmoid(z) * (1 + z (1 - sigmoid(z))) and gy = dy * s * SiLU(z),
 // where pre = s * (merged scan output) is the forward output without the gate.
 template <typename T>
@@ -320,7 +324,7 @@ __global__ void __launch_bounds__(32, BW_MIN_WARPS) bwd_scan_kernel(const BwdPar
             float x = xr, sg = 1.f;
             if (p.softplus) {
                 x = softplus_f(xr);
-                sg = 1.0f / (1.0f + __expf(-xr));
+                sg = sigmoid_f(xr);
             }
             const bool live = st.pos[j] != -2 && dd < D;
             st.x[j][ch] = live ? x : 0.f;
@@ -405,7 +409,7 @@ __global__ void __launch_bounds__(32, BW_MIN_WARPS) bwd_scan_kernel(const BwdPar
             float x = xr, sg = 1.f;
             if (p.softplus) {
                 x = softplus_f(xr);
-                sg = 1.0f / (1.0f + __expf(-xr));
+                sg = sigmoid_f(xr);
             }
             const bool live = rw.pos[j] != -2 && dd < D;
             st.x[j][ch] = live ? x : 0.f;
@@ -452,14 +456,24 @@ __global__ void __launch_bounds__(32, BW_MIN_WARPS) bwd_scan_kernel(const BwdPar
     float2 gs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
     float2 dAs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
     float dDs = 0.f, dbs = 0.f;
+    // dB and dC partials per (step, channel, state) of two steps: B at [slot][channel][16],
+    // C BC_C floats further (16 words past a multiple of 32, so a half-warp reading
+    // both tensors at one channel hits 32 distinct banks). They live in the raw
+    // buffer the current chunk was converted from, which is idle until the chunk after
+    // next is gathered into it.
+    constexpr int BC_C = 2 * BW_CH * 16 + 16;
+    static_assert((BC_C + 2 * BW_CH * 16) * sizeof(float) <= sizeof(BwdRaw<TI>), "partials fit a raw buffer");
     if constexpr (ASYNC) issue(nch - 1, 0);
     for (int c = nch - 1; c >= 0; --c) {
+        float* bcs;
         if constexpr (ASYNC) {
             const int buf = (nch - 1 - c) & 1;
             convert(buf);
             if (c > 0) issue(c - 1, buf ^ 1);  // lands while this chunk's adjoint runs
+            bcs = reinterpret_cast<float*>(&raw[buf]);
         } else {
             stage(c, true);
+            bcs = reinterpret_cast<float*>(&raw[0]);
         }
         float2 hs[BW_TOK + 1][2];  // hs[0] = state entering the chunk, hs[j + 1] after step j
 #pragma unroll
@@ -515,23 +529,29 @@ __global__ void __launch_bounds__(32, BW_MIN_WARPS) bwd_scan_kernel(const BwdPar
                 rd.u[j][cc] = fmaf(Dd, dy, dut);
                 rd.x[j][cc] = draw;
             }
-            {
-                // dB and dC of the step, summed over the 8 channels (lanes 4c + grp, c = 0..7):
-                // a reduce-scatter over lane bits 4, 3, 2 leaves lane 4c + grp with value c of
-                // its group, i.e. tensor c >> 2 (0: B, 1: C) at state 4 grp + (c & 3).
-                const bool b4 = cc & 4, b2 = cc & 2, b1 = cc & 1;
-                float v4[4];
+            // dB and dC of steps j + 1 and j, summed over the 8 channels once both are in
+            // (slot = step & 1; a step past the end is skipped, and so is every later one)
+            *reinterpret_cast<float4*>(&bcs[((j & 1) * BW_CH + cc) * 16 + 4 * grp]) =
+                make_float4(dBv[0], dBv[1], dBv[2], dBv[3]);
+            *reinterpret_cast<float4*>(&bcs[BC_C + ((j & 1) * BW_CH + cc) * 16 + 4 * grp]) =
+                make_float4(dCv[0], dCv[1], dCv[2], dCv[3]);
+            if ((j & 1) == 0) {
+                __syncwarp();
+                // this lane's share: slot lane >> 4, states s_n and s_n + 1, tensor lane & 1
+                const int s_sl = lane >> 4, s_n = 4 * ((lane >> 2) & 3) + 2 * ((lane >> 1) & 1);
+                const bool s_tz = lane & 1;
+                float* const s_dst = s_tz ? p.dC : p.dB;
+                const float* src = bcs + (s_tz ? BC_C : 0) + s_sl * BW_CH * 16 + s_n;
+                float2 acc = *reinterpret_cast<const float2*>(src);
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    v4[i] = (b4 ? dCv[i] : dBv[i]) + __shfl_xor_sync(FULL_MASK, b4 ? dBv[i] : dCv[i], 16);
-                float v2[2];
-#pragma unroll
-                for (int i = 0; i < 2; ++i)
-                    v2[i] = (b2 ? v4[2 + i] : v4[i]) + __shfl_xor_sync(FULL_MASK, b2 ? v4[i] : v4[2 + i], 8);
-                const float v1 = (b1 ? v2[1] : v2[0]) + __shfl_xor_sync(FULL_MASK, b1 ? v2[0] : v2[1], 4);
-                const int n = 4 * grp + (cc & 3);
-                float* dst = b4 ? p.dC : p.dB;
-                if (q >= 0 && n < N && dst) atomicAdd(dst + ki * p.bc_dir + (img + q) * N + n, v1);
+                for (int ch = 1; ch < BW_CH; ++ch) acc = __fadd2_rn(acc, *reinterpret_cast<const float2*>(src + ch * 16));
+                const int qs = st.pos[j + s_sl];
+                if (qs >= 0 && s_dst) {
+                    float* o = s_dst + ki * p.bc_dir + (img + qs) * N + s_n;
+                    if (s_n < N) atomicAdd(o, acc.x);
+                    if (s_n + 1 < N) atomicAdd(o + 1, acc.y);
+                }
+                __syncwarp();
             }
         }
         // add the chunk's token gradients: one atomic per (step, channel), every lane
@@ -631,7 +651,7 @@ __global__ void __launch_bounds__(BWS_THREADS, BWS_MIN_BLOCKS) bwd_scan_split_ke
         sg = 1.f;
         if (p.softplus) {
             x = softplus_f(xr);
-            sg = 1.0f / (1.0f + __expf(-xr));
+            sg = sigmoid_f(xr);
         }
         if (!live) x = 0.f;
     };
