@@ -141,12 +141,12 @@ def peaks():
 
 # device-code files each timed kernel is compiled from (host-side API code excluded)
 KERNEL_SOURCES = {
-    "stream_scan_kernel": ("vscan_stream.cuh", "vscan_common.cuh", "vscan_route.cuh"),
-    "pipe_scan_kernel": ("vscan_pipe.cuh", "vscan_stream.cuh", "vscan_common.cuh", "vscan_route.cuh"),
-    "resident_scan_kernel": ("vscan_resident.cuh", "vscan_stream.cuh", "vscan_common.cuh", "vscan_route.cuh"),
+    "stream_scan_kernel": ("vscan_stream.cuh", "vscan_params.cuh", "vscan_common.cuh", "vscan_route.cuh"),
+    "pipe_scan_kernel": ("vscan_pipe.cuh", "vscan_params.cuh", "vscan_common.cuh", "vscan_route.cuh"),
+    "resident_scan_kernel": ("vscan_resident.cuh", "vscan_params.cuh", "vscan_common.cuh", "vscan_route.cuh"),
     "pool_scan_kernel": ("vscan_pool.cuh", "vscan_common.cuh", "vscan_route.cuh"),
-    "bwd_scan_kernel": ("vscan_backward.cuh", "vscan_common.cuh", "vscan_route.cuh"),
-    "bwd_scan_split_kernel": ("vscan_backward.cuh", "vscan_common.cuh", "vscan_route.cuh"),
+    "bwd_scan_kernel": ("vscan_backward.cuh", "vscan_params.cuh", "vscan_common.cuh", "vscan_route.cuh"),
+    "bwd_scan_split_kernel": ("vscan_backward.cuh", "vscan_params.cuh", "vscan_common.cuh", "vscan_route.cuh"),
 }
 
 

@@ -111,6 +111,14 @@ def test_zoh_all_routes(route, dtype, h, w):
     _case(route, h, w, D, dtype, zoh=True, seq_chunks=1 if route in ("cross4", "atrous2", "bidir") else 0)
 
 
+@pytest.mark.parametrize("batch", [2, 40])
+def test_zoh_atrous_f32_both_consumer_layouts(batch):
+    """The ZOH write term on the float32 atrous streaming kernel with the states split
+    over two consumer warps (at most 8 CTAs per SM) and with one consumer warp (1280
+    CTAs)."""
+    _case("atrous2", 5, 7, 64, "f32", zoh=True, batch=batch, seq_chunks=1)
+
+
 @pytest.mark.parametrize("zoh,conv", [(True, False), (False, True), (True, True)])
 def test_resident_wide_tile_with_optional_steps(zoh, conv):
     """The 8-channel BIDIR resident tile (1188 channels, 149 tiles at batch 1) with the

@@ -81,6 +81,17 @@ def test_resident_chunked_scan(route, nc, h, w):
     _case(route, h, w, 8, 16, "f32", seq_chunks=nc, merge_scale=0.5, gate=False)
 
 
+@pytest.mark.parametrize("batch,D", [(2, 24), (40, 64)])
+def test_atrous_f32_streaming_consumer_layouts(batch, D):
+    """float32 atrous streaming launches of at most 4 CTAs per SM (2 x 3 x 4 = 24 here)
+    split each channel's 16 states over two consumer warps; larger ones (40 x 8 x 4 =
+    1280) keep one consumer warp per 8 channels. Both against the oracle, with a
+    ragged channel tile, per-direction planes and the options."""
+    _case("atrous2", 5, 7, D, 16, "f32", batch=batch, seq_chunks=1)
+    _case("atrous2", 7, 6, D, 16, "f32", batch=batch, seq_chunks=1, pdi=True, pdp=True)
+    _case("atrous2", 5, 7, D, 7, "f32", batch=batch, seq_chunks=1, gate=False, merge_scale=0.5)
+
+
 @pytest.mark.parametrize("nc", [2, 4, 8])
 def test_resident_tile_widths(nc):
     """BIDIR resident tiles are 4 channels wide while 8-channel tiles would leave SMs

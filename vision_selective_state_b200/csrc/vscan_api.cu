@@ -251,20 +251,26 @@ cudaError_t set_smem_once(Kernel* fn, int bytes, int* done_by_device, int max_de
 
 constexpr int kAttrDevices = 64;
 
+// float32 atrous launches whose per-warp chains dominate take the two-warp state
+// split: at most 4 CTAs per SM (b1 56x56: 42.1 -> 36.5 us), or 8 with the ZOH term's
+// longer per-state work (b8: 125 -> 109 us); the plain b8 launch (5.2 CTAs per SM)
+// measured 3 % slower split (61.1 against 63.1 us) and keeps one consumer warp.
+bool atrous_split(long long ctas, bool zoh) { return ctas <= (zoh ? 8LL : 4LL) * num_sms(); }
+
 template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL, int TOK = vscan::ST_TOK,
-          int CH = vscan::ST_CH>
+          int CH = vscan::ST_CH, int SS = 1>
 cudaError_t launch_stream_mode(vscan::ScanParams p, int k_base, int grid_z, cudaStream_t s)
 {
     static_assert(!(FL & vscan::FL_CKPT) || TOK == vscan::BW_TOK, "checkpoints every BW_TOK steps");
-    const size_t smem = vscan::stream_smem_bytes<T, KC, MODE, FL, CH, TOK>();
+    const size_t smem = vscan::stream_smem_bytes<T, KC, MODE, FL, CH, TOK, SS>();
     static int attr_done[kAttrDevices] = {};
-    cudaError_t e = set_smem_once(vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH, TOK>, (int)smem,
+    cudaError_t e = set_smem_once(vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH, TOK, SS>, (int)smem,
                                   attr_done, kAttrDevices);
     if (e != cudaSuccess) return e;
     p.k_base = k_base;
     const dim3 grid((p.D + CH - 1) / CH, p.batch, grid_z);
-    vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH, TOK>
-        <<<grid, vscan::StreamShape<T, KC, MODE, PW, CH, TOK>::THREADS, smem, s>>>(p);
+    vscan::stream_scan_kernel<RK, T, N16, KC, MODE, PW, FL, CH, TOK, SS>
+        <<<grid, vscan::StreamShape<T, KC, MODE, PW, CH, TOK, SS>::THREADS, smem, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -276,7 +282,14 @@ cudaError_t launch_stream_n(const vscan::ScanParams& p, cudaStream_t s)
 {
     using namespace vscan;
     if constexpr (RK == RK_ATROUS2) {
-        if constexpr (sizeof(T) == 4) return launch_stream_mode<RK, T, N16, 1, MODE_OWNER, 1, FL>(p, 0, 4, s);
+        if constexpr (sizeof(T) == 4) {
+            // few CTAs per SM: each channel's states split over two consumer warps and
+            // each chunk's steps over two producer warps, so every warp runs a chain
+            // half as long per chunk
+            if (atrous_split((long long)p.batch * ((p.D + ST_CH - 1) / ST_CH) * 4, (FL & FL_ZOH) != 0))
+                return launch_stream_mode<RK, T, N16, 1, MODE_OWNER, 2, FL, ST_TOK, ST_CH, 2>(p, 0, 4, s);
+            return launch_stream_mode<RK, T, N16, 1, MODE_OWNER, 1, FL>(p, 0, 4, s);
+        }
         else return launch_stream_mode<RK, T, N16, 4, MODE_OWNER, 1, FL>(p, 0, 1, s);
     } else if constexpr (RK == RK_BIDIR) {
         // two producer warps per direction (measured faster on Vim-Small); the fused

@@ -54,7 +54,7 @@
 
 #include "vscan_common.cuh"
 #include "vscan_route.cuh"
-#include "vscan_stream.cuh"
+#include "vscan_params.cuh"
 
 namespace vscan {
 

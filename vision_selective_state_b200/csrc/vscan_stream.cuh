@@ -4,11 +4,13 @@
 // of the route, and runs them as a software pipeline over chunks of TOK = 16
 // steps (32 for the long BIDIR sequences) with two kinds of warps:
 //
-//   consumer warps (CH / 8 per direction) run only the recurrence, each for 8
+//   consumer warps (SS * CH / 8 per direction) run only the recurrence, each for 8
 //     channels of the tile. Lane 4*c + g
 //     owns channel c of the tile and states 4g..4g+3, so the 16 states of a
 //     channel sit on 4 adjacent lanes and the read-out sum over n is a 4-lane
-//     reduction. Per step and state ("Vision Mamba ...", sec. 4;
+//     reduction; with SS = 2 (float32 atrous launches with few CTAs per SM) two
+//     warps share the 8 channels, warp h holding states 8h + 2g, 8h + 2g + 1, and
+//     the epilogue adds their two partial read-outs. Per step and state ("Vision Mamba ...", sec. 4;
 //     "EfficientVMamba", sec. 2), two states per packed f32x2 instruction:
 //         dA = 2^(Delta * A * log2 e)        (one SFU op)
 //         h  = dA * h + (Delta * u) * B      (FMUL + FFMA)
@@ -48,55 +50,16 @@
 #pragma once
 
 #include "vscan_common.cuh"
+#include "vscan_params.cuh"
 #include "vscan_route.cuh"
 
 namespace vscan {
 
 enum StreamMode : int { MODE_OWNER = 0, MODE_PARK = 1 };
 
-struct ScanParams {
-    RouteGeom g;
-    int batch, D, N;
-    const void* u;
-    const void* delta;
-    const void* B;
-    const void* C;
-    const void* z;
-    void* y;
-    const float* A;
-    const float* Dskip;
-    const float* bias;
-    long long in_dir;  // elements between directions of u / delta (0: shared)
-    long long bc_dir;  // elements between directions of B / C (0: shared)
-    int a_dir;         // elements between directions of A (0 or D*N)
-    int v_dir;         // elements between directions of Dskip / bias (0 or D)
-    int softplus;
-    float merge_scale;
-    int k_base;        // first direction of this launch (direction = k_base + blockIdx.z*KC + local)
-    float* scratch;    // PARK: [K][batch][tokens][D] float32
-    const float* conv_w;  // FL_CONV: [Kp][D][4]
-    const float* conv_b;  // FL_CONV: [Kp][D] (nullable)
-    float* ckpt;          // nullable: [K][batch][ceil(L/16)][D][16], the state entering every
-                          // 16-step chunk (saved for the backward pass)
-    int* status;          // nullable device word: bits DEV_STATUS_* OR-ed in by the kernels
-};
-
 constexpr int ST_TOK = 16;  // steps per chunk (default; the checkpointing run always uses 16)
 constexpr int ST_CH = 8;    // channels per consumer warp (a CTA covers CH = 8 or 16 channels)
 constexpr int ST_LOOK = 3;  // chunks between a gather and its discretization
-
-// ---- cp.async (16-byte, L2 only) ------------------------------------------------
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid)
-{
-    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-    const int n = valid ? 16 : 0;  // 0: fill the 16 bytes with zeros, read nothing
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n));
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
 // Gathered per-token rows of one direction's chunk, in the I/O type.
 template <typename T, int CH, int TOK>
@@ -139,7 +102,10 @@ template <int KC, int CH, int TOK> struct ConvRing<true, KC, CH, TOK> {
     float uc[KC][3][TOK][CH];
 };
 
-template <typename T, int KC, int MODE, int PW = 1, int CH = ST_CH, int TOK = ST_TOK>
+// SS: consumer warps sharing a channel's 16 states (1: lane 4c + g holds states
+// 4g..4g+3 of channel c; 2: warp h of the pair holds states 8h..8h+7, lane 4c + g
+// the pair 8h + 2g, 8h + 2g + 1, and the epilogue adds the two partial read-outs).
+template <typename T, int KC, int MODE, int PW = 1, int CH = ST_CH, int TOK = ST_TOK, int SS = 1>
 struct StreamShape {
     static constexpr bool F32 = sizeof(T) == 4;
     static constexpr bool PARK = MODE == MODE_PARK;
@@ -151,7 +117,7 @@ struct StreamShape {
     // B/C slot: until discretized at tau = c-1 (bf16) or consumed at tau = c (f32)
     static constexpr int NBC = LOOK + (F32 ? 2 : 1);
     static constexpr int NY = PARK ? 3 : 2;  // output ring
-    static constexpr int CW = CH / ST_CH;                // consumer warps per direction
+    static constexpr int CW = SS * CH / ST_CH;           // consumer warps per direction
     static constexpr int THREADS = 32 * KC * (CW + PW);  // CW consumers and PW producers per direction
     static constexpr int SPW = TOK / PW;                 // steps of a chunk per producer warp
     static constexpr int RPL = SPW * CH / 32;            // (step, channel) items per producer lane
@@ -159,19 +125,20 @@ struct StreamShape {
     static_assert(PW == 1 || PW == 2, "one or two producer warps per direction");
     static_assert(CH == 8 || CH == 16, "8 or 16 channels per CTA");
     static_assert(TOK == 16 || TOK == 32, "16- or 32-step chunks");
+    static_assert(SS == 1 || SS == 2, "one or two consumer warps per channel");
 };
 
-template <typename T, int KC, int MODE, int FL = 0, int CH = ST_CH, int TOK = ST_TOK>
+template <typename T, int KC, int MODE, int FL = 0, int CH = ST_CH, int TOK = ST_TOK, int SS = 1>
 struct StreamSmem : ConvRing<(FL & FL_CONV) != 0, KC, CH, TOK> {
-    using S = StreamShape<T, KC, MODE, 1, CH, TOK>;
+    using S = StreamShape<T, KC, MODE, 1, CH, TOK, SS>;
     TokStage<T, CH, TOK> tok[KC][S::NR];
     BCStage<T, TOK> bc[KC][S::NBC];
     PrepStage<!S::F32, (FL & FL_ZOH) != 0, CH, TOK> prep[KC][2];
-    float yout[KC][S::NY][TOK][CH];
+    float yout[KC][S::NY][SS][TOK][CH];  // read-outs (SS partial planes) of the last NY chunks
 };
 
-template <typename T, int KC, int MODE, int FL = 0, int CH = ST_CH, int TOK = ST_TOK>
-constexpr size_t stream_smem_bytes() { return sizeof(StreamSmem<T, KC, MODE, FL, CH, TOK>); }
+template <typename T, int KC, int MODE, int FL = 0, int CH = ST_CH, int TOK = ST_TOK, int SS = 1>
+constexpr size_t stream_smem_bytes() { return sizeof(StreamSmem<T, KC, MODE, FL, CH, TOK, SS>); }
 
 // Direction that adds up token p: the one visiting p in the latest chunk.
 template <int RK, int TOK>
@@ -190,10 +157,10 @@ __device__ __forceinline__ int finalizer(const RouteGeom& g, int p)
     return best_k;
 }
 
-template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL, int CH, int TOK>
-__global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH, TOK>::THREADS) stream_scan_kernel(const ScanParams p)
+template <int RK, typename T, bool N16, int KC, int MODE, int PW, int FL, int CH, int TOK, int SS = 1>
+__global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH, TOK, SS>::THREADS) stream_scan_kernel(const ScanParams p)
 {
-    using S = StreamShape<T, KC, MODE, PW, CH, TOK>;
+    using S = StreamShape<T, KC, MODE, PW, CH, TOK, SS>;
     constexpr int LOOK = S::LOOK;
     constexpr int SPW = S::SPW, RPL = S::RPL, CW = S::CW, NBCV = S::NBCV;
     constexpr int RSTEP = 32 / CH;  // rows between a producer lane's items
@@ -207,7 +174,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH, TOK>::THREADS
     constexpr bool F32 = S::F32;
     constexpr int KR = (RK == RK_BIDIR) ? 2 : 4;  // directions of the route
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    StreamSmem<T, KC, MODE, FL, CH, TOK>& sm = *reinterpret_cast<StreamSmem<T, KC, MODE, FL, CH, TOK>*>(smem_raw);
+    StreamSmem<T, KC, MODE, FL, CH, TOK, SS>& sm = *reinterpret_cast<StreamSmem<T, KC, MODE, FL, CH, TOK, SS>*>(smem_raw);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -222,65 +189,92 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH, TOK>::THREADS
         // =============================== consumer =================================
         const int kl = warp / CW;
         const int k = p.k_base + blockIdx.z * KC + kl;
-        const int cc = (warp % CW) * ST_CH + (lane >> 2), grp = lane & 3;  // channel of the tile
+        const int sub = warp % CW;                 // consumer warp of this direction
+        const int half = SS == 2 ? (sub & 1) : 0;  // SS = 2: which 8 states of the channel
+        const int cc = (sub / SS) * ST_CH + (lane >> 2), grp = lane & 3;  // channel of the tile
         const int d = c0 + cc;
         const bool dvalid = d < D;
-        float a2[4];
+        constexpr int NP = 2 / SS;  // state pairs per lane
+        const int n0 = SS == 1 ? 4 * grp : 8 * half + 2 * grp;  // this lane's first state
+        float2 a2p[NP];
+        float ia[2 * NP];  // ZOH: 1 / A per state (0 for A = 0, where x = Delta A = 0 selects the polynomial)
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const int n = 4 * grp + s;
-            a2[s] = (dvalid && n < N) ? __ldg(p.A + (long long)k * p.a_dir + (long long)d * N + n) * LOG2E : 0.f;
+        for (int q = 0; q < NP; ++q) {
+            float av[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int n = n0 + 2 * q + i;
+                av[i] = (dvalid && n < N) ? __ldg(p.A + (long long)k * p.a_dir + (long long)d * N + n) * LOG2E : 0.f;
+                ia[2 * q + i] = (av[i] != 0.f) ? LOG2E / av[i] : 0.f;
+            }
+            a2p[q] = make_float2(av[0], av[1]);
         }
-        const float2 a01 = make_float2(a2[0], a2[1]), a23 = make_float2(a2[2], a2[3]);
-        // ZOH: 1 / A per state (0 for A = 0, where x = Delta A = 0 selects the polynomial)
-        float ia[4];
+        float2 hp[NP];
 #pragma unroll
-        for (int s = 0; s < 4; ++s) ia[s] = (a2[s] != 0.f) ? LOG2E / a2[s] : 0.f;
-        float2 h01 = make_float2(0.f, 0.f), h23 = h01;
+        for (int q = 0; q < NP; ++q) hp[q] = make_float2(0.f, 0.f);
         __syncthreads();  // prologue: chunk 0 discretized
 
         float* ck = (CKPT && dvalid)
-                        ? p.ckpt + (((long long)k * p.batch + b) * nchunks * D + d) * 16 + 4 * grp : nullptr;
+                        ? p.ckpt + (((long long)k * p.batch + b) * nchunks * D + d) * 16 + n0 : nullptr;
         for (int tau = 0; tau <= last_tau; ++tau) {
             if (tau < nchunks) {
                 if constexpr (CKPT) {  // state entering chunk tau
-                    if (ck) *reinterpret_cast<float4*>(ck + (long long)tau * D * 16) = make_float4(h01.x, h01.y, h23.x, h23.y);
+                    if (ck) {
+                        if constexpr (NP == 2)
+                            *reinterpret_cast<float4*>(ck + (long long)tau * D * 16) = make_float4(hp[0].x, hp[0].y, hp[1].x, hp[1].y);
+                        else
+                            *reinterpret_cast<float2*>(ck + (long long)tau * D * 16) = hp[0];
+                    }
                 }
                 const auto& pr = sm.prep[kl][tau & 1];
                 const BCStage<T, TOK>& bcs = sm.bc[kl][tau % NBC];
-                float* yo = &sm.yout[kl][tau % NY][0][0];
+                float* yo = &sm.yout[kl][tau % NY][half][0][0];
                 // Software pipeline over the chunk's TOK steps: the loads, the SFU
                 // exponentials and the input terms of step j + 2 are issued before
                 // the state update of step j, which is the only serial dependency.
-                float2 e01[TOK], e23[TOK], w01[TOK], w23[TOK];
-                float4 cq[TOK];
+                float2 ep[TOK][NP], wp[TOK][NP], cp[TOK][NP];
                 auto front = [&](int j) {
                     const float2 dd = pr.dd[j][cc];
-                    float4 Bv;
+                    float2 Bq[NP], Cq[NP];
                     if constexpr (F32) {
-                        Bv = *reinterpret_cast<const float4*>(&bcs.B[j][4 * grp]);
-                        cq[j] = *reinterpret_cast<const float4*>(&bcs.C[j][4 * grp]);
+                        if constexpr (NP == 2) {
+                            const float4 Bv = *reinterpret_cast<const float4*>(&bcs.B[j][n0]);
+                            const float4 Cv = *reinterpret_cast<const float4*>(&bcs.C[j][n0]);
+                            Bq[0] = make_float2(Bv.x, Bv.y); Bq[1] = make_float2(Bv.z, Bv.w);
+                            Cq[0] = make_float2(Cv.x, Cv.y); Cq[1] = make_float2(Cv.z, Cv.w);
+                        } else {
+                            Bq[0] = *reinterpret_cast<const float2*>(&bcs.B[j][n0]);
+                            Cq[0] = *reinterpret_cast<const float2*>(&bcs.C[j][n0]);
+                        }
                     } else {
-                        Bv = pr.B[j][grp];
-                        cq[j] = pr.C[j][grp];
+                        const float4 Bv = pr.B[j][n0 >> 2], Cv = pr.C[j][n0 >> 2];
+                        if constexpr (NP == 2) {
+                            Bq[0] = make_float2(Bv.x, Bv.y); Bq[1] = make_float2(Bv.z, Bv.w);
+                            Cq[0] = make_float2(Cv.x, Cv.y); Cq[1] = make_float2(Cv.z, Cv.w);
+                        } else {
+                            const bool hi = n0 & 2;
+                            Bq[0] = hi ? make_float2(Bv.z, Bv.w) : make_float2(Bv.x, Bv.y);
+                            Cq[0] = hi ? make_float2(Cv.z, Cv.w) : make_float2(Cv.x, Cv.y);
+                        }
                     }
                     const float2 dsp2 = make_float2(dd.x, dd.x);
                     const float2 du2 = make_float2(dd.y, dd.y);
-                    const float2 x01 = __fmul2_rn(dsp2, a01);
-                    const float2 x23 = __fmul2_rn(dsp2, a23);
-                    e01[j] = make_float2(fast_exp2(x01.x), fast_exp2(x01.y));
-                    e23[j] = make_float2(fast_exp2(x23.x), fast_exp2(x23.y));
-                    w01[j] = __fmul2_rn(du2, make_float2(Bv.x, Bv.y));
-                    w23[j] = __fmul2_rn(du2, make_float2(Bv.z, Bv.w));
+                    float2 xq[NP];
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        xq[q] = __fmul2_rn(dsp2, a2p[q]);
+                        ep[j][q] = make_float2(fast_exp2(xq[q].x), fast_exp2(xq[q].y));
+                        wp[j][q] = __fmul2_rn(du2, Bq[q]);
+                        cp[j][q] = Cq[q];
+                    }
                     if constexpr (ZOH) {
                         const float rd = pr.rd[j][cc];
-                        const float x[4] = {x01.x * LN2, x01.y * LN2, x23.x * LN2, x23.y * LN2};
-                        const float e[4] = {e01[j].x, e01[j].y, e23[j].x, e23[j].y};
-                        float g[4];
 #pragma unroll
-                        for (int s = 0; s < 4; ++s) g[s] = zoh_phi(x[s], e[s], rd * ia[s]);
-                        w01[j] = __fmul2_rn(w01[j], make_float2(g[0], g[1]));
-                        w23[j] = __fmul2_rn(w23[j], make_float2(g[2], g[3]));
+                        for (int q = 0; q < NP; ++q) {
+                            const float g0 = zoh_phi(xq[q].x * LN2, ep[j][q].x, rd * ia[2 * q]);
+                            const float g1 = zoh_phi(xq[q].y * LN2, ep[j][q].y, rd * ia[2 * q + 1]);
+                            wp[j][q] = __fmul2_rn(wp[j][q], make_float2(g0, g1));
+                        }
                     }
                 };
                 front(0);
@@ -293,10 +287,11 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH, TOK>::THREADS
                     for (int jj = 0; jj < 4; ++jj) {
                         const int j = 4 * q + jj;
                         if (j + 2 < TOK) front(j + 2);
-                        h01 = __ffma2_rn(e01[j], h01, w01[j]);
-                        h23 = __ffma2_rn(e23[j], h23, w23[j]);
-                        float2 acc = __fmul2_rn(make_float2(cq[j].x, cq[j].y), h01);
-                        acc = __ffma2_rn(make_float2(cq[j].z, cq[j].w), h23, acc);
+#pragma unroll
+                        for (int r = 0; r < NP; ++r) hp[r] = __ffma2_rn(ep[j][r], hp[r], wp[j][r]);
+                        float2 acc = __fmul2_rn(cp[j][0], hp[0]);
+#pragma unroll
+                        for (int r = 1; r < NP; ++r) acc = __ffma2_rn(cp[j][r], hp[r], acc);
                         yp[jj] = acc.x + acc.y;
                     }
                     // Reduce-scatter over the 4 state-group lanes: lane grp keeps step 4q+grp.
@@ -566,7 +561,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH, TOK>::THREADS
     // Epilogue of chunk c: add the skip term, then store (one owner) or park / keep.
     auto finish_a = [&](int c) {
         const auto& st = sm.tok[kl][c % NR];
-        float* yo = &sm.yout[kl][c % NY][0][0];
+        float* yo = &sm.yout[kl][c % NY][0][0][0];  // SS = 2: the second partial plane follows
         int pj[RPL], fin[RPL];
         float yk[RPL], zz[RPL];
 #pragma unroll
@@ -577,7 +572,8 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH, TOK>::THREADS
             float uj;
             if constexpr (CONV) uj = sm.uc[kl][c % 3][j][ce];
             else uj = to_float(st.u[j][ce]);
-            yk[r] = fmaf(Dk, uj, yo[j * CH + ce]);
+            const float ys = SS == 2 ? yo[j * CH + ce] + yo[(SS - 1) * TOK * CH + j * CH + ce] : yo[j * CH + ce];
+            yk[r] = fmaf(Dk, uj, ys);
             zz[r] = z_base ? to_float(st.z[j][ce]) : 0.f;
         }
         // every row computes its value; only the stores are predicated
@@ -625,7 +621,7 @@ __global__ void __launch_bounds__(StreamShape<T, KC, MODE, PW, CH, TOK>::THREADS
     };
     auto finish_b = [&](int c) {
         const auto& st = sm.tok[kl][c % NR];
-        const float* yo = &sm.yout[kl][c % NY][0][0];
+        const float* yo = &sm.yout[kl][c % NY][0][0][0];  // the finalizer's value, kept by finish_a
 #pragma unroll
         for (int r = 0; r < RPL; ++r) {
             const int j = jl + RSTEP * r;
