@@ -130,7 +130,7 @@ def updates(wl):
 
 
 def roofline_object(bytes_all, upd_all, ms_all, hbm_peak, peak_src, sm_max, traffic, *, kernel,
-                    launch_ms_avg, algorithmic_bytes, backward=False):
+                    launch_ms_avg, algorithmic_bytes, backward=False, steps=1):
     """The bench line's roofline of the dominant kernel. Both floors of the forward are
     computed, compulsory bytes at the HBM peak and one ex2 per state update at the SFU
     peak; the larger one binds. An SFU-bound forward reports "bound": "alu" against the
@@ -154,11 +154,11 @@ def roofline_object(bytes_all, upd_all, ms_all, hbm_peak, peak_src, sm_max, traf
     fp32 = {"lane_ops_per_s": 4 * upd_rate, "peak": fma_peak, "frac": round(4 * upd_rate / fma_peak, 4),
             "note": "4 FP32 ops per state update (Delta*A, Delta*u*B, the state FMA, the "
                     "read-out FMA), 128 FP32 lanes/clk/SM x 148 SMs at max clock"}
-    t_hbm = bytes_all / (hbm_peak * 1e9)
-    t_sfu = upd_all / sfu_peak
+    t_hbm = bytes_all / (hbm_peak * 1e9) / steps  # per step
+    t_sfu = upd_all / sfu_peak / steps
     common = {"traffic": traffic, "kernel": kernel, "launch_ms_avg": launch_ms_avg,
               "algorithmic_bytes_per_launch": algorithmic_bytes,
-              "floors_ms": {"hbm": round(1e3 * t_hbm, 5), "sfu": round(1e3 * t_sfu, 5)}}
+              "floors_ms_per_step": {"hbm": round(1e3 * t_hbm, 5), "sfu": round(1e3 * t_sfu, 5)}}
     if not backward and t_sfu > t_hbm:
         return dict({"bound": "alu", "achieved": round(upd_rate / 1e9, 1), "peak": round(sfu_peak / 1e9, 1),
                      "unit": "G state updates/s", "frac": sfu["frac"],
@@ -548,7 +548,7 @@ def run_ours(args, wls):
     upd_all = sum(updates(w) * K for w in wls)
     roofline = roofline_object(bytes_all, upd_all, ms_all, hbm_peak, peak_src, sm_max, traffic,
                                kernel=kname, launch_ms_avg=round(ms_all / (K * nfw), 5),
-                               algorithmic_bytes=[ab(w) for w in wls], backward=args.backward)
+                               algorithmic_bytes=[ab(w) for w in wls], backward=args.backward, steps=K)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,

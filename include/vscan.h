@@ -363,8 +363,8 @@ typedef struct vscan_grads {
 /*
  * Device scratch bytes vscan_backward needs for these arguments (host only):
  * the pre-gate forward output, the forward's own workspace, the gradient of the
- * merged value, the state at every 16-step chunk boundary of every sequence
- * ([K][batch][ceil(L/16)][D][16] float32), and for the pooled routes the
+ * merged value (grid routes), the state at every 16-step chunk boundary of every
+ * sequence ([K][batch][ceil(L/16)][D][16] float32), and for the pooled routes the
  * pooled inputs and their gradients.
  */
 vscan_status vscan_backward_workspace_size(const vscan_route* route, const vscan_args* args,
@@ -386,8 +386,9 @@ vscan_status vscan_backward_plan_kernel(const vscan_route* route, const vscan_ar
  * Backward pass. args are the forward's arguments (args->y and args->workspace
  * are not used); dy is dL/dy, [batch][tokens][D] in args->dtype, device. The
  * call enqueues on stream: zeroing of the requested gradients, the pre-gate
- * forward pass, the gate's gradient, and the reverse-time adjoint scan of every
- * direction (checkpointed every 16 steps), then the gradients. Token gradients
+ * forward pass, the gate's gradient (for the pooled routes inside the pooling of
+ * the inputs and the merged value's gradient), and the reverse-time adjoint scan
+ * of every direction (checkpointed every 16 steps), then the gradients. Token gradients
  * shared by several directions, channel tiles or images are summed with float
  * atomics, so their low-order bits can vary from run to run.
  * Errors: as vscan_forward; VSCAN_ERR_UNSUPPORTED with the fused convolution,

@@ -14,20 +14,22 @@ SM_MAX = 1965.0
 HBM = 6650.0
 
 
-def _roof(idx, ms=1.0, backward=False):
+def _roof(idx, ms=1.0, backward=False, steps=1):
+    """Roofline of `steps` timed steps of config idx taking ms each."""
     wls = [workloads.WORKLOADS[n] for n in workloads.CONFIG_GROUPS[idx]]
     ab = bench.algorithmic_bytes_bwd if backward else bench.algorithmic_bytes
-    bytes_all = sum(ab(w) for w in wls)
-    upd_all = sum(bench.updates(w) for w in wls)
-    return bench.roofline_object(bytes_all, upd_all, ms, HBM, "fallback", SM_MAX, None, kernel="k",
-                                 launch_ms_avg=ms, algorithmic_bytes=[ab(w) for w in wls], backward=backward)
+    bytes_all = sum(ab(w) for w in wls) * steps
+    upd_all = sum(bench.updates(w) for w in wls) * steps
+    return bench.roofline_object(bytes_all, upd_all, ms * steps, HBM, "fallback", SM_MAX, None, kernel="k",
+                                 launch_ms_avg=ms, algorithmic_bytes=[ab(w) for w in wls], backward=backward,
+                                 steps=steps)
 
 
 def test_sfu_bound_workloads_report_alu_against_the_sfu_peak():
     for idx in (0, 1, 2, 4):
         r = _roof(idx)
         assert r["bound"] == "alu", idx
-        assert r["floors_ms"]["sfu"] > r["floors_ms"]["hbm"], idx
+        assert r["floors_ms_per_step"]["sfu"] > r["floors_ms_per_step"]["hbm"], idx
         sfu_peak_g = 16 * 148 * SM_MAX * 1e6 / 1e9
         assert r["peak"] == round(sfu_peak_g, 1)
         # achieved = state updates per second; frac = achieved / peak
@@ -39,7 +41,7 @@ def test_sfu_bound_workloads_report_alu_against_the_sfu_peak():
 def test_pooled_route_is_hbm_bound():
     r = _roof(3)
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
-    assert r["floors_ms"]["hbm"] > r["floors_ms"]["sfu"]
+    assert r["floors_ms_per_step"]["hbm"] > r["floors_ms_per_step"]["sfu"]
     assert abs(r["frac"] - r["achieved"] / HBM) < 1e-3
     assert "sfu" in r and "fp32" in r
 
@@ -48,10 +50,11 @@ def test_floors_match_the_workload_arithmetic():
     # Vim-Small: 64 images x 2 directions x 4097 steps x 768 channels x 16 states
     r = _roof(4)
     upd = 64 * 2 * 4097 * 768 * 16
-    assert abs(r["floors_ms"]["sfu"] - 1e3 * upd / (16 * 148 * SM_MAX * 1e6)) < 1e-4
-    # at 3.09 ms the SFU fraction is the floor over the time
-    r = _roof(4, ms=3.09)
-    assert abs(r["frac"] - r["floors_ms"]["sfu"] / 3.09) < 1e-3
+    assert abs(r["floors_ms_per_step"]["sfu"] - 1e3 * upd / (16 * 148 * SM_MAX * 1e6)) < 1e-4
+    # at 3.09 ms per step the SFU fraction is the floor over the time, for any step count
+    for steps in (1, 20):
+        r = _roof(4, ms=3.09, steps=steps)
+        assert abs(r["frac"] - r["floors_ms_per_step"]["sfu"] / 3.09) < 1e-3
 
 
 def test_backward_lines_stay_on_hbm():

@@ -393,11 +393,12 @@ class BackwardPlan:
         self._ra, self._rg = ctypes.byref(self.args), ctypes.byref(self.g)
 
     def kernels(self):
-        """Kernel launches of one run(): the pre-gate forward, the gate gradient and the
-        adjoint scan, plus pooling and unpooling for the pooled routes."""
+        """Kernel launches of one run(): the pre-gate forward, then the gate gradient and the
+        adjoint scan (grid routes) or pooling with the gate gradient, the adjoint scan and
+        unpooling (pooled routes)."""
         n = ctypes.c_int32()
         check(lib.vscan_plan_info(self.route.handle, ctypes.byref(self.args), ctypes.byref(n)))
-        return n.value + (4 if self.route.kind_name in ("pool_w", "pool_h") else 2)
+        return n.value + (3 if self.route.kind_name in ("pool_w", "pool_h") else 2)
 
     def kernel_name(self):
         """Name of the kernel that runs the adjoint scan (vscan_backward_plan_kernel)."""

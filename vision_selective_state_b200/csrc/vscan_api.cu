@@ -818,7 +818,7 @@ BwdLayout bwd_layout(const vscan_route* r, const vscan_args* a)
     auto take = [&](size_t bytes) { size_t o = off; off += round256(bytes); return o; };
     Lo.fwd_ws = take(workspace_need(r, a));
     Lo.pre = take(b * T * D * eb);
-    Lo.gy = take(b * T * D * sizeof(float));
+    Lo.gy = take(is_pool(g.kind) ? 0 : b * T * D * sizeof(float));  // pooled routes sum gy while pooling
     Lo.ckpt = take((size_t)g.K * b * nch * D * 16 * sizeof(float));
     if (is_pool(g.kind)) {
         Lo.pu = take(Ki * b * L * D * sizeof(float));
@@ -920,12 +920,15 @@ vscan_status backward_device(const vscan_route* r, const vscan_args* a, const vo
     float* ckpt = reinterpret_cast<float*>(ws + Lo.ckpt);
     vscan_status st = forward_device(r, &fa, s, pooled ? nullptr : ckpt);
     if (st != VSCAN_OK) return st;
-    // gradient of the gate and of the merged value
+    // gradient of the gate and of the merged value (the pooled routes form it inside
+    // their pooling kernel, member by member)
     float* gy = reinterpret_cast<float*>(ws + Lo.gy);
-    const long long n = b * TK * D;
-    const unsigned blocks = (unsigned)std::min<long long>((n + 255) / 256, 148LL * 16);
-    vscan::gate_grad_kernel<T><<<blocks, 256, 0, s>>>(static_cast<const T*>(dy), static_cast<const T*>(a->z),
-                                                      static_cast<const T*>(fa.y), a->merge_scale, n, gy, gr->dz);
+    if (!pooled) {
+        const long long n = b * TK * D;
+        const unsigned blocks = (unsigned)std::min<long long>((n + 255) / 256, 148LL * 16);
+        vscan::gate_grad_kernel<T><<<blocks, 256, 0, s>>>(static_cast<const T*>(dy), static_cast<const T*>(a->z),
+                                                          static_cast<const T*>(fa.y), a->merge_scale, n, gy, gr->dz);
+    }
     vscan::BwdParams p{};
     p.batch = a->batch; p.D = a->channels; p.N = a->d_state;
     p.a_dir = a->per_dir_params ? a->channels * a->d_state : 0;
@@ -956,7 +959,8 @@ vscan_status backward_device(const vscan_route* r, const vscan_args* a, const vo
         const long long in_dir = a->per_dir_inputs ? b * TK * D : 0, bc_dir = a->per_dir_inputs ? b * TK * N : 0;
         vscan::bwd_pool_kernel<T><<<dim3((unsigned)L, (unsigned)b), 256, 0, s>>>(
             g, (int)b, (int)D, (int)N, Ki, static_cast<const T*>(a->u), static_cast<const T*>(a->delta),
-            static_cast<const T*>(a->B), static_cast<const T*>(a->C), in_dir, bc_dir, gy, pu, praw, pB, pC, pg);
+            static_cast<const T*>(a->B), static_cast<const T*>(a->C), in_dir, bc_dir, static_cast<const T*>(dy),
+            static_cast<const T*>(a->z), static_cast<const T*>(fa.y), a->merge_scale, gr->dz, pu, praw, pB, pC, pg);
         // the pooled sequence scanned forward and reversed: a bidirectional route of length L
         vscan::make_geom(vscan::RK_BIDIR, 1, (int)L, -1, &p.g);
         p.u = pu; p.delta = praw; p.B = pB; p.C = pC;

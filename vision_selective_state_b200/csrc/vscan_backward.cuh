@@ -94,11 +94,16 @@ __global__ void gate_grad_kernel(const T* __restrict__ dy, const T* __restrict__
 
 // Pooled routes: pu, praw [Ki][batch][Lp][D] and pB, pC [Ki][batch][Lp][N] are
 // the means over the members of each pooled index, pg [batch][Lp][D] the sum
-// of gy over them. Grid (Lp, batch); threads stride over channels and states.
+// of gy over them. The gate's gradient is formed here, per member token (as
+// gate_grad_kernel does for the grid routes), so gy never goes through HBM:
+// gy = dy * s * SiLU(z) and dz = dy * pre * sigmoid(z) * (1 + z (1 - sigmoid(z))),
+// pre the forward output without the gate. Grid (Lp, batch); threads stride over
+// channels and states.
 template <typename T>
 __global__ void bwd_pool_kernel(RouteGeom g, int batch, int D, int N, int Ki, const T* u, const T* delta,
-                                const T* B, const T* C, long long in_dir, long long bc_dir, const float* gy,
-                                float* pu, float* praw, float* pB, float* pC, float* pg)
+                                const T* B, const T* C, long long in_dir, long long bc_dir, const T* dy,
+                                const T* z, const T* pre, float scale, float* dz, float* pu, float* praw,
+                                float* pB, float* pC, float* pg)
 {
     const int i = blockIdx.x, b = blockIdx.y, Lp = g.L;
     const int cnt = (g.kind == RK_POOL_W) ? g.w : g.h;
@@ -110,20 +115,32 @@ __global__ void bwd_pool_kernel(RouteGeom g, int batch, int D, int N, int Ki, co
             float su = 0.f, sr = 0.f, sg = 0.f;
             constexpr int U = 8;  // members per round, all loads issued before the sums
             for (int j0 = 0; j0 < cnt; j0 += U) {
-                float vu[U], vr[U], vg[U];
+                float vu[U], vr[U], vd[U], vz[U], vp[U];
 #pragma unroll
                 for (int v = 0; v < U; ++v) {
                     const bool in = j0 + v < cnt;
                     const long long o = (img + member(in ? j0 + v : 0)) * D + d;
                     vu[v] = in ? to_float(u[k * in_dir + o]) : 0.f;
                     vr[v] = in ? to_float(delta[k * in_dir + o]) : 0.f;
-                    vg[v] = (in && k == 0) ? gy[o] : 0.f;
+                    const bool gate = in && k == 0;
+                    vd[v] = gate ? to_float(dy[o]) : 0.f;
+                    vz[v] = (gate && z) ? to_float(z[o]) : 0.f;
+                    vp[v] = (gate && z && dz) ? to_float(pre[o]) : 0.f;
                 }
 #pragma unroll
                 for (int v = 0; v < U; ++v) {
                     su += vu[v];
                     sr += vr[v];
-                    sg += vg[v];
+                    if (k == 0) {
+                        if (z) {
+                            const float sgm = 1.0f / (1.0f + __expf(-vz[v]));
+                            sg += vd[v] * scale * vz[v] * sgm;
+                            if (dz && j0 + v < cnt)
+                                dz[(img + member(j0 + v)) * D + d] = vd[v] * vp[v] * sgm * (1.0f + vz[v] * (1.0f - sgm));
+                        } else {
+                            sg += vd[v] * scale;
+                        }
+                    }
                 }
             }
             const long long po = (((long long)k * batch + b) * Lp + i) * D + d;
